@@ -1,0 +1,214 @@
+/*
+ * kda.h — C ABI of the B200 (sm_100a) Kimi Delta Attention layer-forward library.
+ *
+ * The operation (Kimi Linear report, section 3, Eq. 1; "KDA Recurrence"
+ * problem page, problem statement), per batch row b and head h, with the
+ * state S a D_k x D_v matrix:
+ *
+ *   alpha_t = exp(g_min * sigmoid(z_t))                        (decay gate)
+ *   S_t     = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *   o~_t    = S_t^T q_t                          (read from the updated state)
+ *   x_t     = RMSNorm_{D_v}(o~_t) * sigmoid(gate_t),  RMSNorm(u) = u / sqrt(mean(u^2) + eps)
+ *   y_t     = concat_h(x_t) W_o^T                 (W_o is D_model x H*D_v)
+ *
+ * Conventions shared by every entry point
+ * ----------------------------------------
+ * - Every tensor pointer is DEVICE memory owned by the caller, contiguous and
+ *   row-major in exactly the shapes given, and 16-byte aligned.  The library
+ *   allocates nothing; scratch comes from a caller workspace whose size the
+ *   matching *_workspace_size query returns.
+ * - "dtype" tensors hold fp32 (KDA_F32) or bf16 (KDA_BF16) values; all inputs
+ *   of one call share it.  State and log-decay tensors are always fp32.
+ * - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
+ *   the legacy default stream).  A call returns once its kernels are queued.
+ * - Arguments are validated on the host before any launch; on failure nothing
+ *   is launched and a status other than KDA_OK is returned.  kda_last_error()
+ *   then gives a one-line message (thread-local, valid until the next call).
+ * - Outputs must not overlap inputs, except where an entry point says so.
+ * - Kernels never trap.  A device-side wait that runs out sets *dev_status to
+ *   KDA_ERR_TIMEOUT (when the caller passed dev_status) and the kernel returns.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kda_status {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, g_min >= 0, overlap */
+    KDA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (dtype, size) */
+    KDA_ERR_WORKSPACE = 3,    /* workspace NULL or smaller than the size query's answer */
+    KDA_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+    KDA_ERR_TIMEOUT = 5       /* a device-side bounded wait expired (reported via dev_status) */
+} kda_status_t;
+
+typedef enum kda_dtype { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype_t;
+
+/* Engine selection for kda_chunk_fwd. */
+typedef enum kda_engine {
+    KDA_ENGINE_AUTO = 0,   /* tensor-core engine when the shape allows it, else SIMT */
+    KDA_ENGINE_SIMT = 1,   /* exact-fp32 SIMT engine (any D_k, D_v <= 128, chunk <= 64) */
+    KDA_ENGINE_TC = 2      /* tcgen05 engine (bf16, D_k = D_v = 128, chunk = 64) */
+} kda_engine_t;
+
+/* Name of a status code ("KDA_OK", ...).  Never NULL. */
+const char *kda_status_string(kda_status_t status);
+
+/* Message describing the last failure on the calling thread ("" if none). */
+const char *kda_last_error(void);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int kda_version(void);
+
+/* Number of kernel launches this process has issued through the library so
+ * far (all devices and threads).  For counting the kernels of a timed region. */
+uint64_t kda_launch_count(void);
+
+/*
+ * kda_gate — decay gate of the "KDA Recurrence" page:
+ *   log_alpha[i] = g_min * sigmoid(z[i])   for i in [0, n)
+ * so alpha = exp(log_alpha) lies in [exp(g_min), 1].
+ *   z         : n values of `dtype` (the decay logits, same shape as the keys)
+ *   log_alpha : n fp32 values, out
+ * Errors: INVALID_ARG if n < 0, a pointer is NULL/misaligned, or g_min is not
+ * a finite negative number (the page's Constraints require g_min < 0).
+ */
+kda_status_t kda_gate(const void *z, kda_dtype_t dtype, int64_t n, float g_min,
+                      float *log_alpha, void *stream);
+
+/*
+ * kda_chunk_fwd — prefill: the Eq. 1 recurrence over whole sequences with the
+ * chunkwise (gated WY / UT-transform) algorithm of the Kimi Linear report,
+ * section 3.1 and appendix B (Propositions 1-2, Eqs. 16-19).  Sequences are
+ * cut into chunks of `chunk` tokens; inside a chunk the rank-1 updates are
+ * folded into a unit-lower-triangular solve, and the state is carried from
+ * chunk to chunk.  The last chunk of a sequence may be partial.
+ *
+ * Layout ("KDA Recurrence" page, problem statement):
+ *   q, k, z       (B, S, H, D_k)  dtype
+ *   log_decay     (B, S, H, D_k)  fp32 log(alpha) in [g_min, 0], or NULL to use z
+ *   g_min         the lower log-decay bound, finite and < 0 (always required:
+ *                 with log_decay it is the caller's bound on those values)
+ *   v             (B, S, H, D_v)  dtype
+ *   beta          (B, S, H)       dtype, in [0, 1]
+ *   initial_state (B, H, D_k, D_v) fp32, or NULL for zeros; never written
+ *                 unless it is the same pointer as final_state (in-place
+ *                 handoff is allowed: each sequence reads its state first)
+ *   gate_logits   (B, S, H, D_v)  dtype, or NULL
+ *   o             (B, S, H, D_v)  dtype, out.  With gate_logits == NULL it
+ *                 receives o~_t; otherwise RMSNorm(o~_t) * sigmoid(gate_t).
+ *   final_state   (B, H, D_k, D_v) fp32, out, or NULL to skip
+ * S = 0 is allowed (no token: final_state = initial_state).
+ * The tensor-core engine covers bf16, D_k = D_v = 128, chunk 64 and
+ * g_min >= -5.5 (the bound keeps every in-chunk decay factor it forms inside
+ * the fp32/bf16 exponent range); KDA_ENGINE_AUTO falls back to SIMT otherwise.
+ * Errors: INVALID_ARG (see conventions), UNSUPPORTED (D_k or D_v > 128,
+ * chunk > 64, or KDA_ENGINE_TC on a shape it does not cover), WORKSPACE.
+ */
+typedef struct kda_chunk_args {
+    int64_t B, S;
+    int32_t H, D_k, D_v;
+    kda_dtype_t dtype;
+    const void *q;
+    const void *k;
+    const void *v;
+    const void *z;
+    const float *log_decay;
+    float g_min;
+    const void *beta;
+    const float *initial_state;
+    const void *gate_logits;
+    float eps;
+    void *o;
+    float *final_state;
+    void *workspace;
+    size_t workspace_bytes;
+    int32_t chunk;          /* 0 = library default (64) */
+    kda_engine_t engine;
+    int32_t *dev_status;    /* optional device int32, 0 = fine; may be NULL */
+    void *stream;
+} kda_chunk_args;
+
+/* Workspace bytes kda_chunk_fwd needs for these arguments (pointers unused). */
+kda_status_t kda_chunk_workspace_size(const kda_chunk_args *args, size_t *bytes);
+
+kda_status_t kda_chunk_fwd(const kda_chunk_args *args);
+
+/*
+ * kda_decode_step — one token of the Eq. 1 recurrence for B independent
+ * sequences, fused in one pass over the fp32 state (the fused recurrent
+ * form: decay the state, predict k^T S, form the residual beta (v - pred),
+ * write k residual^T, read q^T S), the state updated IN PLACE: decode state
+ * is owned by the caller and advanced by design.
+ *   q, k, z       (B, H, D_k)  dtype;   log_decay (B, H, D_k) fp32 or NULL
+ *   g_min         lower log-decay bound, finite and < 0 (always required)
+ *   v             (B, H, D_v)  dtype;   beta (B, H) dtype
+ *   state         (B, H, D_k, D_v) fp32, read and written
+ *   gate_logits   (B, H, D_v)  dtype or NULL (as in kda_chunk_fwd)
+ *   o             (B, H, D_v)  dtype, out
+ * Errors: INVALID_ARG, UNSUPPORTED (D_k or D_v > 128).
+ */
+typedef struct kda_decode_args {
+    int64_t B;
+    int32_t H, D_k, D_v;
+    kda_dtype_t dtype;
+    const void *q;
+    const void *k;
+    const void *v;
+    const void *z;
+    const float *log_decay;
+    float g_min;
+    const void *beta;
+    float *state;
+    const void *gate_logits;
+    float eps;
+    void *o;
+    void *stream;
+} kda_decode_args;
+
+kda_status_t kda_decode_step(const kda_decode_args *args);
+
+/*
+ * kda_norm_gate — per-head RMS normalisation over D_v then the sigmoid output
+ * gate ("KDA Recurrence" page, problem statement):
+ *   x[n,h,:] = o[n,h,:] / sqrt(mean_j o[n,h,j]^2 + eps) * sigmoid(gate[n,h,:])
+ *   o, gate_logits, x : (N, H, D_v) dtype.  x may equal o (in place).
+ */
+kda_status_t kda_norm_gate(const void *o, const void *gate_logits, int64_t N,
+                           int32_t H, int32_t D_v, float eps, void *x,
+                           kda_dtype_t dtype, void *stream);
+
+/*
+ * kda_out_proj — head concat and output projection ("KDA Recurrence" page):
+ *   y[n, m] = sum_i x[n, i] * W_o[m, i],   i = h * D_v + j
+ *   x (N, K) dtype with K = H * D_v;  W_o (D_model, K) dtype;  y (N, D_model) dtype.
+ * bf16 with K % 64 == 0 and D_model % 16 == 0 runs on the tcgen05 tensor
+ * cores (fp32 accumulation); anything else runs an exact-fp32 SIMT GEMM.
+ */
+kda_status_t kda_out_proj(const void *x, const void *W_o, int64_t N, int32_t K,
+                          int32_t D_model, void *y, kda_dtype_t dtype, void *stream);
+
+/*
+ * kda_out_norm_gate_proj — kda_norm_gate then kda_out_proj:
+ *   y = concat_h(RMSNorm(o_h) * sigmoid(gate_h)) W_o^T
+ *   o, gate_logits (N, H, D_v); W_o (D_model, H*D_v); y (N, D_model); all dtype.
+ * The normalised activations go to the workspace (size query below).
+ */
+kda_status_t kda_out_norm_gate_proj_workspace_size(int64_t N, int32_t H, int32_t D_v,
+                                                   kda_dtype_t dtype, size_t *bytes);
+
+kda_status_t kda_out_norm_gate_proj(const void *o, const void *gate_logits,
+                                    const void *W_o, int64_t N, int32_t H, int32_t D_v,
+                                    int32_t D_model, float eps, void *y, kda_dtype_t dtype,
+                                    void *workspace, size_t workspace_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,11 @@
+"""B200 (sm_100a) Kimi Delta Attention layer forward.
+
+The compute lives in ``libkda.so`` (hand-written CUDA behind the C ABI of
+``include/kda.h``); this package only marshals torch tensors into it.
+"""
+from ._lib import KDAError, load as load_library  # noqa: F401
+from .api import (chunk_fwd, chunk_workspace_bytes, decode_step, gate, kda_decode, kda_forward,  # noqa: F401
+                  norm_gate, out_norm_gate_proj, out_proj)
+
+__all__ = ["chunk_fwd", "chunk_workspace_bytes", "decode_step", "gate", "kda_decode", "kda_forward",
+           "norm_gate", "out_norm_gate_proj", "out_proj", "KDAError", "load_library"]

@@ -1,0 +1,244 @@
+"""Torch-facing binding of libkda: argument marshalling only.
+
+Every step of the layer runs inside libkda's CUDA kernels; torch supplies the
+device memory and the current stream.  Names follow the "KDA Recurrence"
+problem page: query, key (B,S,H,D_k); value, output gate logits (B,S,H,D_v);
+write strength beta (B,S,H); decay logits (B,S,H,D_k); state (B,H,D_k,D_v);
+output projection (D_model, H*D_v).
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+from ._lib import ChunkArgs, DecodeArgs, check
+
+_DT = {torch.float32: _lib.KDA_F32, torch.bfloat16: _lib.KDA_BF16}
+ENGINES = {"auto": _lib.ENGINE_AUTO, "simt": _lib.ENGINE_SIMT, "tc": _lib.ENGINE_TC}
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    try:
+        return _DT[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)") from None
+
+
+def _dev(t, name, dtype=None, shape=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype} (got {t.dtype})")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def gate(z: torch.Tensor, g_min: float) -> torch.Tensor:
+    """log(alpha) = g_min * sigmoid(z), fp32, same shape as z."""
+    _dev(z, "z")
+    out = torch.empty(z.shape, dtype=torch.float32, device=z.device)
+    check("kda_gate", _lib.load().kda_gate(_ptr(z), _dtype_code(z), z.numel(), float(g_min), _ptr(out),
+                                           _stream(z.device)))
+    return out
+
+
+def chunk_fwd(q, k, v, beta, *, z=None, log_decay=None, g_min=-5.0, initial_state=None,
+              gate_logits=None, eps=1e-6, chunk=64, engine="auto", want_final_state=True,
+              out=None, final_state=None, dev_status=None):
+    """Chunkwise prefill.  Returns (o, final_state):
+    o (B,S,H,D_v) in the input dtype holds o~ (gate_logits None) or
+    RMSNorm(o~) * sigmoid(gate_logits); final_state (B,H,D_k,D_v) fp32 or None.
+    ``final_state`` may be the same tensor as ``initial_state`` (in-place handoff)."""
+    _dev(q, "q")
+    dt = q.dtype
+    B, S, H, Dk = q.shape
+    Dv = v.shape[-1]
+    _dev(k, "k", dt, q.shape)
+    _dev(v, "v", dt, (B, S, H, Dv))
+    if beta.dim() == 4 and beta.shape[-1] == 1:
+        beta = beta.view(B, S, H)
+    _dev(beta, "beta", dt, (B, S, H))
+    _dev(z, "z", dt, q.shape)
+    _dev(log_decay, "log_decay", torch.float32, q.shape)
+    _dev(initial_state, "initial_state", torch.float32, (B, H, Dk, Dv))
+    _dev(gate_logits, "gate_logits", dt, (B, S, H, Dv))
+    _dev(dev_status, "dev_status", torch.int32)
+    if out is None:
+        out = torch.empty((B, S, H, Dv), dtype=dt, device=q.device)
+    _dev(out, "out", dt, (B, S, H, Dv))
+    if final_state is None and want_final_state:
+        final_state = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
+    _dev(final_state, "final_state", torch.float32, (B, H, Dk, Dv))
+    a = ChunkArgs(B=B, S=S, H=H, D_k=Dk, D_v=Dv, dtype=_dtype_code(q),
+                  q=_ptr(q), k=_ptr(k), v=_ptr(v), z=_ptr(z), log_decay=_ptr(log_decay),
+                  g_min=float(g_min), beta=_ptr(beta), initial_state=_ptr(initial_state),
+                  gate_logits=_ptr(gate_logits), eps=float(eps), o=_ptr(out),
+                  final_state=_ptr(final_state), workspace=None, workspace_bytes=0,
+                  chunk=int(chunk), engine=ENGINES[engine], dev_status=_ptr(dev_status),
+                  stream=_stream(q.device))
+    lib = _lib.load()
+    nbytes = ctypes.c_size_t(0)
+    check("kda_chunk_workspace_size", lib.kda_chunk_workspace_size(ctypes.byref(a), ctypes.byref(nbytes)))
+    ws = None
+    if nbytes.value:
+        ws = torch.empty(nbytes.value, dtype=torch.uint8, device=q.device)
+        a.workspace = _ptr(ws)
+        a.workspace_bytes = nbytes.value
+    check("kda_chunk_fwd", lib.kda_chunk_fwd(ctypes.byref(a)))
+    return out, final_state
+
+
+def chunk_workspace_bytes(B, S, H, Dk, Dv, dtype=torch.bfloat16, chunk=64, engine="auto", g_min=-5.0):
+    a = ChunkArgs(B=B, S=S, H=H, D_k=Dk, D_v=Dv, dtype=_DT[dtype], g_min=float(g_min), eps=1e-6,
+                  chunk=chunk, engine=ENGINES[engine])
+    n = ctypes.c_size_t(0)
+    check("kda_chunk_workspace_size", _lib.load().kda_chunk_workspace_size(ctypes.byref(a), ctypes.byref(n)))
+    return n.value
+
+
+def decode_step(q, k, v, beta, state, *, z=None, log_decay=None, g_min=-5.0, gate_logits=None, eps=1e-6,
+                out=None):
+    """One token for B sequences: q,k,z (B,H,D_k); v, gate_logits (B,H,D_v); beta (B,H);
+    state (B,H,D_k,D_v) fp32 is advanced IN PLACE.  Returns o (B,H,D_v) in the input dtype."""
+    _dev(q, "q")
+    dt = q.dtype
+    B, H, Dk = q.shape
+    Dv = v.shape[-1]
+    _dev(k, "k", dt, q.shape)
+    _dev(v, "v", dt, (B, H, Dv))
+    if beta.dim() == 3 and beta.shape[-1] == 1:
+        beta = beta.view(B, H)
+    _dev(beta, "beta", dt, (B, H))
+    _dev(z, "z", dt, q.shape)
+    _dev(log_decay, "log_decay", torch.float32, q.shape)
+    _dev(state, "state", torch.float32, (B, H, Dk, Dv))
+    _dev(gate_logits, "gate_logits", dt, (B, H, Dv))
+    if out is None:
+        out = torch.empty((B, H, Dv), dtype=dt, device=q.device)
+    _dev(out, "out", dt, (B, H, Dv))
+    a = DecodeArgs(B=B, H=H, D_k=Dk, D_v=Dv, dtype=_dtype_code(q), q=_ptr(q), k=_ptr(k), v=_ptr(v),
+                   z=_ptr(z), log_decay=_ptr(log_decay), g_min=float(g_min), beta=_ptr(beta),
+                   state=_ptr(state), gate_logits=_ptr(gate_logits), eps=float(eps), o=_ptr(out),
+                   stream=_stream(q.device))
+    check("kda_decode_step", _lib.load().kda_decode_step(ctypes.byref(a)))
+    return out
+
+
+def norm_gate(o, gate_logits, eps=1e-6, out=None):
+    """Per-head RMSNorm over D_v then sigmoid gate; o, gate_logits (..., H, D_v)."""
+    _dev(o, "o")
+    _dev(gate_logits, "gate_logits", o.dtype, o.shape)
+    H, Dv = o.shape[-2], o.shape[-1]
+    N = o.numel() // (H * Dv)
+    if out is None:
+        out = torch.empty_like(o)
+    _dev(out, "out", o.dtype, o.shape)
+    check("kda_norm_gate", _lib.load().kda_norm_gate(_ptr(o), _ptr(gate_logits), N, H, Dv, float(eps),
+                                                     _ptr(out), _dtype_code(o), _stream(o.device)))
+    return out
+
+
+def out_proj(x, W_o, out=None):
+    """y = x W_o^T with x (..., K) and W_o (D_model, K)."""
+    _dev(x, "x")
+    Dm, K = W_o.shape
+    _dev(W_o, "W_o", x.dtype)
+    if x.shape[-1] != K:
+        raise ValueError("x's last dimension must equal W_o's second")
+    N = x.numel() // K
+    if out is None:
+        out = torch.empty((*x.shape[:-1], Dm), dtype=x.dtype, device=x.device)
+    _dev(out, "out", x.dtype, (*x.shape[:-1], Dm))
+    check("kda_out_proj", _lib.load().kda_out_proj(_ptr(x), _ptr(W_o), N, K, Dm, _ptr(out), _dtype_code(x),
+                                                   _stream(x.device)))
+    return out
+
+
+def out_norm_gate_proj(o, gate_logits, W_o, eps=1e-6, out=None):
+    """y = concat_h(RMSNorm(o_h) * sigmoid(gate_h)) W_o^T; o, gate_logits (..., H, D_v)."""
+    _dev(o, "o")
+    _dev(gate_logits, "gate_logits", o.dtype, o.shape)
+    _dev(W_o, "W_o", o.dtype)
+    H, Dv = o.shape[-2], o.shape[-1]
+    Dm = W_o.shape[0]
+    N = o.numel() // (H * Dv)
+    lib = _lib.load()
+    n = ctypes.c_size_t(0)
+    check("kda_out_norm_gate_proj_workspace_size",
+          lib.kda_out_norm_gate_proj_workspace_size(N, H, Dv, _dtype_code(o), ctypes.byref(n)))
+    ws = torch.empty(max(n.value, 16), dtype=torch.uint8, device=o.device)
+    if out is None:
+        out = torch.empty((*o.shape[:-2], Dm), dtype=o.dtype, device=o.device)
+    check("kda_out_norm_gate_proj",
+          lib.kda_out_norm_gate_proj(_ptr(o), _ptr(gate_logits), _ptr(W_o), N, H, Dv, Dm, float(eps), _ptr(out),
+                                     _dtype_code(o), _ptr(ws), n.value, _stream(o.device)))
+    return out
+
+
+def kda_forward(query, key, value, decay_logits, write_strength, output_gate_logits, output_projection,
+                initial_state=None, g_min=-5.0, eps=1e-6, *, state_dtype=None, chunk=64, engine="auto"):
+    """The KDA layer forward with the "KDA Recurrence" page's interface.
+
+    Returns {"outputs": (B,S,D_model), "final_state": (B,H,D_k,D_v)}, both in the
+    input dtype (``state_dtype`` overrides the state's dtype, e.g. torch.float32 to
+    keep the library's fp32 state) and on the inputs' device.  CPU inputs are
+    copied to the current CUDA device and the results copied back; no input is
+    modified.
+    """
+    dt = query.dtype
+    cpu = not query.is_cuda
+    dev = torch.device("cuda", torch.cuda.current_device()) if cpu else query.device
+
+    def up(t, dtype=None):
+        if t is None:
+            return None
+        if t.device != dev:
+            t = t.pin_memory().to(dev, non_blocking=True) if cpu else t.to(dev)
+        if dtype is not None and t.dtype != dtype:
+            t = t.to(dtype)
+        return t.contiguous()
+
+    q, k, v, z, gl, W = (up(t) for t in (query, key, value, decay_logits, output_gate_logits, output_projection))
+    beta = up(write_strength)
+    B, S, H, Dk = q.shape
+    beta = beta.reshape(B, S, H)
+    s0 = up(initial_state, torch.float32)
+    if s0 is not None and s0.data_ptr() == (initial_state.data_ptr() if initial_state is not None else -1):
+        s0 = s0.clone()  # never hand the caller's tensor to a kernel that could write it
+    x, sf = chunk_fwd(q, k, v, beta, z=z, g_min=g_min, initial_state=s0, gate_logits=gl, eps=eps,
+                      chunk=chunk, engine=engine)
+    y = out_proj(x.view(B, S, H * v.shape[-1]), W)
+    sf = sf.to(state_dtype or dt)
+    if cpu:
+        y_h = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+        s_h = torch.empty(sf.shape, dtype=sf.dtype, pin_memory=True)
+        y_h.copy_(y, non_blocking=True)
+        s_h.copy_(sf, non_blocking=True)
+        torch.cuda.current_stream(dev).synchronize()
+        return {"outputs": y_h, "final_state": s_h}
+    return {"outputs": y, "final_state": sf}
+
+
+def kda_decode(query, key, value, decay_logits, write_strength, output_gate_logits, output_projection, state,
+               g_min=-5.0, eps=1e-6):
+    """One decode token through the whole layer: q,k,z (B,H,D_k); v, gate (B,H,D_v);
+    beta (B,H); state (B,H,D_k,D_v) fp32 advanced in place.  Returns y (B, D_model)."""
+    x = decode_step(query, key, value, write_strength, state, z=decay_logits, g_min=g_min,
+                    gate_logits=output_gate_logits, eps=eps)
+    B, H, Dv = x.shape
+    return out_proj(x.view(B, H * Dv), output_projection)

@@ -1,0 +1,244 @@
+// Exact-fp32 SIMT chunk engine for the KDA prefill.
+//
+// Chunkwise form of Eq. 1 (Kimi Linear report, section 3.1 and appendix B,
+// Propositions 1-2): inside a chunk of C tokens with in-chunk cumulative
+// log-decay G_r = sum_{i<=r} log alpha_i (so gamma_{i->r} = exp(G_r - G_i)),
+//
+//   A[r,i] = beta_r sum_c k_rc k_ic exp(G_rc - G_ic)          i < r
+//   (I + A) [W | U] = [Diag(beta)(K * e^G) | Diag(beta) V]   unit-lower, forward substitution
+//   V'     = U - W S_0                 (the "state-corrected" residual values)
+//   M[r,i] = sum_c q_rc k_ic exp(G_rc - G_ic)                 i <= r  (read after update)
+//   O      = (Q * e^G) S_0 + M V'
+//   S_C    = Diag(e^{G_C}) S_0 + (K * e^{G_C - G})^T V'
+//
+// W and U are the stacked w_r, u_r of Eqs. 17 and 19 (beta_r multiplies the
+// whole bracket), and O, S_C follow from Eqs. 16 and 18 inserted into
+// o_r = S_r^T q_r.  Every decay factor is formed as one exp of a difference
+// <= 0, so any g_min is safe.  One CTA owns one (b, h) and a slice of value
+// columns and walks the chunks of that sequence in order.
+//
+// Precision: G reaches |g_min| * C (320 for g_min = -5, C = 64), and
+// exp(G_r - G_i) for nearby r, i takes the difference of two such numbers.  In
+// fp32 that difference carries an absolute error near 1e-5, which is larger
+// than the 1e-6 / 1e-5 fp32 tolerance allows, so for fp32 inputs the per-token
+// log-decay and G are kept in fp64 (GT = double); everything else is fp32.
+#include "kda_internal.cuh"
+
+namespace kda {
+
+namespace {
+
+constexpr int NT = 256;
+constexpr int MAX_VS = 32;
+
+struct SimtParams {
+    int64_t S;
+    int H, Dk, Dv, C, VS;
+    const void *q, *k, *v, *z, *beta;
+    const float *log_decay;
+    float g_min;
+    const float *S0;
+    void *o;
+    float *Sf;
+};
+
+template <typename GT>
+__host__ __device__ inline size_t simt_smem_bytes(int C, int Dk, int VS) {
+    const int LD = Dk + 1;
+    return sizeof(GT) * (size_t)C * LD +
+           sizeof(float) * ((size_t)3 * C * LD + 2 * C * (C + 1) + (size_t)C * VS + (size_t)Dk * VS + C);
+}
+
+template <typename T> struct GType { using type = float; };
+template <> struct GType<float> { using type = double; };
+
+__device__ __forceinline__ double log_alpha_gt(double z, float g_min, double) {
+    return (double)g_min / (1.0 + exp(-z));
+}
+__device__ __forceinline__ float log_alpha_gt(float z, float g_min, float) { return log_alpha_of(z, g_min); }
+
+template <typename T>
+__global__ void __launch_bounds__(NT) chunk_simt_kernel(SimtParams p) {
+    using GT = typename GType<T>::type;
+    extern __shared__ __align__(16) unsigned char smraw[];
+    const int C = p.C, Dk = p.Dk, VS = p.VS, LD = Dk + 1, LC = C + 1;
+    GT *sG = reinterpret_cast<GT *>(smraw);                       // C x LD  cumulative log-decay
+    float *sK = reinterpret_cast<float *>(sG + (size_t)C * LD);   // C x LD  keys, later K * e^{G_C - G}
+    float *sQ = sK + C * LD;        // C x LD   queries, later Q * e^G
+    float *sW = sQ + C * LD;        // C x LD   W
+    float *sA = sW + C * LD;        // C x LC
+    float *sM = sA + C * LC;        // C x LC
+    float *sU = sM + C * LC;        // C x VS   U, then V'
+    float *sS = sU + C * VS;        // Dk x VS  state slice
+    float *sB = sS + Dk * VS;       // C        beta
+
+    const int bh = blockIdx.x;
+    const int b = bh / p.H, h = bh % p.H;
+    const int j0 = blockIdx.y * VS;
+    const int nj = min(VS, p.Dv - j0);
+    const int tid = threadIdx.x;
+    const T *q = (const T *)p.q, *k = (const T *)p.k, *v = (const T *)p.v, *z = (const T *)p.z;
+    const T *beta = (const T *)p.beta;
+    T *o = (T *)p.o;
+    const int64_t strideK = (int64_t)p.H * Dk;
+
+    for (int idx = tid; idx < Dk * VS; idx += NT) {
+        const int c = idx / VS, j = idx % VS;
+        float s = 0.f;
+        if (p.S0 && j < nj) s = p.S0[((int64_t)bh * Dk + c) * p.Dv + j0 + j];
+        sS[idx] = s;
+    }
+
+    for (int64_t t0 = 0; t0 < p.S; t0 += C) {
+        const int len = (int)min((int64_t)C, p.S - t0);
+        const int64_t row0 = (int64_t)b * p.S + t0;  // token row index of the chunk start
+        // ---- loads (rows past the end of the sequence are zero: they change nothing)
+        for (int idx = tid; idx < C * Dk; idx += NT) {
+            const int r = idx / Dk, c = idx % Dk;
+            float kv = 0.f, qv = 0.f;
+            GT g = 0;
+            if (r < len) {
+                const int64_t off = (row0 + r) * strideK + (int64_t)h * Dk + c;
+                kv = load_elem(k, off);
+                qv = load_elem(q, off);
+                g = p.log_decay ? (GT)p.log_decay[off] : log_alpha_gt((GT)load_elem(z, off), p.g_min, GT(0));
+            }
+            sK[r * LD + c] = kv;
+            sQ[r * LD + c] = qv;
+            sG[r * LD + c] = g;
+        }
+        for (int idx = tid; idx < C * VS; idx += NT) {
+            const int r = idx / VS, j = idx % VS;
+            float u = 0.f;
+            if (r < len && j < nj) {
+                const int64_t tok = (row0 + r) * p.H + h;
+                u = load_elem(beta, tok) * load_elem(v, tok * p.Dv + j0 + j);
+            }
+            sU[idx] = u;
+        }
+        for (int r = tid; r < C; r += NT)
+            sB[r] = (r < len) ? load_elem(beta, (row0 + r) * p.H + h) : 0.f;
+        __syncthreads();
+        // ---- in-chunk cumulative log-decay G
+        for (int c = tid; c < Dk; c += NT) {
+            GT acc = 0;
+            for (int r = 0; r < C; ++r) {
+                acc += sG[r * LD + c];
+                sG[r * LD + c] = acc;
+            }
+        }
+        __syncthreads();
+        // ---- A (strictly lower, beta-weighted) and M (lower with diagonal)
+        for (int idx = tid; idx < C * C; idx += NT) {
+            const int r = idx / C, i = idx % C;
+            float a = 0.f, m = 0.f;
+            if (i <= r) {
+                for (int c = 0; c < Dk; ++c) {
+                    const float e = expf((float)(sG[r * LD + c] - sG[i * LD + c]));
+                    const float ki = sK[i * LD + c] * e;
+                    a += sK[r * LD + c] * ki;
+                    m += sQ[r * LD + c] * ki;
+                }
+            }
+            sA[r * LC + i] = (i < r) ? sB[r] * a : 0.f;
+            sM[r * LC + i] = m;
+        }
+        __syncthreads();
+        // ---- forward substitution of (I + A) X = RHS, one column per thread
+        for (int col = tid; col < Dk + VS; col += NT) {
+            if (col < Dk) {
+                const int c = col;
+                for (int r = 0; r < C; ++r) {
+                    float x = sB[r] * sK[r * LD + c] * expf((float)sG[r * LD + c]);
+                    for (int i = 0; i < r; ++i) x -= sA[r * LC + i] * sW[i * LD + c];
+                    sW[r * LD + c] = x;
+                }
+            } else {
+                const int j = col - Dk;
+                for (int r = 0; r < C; ++r) {
+                    float x = sU[r * VS + j];
+                    for (int i = 0; i < r; ++i) x -= sA[r * LC + i] * sU[i * VS + j];
+                    sU[r * VS + j] = x;
+                }
+            }
+        }
+        __syncthreads();
+        // ---- V' = U - W S_0
+        for (int idx = tid; idx < C * VS; idx += NT) {
+            const int r = idx / VS, j = idx % VS;
+            float acc = 0.f;
+            for (int c = 0; c < Dk; ++c) acc += sW[r * LD + c] * sS[c * VS + j];
+            sU[idx] -= acc;
+        }
+        __syncthreads();
+        // ---- Q * e^G and K * e^{G_C - G}
+        for (int idx = tid; idx < C * Dk; idx += NT) {
+            const int r = idx / Dk, c = idx % Dk;
+            const GT G = sG[r * LD + c];
+            sQ[r * LD + c] *= expf((float)G);
+            sK[r * LD + c] *= expf((float)(sG[(C - 1) * LD + c] - G));
+        }
+        __syncthreads();
+        // ---- O = (Q e^G) S_0 + M V'
+        for (int idx = tid; idx < C * VS; idx += NT) {
+            const int r = idx / VS, j = idx % VS;
+            if (r < len && j < nj) {
+                float acc = 0.f;
+                for (int c = 0; c < Dk; ++c) acc += sQ[r * LD + c] * sS[c * VS + j];
+                for (int i = 0; i <= r; ++i) acc += sM[r * LC + i] * sU[i * VS + j];
+                store_elem(o, ((row0 + r) * p.H + h) * (int64_t)p.Dv + j0 + j, acc);
+            }
+        }
+        __syncthreads();
+        // ---- S_C = Diag(e^{G_C}) S_0 + (K e^{G_C - G})^T V'
+        for (int idx = tid; idx < Dk * VS; idx += NT) {
+            const int c = idx / VS, j = idx % VS;
+            float acc = expf((float)sG[(C - 1) * LD + c]) * sS[idx];
+            for (int r = 0; r < C; ++r) acc += sK[r * LD + c] * sU[r * VS + j];
+            sS[idx] = acc;
+        }
+        __syncthreads();
+    }
+    if (p.Sf) {
+        for (int idx = tid; idx < Dk * VS; idx += NT) {
+            const int c = idx / VS, j = idx % VS;
+            if (j < nj) p.Sf[((int64_t)bh * Dk + c) * p.Dv + j0 + j] = sS[idx];
+        }
+    }
+}
+
+}  // namespace
+
+size_t chunk_simt_workspace(const kda_chunk_args &, int) { return 0; }
+
+kda_status_t launch_chunk_simt(const kda_chunk_args &a, int chunk, cudaStream_t st) {
+    SimtParams p;
+    p.S = a.S;
+    p.H = a.H;
+    p.Dk = a.D_k;
+    p.Dv = a.D_v;
+    p.C = chunk;
+    p.VS = a.D_v < MAX_VS ? a.D_v : MAX_VS;
+    p.q = a.q; p.k = a.k; p.v = a.v; p.z = a.z; p.beta = a.beta;
+    p.log_decay = a.log_decay;
+    p.g_min = a.g_min;
+    p.S0 = a.initial_state;
+    p.o = a.o;
+    p.Sf = a.final_state;
+    const int64_t nbh = a.B * a.H;
+    if (nbh > 0x7fffffffLL) return fail(KDA_ERR_UNSUPPORTED, "B*H too large");
+    const dim3 grid((unsigned)nbh, (unsigned)((a.D_v + p.VS - 1) / p.VS));
+    const size_t smem = a.dtype == KDA_F32 ? simt_smem_bytes<double>(p.C, p.Dk, p.VS)
+                                           : simt_smem_bytes<float>(p.C, p.Dk, p.VS);
+    if (a.dtype == KDA_F32) {
+        cudaFuncSetAttribute(chunk_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        chunk_simt_kernel<float><<<grid, NT, smem, st>>>(p);
+    } else {
+        cudaFuncSetAttribute(chunk_simt_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+        chunk_simt_kernel<__nv_bfloat16><<<grid, NT, smem, st>>>(p);
+    }
+    return check_launch("chunk_simt_kernel");
+}
+
+}  // namespace kda

@@ -1,0 +1,59 @@
+// Internal declarations shared by the CUDA translation units of libkda.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+// ----------------------------------------------------------------- host-side error state
+void set_error(const char *fmt, ...);
+kda_status_t fail(kda_status_t s, const char *fmt, ...);
+kda_status_t check_launch(const char *what);
+
+// ----------------------------------------------------------------- element access
+__device__ __forceinline__ float load_elem(const float *p, int64_t i) { return p[i]; }
+__device__ __forceinline__ float load_elem(const __nv_bfloat16 *p, int64_t i) {
+    return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void store_elem(float *p, int64_t i, float v) { p[i] = v; }
+__device__ __forceinline__ void store_elem(__nv_bfloat16 *p, int64_t i, float v) {
+    p[i] = __float2bfloat16_rn(v);
+}
+
+// sigmoid in full fp32 precision (expf, not the fast approximation)
+__device__ __forceinline__ float sigmoid_precise(float x) { return 1.0f / (1.0f + expf(-x)); }
+
+// log(alpha) from the decay logits: g_min * sigmoid(z)
+__device__ __forceinline__ float log_alpha_of(float z, float g_min) {
+    return g_min * sigmoid_precise(z);
+}
+
+// ----------------------------------------------------------------- launchers (one per .cu)
+kda_status_t launch_gate(const void *z, kda_dtype_t dt, int64_t n, float g_min, float *out,
+                         cudaStream_t st);
+
+kda_status_t launch_decode(const kda_decode_args &a, cudaStream_t st);
+
+// SIMT chunk engine: exact fp32 arithmetic, any D_k, D_v <= 128, chunk <= 64.
+kda_status_t launch_chunk_simt(const kda_chunk_args &a, int chunk, cudaStream_t st);
+size_t chunk_simt_workspace(const kda_chunk_args &a, int chunk);
+
+// tcgen05 chunk engine: bf16, D_k = D_v = 128, chunk 64.
+bool chunk_tc_supported(const kda_chunk_args &a, int chunk);
+size_t chunk_tc_workspace(const kda_chunk_args &a);
+kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st);
+
+kda_status_t launch_norm_gate(const void *o, const void *gl, int64_t N, int H, int Dv, float eps,
+                              void *x, kda_dtype_t dt, cudaStream_t st);
+
+kda_status_t launch_proj_simt(const void *x, const void *W, int64_t N, int K, int Dm, void *y,
+                              kda_dtype_t dt, cudaStream_t st);
+bool proj_tc_supported(int64_t N, int K, int Dm, kda_dtype_t dt);
+kda_status_t launch_proj_tc(const void *x, const void *W, int64_t N, int K, int Dm, void *y,
+                            cudaStream_t st);
+
+}  // namespace kda

@@ -125,6 +125,12 @@ def recurrence(q, k, v, beta, *, z=None, log_decay=None, g_min=-5.0,
     return o, sf
 
 
+def log_decay(z, g_min):
+    """The decay gate in log form, g_min * sigmoid(z) = log(alpha) ("KDA Recurrence"
+    page, gate formula), fp64."""
+    return float(g_min) / (1.0 + np.exp(-np.asarray(z, np.float64)))
+
+
 def norm_gate(o_core, gate_logits, eps):
     """Per-head RMS normalisation over D_v with eps inside the root, then the
     sigmoid output gate ("KDA Recurrence" page, problem statement)."""
@@ -158,4 +164,4 @@ def forward(query, key, value, decay_logits, write_strength, output_gate_logits,
     return {"outputs": y, "final_state": sf, "o_core": o}
 
 
-__all__ = ["build", "recurrence", "norm_gate", "project", "forward", "default_threads"]
+__all__ = ["build", "recurrence", "log_decay", "norm_gate", "project", "forward", "default_threads"]

@@ -1,0 +1,156 @@
+"""The C-ABI library on the host: it loads, exports every declared symbol, its
+struct layouts match the header, and argument validation rejects bad calls
+before launching anything (no compute runs here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from kimi_delta_attention_21_b200 import _lib
+from kimi_delta_attention_21_b200._lib import ChunkArgs, DecodeArgs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kda.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(kda_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = _lib.load()
+    names = _declared()
+    assert "kda_chunk_fwd" in names and "kda_decode_step" in names
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _lib.SIGNATURES, f"{n} has no Python signature"
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r" T (kda_\w+)", out))
+    assert set(names) <= exported
+
+
+def test_struct_layout_matches_header(tmp_path):
+    prog = tmp_path / "layout.c"
+    fields_c = [f for f, _ in ChunkArgs._fields_]
+    fields_d = [f for f, _ in DecodeArgs._fields_]
+    lines = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{HEADER}"', "int main(void){",
+             'printf("%zu %zu\\n", sizeof(kda_chunk_args), sizeof(kda_decode_args));']
+    for f in fields_c:
+        lines.append(f'printf("c {f} %zu\\n", offsetof(kda_chunk_args, {f}));')
+    for f in fields_d:
+        lines.append(f'printf("d {f} %zu\\n", offsetof(kda_decode_args, {f}));')
+    lines.append("return 0;}")
+    prog.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.check_call(["gcc", "-std=c11", "-o", str(exe), str(prog)])
+    out = subprocess.check_output([str(exe)], text=True).split("\n")
+    sc, sd = map(int, out[0].split())
+    assert sc == ctypes.sizeof(ChunkArgs) and sd == ctypes.sizeof(DecodeArgs)
+    for line in out[1:]:
+        if not line:
+            continue
+        kind, f, off = line.split()
+        S = ChunkArgs if kind == "c" else DecodeArgs
+        assert getattr(S, f).offset == int(off), (kind, f)
+
+
+def test_status_strings():
+    lib = _lib.load()
+    names = [lib.kda_status_string(i).decode() for i in range(6)]
+    assert names == ["KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_WORKSPACE",
+                     "KDA_ERR_CUDA", "KDA_ERR_TIMEOUT"]
+    assert lib.kda_status_string(99).decode() == "KDA_ERR_UNKNOWN"
+
+
+# Fake device addresses: never dereferenced, because every call below fails
+# validation before anything is launched.
+BASE = 1 << 40
+
+
+def _args(**kw):
+    B, S, H, Dk, Dv = kw.pop("shape", (1, 8, 2, 16, 16))
+    nk = B * S * H * Dk * 2
+    a = ChunkArgs(B=B, S=S, H=H, D_k=Dk, D_v=Dv, dtype=_lib.KDA_BF16, g_min=-5.0, eps=1e-6)
+    a.q = BASE
+    a.k = BASE + 1 * (1 << 30)
+    a.v = BASE + 2 * (1 << 30)
+    a.z = BASE + 3 * (1 << 30)
+    a.beta = BASE + 4 * (1 << 30)
+    a.o = BASE + 5 * (1 << 30)
+    a.final_state = BASE + 6 * (1 << 30)
+    for k_, v_ in kw.items():
+        setattr(a, k_, v_)
+    assert nk < (1 << 30)
+    return a
+
+
+def _chunk_status(a):
+    return _lib.load().kda_chunk_fwd(ctypes.byref(a))
+
+
+@pytest.mark.parametrize("mut,status", [
+    (dict(g_min=0.0), _lib.KDA_ERR_INVALID_ARG),
+    (dict(g_min=float("nan")), _lib.KDA_ERR_INVALID_ARG),
+    (dict(q=None), _lib.KDA_ERR_INVALID_ARG),
+    (dict(q=BASE + 8), _lib.KDA_ERR_INVALID_ARG),            # misaligned
+    (dict(z=None), _lib.KDA_ERR_INVALID_ARG),                # neither z nor log_decay
+    (dict(o=BASE + 256), _lib.KDA_ERR_INVALID_ARG),          # o overlaps q (512 bytes)
+    (dict(final_state=BASE + 2 * (1 << 30)), _lib.KDA_ERR_INVALID_ARG),  # state overlaps v
+    (dict(shape=(1, 8, 2, 256, 16)), _lib.KDA_ERR_UNSUPPORTED),
+    (dict(chunk=128), _lib.KDA_ERR_UNSUPPORTED),
+    (dict(chunk=-1), _lib.KDA_ERR_INVALID_ARG),
+    (dict(dtype=7), _lib.KDA_ERR_UNSUPPORTED),
+    (dict(engine=9), _lib.KDA_ERR_INVALID_ARG),
+    (dict(H=0), _lib.KDA_ERR_INVALID_ARG),
+    (dict(gate_logits=BASE + 7 * (1 << 30), eps=-1.0), _lib.KDA_ERR_INVALID_ARG),
+])
+def test_chunk_validation(mut, status):
+    a = _args(**mut)
+    assert _chunk_status(a) == status
+    assert _lib.load().kda_last_error().decode() != ""
+
+
+def test_tc_engine_refuses_uncovered_shapes():
+    a = _args(shape=(1, 8, 2, 64, 64), engine=_lib.ENGINE_TC)
+    assert _chunk_status(a) == _lib.KDA_ERR_UNSUPPORTED
+    a = _args(shape=(1, 8, 2, 128, 128), engine=_lib.ENGINE_TC, dtype=_lib.KDA_F32)
+    assert _chunk_status(a) == _lib.KDA_ERR_UNSUPPORTED
+    a = _args(shape=(1, 8, 2, 128, 128), engine=_lib.ENGINE_TC, g_min=-8.0)
+    assert _chunk_status(a) == _lib.KDA_ERR_UNSUPPORTED
+
+
+def test_decode_and_gate_validation():
+    lib = _lib.load()
+    d = DecodeArgs(B=2, H=2, D_k=16, D_v=16, dtype=_lib.KDA_BF16, g_min=1.0, eps=1e-6,
+                   q=BASE, k=BASE + (1 << 30), v=BASE + 2 * (1 << 30), z=BASE + 3 * (1 << 30),
+                   beta=BASE + 4 * (1 << 30), state=BASE + 5 * (1 << 30), o=BASE + 6 * (1 << 30))
+    assert lib.kda_decode_step(ctypes.byref(d)) == _lib.KDA_ERR_INVALID_ARG   # g_min > 0
+    d.g_min = -5.0
+    d.o = d.state                                                              # o overlaps state
+    assert lib.kda_decode_step(ctypes.byref(d)) == _lib.KDA_ERR_INVALID_ARG
+    assert lib.kda_gate(BASE, _lib.KDA_BF16, 16, 0.5, BASE + (1 << 30), None) == _lib.KDA_ERR_INVALID_ARG
+    assert lib.kda_gate(BASE, _lib.KDA_BF16, -1, -5.0, BASE + (1 << 30), None) == _lib.KDA_ERR_INVALID_ARG
+    assert lib.kda_gate(BASE, _lib.KDA_BF16, 16, -5.0, BASE + 4, None) == _lib.KDA_ERR_INVALID_ARG
+    assert lib.kda_gate(BASE, _lib.KDA_BF16, 0, -5.0, None, None) == _lib.KDA_OK  # empty: nothing to do
+
+
+def test_projection_validation():
+    lib = _lib.load()
+    assert lib.kda_out_proj(BASE, BASE + (1 << 30), 4, 0, 8, BASE + 2 * (1 << 30), 1, None) == _lib.KDA_ERR_INVALID_ARG
+    # y overlapping x
+    assert lib.kda_out_proj(BASE, BASE + (1 << 30), 4, 8, 8, BASE, 1, None) == _lib.KDA_ERR_INVALID_ARG
+    n = ctypes.c_size_t(0)
+    assert lib.kda_out_norm_gate_proj_workspace_size(10, 2, 4, 1, ctypes.byref(n)) == _lib.KDA_OK
+    assert n.value == 10 * 2 * 4 * 2
+    assert lib.kda_out_norm_gate_proj(BASE, BASE + (1 << 30), BASE + 2 * (1 << 30), 10, 2, 4, 8, 1e-6,
+                                      BASE + 3 * (1 << 30), 1, BASE + 4 * (1 << 30), 8, None) == _lib.KDA_ERR_WORKSPACE
+
+
+def test_workspace_query_needs_no_device():
+    a = _args(shape=(2, 100, 3, 32, 32))
+    n = ctypes.c_size_t(123)
+    assert _lib.load().kda_chunk_workspace_size(ctypes.byref(a), ctypes.byref(n)) == _lib.KDA_OK

@@ -341,3 +341,11 @@ def test_chunk_forms_match_recurrence(C):
         oc, sc = fn(*args, C)
         np.testing.assert_allclose(oc, o[0, :, 0], rtol=1e-10, atol=1e-12)
         np.testing.assert_allclose(sc, sf[0, 0], rtol=1e-10, atol=1e-12)
+
+
+def test_log_decay_gate_limits():
+    z = np.array([0.0, 60.0, -60.0, 1.0])
+    g = oracle.log_decay(z, -5.0)
+    np.testing.assert_allclose(g[:3], [-2.5, -5.0, 0.0], atol=1e-20)
+    # sigmoid(1) = e/(1+e)
+    np.testing.assert_allclose(g[3], -5.0 * np.e / (1 + np.e), rtol=1e-15)
