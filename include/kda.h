@@ -14,9 +14,12 @@
  * Conventions shared by every entry point
  * ----------------------------------------
  * - Every tensor pointer is DEVICE memory owned by the caller, contiguous and
- *   row-major in exactly the shapes given, and 16-byte aligned.  The library
- *   allocates nothing; scratch comes from a caller workspace whose size the
- *   matching *_workspace_size query returns.
+ *   row-major in exactly the shapes given, and aligned to its element size
+ *   (workspaces: 256 bytes).  Tensor-core and vectorised paths additionally
+ *   want 16-byte aligned bases; with a less aligned pointer the call takes an
+ *   exact SIMT path instead (or fails with INVALID_ARG when that engine was
+ *   demanded).  The library allocates nothing; scratch comes from a caller
+ *   workspace whose size the matching *_workspace_size query returns.
  * - "dtype" tensors hold fp32 (KDA_F32) or bf16 (KDA_BF16) values; all inputs
  *   of one call share it.  State and log-decay tensors are always fp32.
  * - All work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is
@@ -68,6 +71,10 @@ int kda_version(void);
 /* Number of kernel launches this process has issued through the library so
  * far (all devices and threads).  For counting the kernels of a timed region. */
 uint64_t kda_launch_count(void);
+
+/* Number of bounded device-side waits that ran out on the current device since
+ * the last reset (0 in a healthy run); reset != 0 clears it.  Synchronous. */
+kda_status_t kda_device_timeouts(uint32_t *count, int reset);
 
 /*
  * kda_gate — decay gate of the "KDA Recurrence" page:

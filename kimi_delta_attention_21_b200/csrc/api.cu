@@ -35,7 +35,7 @@ kda_status_t check_launch(const char *what) {
     return KDA_OK;
 }
 
-static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool aligned_to(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 static size_t esize(kda_dtype_t dt) { return dt == KDA_F32 ? 4 : 2; }
 
@@ -82,15 +82,17 @@ static kda_status_t check_gmin(float g_min) {
         if (s_ != KDA_OK) return s_;       \
     } while (0)
 
-#define KDA_REQ_PTR(p, name)                                                              \
-    do {                                                                                  \
-        if (!(p)) return fail(KDA_ERR_INVALID_ARG, "%s is NULL", name);                   \
-        if (!aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name); \
+// Pointers must be non-NULL (REQ) and aligned to their element size `al`.
+#define KDA_REQ_PTR(p, name, al)                                                               \
+    do {                                                                                       \
+        if (!(p)) return fail(KDA_ERR_INVALID_ARG, "%s is NULL", name);                        \
+        if (!aligned_to(p, al)) return fail(KDA_ERR_INVALID_ARG, "%s is not %d-byte aligned", name, (int)(al)); \
     } while (0)
 
-#define KDA_OPT_PTR(p, name)                                                              \
-    do {                                                                                  \
-        if ((p) && !aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "%s is not 16-byte aligned", name); \
+#define KDA_OPT_PTR(p, name, al)                                                               \
+    do {                                                                                       \
+        if ((p) && !aligned_to(p, al))                                                         \
+            return fail(KDA_ERR_INVALID_ARG, "%s is not %d-byte aligned", name, (int)(al));     \
     } while (0)
 
 static kda_status_t chunk_validate(const kda_chunk_args *a, int *chunk_out, bool *use_tc) {
@@ -149,8 +151,8 @@ kda_status_t kda_gate(const void *z, kda_dtype_t dtype, int64_t n, float g_min, 
     if (n < 0) return fail(KDA_ERR_INVALID_ARG, "n must be >= 0");
     KDA_TRY(check_gmin(g_min));
     if (n == 0) return KDA_OK;
-    KDA_REQ_PTR(z, "z");
-    KDA_REQ_PTR(log_alpha, "log_alpha");
+    KDA_REQ_PTR(z, "z", esize(dtype));
+    KDA_REQ_PTR(log_alpha, "log_alpha", 4);
     Buf in{z, (size_t)n * esize(dtype), "z"};
     KDA_TRY(check_no_overlap(Buf{log_alpha, (size_t)n * 4, "log_alpha"}, &in, 1));
     return launch_gate(z, dtype, n, g_min, log_alpha, (cudaStream_t)stream);
@@ -178,19 +180,22 @@ kda_status_t kda_chunk_fwd(const kda_chunk_args *a) {
     const size_t nb = (size_t)a->B * a->S * a->H;
     const size_t ns = (size_t)a->B * a->H * a->D_k * a->D_v * 4;
     if (a->S > 0) {
-        KDA_REQ_PTR(a->q, "q");
-        KDA_REQ_PTR(a->k, "k");
-        KDA_REQ_PTR(a->v, "v");
-        KDA_REQ_PTR(a->beta, "beta");
-        KDA_REQ_PTR(a->o, "o");
-        if (!a->log_decay) KDA_REQ_PTR(a->z, "z (or log_decay)");
-        KDA_OPT_PTR(a->log_decay, "log_decay");
-        KDA_OPT_PTR(a->gate_logits, "gate_logits");
+        KDA_REQ_PTR(a->q, "q", es);
+        KDA_REQ_PTR(a->k, "k", es);
+        KDA_REQ_PTR(a->v, "v", es);
+        KDA_REQ_PTR(a->beta, "beta", es);
+        KDA_REQ_PTR(a->o, "o", es);
+        if (!a->log_decay) KDA_REQ_PTR(a->z, "z (or log_decay)", es);
+        KDA_OPT_PTR(a->log_decay, "log_decay", 4);
+        KDA_OPT_PTR(a->gate_logits, "gate_logits", es);
     }
-    KDA_OPT_PTR(a->initial_state, "initial_state");
-    KDA_OPT_PTR(a->final_state, "final_state");
-    KDA_OPT_PTR(a->workspace, "workspace");
-    KDA_OPT_PTR(a->dev_status, "dev_status");
+    KDA_OPT_PTR(a->initial_state, "initial_state", 4);
+    KDA_OPT_PTR(a->final_state, "final_state", 4);
+    KDA_OPT_PTR(a->workspace, "workspace", 256);
+    KDA_OPT_PTR(a->dev_status, "dev_status", 4);
+    if (tc && a->engine == KDA_ENGINE_TC && !chunk_tc_aligned(*a))
+        return fail(KDA_ERR_INVALID_ARG, "the tensor-core engine needs 16-byte aligned q, k, v, z, beta, o");
+    if (tc && !chunk_tc_aligned(*a)) tc = false;
     const size_t need = tc ? chunk_tc_workspace(*a) : chunk_simt_workspace(*a, chunk);
     if (need > 0 && (!a->workspace || a->workspace_bytes < need))
         return fail(KDA_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", need,
@@ -231,19 +236,19 @@ kda_status_t kda_decode_step(const kda_decode_args *a) {
     if (a->D_k > 128 || a->D_v > 128)
         return fail(KDA_ERR_UNSUPPORTED, "D_k and D_v must be <= 128");
     if (a->B == 0) return KDA_OK;
-    KDA_REQ_PTR(a->q, "q");
-    KDA_REQ_PTR(a->k, "k");
-    KDA_REQ_PTR(a->v, "v");
-    KDA_REQ_PTR(a->beta, "beta");
-    KDA_REQ_PTR(a->state, "state");
-    KDA_REQ_PTR(a->o, "o");
+    const size_t es = esize(a->dtype);
+    KDA_REQ_PTR(a->q, "q", es);
+    KDA_REQ_PTR(a->k, "k", es);
+    KDA_REQ_PTR(a->v, "v", es);
+    KDA_REQ_PTR(a->beta, "beta", es);
+    KDA_REQ_PTR(a->state, "state", 4);
+    KDA_REQ_PTR(a->o, "o", es);
     KDA_TRY(check_gmin(a->g_min));
-    if (!a->log_decay) KDA_REQ_PTR(a->z, "z (or log_decay)");
-    KDA_OPT_PTR(a->log_decay, "log_decay");
-    KDA_OPT_PTR(a->gate_logits, "gate_logits");
+    if (!a->log_decay) KDA_REQ_PTR(a->z, "z (or log_decay)", es);
+    KDA_OPT_PTR(a->log_decay, "log_decay", 4);
+    KDA_OPT_PTR(a->gate_logits, "gate_logits", es);
     if (a->gate_logits && !(isfinite(a->eps) && a->eps >= 0.0f))
         return fail(KDA_ERR_INVALID_ARG, "eps must be finite and >= 0");
-    const size_t es = esize(a->dtype);
     const size_t nk = (size_t)a->B * a->H * a->D_k, nv = (size_t)a->B * a->H * a->D_v;
     const size_t ns = (size_t)a->B * a->H * a->D_k * a->D_v * 4;
     const Buf ins[] = {
@@ -265,9 +270,9 @@ kda_status_t kda_norm_gate(const void *o, const void *gl, int64_t N, int32_t H, 
     if (N < 0 || H < 1 || Dv < 1) return fail(KDA_ERR_INVALID_ARG, "bad sizes");
     if (!(isfinite(eps) && eps >= 0.0f)) return fail(KDA_ERR_INVALID_ARG, "eps must be finite and >= 0");
     if (N == 0) return KDA_OK;
-    KDA_REQ_PTR(o, "o");
-    KDA_REQ_PTR(gl, "gate_logits");
-    KDA_REQ_PTR(x, "x");
+    KDA_REQ_PTR(o, "o", esize(dtype));
+    KDA_REQ_PTR(gl, "gate_logits", esize(dtype));
+    KDA_REQ_PTR(x, "x", esize(dtype));
     const size_t n = (size_t)N * H * Dv * esize(dtype);
     const Buf ins[] = {{x == o ? nullptr : o, n, "o"}, {gl, n, "gate_logits"}};
     KDA_TRY(check_no_overlap(Buf{x, n, "x"}, ins, 2));
@@ -281,13 +286,14 @@ kda_status_t kda_out_proj(const void *x, const void *W, int64_t N, int32_t K, in
     KDA_TRY(check_dtype(dtype));
     if (N < 0 || K < 1 || Dm < 1) return fail(KDA_ERR_INVALID_ARG, "bad sizes");
     if (N == 0) return KDA_OK;
-    KDA_REQ_PTR(x, "x");
-    KDA_REQ_PTR(W, "W_o");
-    KDA_REQ_PTR(y, "y");
     const size_t es = esize(dtype);
+    KDA_REQ_PTR(x, "x", es);
+    KDA_REQ_PTR(W, "W_o", es);
+    KDA_REQ_PTR(y, "y", es);
     const Buf ins[] = {{x, (size_t)N * K * es, "x"}, {W, (size_t)Dm * K * es, "W_o"}};
     KDA_TRY(check_no_overlap(Buf{y, (size_t)N * Dm * es, "y"}, ins, 2));
-    if (proj_tc_supported(N, K, Dm, dtype)) return launch_proj_tc(x, W, N, K, Dm, y, (cudaStream_t)stream);
+    if (proj_tc_supported(N, K, Dm, dtype) && aligned_to(x, 16) && aligned_to(W, 16) && aligned_to(y, 16))
+        return launch_proj_tc(x, W, N, K, Dm, y, (cudaStream_t)stream);
     return launch_proj_simt(x, W, N, K, Dm, y, dtype, (cudaStream_t)stream);
 }
 
@@ -309,12 +315,12 @@ kda_status_t kda_out_norm_gate_proj(const void *o, const void *gl, const void *W
     if (N < 0 || H < 1 || Dv < 1 || Dm < 1) return fail(KDA_ERR_INVALID_ARG, "bad sizes");
     if (!(isfinite(eps) && eps >= 0.0f)) return fail(KDA_ERR_INVALID_ARG, "eps must be finite and >= 0");
     if (N == 0) return KDA_OK;
-    KDA_REQ_PTR(o, "o");
-    KDA_REQ_PTR(gl, "gate_logits");
-    KDA_REQ_PTR(W, "W_o");
-    KDA_REQ_PTR(y, "y");
-    KDA_REQ_PTR(ws, "workspace");
     const size_t es = esize(dtype);
+    KDA_REQ_PTR(o, "o", es);
+    KDA_REQ_PTR(gl, "gate_logits", es);
+    KDA_REQ_PTR(W, "W_o", es);
+    KDA_REQ_PTR(y, "y", es);
+    KDA_REQ_PTR(ws, "workspace", 256);
     const size_t nx = (size_t)N * H * Dv * es;
     if (ws_bytes < nx) return fail(KDA_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", nx, ws_bytes);
     const Buf ins[] = {{o, nx, "o"}, {gl, nx, "gate_logits"}, {W, (size_t)Dm * H * Dv * es, "W_o"}};
@@ -324,7 +330,8 @@ kda_status_t kda_out_norm_gate_proj(const void *o, const void *gl, const void *W
     cudaStream_t st = (cudaStream_t)stream;
     KDA_TRY(launch_norm_gate(o, gl, N, H, Dv, eps, ws, dtype, st));
     const int K = H * Dv;
-    if (proj_tc_supported(N, K, Dm, dtype)) return launch_proj_tc(ws, W, N, K, Dm, y, st);
+    if (proj_tc_supported(N, K, Dm, dtype) && aligned_to(W, 16) && aligned_to(y, 16))
+        return launch_proj_tc(ws, W, N, K, Dm, y, st);
     return launch_proj_simt(ws, W, N, K, Dm, y, dtype, st);
 }
 

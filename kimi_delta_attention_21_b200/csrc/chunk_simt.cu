@@ -60,6 +60,7 @@ __device__ __forceinline__ float log_alpha_gt(float z, float g_min, float) { ret
 template <typename T>
 __global__ void __launch_bounds__(NT) chunk_simt_kernel(SimtParams p) {
     using GT = typename GType<T>::type;
+    using AT = typename AccT<T>::type;
     extern __shared__ __align__(16) unsigned char smraw[];
     const int C = p.C, Dk = p.Dk, VS = p.VS, LD = Dk + 1, LC = C + 1;
     GT *sG = reinterpret_cast<GT *>(smraw);                       // C x LD  cumulative log-decay
@@ -131,17 +132,17 @@ __global__ void __launch_bounds__(NT) chunk_simt_kernel(SimtParams p) {
         // ---- A (strictly lower, beta-weighted) and M (lower with diagonal)
         for (int idx = tid; idx < C * C; idx += NT) {
             const int r = idx / C, i = idx % C;
-            float a = 0.f, m = 0.f;
+            AT a = 0, m = 0;
             if (i <= r) {
                 for (int c = 0; c < Dk; ++c) {
-                    const float e = expf((float)(sG[r * LD + c] - sG[i * LD + c]));
-                    const float ki = sK[i * LD + c] * e;
+                    const AT e = expf((float)(sG[r * LD + c] - sG[i * LD + c]));
+                    const AT ki = sK[i * LD + c] * e;
                     a += sK[r * LD + c] * ki;
                     m += sQ[r * LD + c] * ki;
                 }
             }
-            sA[r * LC + i] = (i < r) ? sB[r] * a : 0.f;
-            sM[r * LC + i] = m;
+            sA[r * LC + i] = (i < r) ? (float)(sB[r] * a) : 0.f;
+            sM[r * LC + i] = (float)m;
         }
         __syncthreads();
         // ---- forward substitution of (I + A) X = RHS, one column per thread
@@ -149,16 +150,16 @@ __global__ void __launch_bounds__(NT) chunk_simt_kernel(SimtParams p) {
             if (col < Dk) {
                 const int c = col;
                 for (int r = 0; r < C; ++r) {
-                    float x = sB[r] * sK[r * LD + c] * expf((float)sG[r * LD + c]);
-                    for (int i = 0; i < r; ++i) x -= sA[r * LC + i] * sW[i * LD + c];
-                    sW[r * LD + c] = x;
+                    AT x = (AT)sB[r] * sK[r * LD + c] * expf((float)sG[r * LD + c]);
+                    for (int i = 0; i < r; ++i) x -= (AT)sA[r * LC + i] * sW[i * LD + c];
+                    sW[r * LD + c] = (float)x;
                 }
             } else {
                 const int j = col - Dk;
                 for (int r = 0; r < C; ++r) {
-                    float x = sU[r * VS + j];
-                    for (int i = 0; i < r; ++i) x -= sA[r * LC + i] * sU[i * VS + j];
-                    sU[r * VS + j] = x;
+                    AT x = sU[r * VS + j];
+                    for (int i = 0; i < r; ++i) x -= (AT)sA[r * LC + i] * sU[i * VS + j];
+                    sU[r * VS + j] = (float)x;
                 }
             }
         }
@@ -166,9 +167,9 @@ __global__ void __launch_bounds__(NT) chunk_simt_kernel(SimtParams p) {
         // ---- V' = U - W S_0
         for (int idx = tid; idx < C * VS; idx += NT) {
             const int r = idx / VS, j = idx % VS;
-            float acc = 0.f;
-            for (int c = 0; c < Dk; ++c) acc += sW[r * LD + c] * sS[c * VS + j];
-            sU[idx] -= acc;
+            AT acc = sU[idx];
+            for (int c = 0; c < Dk; ++c) acc -= (AT)sW[r * LD + c] * sS[c * VS + j];
+            sU[idx] = (float)acc;
         }
         __syncthreads();
         // ---- Q * e^G and K * e^{G_C - G}
@@ -183,19 +184,19 @@ __global__ void __launch_bounds__(NT) chunk_simt_kernel(SimtParams p) {
         for (int idx = tid; idx < C * VS; idx += NT) {
             const int r = idx / VS, j = idx % VS;
             if (r < len && j < nj) {
-                float acc = 0.f;
-                for (int c = 0; c < Dk; ++c) acc += sQ[r * LD + c] * sS[c * VS + j];
-                for (int i = 0; i <= r; ++i) acc += sM[r * LC + i] * sU[i * VS + j];
-                store_elem(o, ((row0 + r) * p.H + h) * (int64_t)p.Dv + j0 + j, acc);
+                AT acc = 0;
+                for (int c = 0; c < Dk; ++c) acc += (AT)sQ[r * LD + c] * sS[c * VS + j];
+                for (int i = 0; i <= r; ++i) acc += (AT)sM[r * LC + i] * sU[i * VS + j];
+                store_elem(o, ((row0 + r) * p.H + h) * (int64_t)p.Dv + j0 + j, (float)acc);
             }
         }
         __syncthreads();
         // ---- S_C = Diag(e^{G_C}) S_0 + (K e^{G_C - G})^T V'
         for (int idx = tid; idx < Dk * VS; idx += NT) {
             const int c = idx / VS, j = idx % VS;
-            float acc = expf((float)sG[(C - 1) * LD + c]) * sS[idx];
-            for (int r = 0; r < C; ++r) acc += sK[r * LD + c] * sU[r * VS + j];
-            sS[idx] = acc;
+            AT acc = (AT)expf((float)sG[(C - 1) * LD + c]) * sS[idx];
+            for (int r = 0; r < C; ++r) acc += (AT)sK[r * LD + c] * sU[r * VS + j];
+            sS[idx] = (float)acc;
         }
         __syncthreads();
     }

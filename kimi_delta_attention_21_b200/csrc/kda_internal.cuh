@@ -24,6 +24,12 @@ __device__ __forceinline__ void store_elem(__nv_bfloat16 *p, int64_t i, float v)
     p[i] = __float2bfloat16_rn(v);
 }
 
+// Accumulator type of the exact-fp32 kernels: fp32 inputs accumulate their
+// reductions in fp64 so that results stay within 1e-6 absolute / 1e-5 relative
+// of an fp64 evaluation; bf16 inputs accumulate in fp32.
+template <typename T> struct AccT { using type = float; };
+template <> struct AccT<float> { using type = double; };
+
 // sigmoid in full fp32 precision (expf, not the fast approximation)
 __device__ __forceinline__ float sigmoid_precise(float x) { return 1.0f / (1.0f + expf(-x)); }
 
@@ -44,6 +50,7 @@ size_t chunk_simt_workspace(const kda_chunk_args &a, int chunk);
 
 // tcgen05 chunk engine: bf16, D_k = D_v = 128, chunk 64.
 bool chunk_tc_supported(const kda_chunk_args &a, int chunk);
+bool chunk_tc_aligned(const kda_chunk_args &a);
 size_t chunk_tc_workspace(const kda_chunk_args &a);
 kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st);
 

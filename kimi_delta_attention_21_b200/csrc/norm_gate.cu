@@ -12,18 +12,19 @@ __global__ void __launch_bounds__(256) norm_gate_kernel(const T *o, const T *__r
     const int lane = threadIdx.x & 31;
     const int64_t row = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (row >= rows) return;
+    using AT = typename AccT<T>::type;
     const T *src = o + row * Dv;
-    float ss = 0.f;
+    AT ss = 0;
     for (int j = lane; j < Dv; j += 32) {
-        const float u = load_elem(src, j);
+        const AT u = load_elem(src, j);
         ss += u * u;
     }
 #pragma unroll
     for (int m = 16; m > 0; m >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, m);
-    const float inv = 1.0f / sqrtf(ss / (float)Dv + eps);
+    const AT inv = AT(1) / sqrt(ss / (AT)Dv + (AT)eps);
     for (int j = lane; j < Dv; j += 32) {
-        const float u = load_elem(src, j);
-        store_elem(x, row * Dv + j, u * inv * sigmoid_precise(load_elem(gl, row * Dv + j)));
+        const AT u = load_elem(src, j);
+        store_elem(x, row * Dv + j, (float)(u * inv * (AT)sigmoid_precise(load_elem(gl, row * Dv + j))));
     }
 }
 

@@ -17,7 +17,8 @@ __global__ void __launch_bounds__(256) proj_simt_kernel(const T *__restrict__ x,
     const int tx = tid % 16, ty = tid / 16;
     const int64_t n0 = (int64_t)blockIdx.y * BM;
     const int m0 = blockIdx.x * BN;
-    float acc[4][4] = {};
+    using AT = typename AccT<T>::type;
+    AT acc[4][4] = {};
     for (int k0 = 0; k0 < K; k0 += BK) {
         for (int e = tid; e < BM * BK; e += 256) {
             const int r = e / BK, kk = e % BK;
@@ -38,7 +39,7 @@ __global__ void __launch_bounds__(256) proj_simt_kernel(const T *__restrict__ x,
 #pragma unroll
             for (int i = 0; i < 4; ++i)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] += a[i] * b[j];
+                for (int j = 0; j < 4; ++j) acc[i][j] += (AT)a[i] * (AT)b[j];
         }
         __syncthreads();
     }
@@ -49,7 +50,7 @@ __global__ void __launch_bounds__(256) proj_simt_kernel(const T *__restrict__ x,
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             const int m = m0 + tx * 4 + j;
-            if (m < Dm) store_elem(y, n * Dm + m, acc[i][j]);
+            if (m < Dm) store_elem(y, n * Dm + m, (float)acc[i][j]);
         }
     }
 }

@@ -5,14 +5,10 @@
 namespace kda {
 
 bool chunk_tc_supported(const kda_chunk_args &, int) { return false; }
+bool chunk_tc_aligned(const kda_chunk_args &) { return false; }
 size_t chunk_tc_workspace(const kda_chunk_args &) { return 0; }
 kda_status_t launch_chunk_tc(const kda_chunk_args &, cudaStream_t) {
     return fail(KDA_ERR_UNSUPPORTED, "tensor-core chunk engine not built");
-}
-
-bool proj_tc_supported(int64_t, int, int, kda_dtype_t) { return false; }
-kda_status_t launch_proj_tc(const void *, const void *, int64_t, int, int, void *, cudaStream_t) {
-    return fail(KDA_ERR_UNSUPPORTED, "tensor-core projection not built");
 }
 
 }  // namespace kda

@@ -1,0 +1,87 @@
+// TMA tensor-map encoding and the device wait-timeout counter.
+#include <atomic>
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
+#include "kda_internal.cuh"
+#include "tma_host.cuh"
+
+namespace kda {
+
+// Counts bounded device-side waits that ran out (all kernels of this library).
+__device__ unsigned int g_kda_wait_timeouts;
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+kda_status_t make_tmap_2d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes,
+                          uint64_t rows, uint64_t cols, uint64_t row_stride, uint32_t box_rows, uint32_t box_cols,
+                          CUtensorMapSwizzle swizzle) {
+    auto fn = encode_fn();
+    if (!fn) return fail(KDA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {row_stride * (uint64_t)elem_bytes};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dtype, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(KDA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return KDA_OK;
+}
+
+kda_status_t make_tmap_3d(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes,
+                          uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t box0,
+                          uint32_t box1, uint32_t box2, CUtensorMapSwizzle swizzle) {
+    auto fn = encode_fn();
+    if (!fn) return fail(KDA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {stride1 * (uint64_t)elem_bytes, stride2 * (uint64_t)elem_bytes};
+    cuuint32_t box[3] = {box0, box1, box2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, dtype, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(KDA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return KDA_OK;
+}
+
+unsigned int *device_timeout_counter() {
+    static std::atomic<unsigned int *> ptrs[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    unsigned int *p = ptrs[dev].load();
+    if (!p) {
+        void *q = nullptr;
+        if (cudaGetSymbolAddress(&q, g_kda_wait_timeouts) != cudaSuccess) return nullptr;
+        p = static_cast<unsigned int *>(q);
+        ptrs[dev].store(p);
+    }
+    return p;
+}
+
+}  // namespace kda
+
+extern "C" kda_status_t kda_device_timeouts(uint32_t *count, int reset) {
+    using namespace kda;
+    if (!count) return fail(KDA_ERR_INVALID_ARG, "count is NULL");
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_kda_wait_timeouts, sizeof(v));
+    if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "reading the timeout counter: %s", cudaGetErrorString(e));
+    *count = v;
+    if (reset) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_kda_wait_timeouts, &zero, sizeof(zero));
+        if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "resetting the timeout counter: %s", cudaGetErrorString(e));
+    }
+    return KDA_OK;
+}

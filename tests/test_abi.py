@@ -96,7 +96,7 @@ def _chunk_status(a):
     (dict(g_min=0.0), _lib.KDA_ERR_INVALID_ARG),
     (dict(g_min=float("nan")), _lib.KDA_ERR_INVALID_ARG),
     (dict(q=None), _lib.KDA_ERR_INVALID_ARG),
-    (dict(q=BASE + 8), _lib.KDA_ERR_INVALID_ARG),            # misaligned
+    (dict(q=BASE + 1), _lib.KDA_ERR_INVALID_ARG),            # misaligned for bf16
     (dict(z=None), _lib.KDA_ERR_INVALID_ARG),                # neither z nor log_decay
     (dict(o=BASE + 256), _lib.KDA_ERR_INVALID_ARG),          # o overlaps q (512 bytes)
     (dict(final_state=BASE + 2 * (1 << 30)), _lib.KDA_ERR_INVALID_ARG),  # state overlaps v
@@ -134,7 +134,7 @@ def test_decode_and_gate_validation():
     assert lib.kda_decode_step(ctypes.byref(d)) == _lib.KDA_ERR_INVALID_ARG
     assert lib.kda_gate(BASE, _lib.KDA_BF16, 16, 0.5, BASE + (1 << 30), None) == _lib.KDA_ERR_INVALID_ARG
     assert lib.kda_gate(BASE, _lib.KDA_BF16, -1, -5.0, BASE + (1 << 30), None) == _lib.KDA_ERR_INVALID_ARG
-    assert lib.kda_gate(BASE, _lib.KDA_BF16, 16, -5.0, BASE + 4, None) == _lib.KDA_ERR_INVALID_ARG
+    assert lib.kda_gate(BASE, _lib.KDA_BF16, 16, -5.0, BASE + 2, None) == _lib.KDA_ERR_INVALID_ARG
     assert lib.kda_gate(BASE, _lib.KDA_BF16, 0, -5.0, None, None) == _lib.KDA_OK  # empty: nothing to do
 
 

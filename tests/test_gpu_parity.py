@@ -248,3 +248,34 @@ def test_prefill_4k_layer(K, engine):
     want = oracle_layer(inp, w)
     assert_bf16_outputs(to_np(out["outputs"]), want["outputs"], "outputs")
     assert_bf16_state(to_np(out["final_state"]), want["final_state"], "final_state")
+
+
+@pytest.mark.parametrize("N,K,Dm", [(1, 8, 8), (128, 64, 256), (129, 64, 264), (300, 200, 96), (4096, 2048, 2048),
+                                    (256, 4096, 4096), (77, 4096, 520)])
+def test_projection_tensor_core_shapes(K, N, Dm):
+    rng = np.random.default_rng(N * 3 + K)
+    x = ki.round_bf16(rng.standard_normal((N, K)).astype(np.float32))
+    W = ki.round_bf16((rng.standard_normal((Dm, K)) / np.sqrt(K)).astype(np.float32))
+    import kimi_delta_attention_21_b200 as KK
+    y = KK.out_proj(to_dev(x, torch.bfloat16), to_dev(W, torch.bfloat16))
+    want = oracle.project(x[:, None, :], W)  # one "head" of width K
+    # bf16 output rounding dominates: |y| <~ 5, half an ulp of bf16 at 4..8 is 1.6e-2
+    err = np.abs(to_np(y) - want)
+    assert float(err.max()) <= 2e-2
+    assert float(np.median(err)) <= 2e-3
+
+
+def test_unaligned_views_take_exact_paths(K):
+    # token slices of (B, S, H, .) tensors start at element offsets that are not
+    # 16-byte aligned: decode and the gate must still run and agree
+    w = small("u", 1, 5, 1, 128, 128, 16, "bf16", seed=33, s0_std=0.02)
+    inp = ki.make_inputs(w)
+    d = upload(inp, w)
+    st = d["S0"].clone()
+    xs = [K.decode_step(d["q"][:, t], d["k"][:, t], d["v"][:, t], d["beta"][:, t], st, z=d["z"][:, t],
+                        gate_logits=d["gate"][:, t]) for t in range(5)]
+    o_ref, s_ref = oracle.recurrence(inp["q"], inp["k"], inp["v"], inp["beta"], z=inp["z"], initial_state=inp["S0"])
+    assert_bf16_outputs(to_np(torch.stack(xs, 1)), oracle.norm_gate(o_ref, inp["gate"], 1e-6))
+    assert_bf16_state(to_np(st), s_ref)
+    zz = d["z"].flatten()[3:1000]
+    np.testing.assert_allclose(to_np(K.gate(zz, -5.0)), oracle.log_decay(to_np(zz), -5.0), rtol=1e-6, atol=1e-6)
