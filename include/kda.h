@@ -214,6 +214,30 @@ kda_status_t kda_out_norm_gate_proj(const void *o, const void *gate_logits,
                                     int32_t D_model, float eps, void *y, kda_dtype_t dtype,
                                     void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * kda_out_norm_gate_proj_noalloc — the same computation as
+ * kda_out_norm_gate_proj for callers that cannot allocate device memory: an
+ * integration point that passes the library only its input and output
+ * buffers, or a loop that must not call cudaMalloc while it runs because the
+ * call can synchronise the device.  No page describes this variant; it exists
+ * for those callers only.
+ *   o, gate_logits (N, H, D_v); W_o (D_model, H*D_v); y (N, D_model); all dtype.
+ * The normalised activations live in a fixed 8 MiB scratch array inside the
+ * library's device memory (held by every GPU that loads the library until the
+ * process exits) instead of a caller workspace, so this call never allocates.
+ * Limit: N * H * D_v * element_size <= 8 MiB, else KDA_ERR_UNSUPPORTED and
+ * nothing is launched.  The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress); make that first call before any stream
+ * capture.  All calls on a device share the array and it keeps the last call's
+ * contents (each call writes every byte it reads, so nothing needs clearing);
+ * calls whose kernels overlap on the GPU race on it and must be ordered by the
+ * caller.
+ */
+kda_status_t kda_out_norm_gate_proj_noalloc(const void *o, const void *gate_logits,
+                                            const void *W_o, int64_t N, int32_t H, int32_t D_v,
+                                            int32_t D_model, float eps, void *y, kda_dtype_t dtype,
+                                            void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -66,6 +66,8 @@ SIGNATURES = {
                                                              ctypes.POINTER(ctypes.c_size_t)]),
     "kda_out_norm_gate_proj": (ctypes.c_int, [_p, _p, _p, _i64, _i32, _i32, _i32, _f32, _p, ctypes.c_int,
                                               _p, ctypes.c_size_t, _p]),
+    "kda_out_norm_gate_proj_noalloc": (ctypes.c_int, [_p, _p, _p, _i64, _i32, _i32, _i32, _f32, _p, ctypes.c_int,
+                                                      _p]),
 }
 
 _lib = None
