@@ -59,11 +59,13 @@ def gate(z: torch.Tensor, g_min: float) -> torch.Tensor:
 
 def chunk_fwd(q, k, v, beta, *, z=None, log_decay=None, g_min=-5.0, initial_state=None,
               gate_logits=None, eps=1e-6, chunk=64, engine="auto", want_final_state=True,
-              out=None, final_state=None, dev_status=None):
+              out=None, final_state=None, dev_status=None, workspace=None):
     """Chunkwise prefill.  Returns (o, final_state):
     o (B,S,H,D_v) in the input dtype holds o~ (gate_logits None) or
     RMSNorm(o~) * sigmoid(gate_logits); final_state (B,H,D_k,D_v) fp32 or None.
-    ``final_state`` may be the same tensor as ``initial_state`` (in-place handoff)."""
+    ``final_state`` may be the same tensor as ``initial_state`` (in-place handoff).
+    ``workspace`` is an optional uint8 CUDA tensor at least
+    ``chunk_workspace_bytes(...)`` long (allocated per call when omitted)."""
     _dev(q, "q")
     dt = q.dtype
     B, S, H, Dk = q.shape
@@ -94,11 +96,13 @@ def chunk_fwd(q, k, v, beta, *, z=None, log_decay=None, g_min=-5.0, initial_stat
     lib = _lib.load()
     nbytes = ctypes.c_size_t(0)
     check("kda_chunk_workspace_size", lib.kda_chunk_workspace_size(ctypes.byref(a), ctypes.byref(nbytes)))
-    ws = None
+    ws = workspace
     if nbytes.value:
-        ws = torch.empty(nbytes.value, dtype=torch.uint8, device=q.device)
+        if ws is None:
+            ws = torch.empty(nbytes.value, dtype=torch.uint8, device=q.device)
+        _dev(ws, "workspace", torch.uint8)
         a.workspace = _ptr(ws)
-        a.workspace_bytes = nbytes.value
+        a.workspace_bytes = ws.numel()
     check("kda_chunk_fwd", lib.kda_chunk_fwd(ctypes.byref(a)))
     return out, final_state
 

@@ -55,6 +55,27 @@ kda_status_t make_tmap_3d(CUtensorMap *map, const void *base, CUtensorMapDataTyp
     return KDA_OK;
 }
 
+kda_status_t make_tmap_nd(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes, int rank,
+                          const uint64_t *dims, const uint64_t *strides, const uint32_t *box,
+                          CUtensorMapSwizzle swizzle) {
+    auto fn = encode_fn();
+    if (!fn) return fail(KDA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    if (rank < 1 || rank > 5) return fail(KDA_ERR_INVALID_ARG, "tensor map rank %d", rank);
+    cuuint64_t d[5], st[4];
+    cuuint32_t bx[5], es[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        bx[i] = box[i];
+        es[i] = 1;
+    }
+    for (int i = 0; i + 1 < rank; ++i) st[i] = strides[i] * (uint64_t)elem_bytes;
+    CUresult r = fn(map, dtype, (cuuint32_t)rank, const_cast<void *>(base), d, st, bx, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(KDA_ERR_CUDA, "cuTensorMapEncodeTiled (rank %d) failed (%d)", rank, (int)r);
+    return KDA_OK;
+}
+
 unsigned int *device_timeout_counter() {
     static std::atomic<unsigned int *> ptrs[64];
     int dev = 0;

@@ -23,6 +23,12 @@ kda_status_t make_tmap_3d(CUtensorMap *map, const void *base, CUtensorMapDataTyp
                           uint64_t d0, uint64_t d1, uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t box0,
                           uint32_t box1, uint32_t box2, CUtensorMapSwizzle swizzle);
 
+// N-D tensor (rank <= 5): dims[0] contiguous, strides[i] (elements) for dims[i+1],
+// box[i] elements per dimension.
+kda_status_t make_tmap_nd(CUtensorMap *map, const void *base, CUtensorMapDataType dtype, int elem_bytes, int rank,
+                          const uint64_t *dims, const uint64_t *strides, const uint32_t *box,
+                          CUtensorMapSwizzle swizzle);
+
 // Device address of this library's wait-timeout counter on the current device.
 unsigned int *device_timeout_counter();
 

@@ -1,0 +1,177 @@
+"""The tcgen05 chunk engine (bf16, D_k = D_v = 128, chunk 64) against the oracle,
+the fp64 chunk mirror (its workspace intermediates) and the exact SIMT engine."""
+import numpy as np
+import pytest
+
+import kda_inputs as ki
+import oracle
+from oracle import chunk_mirror
+from kda_testlib import (assert_bf16_outputs, assert_bf16_state, oracle_layer, rel_fro, small, to_np, upload)
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+REC = 74240  # workspace bytes per (b, h, chunk)
+
+
+@pytest.fixture(scope="module")
+def K():
+    import kimi_delta_attention_21_b200 as K
+    K.load_library()
+    return K
+
+
+def _timeouts(K):
+    import ctypes
+    n = ctypes.c_uint32(0)
+    assert K.load_library().kda_device_timeouts(ctypes.byref(n), 1) == 0
+    return n.value
+
+
+def _bf16_view(ws_bytes):
+    return np.frombuffer(ws_bytes.tobytes(), dtype=np.uint16)
+
+
+def _bf(u16):
+    return (u16.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _kmajor_image(buf, rows=64):
+    """[2 atoms][rows][128 B] 128-byte-swizzled bf16 image -> (rows, 128)."""
+    u = np.frombuffer(buf, dtype=np.uint16)
+    out = np.zeros((rows, 128))
+    for r in range(rows):
+        for c in range(128):
+            atom, chunk, e = c // 64, (c % 64) // 8, c % 8
+            off = atom * rows * 128 + r * 128 + ((chunk ^ (r % 8)) * 16) + e * 2
+            out[r, c] = _bf(u[off // 2:off // 2 + 1])[0]
+    return out
+
+
+def _mt_image(buf):
+    u = np.frombuffer(buf, dtype=np.uint16)
+    out = np.zeros((64, 64))
+    for i in range(64):
+        for r in range(64):
+            off = i * 128 + (((r // 8) ^ (i % 8)) * 16) + (r % 8) * 2
+            out[i, r] = _bf(u[off // 2:off // 2 + 1])[0]
+    return out
+
+
+def _close(got, want, what, tol=2e-2):
+    scale = max(1.0, float(np.max(np.abs(want))))
+    err = float(np.max(np.abs(got - want)))
+    assert err <= tol * scale, f"{what}: max-abs {err:.3e} (scale {scale:.3e})"
+
+
+def test_workspace_intermediates_match_chunk_mirror(K):
+    w = small("wsi", 1, 100, 2, 128, 128, 16, "bf16", seed=41)
+    inp = ki.make_inputs(w)
+    d = upload(inp, w)
+    nb = K.chunk_workspace_bytes(1, 100, 2, 128, 128)
+    assert nb == 1 * 2 * 2 * REC
+    ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=d["z"], engine="tc", workspace=ws)
+    torch.cuda.synchronize()
+    assert _timeouts(K) == 0
+    wsh = ws.cpu().numpy()
+    la = oracle.log_decay(inp["z"], w.g_min)
+    nv = 16  # B*H = 2 -> 16-column value slices
+    for h in range(2):
+        for n in range(2):
+            t0, t1 = 64 * n, min(100, 64 * n + 64)
+            L = t1 - t0
+            pad = lambda a: np.concatenate([a, np.zeros((64 - L,) + a.shape[1:])]) if L < 64 else a
+            q = pad(inp["q"][0, t0:t1, h].astype(np.float64)); k = pad(inp["k"][0, t0:t1, h].astype(np.float64))
+            v = pad(inp["v"][0, t0:t1, h].astype(np.float64)); beta = pad(inp["beta"][0, t0:t1, h].astype(np.float64))
+            g = pad(la[0, t0:t1, h])
+            mir = chunk_mirror.matrix_chunk(q, k, v, beta, g, np.zeros((128, 128)))
+            G = mir["G"]
+            rec = wsh[(h * 2 + n) * REC:(h * 2 + n + 1) * REC]
+            _close(_kmajor_image(rec[0:16384]), q * np.exp(G), f"Qg h{h} n{n}")
+            _close(_kmajor_image(rec[16384:32768]), k * np.exp(G[-1] - G), f"Kt h{h} n{n}")
+            _close(_kmajor_image(rec[32768:49152]), mir["W"], f"W h{h} n{n}")
+            _close(_mt_image(rec[49152:57344]), mir["M"].T, f"M h{h} n{n}")
+            U = np.zeros((64, 128))
+            uu = _bf(np.frombuffer(rec[57344:73728].tobytes(), dtype=np.uint16))
+            for s in range(128 // nv):
+                U[:, s * nv:(s + 1) * nv] = uu[s * 64 * nv:(s + 1) * 64 * nv].reshape(64, nv)
+            _close(U, mir["U"], f"U h{h} n{n}")
+            gam = np.frombuffer(rec[73728:74240].tobytes(), dtype=np.float32)
+            np.testing.assert_allclose(gam, np.exp(G[-1]), rtol=1e-4, atol=1e-30)
+
+
+@pytest.mark.parametrize("B,S,H", [(1, 1, 1), (1, 64, 1), (1, 65, 2), (2, 130, 3), (1, 200, 2), (3, 257, 27),
+                                   (2, 300, 80)])
+def test_tc_core_matches_oracle(K, B, S, H):
+    w = small("tc", B, S, H, 128, 128, 16, "bf16", seed=S + 3 * H, s0_std=0.02)
+    inp = ki.make_inputs(w)
+    d = upload(inp, w)
+    o, sf = K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=d["z"], initial_state=d["S0"], engine="tc")
+    torch.cuda.synchronize()
+    assert _timeouts(K) == 0
+    o_ref, s_ref = oracle.recurrence(inp["q"], inp["k"], inp["v"], inp["beta"], z=inp["z"], g_min=w.g_min,
+                                     initial_state=inp["S0"])
+    assert_bf16_outputs(to_np(o), o_ref, "o~")
+    assert_bf16_state(to_np(sf), s_ref, "final_state")
+
+
+def test_tc_matches_simt_engine(K):
+    w = small("ts", 2, 333, 4, 128, 128, 16, "bf16", seed=5, s0_std=0.02, z_std=2.0)
+    inp = ki.make_inputs(w)
+    d = upload(inp, w)
+    o1, s1 = K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=d["z"], initial_state=d["S0"], engine="tc")
+    o2, s2 = K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=d["z"], initial_state=d["S0"], engine="simt")
+    assert_bf16_outputs(to_np(o1), to_np(o2), "tc vs simt o~")
+    assert rel_fro(to_np(s1), to_np(s2)) <= 1e-2
+
+
+def test_tc_special_cases(K):
+    w = small("sp", 1, 150, 2, 128, 128, 16, "bf16", seed=9, s0_std=0.1)
+    inp = ki.make_inputs(w)
+    d = upload(inp, w)
+    zero_ld = torch.zeros(d["z"].shape, dtype=torch.float32, device="cuda")
+    # alpha = 1, beta = 0: the state never changes and o_t = S_0^T q_t
+    o, sf = K.chunk_fwd(d["q"], d["k"], d["v"], torch.zeros_like(d["beta"]), log_decay=zero_ld,
+                        initial_state=d["S0"], engine="tc")
+    assert rel_fro(to_np(sf), inp["S0"]) <= 1e-6
+    assert_bf16_outputs(to_np(o), np.einsum("bshc,bhcj->bshj", inp["q"].astype(np.float64),
+                                            inp["S0"].astype(np.float64)))
+    # alpha = 1 with writes (DeltaNet)
+    o, sf = K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], log_decay=zero_ld, initial_state=d["S0"], engine="tc")
+    o_ref, s_ref = oracle.recurrence(inp["q"], inp["k"], inp["v"], inp["beta"], log_decay=np.zeros_like(inp["z"]),
+                                     initial_state=inp["S0"])
+    assert_bf16_outputs(to_np(o), o_ref)
+    assert_bf16_state(to_np(sf), s_ref)
+    # empty sequence: final state = initial state
+    e = torch.empty(1, 0, 2, 128, dtype=torch.bfloat16, device="cuda")
+    o, sf = K.chunk_fwd(e, e, e, torch.empty(1, 0, 2, dtype=torch.bfloat16, device="cuda"), z=e,
+                        initial_state=d["S0"], engine="tc")
+    assert torch.equal(sf, d["S0"])
+
+
+def test_tc_state_handoff_in_place(K):
+    w = small("ho", 1, 300, 2, 128, 128, 16, "bf16", seed=12, s0_std=0.02)
+    inp = ki.make_inputs(w)
+    d = upload(inp, w)
+    o_all, s_all = K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=d["z"], initial_state=d["S0"], engine="tc")
+    st = d["S0"].clone()
+    outs = []
+    for a, b in ((0, 64), (64, 100), (100, 300)):
+        sl = lambda t: t[:, a:b].contiguous()
+        o, _ = K.chunk_fwd(sl(d["q"]), sl(d["k"]), sl(d["v"]), sl(d["beta"]), z=sl(d["z"]), initial_state=st,
+                           final_state=st, engine="tc")
+        outs.append(o)
+    assert_bf16_outputs(to_np(torch.cat(outs, 1)), to_np(o_all))
+    assert rel_fro(to_np(st), to_np(s_all)) <= 1e-2
+
+
+def test_tc_layer_with_fused_gate(K):
+    w = ki.custom("lay", 2, 500, 4, 128, 128, 256, "bf16", seed=77)
+    inp = ki.make_inputs(w)
+    d = upload(inp, w)
+    out = K.kda_forward(d["q"], d["k"], d["v"], d["z"], d["beta"], d["gate"], d["W_o"], None,
+                        g_min=w.g_min, eps=w.eps, state_dtype=torch.float32, engine="tc")
+    want = oracle_layer(inp, w)
+    assert_bf16_outputs(to_np(out["outputs"]), want["outputs"], "outputs")
+    assert_bf16_state(to_np(out["final_state"]), want["final_state"], "final_state")

@@ -25,7 +25,7 @@ def K():
     return K
 
 
-ENGINES = ["simt"]
+ENGINES = ["simt", "tc"]
 
 
 # ------------------------------------------------------------------ the page's examples
