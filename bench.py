@@ -253,6 +253,14 @@ def run_ours(args, rank, world, local):
     t_step = t_chunk + t_proj
     t_step_max, t_chunk_max, t_proj_max = reduce_max([t_step, t_chunk, t_proj], world, dev)
 
+    if args.only == "decode":
+        dec = run_decode(args, rank, world, local, K, dev, peaks)
+        return {"metric": METRIC, "decode": dec, "n_gpus": world} if rank == 0 else None
+    if args.only == "prefill":
+        return {"metric": METRIC, "value": round(N * world / t_step_max, 1), "unit": "tokens/s",
+                "kernels_ms": {"chunk_engine": round(t_chunk * 1e3, 4), "out_proj": round(t_proj * 1e3, 4)},
+                "gpu_launches": int(launches)} if rank == 0 else None
+
     # ---------------- end to end through the public API, host buffers
     hin = {n: torch.from_numpy(inp[n]).to(dt).pin_memory() for n in ("q", "k", "v", "z", "beta", "gate")}
     h2d = sum(t.numel() * t.element_size() for t in hin.values())
@@ -427,6 +435,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                    help="run one engine only (for profiling); the default runs both plus e2e")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
