@@ -67,3 +67,43 @@ def oracle_layer(inp, w, threads=None):
 
 def small(name, B, S, H, Dk, Dv, Dm, dtype, seed, **kw):
     return ki.custom(name, B, S, H, Dk, Dv, Dm, dtype, seed=seed, **kw)
+
+
+def upload_by_head(w, device="cuda"):
+    """Device tensors in the page's layout, generated one head at a time (host
+    memory stays at one head's worth even for the 1M-token workload)."""
+    import torch
+    dt = torch_dtype(w)
+    d = {
+        "q": torch.empty((w.B, w.S, w.H, w.Dk), dtype=dt, device=device),
+        "k": torch.empty((w.B, w.S, w.H, w.Dk), dtype=dt, device=device),
+        "z": torch.empty((w.B, w.S, w.H, w.Dk), dtype=dt, device=device),
+        "v": torch.empty((w.B, w.S, w.H, w.Dv), dtype=dt, device=device),
+        "gate": torch.empty((w.B, w.S, w.H, w.Dv), dtype=dt, device=device),
+        "beta": torch.empty((w.B, w.S, w.H), dtype=dt, device=device),
+    }
+    s0 = None
+    for h in range(w.H):
+        hd = ki.head_inputs(w, h)
+        for n in ("q", "k", "z", "v", "gate"):
+            d[n][:, :, h, :] = torch.from_numpy(hd[n]).to(device).to(dt)
+        d["beta"][:, :, h] = torch.from_numpy(hd["beta"]).to(device).to(dt)
+        if hd["S0"] is not None:
+            if s0 is None:
+                s0 = torch.empty((w.B, w.H, w.Dk, w.Dv), dtype=torch.float32, device=device)
+            s0[:, h] = torch.from_numpy(hd["S0"]).to(device)
+    d["S0"] = s0
+    d["W_o"] = to_dev(ki.weights(w), dt, device)
+    return d
+
+
+def oracle_head(w, b, h, t_rec=None, threads=1):
+    """Oracle o~ (at t_rec tokens) and final state for one (b, h) of a workload,
+    regenerating only that head's inputs."""
+    hd = ki.head_inputs(w, h)
+    sl = lambda a: a[b:b + 1, :, None, :]
+    s0 = None if hd["S0"] is None else hd["S0"][b:b + 1, None]
+    o, sf = oracle.recurrence(sl(hd["q"]), sl(hd["k"]), sl(hd["v"]), hd["beta"][b:b + 1, :, None],
+                              z=sl(hd["z"]), g_min=w.g_min, initial_state=s0, t_rec=t_rec, threads=threads)
+    gate = hd["gate"][b, t_rec if t_rec is not None else slice(None)]
+    return o[0, :, 0], sf[0, 0], gate
