@@ -103,6 +103,18 @@ __device__ __forceinline__ void load8f(const float *p, float (&f)[8]) {
     f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
+// The tensor-core engine works on bf16 data and every exponent it takes is
+// bounded (|x| <= 8 |g_min| + |g_min| * 64), so the hardware exp2 approximation
+// (a few ulp of fp32) is far below the bf16 rounding it feeds.
+__device__ __forceinline__ float fexp(float x) { return __expf(x); }
+__device__ __forceinline__ float log_alpha_fast(float z, float g_min) {
+    return g_min * __fdividef(1.0f, 1.0f + __expf(-z));
+}
+
+// A descriptor for base + off: the start-address field holds address >> 4 in 14
+// bits, which cannot carry for shared-memory addresses below 256 KB.
+__device__ __forceinline__ uint64_t dadd(uint64_t d, uint32_t off_bytes) { return d + (off_bytes >> 4); }
+
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
@@ -113,27 +125,32 @@ __device__ __forceinline__ void report_timeout(unsigned int *timeouts, int *dev_
 }
 
 // ================================================================ K2a: chunk_prep_kernel
+// Persistent: one CTA per SM walks (chunk, head, batch) units.  The next unit's
+// q, k and z tiles are loaded by TMA as soon as this unit's copies of them are
+// dead (after the A/M MMAs), v after the W/U MMA, and the workspace bulk
+// stores drain while the next unit is computed.
 // Shared-memory map (bytes from a 1024-aligned base).
-constexpr uint32_t P_QI = 0;         // q image, becomes Q e^G
-constexpr uint32_t P_KI = 16384;     // k image, becomes K e^{G_C - G}
-constexpr uint32_t P_VI = 32768;     // v image; later lo parts of the diagonal column operands
-constexpr uint32_t P_ZI = 49152;     // z image; later lo parts of the q row operand, then M^T image (8 KB) + T image (8 KB)
-constexpr uint32_t P_KC = 65536;     // column operands, 4 versions packed: [2 atoms][160 rows][128 B]; later W, U
-constexpr uint32_t P_KR = 106496;    // row operand from k: [2 atoms][64 rows][128 B]
-constexpr uint32_t P_QR = 122880;    // row operand from q
-constexpr uint32_t P_RH = 139264;    // [beta K e^G | beta V]^T: [256 rows][128 B]
-constexpr uint32_t P_SG = 172032;    // G fp32 [64][132]; later A, T fp32 [64][65] each
-constexpr uint32_t P_TAB = 205824;   // per-channel block constants [26][128] fp32
-constexpr uint32_t P_XS = 219136;    // scratch for the blocked inverse [3][256] fp32
-constexpr uint32_t P_BETA = 222208;  // beta [64] fp32
-constexpr uint32_t P_GAM = 222464;   // e^{G_C} [128] fp32
-constexpr uint32_t P_BAR = 222976;   // 3 mbarriers + TMEM slot
-constexpr uint32_t P_END = 223056;
+constexpr uint32_t P_QI = 0;         // q image; becomes Q e^G (stored as soon as P2 ends)
+constexpr uint32_t P_KI = 16384;     // k image; becomes K e^{G_C - G}
+constexpr uint32_t P_VI = 32768;     // v image; becomes beta V (MN-major B operand of the W|U MMA)
+constexpr uint32_t P_ZI = 49152;     // z image; becomes lo part of the q row operand
+constexpr uint32_t P_KC = 65536;     // column operands, 4 versions packed [2 atoms][160 rows][128 B]; later W, U
+constexpr uint32_t P_KR = 106496;    // row operand from k [2 atoms][64 rows][128 B]; later the M^T image
+constexpr uint32_t P_QR = 122880;    // row operand from q; later the T image
+constexpr uint32_t P_RH = 139264;    // beta K e^G image (MN-major B) + lo part of the diagonal column operand
+constexpr uint32_t P_SG = 172032;    // G fp32 [64][132]; later A [64][65] and T [64][68] fp32
+constexpr uint32_t P_TAB = 206080;   // per-channel block constants [26][128] fp32
+constexpr uint32_t P_XS = 219392;    // scratch for the blocked inverse [3][256] fp32
+constexpr uint32_t P_BETA = 222464;  // beta [64] fp32
+constexpr uint32_t P_GAM = 222720;   // e^{G_C} [128] fp32
+constexpr uint32_t P_BAR = 223232;   // 3 mbarriers + TMEM slot
+constexpr uint32_t P_END = 223312;
 constexpr size_t PREP_SMEM = P_END + 1024;
-constexpr uint32_t P_MT = P_ZI, P_TI = P_ZI + 8192;
+constexpr uint32_t P_MT = P_KR, P_TI = P_QR;
+constexpr uint32_t P_KLO = P_RH + 16384;
 constexpr uint32_t P_SA = P_SG, P_ST = P_SG + 16640;
 constexpr uint32_t P_WI = P_KC, P_UI = P_KC + 16384;
-constexpr int SG_LD = 132;
+constexpr int SG_LD = 132, SA_LD = 65, ST_LD = 68;
 constexpr uint32_t KC_ATOM = 160 * 128;  // bytes per atom column of the packed column operand
 
 // table rows: b_R (0-3), F_R = e^{b_{R-1} - m_R} (4-7), E_R = e^{b_{R-1}} (8-11),
@@ -143,6 +160,7 @@ __device__ __forceinline__ int kc_row0(int V) { return 8 * V * (V + 1); }  // 0,
 
 struct PrepArgs {
     int S, H, Nc, Nv;
+    int64_t units;  // Nc * H * B
     float g_min;
     const __nv_bfloat16 *beta;
     const float *log_decay;
@@ -157,9 +175,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = align1024(smraw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int t0 = n * CH;
-    const int len = min(CH, p.S - t0);
     uint64_t *bar_in = reinterpret_cast<uint64_t *>(sm + P_BAR);
     uint64_t *bar_am = bar_in + 1;
     uint64_t *bar_wu = bar_in + 2;
@@ -168,59 +183,98 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     float *tab = reinterpret_cast<float *>(sm + P_TAB);
     float *sbeta = reinterpret_cast<float *>(sm + P_BETA);
     float *sgam = reinterpret_cast<float *>(sm + P_GAM);
+    const uint32_t in_bytes = (p.log_decay ? 6u : 8u) * 8192u;
+
+    auto unit_coords = [&](int64_t u, int &n, int &h, int &b) {
+        n = (int)(u % p.Nc);
+        const int64_t bh = u / p.Nc;
+        h = (int)(bh % p.H);
+        b = (int)(bh / p.H);
+    };
+    auto load_qkz = [&](int64_t u) {  // arms bar_in for the whole unit
+        int n, h, b;
+        unit_coords(u, n, h, b);
+        mbar_arrive_expect_tx(bar_in, in_bytes);
+        for (int a = 0; a < 2; ++a) {
+            tma_load_4d(sm + P_QI + a * 8192, &tq, bar_in, 64 * a, h, n * CH, b);
+            tma_load_4d(sm + P_KI + a * 8192, &tk, bar_in, 64 * a, h, n * CH, b);
+            if (!p.log_decay) tma_load_4d(sm + P_ZI + a * 8192, &tz, bar_in, 64 * a, h, n * CH, b);
+        }
+    };
+    auto load_v = [&](int64_t u) {
+        int n, h, b;
+        unit_coords(u, n, h, b);
+        for (int a = 0; a < 2; ++a) tma_load_4d(sm + P_VI + a * 8192, &tv, bar_in, 64 * a, h, n * CH, b);
+    };
 
     if (tid == 0) {
         mbar_init(bar_in, 1);
         mbar_init(bar_am, 1);
         mbar_init(bar_wu, 1);
         fence_barrier_init();
-        mbar_arrive_expect_tx(bar_in, (p.log_decay ? 6u : 8u) * 8192u);
-        for (int a = 0; a < 2; ++a) {
-            tma_load_4d(sm + P_QI + a * 8192, &tq, bar_in, 64 * a, h, t0, b);
-            tma_load_4d(sm + P_KI + a * 8192, &tk, bar_in, 64 * a, h, t0, b);
-            tma_load_4d(sm + P_VI + a * 8192, &tv, bar_in, 64 * a, h, t0, b);
-            if (!p.log_decay) tma_load_4d(sm + P_ZI + a * 8192, &tz, bar_in, 64 * a, h, t0, b);
+        if ((int64_t)blockIdx.x < p.units) {
+            load_qkz(blockIdx.x);
+            load_v(blockIdx.x);
         }
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 256);
         tmem_relinquish();
     }
-    if (tid < CH)
-        sbeta[tid] = (tid < len) ? __bfloat162float(p.beta[((int64_t)b * p.S + t0 + tid) * p.H + h]) : 0.f;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    bool ok = mbar_wait(bar_in, 0);
-    ok = __syncthreads_and(ok);
+    bool ok = true;
 
-    if (ok) {
+    int it = 0;
+    for (int64_t u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++it) {
+        int n, h, b;
+        unit_coords(u, n, h, b);
+        const int t0 = n * CH;
+        const int len = min(CH, p.S - t0);
+        const int64_t u_next = u + gridDim.x;
+        const uint32_t par = it & 1;
+        // the previous unit's bulk stores must have read their shared sources
+        if (tid == 0) bulk_wait_read_all();
+        if (tid < CH)
+            sbeta[tid] = (tid < len) ? __bfloat162float(p.beta[((int64_t)b * p.S + t0 + tid) * p.H + h]) : 0.f;
+        ok = mbar_wait(bar_in, par);
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
+
         // ---------------- P1: G = in-chunk cumulative log-decay (rows past the sequence end: no decay)
         {
             const int c = tid & 127, half = tid >> 7;
-            float acc = 0.f;
-            for (int rr = 0; rr < 32; ++rr) {
-                const int r = half * 32 + rr;
-                float g = 0.f;
-                if (r < len) {
-                    if (p.log_decay) {
-                        g = p.log_decay[(((int64_t)b * p.S + t0 + r) * p.H + h) * DD + c];
-                    } else {
-                        const __nv_bfloat16 *zr = reinterpret_cast<const __nv_bfloat16 *>(
-                            sm + P_ZI + (c >> 6) * 8192 + sw128(r, (c & 63) >> 3));
-                        g = log_alpha_of(__bfloat162float(zr[c & 7]), p.g_min);
-                    }
+            float g[32];
+            if (p.log_decay) {
+#pragma unroll
+                for (int rr = 0; rr < 32; ++rr) {
+                    const int r = half * 32 + rr;
+                    g[rr] = (r < len) ? p.log_decay[(((int64_t)b * p.S + t0 + r) * p.H + h) * DD + c] : 0.f;
                 }
-                acc += g;
-                sG[r * SG_LD + c] = acc;
+            } else {
+                const uint8_t *zc = sm + P_ZI + (c >> 6) * 8192 + (c & 7) * 2;
+                const uint32_t ch = (c & 63) >> 3;
+#pragma unroll
+                for (int rr = 0; rr < 32; ++rr) {
+                    const int r = half * 32 + rr;
+                    const float zv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(zc + sw128(r, ch)));
+                    g[rr] = (r < len) ? log_alpha_fast(zv, p.g_min) : 0.f;
+                }
             }
-        }
-        __syncthreads();
-        if (tid >= 128) {
-            const int c = tid & 127;
-            const float base = sG[31 * SG_LD + c];
-            for (int r = 32; r < 64; ++r) sG[r * SG_LD + c] += base;
+            float acc = 0.f;
+#pragma unroll
+            for (int rr = 0; rr < 32; ++rr) {
+                acc += g[rr];
+                g[rr] = acc;
+            }
+            if (half == 0) sG[31 * SG_LD + c] = acc;
+            __syncthreads();
+            const float base = half ? sG[31 * SG_LD + c] : 0.f;
+            __syncthreads();
+#pragma unroll
+            for (int rr = 0; rr < 32; ++rr) sG[(half * 32 + rr) * SG_LD + c] = g[rr] + base;
         }
         __syncthreads();
         // ---------------- per-channel block constants
@@ -236,15 +290,15 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             for (int R = 0; R < 4; ++R) {
                 const float bm1 = R ? bb[R - 1] : 0.f;
                 tab[R * 128 + c] = bb[R];
-                tab[(4 + R) * 128 + c] = expf(bm1 - mm[R]);
-                tab[(8 + R) * 128 + c] = expf(bm1);
-                tab[(12 + R) * 128 + c] = expf(bb[3] - bb[R]);
+                tab[(4 + R) * 128 + c] = fexp(bm1 - mm[R]);
+                tab[(8 + R) * 128 + c] = fexp(bm1);
+                tab[(12 + R) * 128 + c] = fexp(bb[3] - bb[R]);
             }
 #pragma unroll
             for (int V = 0; V < 4; ++V)
 #pragma unroll
-                for (int R = 0; R <= V; ++R) tab[tab_c(V, R) * 128 + c] = expf(mm[V] - bb[R]);
-            sgam[c] = expf(bb[3]);
+                for (int R = 0; R <= V; ++R) tab[tab_c(V, R) * 128 + c] = fexp(mm[V] - bb[R]);
+            sgam[c] = fexp(bb[3]);
         }
         __syncthreads();
         // ---------------- P2: decay-scaled operands (one thread per row r and 4 chunks of 8 channels)
@@ -274,8 +328,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 float e1[8], e3[8], t[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    e1[e] = expf(G[e] - bRm1[e]);
-                    e3[e] = expf(bR[e] - G[e]);
+                    e1[e] = fexp(G[e] - bRm1[e]);
+                    e3[e] = fexp(bR[e] - G[e]);
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) t[e] = kv[e] * e1[e] * F[e];
@@ -303,8 +357,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                         unpack8(hi, hf);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) lo[e] = t[e] - hf[e];
-                        // same (row, chunk) as this thread's v chunk, which is already in registers
-                        *reinterpret_cast<uint4 *>(sm + P_VI + img) = pack8(lo);
+                        *reinterpret_cast<uint4 *>(sm + P_KLO + img) = pack8(lo);
                     }
                 }
 #pragma unroll
@@ -314,212 +367,233 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 for (int e = 0; e < 8; ++e) t[e] = kv[e] * e3[e] * Dd[e];
                 *reinterpret_cast<uint4 *>(sm + P_KI + img) = pack8(t);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int c = c0 + e;
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + P_RH + sw128(c, r >> 3) + (r & 7) * 2) =
-                        __float2bfloat16_rn(beta_r * kv[e] * e1[e] * E[e]);
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + P_RH + sw128(128 + c, r >> 3) + (r & 7) * 2) =
-                        __float2bfloat16_rn(beta_r * vv[e]);
-                }
+                for (int e = 0; e < 8; ++e) t[e] = beta_r * kv[e] * e1[e] * E[e];
+                *reinterpret_cast<uint4 *>(sm + P_RH + img) = pack8(t);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) t[e] = beta_r * vv[e];
+                *reinterpret_cast<uint4 *>(sm + P_VI + img) = pack8(t);
             }
         }
         fence_proxy_async_smem();
-    }
-    tc_fence_before();
-    __syncthreads();
-
-    // ---------------- tcgen05: A^T (cols 0-63) and M^T (cols 64-127), one N=16 block per V
-    if (tid == 0 && ok) {
-        tc_fence_after();
-        constexpr uint32_t id = idesc_f16(64, 16, 0, 0);
-        const uint32_t kc = smem_u32(sm + P_KC), kr = smem_u32(sm + P_KR), qr = smem_u32(sm + P_QR);
-        for (int V = 0; V < 4; ++V) {
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                const uint32_t ko = (s >> 2), kb = (s & 3) * 32;
-                const uint64_t a = smem_desc(kc + ko * KC_ATOM + kc_row0(V) * 128 + kb, 16, 1024, LAYOUT_SW128);
-                const uint64_t bk = smem_desc(kr + ko * 8192 + V * 2048 + kb, 16, 1024, LAYOUT_SW128);
-                const uint64_t bq = smem_desc(qr + ko * 8192 + V * 2048 + kb, 16, 1024, LAYOUT_SW128);
-                mma_f16_ss(tmem + 16 * V, a, bk, id, s > 0);
-                mma_f16_ss(tmem + 64 + 16 * V, a, bq, id, s > 0);
-            }
-        }
-        // residue products of the diagonal blocks of M: lo(k) * hi(q) + hi(k) * lo(q)
-        const uint32_t klo = smem_u32(sm + P_VI), qlo = smem_u32(sm + P_ZI);
-        for (int V = 0; V < 4; ++V) {
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                const uint32_t ko = (s >> 2), kb = (s & 3) * 32;
-                const uint64_t a_lo = smem_desc(klo + ko * 8192 + kb, 16, 1024, LAYOUT_SW128);
-                const uint64_t a_hi = smem_desc(kc + ko * KC_ATOM + kc_row0(V) * 128 + kb, 16, 1024, LAYOUT_SW128);
-                const uint64_t b_hi = smem_desc(qr + ko * 8192 + V * 2048 + kb, 16, 1024, LAYOUT_SW128);
-                const uint64_t b_lo = smem_desc(qlo + ko * 8192 + V * 2048 + kb, 16, 1024, LAYOUT_SW128);
-                mma_f16_ss(tmem + 128 + 16 * V, a_lo, b_hi, id, s > 0);
-                mma_f16_ss(tmem + 128 + 16 * V, a_hi, b_lo, id, 1);
-            }
-        }
-        mma_commit(bar_am);
-    }
-    if (ok) ok = mbar_wait(bar_am, 0);
-    ok = __syncthreads_and(ok);
-    tc_fence_after();
-
-    // ---------------- P3: A (masked, beta-weighted, fp32) and the M^T image
-    if (ok) {
-        const int q4 = warp & 3, role = warp >> 2;
-        const int i = 16 * q4 + lane;
-        uint32_t va[32], vb[32], vd[16];
-        const uint32_t taddr = tmem + ((uint32_t)(32 * q4) << 16) + 64 * role;
-        tmem_ld_32x32b_x32(taddr, va);
-        tmem_ld_32x32b_x32(taddr + 32, vb);
-        // residue of M's diagonal block of row i (columns r in 16*q4 .. 16*q4+15)
-        tmem_ld_32x32b_x16(tmem + ((uint32_t)(32 * q4) << 16) + 128 + 16 * q4, vd);
-        tmem_wait_ld();
-        if (lane < 16) {
-            if (role == 0) {
-                float *sA = reinterpret_cast<float *>(sm + P_SA);
-#pragma unroll
-                for (int r = 0; r < 64; ++r) {
-                    const float v = __uint_as_float(r < 32 ? va[r] : vb[r - 32]);
-                    sA[r * 65 + i] = (i < r) ? sbeta[r] * v : 0.f;
-                }
-            } else {
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    float t[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int r = 8 * cc + e;
-                        float v = __uint_as_float(r < 32 ? va[r] : vb[r - 32]);
-                        if ((r >> 4) == q4) v += __uint_as_float(vd[r & 15]);
-                        t[e] = (i <= r) ? v : 0.f;
-                    }
-                    *reinterpret_cast<uint4 *>(sm + P_MT + sw128(i, cc)) = pack8(t);
-                }
-            }
-        }
-    }
-    tc_fence_before();
-    __syncthreads();
-
-    // ---------------- P4: T = (I + A)^{-1} by blocks of 16 (fp32)
-    if (ok) {
-        const float *sA = reinterpret_cast<const float *>(sm + P_SA);
-        float *sT = reinterpret_cast<float *>(sm + P_ST);
-        float *xs = reinterpret_cast<float *>(sm + P_XS);
-        for (int e = tid; e < 64 * 65; e += 256) sT[e] = 0.f;
+        tc_fence_before();
         __syncthreads();
-        if (tid < 64) {  // diagonal blocks: column jc of block R by forward substitution
-            const int R = tid >> 4, jc = tid & 15, o = 16 * R;
-            float col[16];
-#pragma unroll
-            for (int a = 0; a < 16; ++a) {
-                float x = (a == jc) ? 1.f : 0.f;
-#pragma unroll
-                for (int m = 0; m < a; ++m) x -= sA[(o + a) * 65 + o + m] * col[m];
-                col[a] = (a < jc) ? 0.f : x;
-            }
-#pragma unroll
-            for (int a = 0; a < 16; ++a) sT[(o + a) * 65 + o + jc] = col[a];
-        }
-        __syncthreads();
-        for (int d = 1; d < 4; ++d) {
-            const int total = (4 - d) * 256;
-            for (int e = tid; e < total; e += 256) {
-                const int blk = e >> 8, R = d + blk, I = R - d, a = (e >> 4) & 15, bc = e & 15;
-                float x = 0.f;
-                for (int k = 16 * I; k < 16 * R; ++k) x += sA[(16 * R + a) * 65 + k] * sT[k * 65 + 16 * I + bc];
-                xs[blk * 256 + a * 16 + bc] = x;
-            }
-            __syncthreads();
-            for (int e = tid; e < total; e += 256) {
-                const int blk = e >> 8, R = d + blk, I = R - d, a = (e >> 4) & 15, bc = e & 15;
-                float x = 0.f;
-                for (int m = 0; m <= a; ++m) x += sT[(16 * R + a) * 65 + 16 * R + m] * xs[blk * 256 + m * 16 + bc];
-                sT[(16 * R + a) * 65 + 16 * I + bc] = -x;
-            }
-            __syncthreads();
-        }
-        {  // T image (K-major, 64 rows x 64 cols)
-            const int r = tid >> 2, part = tid & 3;
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int cc = 2 * part + u;
-                float t[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) t[e] = sT[r * 65 + 8 * cc + e];
-                *reinterpret_cast<uint4 *>(sm + P_TI + sw128(r, cc)) = pack8(t);
-            }
-        }
-        fence_proxy_async_smem();
-    }
-    tc_fence_before();
-    __syncthreads();
 
-    // ---------------- tcgen05: [W | U] = T [beta K e^G | beta V]   (M=64, N=256, K=64)
-    if (tid == 0 && ok) {
-        tc_fence_after();
-        constexpr uint32_t id = idesc_f16(64, 256, 0, 0);
-        const uint32_t ti = smem_u32(sm + P_TI), rh = smem_u32(sm + P_RH);
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            const uint64_t a = smem_desc(ti + s * 32, 16, 1024, LAYOUT_SW128);
-            const uint64_t bd = smem_desc(rh + s * 32, 16, 1024, LAYOUT_SW128);
-            mma_f16_ss(tmem, a, bd, id, s > 0);
-        }
-        mma_commit(bar_wu);
-    }
-    if (ok) ok = mbar_wait(bar_wu, 0);
-    ok = __syncthreads_and(ok);
-    tc_fence_after();
-
-    // ---------------- P5: W image and U slices
-    if (ok) {
-        const int q4 = warp & 3, half = warp >> 2;
-        const int r = 16 * q4 + lane;
-#pragma unroll 1
-        for (int cb = 0; cb < 4; ++cb) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q4) << 16) + 128 * half + 32 * cb, v);
-            tmem_wait_ld();
-            if (lane < 16) {
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    float t[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) t[e] = __uint_as_float(v[8 * g + e]);
-                    if (half == 0) {
-                        const int j = 4 * cb + g;
-                        *reinterpret_cast<uint4 *>(sm + P_WI + (j >> 3) * 8192 + sw128(r, j & 7)) = pack8(t);
-                    } else {
-                        const int jv = 32 * cb + 8 * g;
-                        const int slice = jv / p.Nv, within = jv % p.Nv;
-                        *reinterpret_cast<uint4 *>(sm + P_UI + slice * (64 * p.Nv * 2) + (r * p.Nv + within) * 2) =
-                            pack8(t);
-                    }
-                }
-            }
-        }
-        fence_proxy_async_smem();
-    }
-    tc_fence_before();
-    __syncthreads();
-
-    if (tid == 0) {
-        if (ok) {
-            uint8_t *rec = p.ws + ((size_t)(b * p.H + h) * p.Nc + n) * REC_BYTES;
+        uint8_t *rec = p.ws + ((size_t)(b * p.H + h) * p.Nc + n) * REC_BYTES;
+        // ---------------- Q e^G and K e^{G_C - G} leave now; tcgen05: A^T (cols 0-63), M^T (64-127),
+        // residues of M's diagonal blocks (128-191)
+        if (tid == 0) {
             bulk_store(rec + REC_QG, sm + P_QI, 16384);
             bulk_store(rec + REC_KT, sm + P_KI, 16384);
+            bulk_commit();
+            tc_fence_after();
+            constexpr uint32_t id = idesc_f16(64, 16, 0, 0);
+            const uint64_t kc = smem_desc(smem_u32(sm + P_KC), 16, 1024, LAYOUT_SW128);
+            const uint64_t kr = smem_desc(smem_u32(sm + P_KR), 16, 1024, LAYOUT_SW128);
+            const uint64_t qr = smem_desc(smem_u32(sm + P_QR), 16, 1024, LAYOUT_SW128);
+            const uint64_t klo = smem_desc(smem_u32(sm + P_KLO), 16, 1024, LAYOUT_SW128);
+            const uint64_t qlo = smem_desc(smem_u32(sm + P_ZI), 16, 1024, LAYOUT_SW128);
+#pragma unroll
+            for (int V = 0; V < 4; ++V) {
+#pragma unroll
+                for (int s8 = 0; s8 < 8; ++s8) {
+                    const uint32_t ko = (s8 >> 2), kb = (s8 & 3) * 32;
+                    const uint64_t a = dadd(kc, ko * KC_ATOM + kc_row0(V) * 128 + kb);
+                    const uint64_t bk = dadd(kr, ko * 8192 + V * 2048 + kb);
+                    const uint64_t bq = dadd(qr, ko * 8192 + V * 2048 + kb);
+                    mma_f16_ss(tmem + 16 * V, a, bk, id, s8 > 0);
+                    mma_f16_ss(tmem + 64 + 16 * V, a, bq, id, s8 > 0);
+                    mma_f16_ss(tmem + 128 + 16 * V, dadd(klo, ko * 8192 + kb), bq, id, s8 > 0);
+                    mma_f16_ss(tmem + 128 + 16 * V, a, dadd(qlo, ko * 8192 + V * 2048 + kb), id, 1);
+                }
+            }
+            mma_commit(bar_am);
+        }
+        ok = mbar_wait(bar_am, par);
+        ok = __syncthreads_and(ok);
+        tc_fence_after();
+        if (!ok) break;
+        // q, k, z images are dead (their stores have read them once the group drains): prefetch
+        if (tid == 0 && u_next < p.units) {
+            bulk_wait_read_all();
+            load_qkz(u_next);
+        }
+
+        // ---------------- P3: A (masked, beta-weighted, fp32) and the M^T image
+        {
+            const int q4 = warp & 3, role = warp >> 2;
+            const int i = 16 * q4 + lane;
+            uint32_t va[32], vb[32], vd[16];
+            const uint32_t taddr = tmem + ((uint32_t)(32 * q4) << 16) + 64 * role;
+            tmem_ld_32x32b_x32(taddr, va);
+            tmem_ld_32x32b_x32(taddr + 32, vb);
+            tmem_ld_32x32b_x16(tmem + ((uint32_t)(32 * q4) << 16) + 128 + 16 * q4, vd);
+            tmem_wait_ld();
+            if (lane < 16) {
+                if (role == 0) {
+                    float *sA = reinterpret_cast<float *>(sm + P_SA);
+#pragma unroll
+                    for (int r = 0; r < 64; ++r) {
+                        const float v = __uint_as_float(r < 32 ? va[r] : vb[r - 32]);
+                        sA[r * SA_LD + i] = (i < r) ? sbeta[r] * v : 0.f;
+                    }
+                } else {
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        float t[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int r = 8 * cc + e;
+                            float v = __uint_as_float(r < 32 ? va[r] : vb[r - 32]);
+                            if ((r >> 4) == q4) v += __uint_as_float(vd[r & 15]);
+                            t[e] = (i <= r) ? v : 0.f;
+                        }
+                        *reinterpret_cast<uint4 *>(sm + P_MT + sw128(i, cc)) = pack8(t);
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+        __syncthreads();
+
+        // ---------------- P4: T = (I + A)^{-1} by blocks of 16 (fp32)
+        {
+            const float *sA = reinterpret_cast<const float *>(sm + P_SA);
+            float *sT = reinterpret_cast<float *>(sm + P_ST);
+            float *xs = reinterpret_cast<float *>(sm + P_XS);
+            for (int e = tid; e < 64 * ST_LD / 4; e += 256)
+                reinterpret_cast<float4 *>(sT)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+            __syncthreads();
+            if (tid < 64) {  // diagonal block R, column jc: forward substitution
+                const int R = tid >> 4, jc = tid & 15, o = 16 * R;
+                float col[16];
+#pragma unroll
+                for (int a = 0; a < 16; ++a) {
+                    float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int m = 0; m < a; ++m) part[m & 3] += sA[(o + a) * SA_LD + o + m] * col[m];
+                    const float x = ((a == jc) ? 1.f : 0.f) - ((part[0] + part[1]) + (part[2] + part[3]));
+                    col[a] = (a < jc) ? 0.f : x;
+                }
+#pragma unroll
+                for (int a = 0; a < 16; ++a) sT[(o + a) * ST_LD + o + jc] = col[a];
+            }
+            __syncthreads();
+            // blocks below the diagonal, one distance d = R - I at a time, 4 columns per thread:
+            //   X = A[16R+a, 16I:16R] T[16I:16R, 16I+bc..+3],  T_RI = -T_RR X
+#pragma unroll
+            for (int d = 1; d < 4; ++d) {
+                const int e = tid;
+                const bool act = e < (4 - d) * 64;
+                const int blk = e >> 6, R = d + blk, I = R - d, a = (e >> 2) & 15, bc = (e & 3) * 4;
+                if (act) {
+                    const float *arow = sA + (16 * R + a) * SA_LD + 16 * I;
+                    const float *tblk = sT + 16 * I * ST_LD + 16 * I + bc;
+                    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int k = 0; k < 16 * d; ++k) {
+                        const float av = arow[k];
+                        const float4 tv = *reinterpret_cast<const float4 *>(tblk + k * ST_LD);
+                        x.x += av * tv.x; x.y += av * tv.y; x.z += av * tv.z; x.w += av * tv.w;
+                    }
+                    *reinterpret_cast<float4 *>(xs + blk * 256 + a * 16 + bc) = x;
+                }
+                __syncthreads();
+                if (act) {
+                    const float *trow = sT + (16 * R + a) * ST_LD + 16 * R;
+                    const float *xb = xs + blk * 256 + bc;
+                    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int m = 0; m < 16; ++m) {
+                        const float tv = trow[m];  // zero above the diagonal
+                        const float4 xv = *reinterpret_cast<const float4 *>(xb + m * 16);
+                        y.x += tv * xv.x; y.y += tv * xv.y; y.z += tv * xv.z; y.w += tv * xv.w;
+                    }
+                    *reinterpret_cast<float4 *>(sT + (16 * R + a) * ST_LD + 16 * I + bc) =
+                        make_float4(-y.x, -y.y, -y.z, -y.w);
+                }
+                __syncthreads();
+            }
+            {  // T image (K-major, 64 rows x 64 cols)
+                const int r = tid >> 2, part = tid & 3;
+#pragma unroll
+                for (int uu = 0; uu < 2; ++uu) {
+                    const int cc = 2 * part + uu;
+                    float t[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) t[e] = sT[r * ST_LD + 8 * cc + e];
+                    *reinterpret_cast<uint4 *>(sm + P_TI + sw128(r, cc)) = pack8(t);
+                }
+            }
+            fence_proxy_async_smem();
+        }
+        tc_fence_before();
+        __syncthreads();
+
+        // ---------------- tcgen05: W = T (beta K e^G), U = T (beta V)   (M=64, N=128+128, K=64, B MN-major)
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t id = idesc_f16(64, 128, 0, 1);
+            const uint64_t ti = smem_desc(smem_u32(sm + P_TI), 16, 1024, LAYOUT_SW128);
+            const uint64_t rw = smem_desc(smem_u32(sm + P_RH), 8192, 1024, LAYOUT_SW128);
+            const uint64_t ru = smem_desc(smem_u32(sm + P_VI), 8192, 1024, LAYOUT_SW128);
+#pragma unroll
+            for (int s4 = 0; s4 < 4; ++s4) {
+                mma_f16_ss(tmem, dadd(ti, s4 * 32), dadd(rw, s4 * 2048), id, s4 > 0);
+                mma_f16_ss(tmem + 128, dadd(ti, s4 * 32), dadd(ru, s4 * 2048), id, s4 > 0);
+            }
+            mma_commit(bar_wu);
+        }
+        ok = mbar_wait(bar_wu, par);
+        ok = __syncthreads_and(ok);
+        tc_fence_after();
+        if (!ok) break;
+        if (tid == 0 && u_next < p.units) load_v(u_next);  // beta V has been consumed
+
+        // ---------------- P5: W image and U slices
+        {
+            const int q4 = warp & 3, half = warp >> 2;
+            const int r = 16 * q4 + lane;
+#pragma unroll 1
+            for (int cb = 0; cb < 4; ++cb) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q4) << 16) + 128 * half + 32 * cb, v);
+                tmem_wait_ld();
+                if (lane < 16) {
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        float t[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) t[e] = __uint_as_float(v[8 * g + e]);
+                        if (half == 0) {
+                            const int j = 4 * cb + g;
+                            *reinterpret_cast<uint4 *>(sm + P_WI + (j >> 3) * 8192 + sw128(r, j & 7)) = pack8(t);
+                        } else {
+                            const int jv = 32 * cb + 8 * g;
+                            const int slice = jv / p.Nv, within = jv % p.Nv;
+                            *reinterpret_cast<uint4 *>(sm + P_UI + slice * (64 * p.Nv * 2) +
+                                                       (r * p.Nv + within) * 2) = pack8(t);
+                        }
+                    }
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
             bulk_store(rec + REC_W, sm + P_WI, 16384);
             bulk_store(rec + REC_MT, sm + P_MT, 8192);
             bulk_store(rec + REC_U, sm + P_UI, 16384);
             bulk_store(rec + REC_GAM, sgam, 512);
             bulk_commit();
-            bulk_wait_all();
-        } else {
-            report_timeout(p.timeouts, p.dev_status);
         }
     }
+
+    if (tid == 0) {
+        bulk_wait_all();
+        if (!ok) report_timeout(p.timeouts, p.dev_status);
+    }
+    tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 256);
 }
@@ -629,64 +703,99 @@ __global__ void __launch_bounds__(128, 1) chunk_state_kernel(StateArgs p) {
     const uint32_t S_COL = 0, P_COL = NV, O_COL0 = 2 * NV;
     const int c = tid;  // state row (key channel) owned by this thread
 
-    // ---------------- initial state -> TMEM accumulator and the bf16 S^T operand
+    // ---------------- initial state -> TMEM accumulator
     {
-        float sv[NV];
         uint32_t su[NV];
         if (p.S0) {
             const float4 *src = reinterpret_cast<const float4 *>(p.S0 + ((size_t)bh * DD + c) * DD + j0);
 #pragma unroll
             for (int k = 0; k < NV / 4; ++k) {
                 const float4 x = src[k];
-                sv[4 * k] = x.x; sv[4 * k + 1] = x.y; sv[4 * k + 2] = x.z; sv[4 * k + 3] = x.w;
+                su[4 * k] = __float_as_uint(x.x); su[4 * k + 1] = __float_as_uint(x.y);
+                su[4 * k + 2] = __float_as_uint(x.z); su[4 * k + 3] = __float_as_uint(x.w);
             }
         } else {
 #pragma unroll
-            for (int j = 0; j < NV; ++j) sv[j] = 0.f;
+            for (int j = 0; j < NV; ++j) su[j] = 0u;
         }
-#pragma unroll
-        for (int j = 0; j < NV; ++j) su[j] = __float_as_uint(sv[j]);
         tmem_st_cols<NV>(tmem + lane_base + S_COL, su);
         tmem_wait_st();
-        write_st_row<NV>(st_img, c, sv);
     }
-    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
+
+    constexpr uint32_t id_p = idesc_f16(64, NV, 0, 0);
+    constexpr uint32_t id_o = idesc_f16(64, NV, 1, 0);
+    constexpr uint32_t id_s = idesc_f16(128, NV, 1, 0);
+    const uint64_t d_st = smem_desc(smem_u32(st_img), 16, 1024, LAYOUT_SW128);
+    const uint64_t d_vt = smem_desc(smem_u32(vt_img), 16, 1024, LAYOUT_SW128);
+    const uint64_t d_k16 = smem_desc(smem_u32(sm), 16, 1024, LAYOUT_SW128);     // K-major images
+    const uint64_t d_mn = smem_desc(smem_u32(sm), 8192, 1024, LAYOUT_SW128);    // MN-major images
+
+    // O of chunk m (TMEM buffer m & 1) -> o~ rows of the chunk (this thread's token row)
+    auto store_o = [&](int m) {
+        uint32_t ov[NV];
+        tmem_ld_cols<NV>(tmem + lane_base + O_COL0 + (m & 1) * NV, ov);
+        tmem_wait_ld();
+        const int r = 16 * warp + lane;
+        const int t = m * CH + r;
+        if (lane < 16 && t < p.S) {
+            __nv_bfloat16 *dst = p.o + (((size_t)b * p.S + t) * p.H + h) * DD + j0;
+#pragma unroll
+            for (int k = 0; k < NV / 8; ++k) {
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(ov[8 * k + e]);
+                reinterpret_cast<uint4 *>(dst)[k] = pack8(f);
+            }
+        }
+    };
 
     bool ok = true;
     for (int n = 0; n < p.Nc; ++n) {
         const int stg = n & 1;
         uint8_t *sg = sm + stg * Cfg::STAGE;
+        const uint32_t sgo = stg * Cfg::STAGE;
         const uint32_t ocol = O_COL0 + (n & 1) * NV;
-        // ---------- P = W S and O = (Q e^G) S
-        if (tid == 0) {
-            if (!mbar_wait(&full[stg], (n >> 1) & 1)) {
-                s_fail = 1;
-            } else {
-                tc_fence_after();
-                constexpr uint32_t id = idesc_f16(64, NV, 0, 0);
-                const uint32_t w = smem_u32(sg + REC_W), qg = smem_u32(sg + REC_QG), sti = smem_u32(st_img);
+        // ---------- this chunk's record; S_n -> bf16 operand; S <- Diag(e^{G_C}) S_n in TMEM
+        if (!mbar_wait(&full[stg], (n >> 1) & 1)) s_fail = 1;
+        {
+            uint32_t sv[NV];
+            tmem_ld_cols<NV>(tmem + lane_base + S_COL, sv);
+            tmem_wait_ld();
+            float sf[NV];
 #pragma unroll
-                for (int s = 0; s < 8; ++s) {
-                    const uint32_t ko = s >> 2, kb = (s & 3) * 32;
-                    const uint64_t bd = smem_desc(sti + ko * (NV * 128) + kb, 16, 1024, LAYOUT_SW128);
-                    mma_f16_ss(tmem + P_COL, smem_desc(w + ko * 8192 + kb, 16, 1024, LAYOUT_SW128), bd, id, s > 0);
-                    mma_f16_ss(tmem + ocol, smem_desc(qg + ko * 8192 + kb, 16, 1024, LAYOUT_SW128), bd, id, s > 0);
-                }
-                mma_commit(bar_po);
-            }
+            for (int j = 0; j < NV; ++j) sf[j] = __uint_as_float(sv[j]);
+            write_st_row<NV>(st_img, c, sf);
+            const float gam = reinterpret_cast<const float *>(sg + Cfg::S_GAM)[c];
+#pragma unroll
+            for (int j = 0; j < NV; ++j) sv[j] = __float_as_uint(sf[j] * gam);
+            tmem_st_cols<NV>(tmem + lane_base + S_COL, sv);
+            tmem_wait_st();
         }
+        fence_proxy_async_smem();
+        tc_fence_before();
         __syncthreads();
         if (s_fail) { ok = false; break; }
+        // ---------- P = W S and O = (Q e^G) S
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int s = 0; s < 8; ++s) {
+                const uint32_t ko = s >> 2, kb = (s & 3) * 32;
+                const uint64_t bd = dadd(d_st, ko * (NV * 128) + kb);
+                mma_f16_ss(tmem + P_COL, dadd(d_k16, sgo + REC_W + ko * 8192 + kb), bd, id_p, s > 0);
+                mma_f16_ss(tmem + ocol, dadd(d_k16, sgo + REC_QG + ko * 8192 + kb), bd, id_p, s > 0);
+            }
+            mma_commit(bar_po);
+        }
+        if (n > 0) store_o(n - 1);  // overlaps the MMAs just issued
         if (!mbar_wait(bar_po, n & 1)) s_fail = 1;
         tc_fence_after();
-        // ---------- V' = U - P (token rows), S <- Diag(e^{G_C}) S (channel rows)
+        // ---------- V' = U - P (token rows of the M=64 accumulator layout)
         {
             uint32_t pv[NV];
             tmem_ld_cols<NV>(tmem + lane_base + P_COL, pv);
-            uint32_t sv[NV];
-            tmem_ld_cols<NV>(tmem + lane_base + S_COL, sv);
             tmem_wait_ld();
             if (lane < 16) {
                 const int r = 16 * warp + lane;
@@ -698,11 +807,6 @@ __global__ void __launch_bounds__(128, 1) chunk_state_kernel(StateArgs p) {
                         __float2bfloat16_rn(vp);
                 }
             }
-            const float gam = reinterpret_cast<const float *>(sg + Cfg::S_GAM)[c];
-#pragma unroll
-            for (int j = 0; j < NV; ++j) sv[j] = __float_as_uint(__uint_as_float(sv[j]) * gam);
-            tmem_st_cols<NV>(tmem + lane_base + S_COL, sv);
-            tmem_wait_st();
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -711,14 +815,11 @@ __global__ void __launch_bounds__(128, 1) chunk_state_kernel(StateArgs p) {
         // ---------- O += M V' and S += (K e^{G_C - G})^T V'
         if (tid == 0) {
             tc_fence_after();
-            constexpr uint32_t id_o = idesc_f16(64, NV, 1, 0);
-            constexpr uint32_t id_s = idesc_f16(128, NV, 1, 0);
-            const uint32_t mt = smem_u32(sg + REC_MT), kt = smem_u32(sg + REC_KT), vti = smem_u32(vt_img);
 #pragma unroll
             for (int s = 0; s < 4; ++s) {
-                const uint64_t bd = smem_desc(vti + s * 32, 16, 1024, LAYOUT_SW128);
-                mma_f16_ss(tmem + ocol, smem_desc(mt + s * 2048, 8192, 1024, LAYOUT_SW128), bd, id_o, 1);
-                mma_f16_ss(tmem + S_COL, smem_desc(kt + s * 2048, 8192, 1024, LAYOUT_SW128), bd, id_s, 1);
+                const uint64_t bd = dadd(d_vt, s * 32);
+                mma_f16_ss(tmem + ocol, dadd(d_mn, sgo + REC_MT + s * 2048), bd, id_o, 1);
+                mma_f16_ss(tmem + S_COL, dadd(d_mn, sgo + REC_KT + s * 2048), bd, id_s, 1);
             }
             mma_commit(bar_so);
         }
@@ -727,37 +828,8 @@ __global__ void __launch_bounds__(128, 1) chunk_state_kernel(StateArgs p) {
         __syncthreads();
         if (s_fail) { ok = false; break; }
         if (tid == 0 && n + 2 < p.Nc) issue_chunk(n + 2, stg);
-        // ---------- next S^T operand, then this chunk's outputs
-        if (n + 1 < p.Nc) {
-            uint32_t sv[NV];
-            tmem_ld_cols<NV>(tmem + lane_base + S_COL, sv);
-            tmem_wait_ld();
-            float sf[NV];
-#pragma unroll
-            for (int j = 0; j < NV; ++j) sf[j] = __uint_as_float(sv[j]);
-            write_st_row<NV>(st_img, c, sf);
-        }
-        {
-            uint32_t ov[NV];
-            tmem_ld_cols<NV>(tmem + lane_base + ocol, ov);
-            tmem_wait_ld();
-            const int r = 16 * warp + lane;
-            const int t = n * CH + r;
-            if (lane < 16 && t < p.S) {
-                __nv_bfloat16 *dst = p.o + (((size_t)b * p.S + t) * p.H + h) * DD + j0;
-#pragma unroll
-                for (int k = 0; k < NV / 8; ++k) {
-                    float f[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(ov[8 * k + e]);
-                    reinterpret_cast<uint4 *>(dst)[k] = pack8(f);
-                }
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
     }
+    if (ok && p.Nc > 0) store_o(p.Nc - 1);
 
     if (ok) {
         if (p.Sf) {
@@ -850,14 +922,19 @@ kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
         pa.H = a.H;
         pa.Nc = (int)Nc;
         pa.Nv = nv;
+        pa.units = Nc * a.H * a.B;
         pa.g_min = a.g_min;
         pa.beta = (const __nv_bfloat16 *)a.beta;
         pa.log_decay = a.log_decay;
         pa.ws = (uint8_t *)a.workspace;
         pa.timeouts = timeouts;
         pa.dev_status = a.dev_status;
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int64_t grid = pa.units < sms ? pa.units : sms;
         cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PREP_SMEM);
-        chunk_prep_kernel<<<dim3((unsigned)Nc, a.H, (unsigned)a.B), 256, PREP_SMEM, st>>>(tq, tk, tv, tz, pa);
+        chunk_prep_kernel<<<(unsigned)grid, 256, PREP_SMEM, st>>>(tq, tk, tv, tz, pa);
         s = check_launch("chunk_prep_kernel");
         if (s != KDA_OK) return s;
     }
