@@ -76,6 +76,13 @@ uint64_t kda_launch_count(void);
  * the last reset (0 in a healthy run); reset != 0 clears it.  Synchronous. */
 kda_status_t kda_device_timeouts(uint32_t *count, int reset);
 
+/* Self-test of the bounded-wait path the tensor-core kernels use: launches a
+ * one-CTA kernel that waits on a barrier nothing completes, gives up after
+ * limit_us microseconds (1 .. 1e6), writes KDA_ERR_TIMEOUT to *dev_status (a
+ * device int32), counts one timeout and returns.  Nothing traps or faults and
+ * the context stays usable.  Asynchronous on `stream`. */
+kda_status_t kda_selftest_wait_timeout(int32_t *dev_status, uint32_t limit_us, void *stream);
+
 /*
  * kda_gate — decay gate of the "KDA Recurrence" page:
  *   log_alpha[i] = g_min * sigmoid(z[i])   for i in [0, n)

@@ -56,6 +56,7 @@ SIGNATURES = {
     "kda_version": (ctypes.c_int, []),
     "kda_launch_count": (ctypes.c_uint64, []),
     "kda_device_timeouts": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]),
+    "kda_selftest_wait_timeout": (ctypes.c_int, [_p, ctypes.c_uint32, _p]),
     "kda_gate": (ctypes.c_int, [_p, ctypes.c_int, _i64, _f32, _p, _p]),
     "kda_chunk_workspace_size": (ctypes.c_int, [ctypes.POINTER(ChunkArgs), ctypes.POINTER(ctypes.c_size_t)]),
     "kda_chunk_fwd": (ctypes.c_int, [ctypes.POINTER(ChunkArgs)]),

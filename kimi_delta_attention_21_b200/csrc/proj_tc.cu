@@ -2,12 +2,13 @@
 //   y[n, m] = sum_i x[n, i] * W_o[m, i]      (head concat is x's row-major layout)
 // bf16 operands, fp32 accumulation in TMEM, bf16 output.
 //
-// One CTA computes a 128 x 256 tile of y.  Warp 0 (one thread) streams
-// 128x64 tiles of x and 256x64 tiles of W_o into a 4-stage shared-memory ring
-// with TMA (128-byte swizzle); warp 1 (one thread) issues tcgen05.mma
-// (M=128, N=256, K=16) into a 256-column TMEM accumulator and releases each
-// stage with tcgen05.commit; then all four warps read the accumulator back
-// (tcgen05.ld 32x32b, one row per thread) and store bf16.
+// One CTA computes a 128 x BN tile of y (BN = 256, or 64 when there are few
+// rows, as in decode, so that the grid still covers the SMs).  Warp 0 (one
+// thread) streams 128x64 tiles of x and BNx64 tiles of W_o into a 4-stage
+// shared-memory ring with TMA (128-byte swizzle); warp 1 (one thread) issues
+// tcgen05.mma (M=128, N=BN, K=16) into a BN-column TMEM accumulator and
+// releases each stage with tcgen05.commit; then all four warps read the
+// accumulator back (tcgen05.ld 32x32b, one row per thread) and store bf16.
 #include "kda_internal.cuh"
 #include "sm100_ptx.cuh"
 #include "tma_host.cuh"
@@ -18,16 +19,23 @@ namespace {
 
 using namespace sm100;
 
-constexpr int BM = 128, BN = 256, BK = 64, ST = 4;
-constexpr uint32_t A_BYTES = BM * BK * 2;
-constexpr uint32_t B_BYTES = BN * BK * 2;
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr size_t SMEM_BYTES = ST * STAGE_BYTES + 1024 /*alignment slack*/ + 256 /*barriers*/;
-constexpr uint32_t TMEM_COLS = 256;
+constexpr int BM = 128, BK = 64, ST = 4;
 
+template <int BN> struct ProjCfg {
+    static constexpr uint32_t A_BYTES = BM * BK * 2;
+    static constexpr uint32_t B_BYTES = BN * BK * 2;
+    static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr size_t SMEM_BYTES = ST * STAGE_BYTES + 1024 /*alignment slack*/ + 256 /*barriers*/;
+    static constexpr uint32_t TMEM_COLS = BN < 32 ? 32 : BN;
+};
+
+template <int BN>
 __global__ void __launch_bounds__(128, 1)
 proj_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
                int K, __nv_bfloat16 *__restrict__ y, unsigned int *timeouts) {
+    using Cfg = ProjCfg<BN>;
+    constexpr uint32_t A_BYTES = Cfg::A_BYTES, B_BYTES = Cfg::B_BYTES, STAGE_BYTES = Cfg::STAGE_BYTES;
+    constexpr uint32_t TMEM_COLS = Cfg::TMEM_COLS;
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = sm;
@@ -145,19 +153,33 @@ bool proj_tc_supported(int64_t N, int K, int Dm, kda_dtype_t dt) {
     return dt == KDA_BF16 && K % 8 == 0 && Dm % 8 == 0 && N <= 0x7fffffff && (N + BM - 1) / BM <= 65535;
 }
 
+template <int BN>
+static kda_status_t launch_proj_tc_bn(const CUtensorMap &ta, const void *W, int64_t N, int K, int Dm, void *y,
+                                      cudaStream_t st) {
+    using Cfg = ProjCfg<BN>;
+    CUtensorMap tb;
+    kda_status_t s = make_tmap_2d(&tb, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)Dm, (uint64_t)K,
+                                  (uint64_t)K, BN, BK, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (s != KDA_OK) return s;
+    cudaFuncSetAttribute(proj_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_BYTES);
+    const dim3 grid((unsigned)((Dm + BN - 1) / BN), (unsigned)((N + BM - 1) / BM));
+    proj_tc_kernel<BN><<<grid, 128, Cfg::SMEM_BYTES, st>>>(ta, tb, (int)N, Dm, K, (__nv_bfloat16 *)y,
+                                                          device_timeout_counter());
+    return check_launch("proj_tc_kernel");
+}
+
 kda_status_t launch_proj_tc(const void *x, const void *W, int64_t N, int K, int Dm, void *y, cudaStream_t st) {
-    CUtensorMap ta, tb;
+    CUtensorMap ta;
     kda_status_t s = make_tmap_2d(&ta, x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)N, (uint64_t)K,
                                   (uint64_t)K, BM, BK, CU_TENSOR_MAP_SWIZZLE_128B);
     if (s != KDA_OK) return s;
-    s = make_tmap_2d(&tb, W, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)Dm, (uint64_t)K, (uint64_t)K, BN, BK,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
-    if (s != KDA_OK) return s;
-    cudaFuncSetAttribute(proj_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
-    const dim3 grid((unsigned)((Dm + BN - 1) / BN), (unsigned)((N + BM - 1) / BM));
-    proj_tc_kernel<<<grid, 128, SMEM_BYTES, st>>>(ta, tb, (int)N, Dm, K, (__nv_bfloat16 *)y,
-                                                 device_timeout_counter());
-    return check_launch("proj_tc_kernel");
+    // few rows (decode): narrow tiles so that the grid covers the SMs
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t tiles256 = ((N + BM - 1) / BM) * ((Dm + 255) / 256);
+    if (tiles256 < sms) return launch_proj_tc_bn<64>(ta, W, N, K, Dm, y, st);
+    return launch_proj_tc_bn<256>(ta, W, N, K, Dm, y, st);
 }
 
 }  // namespace kda
