@@ -392,6 +392,15 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             const uint64_t qr = smem_desc(smem_u32(sm + P_QR), 16, 1024, LAYOUT_SW128);
             const uint64_t klo = smem_desc(smem_u32(sm + P_KLO), 16, 1024, LAYOUT_SW128);
             const uint64_t qlo = smem_desc(smem_u32(sm + P_ZI), 16, 1024, LAYOUT_SW128);
+            // lo(k) * hi(q) for all four diagonal blocks at once: rows i of the residue image
+            // carry the scaling of their own block, so the products are right wherever i and
+            // r share a block (the only entries read)
+            constexpr uint32_t id64 = idesc_f16(64, 64, 0, 0);
+#pragma unroll
+            for (int s8 = 0; s8 < 8; ++s8) {
+                const uint32_t ko = (s8 >> 2), kb = (s8 & 3) * 32;
+                mma_f16_ss(tmem + 128, dadd(klo, ko * 8192 + kb), dadd(qr, ko * 8192 + kb), id64, s8 > 0);
+            }
 #pragma unroll
             for (int V = 0; V < 4; ++V) {
 #pragma unroll
@@ -402,7 +411,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                     const uint64_t bq = dadd(qr, ko * 8192 + V * 2048 + kb);
                     mma_f16_ss(tmem + 16 * V, a, bk, id, s8 > 0);
                     mma_f16_ss(tmem + 64 + 16 * V, a, bq, id, s8 > 0);
-                    mma_f16_ss(tmem + 128 + 16 * V, dadd(klo, ko * 8192 + kb), bq, id, s8 > 0);
+                    // hi(k) * lo(q) on block V's columns, added to the residue above
                     mma_f16_ss(tmem + 128 + 16 * V, a, dadd(qlo, ko * 8192 + V * 2048 + kb), id, 1);
                 }
             }
