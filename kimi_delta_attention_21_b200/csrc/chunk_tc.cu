@@ -44,6 +44,10 @@
 // output error for tokens whose o~ is small.  The diagonal blocks of M are
 // therefore computed with split operands, x = hi + lo (both bf16): the MMA
 // adds hi*lo + lo*hi on top of hi*hi, which leaves ~2^-17 relative error.
+#include <cstring>
+
+#include <cuda_fp16.h>
+
 #include "kda_internal.cuh"
 #include "sm100_ptx.cuh"
 #include "tma_host.cuh"
@@ -59,14 +63,17 @@ constexpr int DD = 128;  // D_k = D_v
 constexpr float TC_GMIN_LIMIT = -5.5f;
 
 // ---------------------------------------------------------------- workspace record (per b, h, chunk)
-constexpr uint32_t REC_QG = 0;        // Q * e^G          K-major SW128 image [2 atoms][64 rows][128 B]
-constexpr uint32_t REC_KT = 16384;    // K * e^{G_C - G}  same image (MN-major A operand of K~^T V')
-constexpr uint32_t REC_W = 32768;     // W                same image
-constexpr uint32_t REC_MT = 49152;    // M^T              [64 rows i][128 B: r] (MN-major A operand of M V')
-constexpr uint32_t REC_U = 57344;     // U                [128/NV slices][64 rows][NV] bf16
-constexpr uint32_t REC_GAM = 73728;   // e^{G_C}          128 fp32
-constexpr uint32_t REC_IMG = 57344;   // bytes of the four images
+// All images are 128-byte-swizzled bf16 tiles in the layout the state kernel's
+// MMAs read them in, so a record is one contiguous bulk copy away from use.
+constexpr uint32_t REC_WQ = 0;        // [2 atoms (c / 64)][128 rows: -W rows 0-63, Q e^G rows 64-127][128 B]
+                                      //   K-major A operand of [-W; Q e^G] S (M = 128)
+constexpr uint32_t REC_KT = 32768;    // K e^{G_C - G}  [2 atoms (c / 64)][64 rows i][128 B], MN-major A of K~^T V'
+constexpr uint32_t REC_MT = 49152;    // M^T            [64 rows i][128 B: r]; with the K~ atom in front of it,
+                                      //   the MN-major A operand of [*; M] V' (M = 128, rows 64-127 = M)
+constexpr uint32_t REC_U = 57344;     // U^T            [128 rows j][128 B: r]
+constexpr uint32_t REC_GAM = 73728;   // e^{G_C}        128 fp32
 constexpr uint32_t REC_BYTES = 74240;
+constexpr uint32_t SIG_BYTES = CH * 128 * 2;  // per chunk: sigmoid of the output-gate logits, [64][128] f16
 
 __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
@@ -159,12 +166,14 @@ __device__ __forceinline__ int tab_c(int V, int R) { return 16 + V * (V + 1) / 2
 __device__ __forceinline__ int kc_row0(int V) { return 8 * V * (V + 1); }  // 0, 16, 48, 96
 
 struct PrepArgs {
-    int S, H, Nc, Nv;
+    int S, H, Nc;
     int64_t units;  // Nc * H * B
     float g_min;
     const __nv_bfloat16 *beta;
     const float *log_decay;
+    const __nv_bfloat16 *gate;  // output-gate logits (B, S, H, 128), or null
     uint8_t *ws;
+    __half *sig;                // sigmoid(gate) per (b, h, chunk): [2 atoms (j / 64)][64 rows r][128 B] f16, swizzled
     unsigned int *timeouts;
     int *dev_status;
 };
@@ -382,7 +391,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         // ---------------- Q e^G and K e^{G_C - G} leave now; tcgen05: A^T (cols 0-63), M^T (64-127),
         // residues of M's diagonal blocks (128-191)
         if (tid == 0) {
-            bulk_store(rec + REC_QG, sm + P_QI, 16384);
+            // Q e^G fills rows 64-127 of each atom of the stacked [W; Q e^G] image
+            bulk_store(rec + REC_WQ + 8192, sm + P_QI, 8192);
+            bulk_store(rec + REC_WQ + 16384 + 8192, sm + P_QI + 8192, 8192);
             bulk_store(rec + REC_KT, sm + P_KI, 16384);
             bulk_commit();
             tc_fence_after();
@@ -417,14 +428,42 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             }
             mma_commit(bar_am);
         }
+        // while the MMAs run: sigmoid of the output-gate logits (full fp32, stored as f16) for the state
+        // kernel's output stage, in its tile layout [2 atoms (j / 64)][64 rows r][128 B], 128-byte swizzled
+        if (p.gate) {
+            const int row = tid >> 2, part = tid & 3;
+            if (row < len) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    p.gate + (((int64_t)b * p.S + t0 + row) * p.H + h) * DD + part * 32);
+                uint8_t *dst = reinterpret_cast<uint8_t *>(p.sig + ((size_t)(b * p.H + h) * p.Nc + n) * (CH * DD)) +
+                               (part >> 1) * 8192;
+                uint4 gv[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) gv[k] = src[k];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    float g[8];
+                    unpack8(gv[k], g);
+                    uint4 o;
+                    __half2 *oh = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        oh[e] = __floats2half2_rn(__fdividef(1.0f, 1.0f + __expf(-g[2 * e])),
+                                                  __fdividef(1.0f, 1.0f + __expf(-g[2 * e + 1])));
+                    *reinterpret_cast<uint4 *>(dst + sw128(row, 4 * (part & 1) + k)) = o;
+                }
+            }
+        }
         ok = mbar_wait(bar_am, par);
         ok = __syncthreads_and(ok);
         tc_fence_after();
         if (!ok) break;
         // q, k, z images are dead (their stores have read them once the group drains): prefetch
-        if (tid == 0 && u_next < p.units) {
-            bulk_wait_read_all();
-            load_qkz(u_next);
+        if (tid == 0) {
+            if (u_next < p.units) {
+                bulk_wait_read_all();
+                load_qkz(u_next);
+            }
         }
 
         // ---------------- P3: A (masked, beta-weighted, fp32) and the M^T image
@@ -538,17 +577,19 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         tc_fence_before();
         __syncthreads();
 
-        // ---------------- tcgen05: W = T (beta K e^G), U = T (beta V)   (M=64, N=128+128, K=64, B MN-major)
+        // ---------------- tcgen05: W = T (beta K e^G)            (M=64, N=128, K=64: A = T, B MN-major)
+        //                   U^T = (beta V)^T T^T              (M=128, N=64, K=64: A MN-major, B = T K-major)
         if (tid == 0) {
             tc_fence_after();
-            constexpr uint32_t id = idesc_f16(64, 128, 0, 1);
+            constexpr uint32_t idw = idesc_f16(64, 128, 0, 1);
+            constexpr uint32_t idu = idesc_f16(128, 64, 1, 0);
             const uint64_t ti = smem_desc(smem_u32(sm + P_TI), 16, 1024, LAYOUT_SW128);
             const uint64_t rw = smem_desc(smem_u32(sm + P_RH), 8192, 1024, LAYOUT_SW128);
-            const uint64_t ru = smem_desc(smem_u32(sm + P_VI), 8192, 1024, LAYOUT_SW128);
+            const uint64_t vt = smem_desc(smem_u32(sm + P_VI), 8192, 1024, LAYOUT_SW128);
 #pragma unroll
             for (int s4 = 0; s4 < 4; ++s4) {
-                mma_f16_ss(tmem, dadd(ti, s4 * 32), dadd(rw, s4 * 2048), id, s4 > 0);
-                mma_f16_ss(tmem + 128, dadd(ti, s4 * 32), dadd(ru, s4 * 2048), id, s4 > 0);
+                mma_f16_ss(tmem, dadd(ti, s4 * 32), dadd(rw, s4 * 2048), idw, s4 > 0);
+                mma_f16_ss(tmem + 128, dadd(vt, s4 * 2048), dadd(ti, s4 * 32), idu, s4 > 0);
             }
             mma_commit(bar_wu);
         }
@@ -558,30 +599,41 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         if (!ok) break;
         if (tid == 0 && u_next < p.units) load_v(u_next);  // beta V has been consumed
 
-        // ---------------- P5: W image and U slices
+        // ---------------- P5: -W image (warps 0-3, M = 64 accumulator rows) and U^T image (warps 4-7,
+        // one value column j per lane)
         {
-            const int q4 = warp & 3, half = warp >> 2;
-            const int r = 16 * q4 + lane;
+            const int q4 = warp & 3;
+            if (warp < 4) {
+                const int r = 16 * q4 + lane;
 #pragma unroll 1
-            for (int cb = 0; cb < 4; ++cb) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q4) << 16) + 128 * half + 32 * cb, v);
-                tmem_wait_ld();
-                if (lane < 16) {
+                for (int cb = 0; cb < 4; ++cb) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q4) << 16) + 32 * cb, v);
+                    tmem_wait_ld();
+                    if (lane < 16) {
+#pragma unroll
+                        for (int g = 0; g < 4; ++g) {
+                            float t[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) t[e] = -__uint_as_float(v[8 * g + e]);
+                            const int j = 4 * cb + g;  // 8-column group
+                            *reinterpret_cast<uint4 *>(sm + P_WI + (j >> 3) * 8192 + sw128(r, j & 7)) = pack8(t);
+                        }
+                    }
+                }
+            } else {
+                const int jv = 32 * q4 + lane;
+#pragma unroll 1
+                for (int cb = 0; cb < 2; ++cb) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q4) << 16) + 128 + 32 * cb, v);
+                    tmem_wait_ld();
 #pragma unroll
                     for (int g = 0; g < 4; ++g) {
                         float t[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) t[e] = __uint_as_float(v[8 * g + e]);
-                        if (half == 0) {
-                            const int j = 4 * cb + g;
-                            *reinterpret_cast<uint4 *>(sm + P_WI + (j >> 3) * 8192 + sw128(r, j & 7)) = pack8(t);
-                        } else {
-                            const int jv = 32 * cb + 8 * g;
-                            const int slice = jv / p.Nv, within = jv % p.Nv;
-                            *reinterpret_cast<uint4 *>(sm + P_UI + slice * (64 * p.Nv * 2) +
-                                                       (r * p.Nv + within) * 2) = pack8(t);
-                        }
+                        *reinterpret_cast<uint4 *>(sm + P_UI + sw128(jv, 4 * cb + g)) = pack8(t);
                     }
                 }
             }
@@ -590,7 +642,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         tc_fence_before();
         __syncthreads();
         if (tid == 0) {
-            bulk_store(rec + REC_W, sm + P_WI, 16384);
+            bulk_store(rec + REC_WQ, sm + P_WI, 8192);
+            bulk_store(rec + REC_WQ + 16384, sm + P_WI + 8192, 8192);
             bulk_store(rec + REC_MT, sm + P_MT, 8192);
             bulk_store(rec + REC_U, sm + P_UI, 16384);
             bulk_store(rec + REC_GAM, sgam, 512);
@@ -608,264 +661,381 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
 }
 
 // ================================================================ K2b: chunk_state_kernel
+// One CTA per (head, batch) walks the chunks in order.  The state is kept
+// transposed in TMEM: lane j (value column) holds S[:, j] in fp32, so every
+// per-chunk product takes its A operand straight from TMEM and the register
+// work of the chain is spread over all 128 lanes.  Warp 8 issues the MMAs and
+// the record copies; warps 0-7 (lane quarter = warp % 4, column half =
+// warp / 4) do the register work.  Per chunk n:
+//   warps:    S^T -> bf16 copy in TMEM; S^T <- S^T Diag(e^{G_C})
+//   MMA:      PO  = S^T [-W; Q e^G]^T           PO[j, r] = -(W S)[r, j],  PO[j, 64 + r] = (Q e^G S)[r, j]
+//   warps:    V'^T = U^T + PO[:, 0:64] -> bf16 copy in TMEM
+//   MMA:      S^T += V'^T K~,  PO[:, 64:128] += V'^T M^T      (= O^T of chunk n)
+// and, one chunk behind, the output: the warps write O^T (bf16) as an operand
+// image, one MMA with [I; I] turns it back into token rows (into the PO
+// buffer, now free; lanes 64-127 repeat lanes 0-63), and the eight warps, 32
+// rows x 32 columns each, apply the RMS normalisation over the head and the
+// sigmoid output gate (precomputed by the prep kernel) and store the tile with
+// a TMA tensor store.
+// Records stream in by bulk copies, two stages deep.
 struct StateArgs {
     int S, H, Nc;
     const uint8_t *ws;
+    const __half *sig;  // sigmoid of the output-gate logits per chunk (tile layout), or null: write o~
     const float *S0;
     float *Sf;
-    __nv_bfloat16 *o;
+    float eps;
     unsigned int *timeouts;
     int *dev_status;
 };
 
-template <int NV> struct StateCfg {
-    static constexpr uint32_t U_BYTES = 64 * NV * 2;
-    static constexpr uint32_t STAGE_RAW = REC_IMG + U_BYTES + 512;
-    static constexpr uint32_t STAGE = (STAGE_RAW + 1023) & ~1023u;
-    static constexpr uint32_t S_U = REC_IMG;
-    static constexpr uint32_t S_GAM = REC_IMG + U_BYTES;
-    static constexpr uint32_t B_ST = 2 * STAGE;          // S^T image [2 atoms][NV rows][128 B]
-    static constexpr uint32_t B_VT = B_ST + NV * 256;    // V'^T image [NV rows][128 B]
-    static constexpr uint32_t B_BAR = B_VT + NV * 128;
-    static constexpr uint32_t END = B_BAR + 64;
-    static constexpr size_t SMEM = END + 1024;
-    static constexpr uint32_t TCOLS = 4 * NV <= 32 ? 32 : (4 * NV <= 64 ? 64 : (4 * NV <= 128 ? 128 : 256));
-    static constexpr uint32_t EXPECT = REC_IMG + U_BYTES + 512;
-};
+constexpr int ST_THREADS = 288;                // warps 0-7 register work, warp 8 MMA + copies
+constexpr uint32_t ST_STAGE = REC_GAM;         // the image part of a record (73728 B)
+constexpr uint32_t ST_GAM = 2 * ST_STAGE;      // e^{G_C} [2 stages][128] fp32
+constexpr uint32_t ST_OIMG = ST_GAM + 1024;    // output tile [2 atoms (j / 64)][64 rows r][128 B]
+constexpr uint32_t ST_SIGT = ST_OIMG + 16384;  // sigmoid(gate) tile, same layout, f16
+constexpr uint32_t ST_OT = ST_SIGT + 16384;    // O^T image, K-major B [128 rows j][128 B: 64 r]
+constexpr uint32_t ST_ID = ST_OT + 16384;      // [I_64; I_64], K-major A [128 rows][128 B: 64 k]
+constexpr uint32_t ST_RED = ST_ID + 16384;     // per-row partial sums of squares [64][4] fp32
+constexpr uint32_t ST_BAR = ST_RED + 1024;     // mbarriers + TMEM slot
+constexpr uint32_t ST_END = ST_BAR + 128;
+constexpr size_t STATE_SMEM = ST_END + 1024;
+static_assert(STATE_SMEM <= 232448, "state kernel shared memory");
+// TMEM columns
+constexpr uint32_t T_S32 = 0;     // S^T fp32 [j][c]
+constexpr uint32_t T_S16 = 128;   // S^T bf16 pairs (A operand, K = c)
+constexpr uint32_t T_PO = 192;    // two [128][128] accumulators
+constexpr uint32_t T_V16 = 448;   // V'^T bf16 pairs (A operand, K = r)
+constexpr uint32_t ST_TCOLS = 512;
 
-template <int NV>
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&v)[NV]) {
-#pragma unroll
-    for (int k = 0; k < NV / 16; ++k) {
-        uint32_t t[16];
-        tmem_ld_32x32b_x16(taddr + 16 * k, t);
-#pragma unroll
-        for (int e = 0; e < 16; ++e) v[16 * k + e] = t[e];
-    }
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-template <int NV>
-__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t (&v)[NV]) {
-#pragma unroll
-    for (int k = 0; k < NV / 16; ++k) {
-        uint32_t t[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) t[e] = v[16 * k + e];
-        tmem_st_32x32b_x16(taddr + 16 * k, t);
-    }
-}
-
-// S^T image element (row j, column c) for the K-major B operand [2 atoms][NV rows][128 B]
-template <int NV>
-__device__ __forceinline__ void write_st_row(uint8_t *img, int c, const float *vals) {
-#pragma unroll
-    for (int j = 0; j < NV; ++j)
-        *reinterpret_cast<__nv_bfloat16 *>(img + (c >> 6) * (NV * 128) + sw128(j, (c & 63) >> 3) + (c & 7) * 2) =
-            __float2bfloat16_rn(vals[j]);
-}
-
-template <int NV>
-__global__ void __launch_bounds__(128, 1) chunk_state_kernel(StateArgs p) {
-    using Cfg = StateCfg<NV>;
+__global__ void __launch_bounds__(ST_THREADS, 1)
+chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = align1024(smraw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int slice = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int j0 = slice * NV;
+    const int q4 = warp & 3, hf = (warp >> 2) & 1;  // TMEM lane quarter, column half (warps 0-7)
+    const int h = blockIdx.x, b = blockIdx.y;
     const int bh = b * p.H + h;
-    uint64_t *full = reinterpret_cast<uint64_t *>(sm + Cfg::B_BAR);
-    uint64_t *bar_po = full + 2;
-    uint64_t *bar_so = full + 3;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + Cfg::B_BAR + 32);
-    uint8_t *st_img = sm + Cfg::B_ST;
-    uint8_t *vt_img = sm + Cfg::B_VT;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ST_BAR);
+    uint64_t *full = bars;           // [2] record stage landed
+    uint64_t *bar_p = bars + 2;      // PO group done
+    uint64_t *bar_s = bars + 3;      // S^T += V'^T K~ done (and every earlier group)
+    uint64_t *bar_o = bars + 4;      // PO += V'^T M^T done
+    uint64_t *bar_t = bars + 5;      // transposition of O done
+    uint64_t *bar_simg = bars + 6;   // bf16 copy of S^T written (8 warps)
+    uint64_t *bar_vimg = bars + 7;   // bf16 copy of V'^T written (8 warps)
+    uint64_t *bar_ot = bars + 8;     // O^T image written (8 warps)
+    uint64_t *bar_sig = bars + 9;    // sigmoid tile landed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
+    float *sgam = reinterpret_cast<float *>(sm + ST_GAM);
+    float *red = reinterpret_cast<float *>(sm + ST_RED);
     const uint8_t *rec0 = p.ws + (size_t)bh * p.Nc * REC_BYTES;
-    __shared__ int s_fail;
-
-    auto issue_chunk = [&](int n, int stg) {
-        uint8_t *dst = sm + stg * Cfg::STAGE;
-        const uint8_t *src = rec0 + (size_t)n * REC_BYTES;
-        mbar_arrive_expect_tx(&full[stg], Cfg::EXPECT);
-        bulk_load(dst, src, REC_IMG, &full[stg]);
-        bulk_load(dst + Cfg::S_U, src + REC_U + slice * Cfg::U_BYTES, Cfg::U_BYTES, &full[stg]);
-        bulk_load(dst + Cfg::S_GAM, src + REC_GAM, 512, &full[stg]);
-    };
+    __shared__ volatile int s_fail;
 
     if (tid == 0) {
         s_fail = 0;
-        mbar_init(&full[0], 1);
-        mbar_init(&full[1], 1);
-        mbar_init(bar_po, 1);
-        mbar_init(bar_so, 1);
+        for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
+        mbar_init(bar_simg, 8);
+        mbar_init(bar_vimg, 8);
+        mbar_init(bar_ot, 8);
+        mbar_init(bar_sig, 1);
         fence_barrier_init();
-        for (int n = 0; n < 2 && n < p.Nc; ++n) issue_chunk(n, n);
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, Cfg::TCOLS);
+        tmem_alloc(tmem_slot, ST_TCOLS);
         tmem_relinquish();
     }
+    for (int e = tid; e < 128 * 8; e += ST_THREADS) {  // [I_64; I_64]
+        const int row = e >> 3, ch = e & 7;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (((row & 63) >> 3) == ch) reinterpret_cast<uint16_t *>(&v)[row & 7] = 0x3F80;  // bf16 1.0
+        *reinterpret_cast<uint4 *>(sm + ST_ID + sw128(row, ch)) = v;
+    }
+    fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-    const uint32_t S_COL = 0, P_COL = NV, O_COL0 = 2 * NV;
-    const int c = tid;  // state row (key channel) owned by this thread
-
-    // ---------------- initial state -> TMEM accumulator
-    {
-        uint32_t su[NV];
-        if (p.S0) {
-            const float4 *src = reinterpret_cast<const float4 *>(p.S0 + ((size_t)bh * DD + c) * DD + j0);
-#pragma unroll
-            for (int k = 0; k < NV / 4; ++k) {
-                const float4 x = src[k];
-                su[4 * k] = __float_as_uint(x.x); su[4 * k + 1] = __float_as_uint(x.y);
-                su[4 * k + 2] = __float_as_uint(x.z); su[4 * k + 3] = __float_as_uint(x.w);
-            }
-        } else {
-#pragma unroll
-            for (int j = 0; j < NV; ++j) su[j] = 0u;
-        }
-        tmem_st_cols<NV>(tmem + lane_base + S_COL, su);
-        tmem_wait_st();
-    }
-    tc_fence_before();
-    __syncthreads();
-
-    constexpr uint32_t id_p = idesc_f16(64, NV, 0, 0);
-    constexpr uint32_t id_o = idesc_f16(64, NV, 1, 0);
-    constexpr uint32_t id_s = idesc_f16(128, NV, 1, 0);
-    const uint64_t d_st = smem_desc(smem_u32(st_img), 16, 1024, LAYOUT_SW128);
-    const uint64_t d_vt = smem_desc(smem_u32(vt_img), 16, 1024, LAYOUT_SW128);
-    const uint64_t d_k16 = smem_desc(smem_u32(sm), 16, 1024, LAYOUT_SW128);     // K-major images
-    const uint64_t d_mn = smem_desc(smem_u32(sm), 8192, 1024, LAYOUT_SW128);    // MN-major images
-
-    // O of chunk m (TMEM buffer m & 1) -> o~ rows of the chunk (this thread's token row)
-    auto store_o = [&](int m) {
-        uint32_t ov[NV];
-        tmem_ld_cols<NV>(tmem + lane_base + O_COL0 + (m & 1) * NV, ov);
-        tmem_wait_ld();
-        const int r = 16 * warp + lane;
-        const int t = m * CH + r;
-        if (lane < 16 && t < p.S) {
-            __nv_bfloat16 *dst = p.o + (((size_t)b * p.S + t) * p.H + h) * DD + j0;
-#pragma unroll
-            for (int k = 0; k < NV / 8; ++k) {
-                float f[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(ov[8 * k + e]);
-                reinterpret_cast<uint4 *>(dst)[k] = pack8(f);
-            }
-        }
-    };
-
     bool ok = true;
-    for (int n = 0; n < p.Nc; ++n) {
-        const int stg = n & 1;
-        uint8_t *sg = sm + stg * Cfg::STAGE;
-        const uint32_t sgo = stg * Cfg::STAGE;
-        const uint32_t ocol = O_COL0 + (n & 1) * NV;
-        // ---------- this chunk's record; S_n -> bf16 operand; S <- Diag(e^{G_C}) S_n in TMEM
-        if (!mbar_wait(&full[stg], (n >> 1) & 1)) s_fail = 1;
-        {
-            uint32_t sv[NV];
-            tmem_ld_cols<NV>(tmem + lane_base + S_COL, sv);
-            tmem_wait_ld();
-            float sf[NV];
+    int issued = 0, landed = 0;  // records requested / seen complete (MMA warp)
+
+    if (warp == 8) {
+        // ======================================== MMA and copy issue (one thread)
+        if (lane == 0) {
+            constexpr uint32_t id_kk = idesc_f16(128, 128, 0, 0);  // A, B K-major (A may be in TMEM)
+            constexpr uint32_t id_s = idesc_f16(128, 128, 0, 1);   // B MN-major
+            constexpr uint32_t id_o = idesc_f16(128, 64, 0, 1);    // B MN-major
+            const uint64_t d_k = smem_desc(smem_u32(sm), 16, 1024, LAYOUT_SW128);     // K-major images
+            const uint64_t d_mn = smem_desc(smem_u32(sm), 8192, 1024, LAYOUT_SW128);  // K~ and M^T images
+            auto issue_record = [&](int n) {
+                const int stg = n & 1;
+                mbar_arrive_expect_tx(&full[stg], ST_STAGE + 512);
+                const uint8_t *src = rec0 + (size_t)n * REC_BYTES;
+                bulk_load(sm + stg * ST_STAGE, src, ST_STAGE, &full[stg]);
+                bulk_load(sgam + stg * 128, src + REC_GAM, 512, &full[stg]);
+                ++issued;
+            };
+            // O of chunk m back to token rows: PO[m & 1][r, j] = sum_k [I; I][r, k] O^T[j, k]
+            auto transpose_o = [&](int m) -> bool {
+                if (!mbar_wait(bar_ot, m & 1)) return false;
+                tc_fence_after();
+                const uint32_t d = tmem + T_PO + (uint32_t)(m & 1) * 128;
 #pragma unroll
-            for (int j = 0; j < NV; ++j) sf[j] = __uint_as_float(sv[j]);
-            write_st_row<NV>(st_img, c, sf);
-            const float gam = reinterpret_cast<const float *>(sg + Cfg::S_GAM)[c];
+                for (int s4 = 0; s4 < 4; ++s4)
+                    mma_f16_ss(d, dadd(d_k, ST_ID + s4 * 32), dadd(d_k, ST_OT + s4 * 32), id_kk, s4 > 0);
+                mma_commit(bar_t);
+                return true;
+            };
+            for (int n = 0; n < 2 && n < p.Nc; ++n) issue_record(n);
+            int n = 0;
+            for (; n < p.Nc; ++n) {
+                if (s_fail) { ok = false; break; }
+                const uint32_t sgo = (n & 1) * ST_STAGE;
+                const uint32_t po = tmem + T_PO + (uint32_t)(n & 1) * 128;
+                if (!mbar_wait(&full[n & 1], (n >> 1) & 1)) { ok = false; break; }
+                landed = n + 1;
+                // PO = S_n^T [-W; Q e^G]^T
+                if (!mbar_wait(bar_simg, n & 1)) { ok = false; break; }
+                tc_fence_after();
 #pragma unroll
-            for (int j = 0; j < NV; ++j) sv[j] = __float_as_uint(sf[j] * gam);
-            tmem_st_cols<NV>(tmem + lane_base + S_COL, sv);
+                for (int s8 = 0; s8 < 8; ++s8) {
+                    const uint32_t ko = s8 >> 2, kb = (s8 & 3) * 32;
+                    mma_f16_ts(po, tmem + T_S16 + 8 * s8, dadd(d_k, sgo + REC_WQ + ko * 16384 + kb), id_kk, s8 > 0);
+                }
+                mma_commit(bar_p);
+                // record n - 1 is consumed once its last group is done: refill its stage
+                if (n >= 1 && n + 1 < p.Nc) {
+                    if (!mbar_wait(bar_o, (n - 1) & 1)) { ok = false; break; }
+                    issue_record(n + 1);
+                }
+                if (n >= 1 && !transpose_o(n - 1)) { ok = false; break; }
+                // S^T += V'^T K~, then PO[:, 64:] += V'^T M^T
+                if (!mbar_wait(bar_vimg, n & 1)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int s4 = 0; s4 < 4; ++s4)
+                    mma_f16_ts(tmem + T_S32, tmem + T_V16 + 8 * s4, dadd(d_mn, sgo + REC_KT + s4 * 2048), id_s, 1);
+                mma_commit(bar_s);
+#pragma unroll
+                for (int s4 = 0; s4 < 4; ++s4)
+                    mma_f16_ts(po + 64, tmem + T_V16 + 8 * s4, dadd(d_mn, sgo + REC_MT + s4 * 2048), id_o, 1);
+                mma_commit(bar_o);
+            }
+            if (ok && p.Nc > 0 && !transpose_o(p.Nc - 1)) ok = false;
+            if (!ok) s_fail = 1;
+        }
+    } else {
+        // ======================================== register work (warps 0-7)
+        const uint32_t lrow = (uint32_t)(32 * q4) << 16;
+        const int j = 32 * q4 + lane;  // value column (TMEM lane) of this thread
+        {   // initial state -> TMEM (S^T[j, c] = S0[c, j]: a warp reads 128 contiguous bytes per c)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t su[32];
+                if (p.S0) {
+                    const float *src = p.S0 + (size_t)bh * DD * DD + (size_t)(64 * hf + 32 * hh) * DD + j;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) su[e] = __float_as_uint(src[(size_t)e * DD]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) su[e] = 0u;
+                }
+                tmem_st_32x32b_x32(tmem + lrow + T_S32 + 64 * hf + 32 * hh, su);
+            }
             tmem_wait_st();
         }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (s_fail) { ok = false; break; }
-        // ---------- P = W S and O = (Q e^G) S
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int s = 0; s < 8; ++s) {
-                const uint32_t ko = s >> 2, kb = (s & 3) * 32;
-                const uint64_t bd = dadd(d_st, ko * (NV * 128) + kb);
-                mma_f16_ss(tmem + P_COL, dadd(d_k16, sgo + REC_W + ko * 8192 + kb), bd, id_p, s > 0);
-                mma_f16_ss(tmem + ocol, dadd(d_k16, sgo + REC_QG + ko * 8192 + kb), bd, id_p, s > 0);
+        auto load_sig = [&](int m) {  // sigmoid tile of chunk m -> shared memory (thread 0)
+            if (tid == 0 && p.sig && m < p.Nc) {
+                mbar_arrive_expect_tx(bar_sig, SIG_BYTES);
+                bulk_load(sm + ST_SIGT, p.sig + ((size_t)bh * p.Nc + m) * (CH * DD), SIG_BYTES, bar_sig);
             }
-            mma_commit(bar_po);
-        }
-        if (n > 0) store_o(n - 1);  // overlaps the MMAs just issued
-        if (!mbar_wait(bar_po, n & 1)) s_fail = 1;
-        tc_fence_after();
-        // ---------- V' = U - P (token rows of the M=64 accumulator layout)
-        {
-            uint32_t pv[NV];
-            tmem_ld_cols<NV>(tmem + lane_base + P_COL, pv);
+        };
+        // O^T of chunk m (PO[m & 1][j, 64 + r]) -> bf16 operand image (all warps; after bar_o(m))
+        auto write_ot = [&](int m) {
+            uint32_t ov[32];
+            tmem_ld_32x32b_x32(tmem + lrow + T_PO + (uint32_t)(m & 1) * 128 + 64 + 32 * hf, ov);
             tmem_wait_ld();
-            if (lane < 16) {
-                const int r = 16 * warp + lane;
-                const __nv_bfloat16 *u = reinterpret_cast<const __nv_bfloat16 *>(sg + Cfg::S_U) + r * NV;
 #pragma unroll
-                for (int j = 0; j < NV; ++j) {
-                    const float vp = __bfloat162float(u[j]) - __uint_as_float(pv[j]);
-                    *reinterpret_cast<__nv_bfloat16 *>(vt_img + sw128(j, r >> 3) + (r & 7) * 2) =
-                        __float2bfloat16_rn(vp);
+            for (int k = 0; k < 4; ++k) {
+                uint4 u;
+                u.x = pack_bf16x2(__uint_as_float(ov[8 * k]), __uint_as_float(ov[8 * k + 1]));
+                u.y = pack_bf16x2(__uint_as_float(ov[8 * k + 2]), __uint_as_float(ov[8 * k + 3]));
+                u.z = pack_bf16x2(__uint_as_float(ov[8 * k + 4]), __uint_as_float(ov[8 * k + 5]));
+                u.w = pack_bf16x2(__uint_as_float(ov[8 * k + 6]), __uint_as_float(ov[8 * k + 7]));
+                *reinterpret_cast<uint4 *>(sm + ST_OT + sw128(j, 4 * hf + k)) = u;
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_ot);
+        };
+        // token rows of chunk m (PO[m & 1][r, j], lane r and r + 64) -> normalised, gated output tile;
+        // each warp takes rows 32 (q4 & 1) .. +32 and value columns 32 cq .. +32
+        auto store_o = [&](int m) -> bool {
+            const int r = 32 * (q4 & 1) + lane;
+            const int cq = (q4 >> 1) + 2 * hf;
+            const uint32_t ocol = tmem + lrow + T_PO + (uint32_t)(m & 1) * 128 + 32 * cq;
+            if (!mbar_wait(bar_t, m & 1)) return false;
+            tc_fence_after();
+            bool okw = true;
+            float inv = 1.f;
+            if (p.sig) {
+                uint32_t ov[32];
+                tmem_ld_32x32b_x32(ocol, ov);
+                tmem_wait_ld();
+                float ss = 0.f;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) ss += __uint_as_float(ov[e]) * __uint_as_float(ov[e]);
+                red[r * 4 + cq] = ss;
+            }
+            if (tid == 0) bulk_wait_read_all();  // the previous tile's store has left shared memory
+            named_sync(1, 256);
+            if (p.sig) {
+                const float4 rr = *reinterpret_cast<const float4 *>(red + r * 4);
+                inv = rsqrtf(((rr.x + rr.y) + (rr.z + rr.w)) * (1.0f / 128.0f) + p.eps);
+                okw = mbar_wait(bar_sig, m & 1);
+            }
+            {
+                uint32_t ov[32];
+                tmem_ld_32x32b_x32(ocol, ov);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint32_t off = (cq >> 1) * 8192 + sw128(r, 4 * (cq & 1) + k);
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(ov[8 * k + e]);
+                    if (p.sig) {
+                        const uint4 g8 = *reinterpret_cast<const uint4 *>(sm + ST_SIGT + off);
+                        const __half2 *gh = reinterpret_cast<const __half2 *>(&g8);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 g = __half22float2(gh[e]);
+                            f[2 * e] *= inv * g.x;
+                            f[2 * e + 1] *= inv * g.y;
+                        }
+                    }
+                    *reinterpret_cast<uint4 *>(sm + ST_OIMG + off) = pack8(f);
                 }
             }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (s_fail) { ok = false; break; }
-        // ---------- O += M V' and S += (K e^{G_C - G})^T V'
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int s = 0; s < 4; ++s) {
-                const uint64_t bd = dadd(d_vt, s * 32);
-                mma_f16_ss(tmem + ocol, dadd(d_mn, sgo + REC_MT + s * 2048), bd, id_o, 1);
-                mma_f16_ss(tmem + S_COL, dadd(d_mn, sgo + REC_KT + s * 2048), bd, id_s, 1);
+            fence_proxy_async_smem();
+            named_sync(1, 256);
+            if (tid == 0) {  // rows past the end of the sequence are clipped by the tensor map
+                tma_store_4d(&tmo, sm + ST_OIMG, 0, h, m * CH, b);
+                tma_store_4d(&tmo, sm + ST_OIMG + 8192, 64, h, m * CH, b);
+                bulk_commit();
             }
-            mma_commit(bar_so);
-        }
-        if (!mbar_wait(bar_so, n & 1)) s_fail = 1;
-        tc_fence_after();
-        __syncthreads();
-        if (s_fail) { ok = false; break; }
-        if (tid == 0 && n + 2 < p.Nc) issue_chunk(n + 2, stg);
-    }
-    if (ok && p.Nc > 0) store_o(p.Nc - 1);
+            load_sig(m + 1);  // every reader is past the barrier above
+            return okw;
+        };
+        load_sig(0);
 
-    if (ok) {
-        if (p.Sf) {
-            uint32_t sv[NV];
-            tmem_ld_cols<NV>(tmem + lane_base + S_COL, sv);
-            tmem_wait_ld();
-            float4 *dst = reinterpret_cast<float4 *>(p.Sf + ((size_t)bh * DD + c) * DD + j0);
+        for (int n = 0; n < p.Nc; ++n) {
+            if (s_fail) { ok = false; break; }
+            const uint32_t po = tmem + lrow + T_PO + (uint32_t)(n & 1) * 128;
+            // ---------- S_n^T (after the previous chunk's update) -> bf16 copy; S^T <- S^T Diag(e^{G_C})
+            if (n >= 1 && !mbar_wait(bar_s, (n - 1) & 1)) { ok = false; break; }
+            if (!mbar_wait(&full[n & 1], (n >> 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+            {
+                const float4 *g4 = reinterpret_cast<const float4 *>(sgam + (n & 1) * 128 + 64 * hf);
 #pragma unroll
-            for (int k = 0; k < NV / 4; ++k)
-                dst[k] = make_float4(__uint_as_float(sv[4 * k]), __uint_as_float(sv[4 * k + 1]),
-                                     __uint_as_float(sv[4 * k + 2]), __uint_as_float(sv[4 * k + 3]));
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t sv[32], pk[16];
+                    tmem_ld_32x32b_x32(tmem + lrow + T_S32 + 64 * hf + 32 * hh, sv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1]));
+                    tmem_st_32x32b_x16(tmem + lrow + T_S16 + 32 * hf + 16 * hh, pk);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float4 g = g4[8 * hh + e];
+                        sv[4 * e] = __float_as_uint(__uint_as_float(sv[4 * e]) * g.x);
+                        sv[4 * e + 1] = __float_as_uint(__uint_as_float(sv[4 * e + 1]) * g.y);
+                        sv[4 * e + 2] = __float_as_uint(__uint_as_float(sv[4 * e + 2]) * g.z);
+                        sv[4 * e + 3] = __float_as_uint(__uint_as_float(sv[4 * e + 3]) * g.w);
+                    }
+                    tmem_st_32x32b_x32(tmem + lrow + T_S32 + 64 * hf + 32 * hh, sv);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_simg);
+            // ---------- O^T of the previous chunk -> operand image (turned back into rows by the MMA warp)
+            if (n >= 1) {
+                if (!mbar_wait(bar_o, (n - 1) & 1)) { ok = false; break; }
+                tc_fence_after();
+                write_ot(n - 1);
+            }
+            // ---------- V'^T = U^T - (W S_n)^T -> bf16 copy in TMEM
+            {
+                const uint8_t *ut = sm + (n & 1) * ST_STAGE + REC_U;
+                uint4 uu[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) uu[k] = *reinterpret_cast<const uint4 *>(ut + sw128(j, 4 * hf + k));
+                if (!mbar_wait(bar_p, n & 1)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t pv[32], pk[16];
+                tmem_ld_32x32b_x32(po + 32 * hf, pv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    float u[8];
+                    unpack8(uu[k], u);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        pk[4 * k + e] = pack_bf16x2(u[2 * e] + __uint_as_float(pv[8 * k + 2 * e]),
+                                                    u[2 * e + 1] + __uint_as_float(pv[8 * k + 2 * e + 1]));
+                }
+                tmem_st_32x32b_x16(tmem + lrow + T_V16 + 16 * hf, pk);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_vimg);
+            // ---------- the previous chunk's output tile, while this chunk's state update runs
+            if (n >= 1 && !store_o(n - 1)) { ok = false; break; }
         }
-    } else if (tid == 0) {
-        report_timeout(p.timeouts, p.dev_status);
-        // let bulk copies already issued land before the CTA exits
-        for (int s = 0; s < 2; ++s) mbar_wait(&full[s], 0, 100000000ull);
+        if (ok && p.Nc > 0) {
+            if (!mbar_wait(bar_s, (p.Nc - 1) & 1) || !mbar_wait(bar_o, (p.Nc - 1) & 1)) ok = false;
+            tc_fence_after();
+            if (ok) write_ot(p.Nc - 1);
+            if (ok && !store_o(p.Nc - 1)) ok = false;
+        }
+        if (ok && p.Sf) {  // (with no chunks TMEM still holds the initial state)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t sv[32];
+                tmem_ld_32x32b_x32(tmem + lrow + T_S32 + 64 * hf + 32 * hh, sv);
+                tmem_wait_ld();
+                float *dst = p.Sf + (size_t)bh * DD * DD + (size_t)(64 * hf + 32 * hh) * DD + j;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) dst[(size_t)e * DD] = __uint_as_float(sv[e]);
+            }
+        }
+        if (!ok) s_fail = 1;
+        if (tid == 0) bulk_wait_all();
     }
+    __syncthreads();
+    if (warp == 8 && lane == 0 && s_fail) {
+        report_timeout(p.timeouts, p.dev_status);
+        // let the bulk copies already issued land before the CTA exits
+        for (int m = landed; m < issued; ++m) mbar_wait(&full[m & 1], (m >> 1) & 1, 100000000ull);
+    }
+    if (tid == 0 && s_fail && p.sig) mbar_wait(bar_sig, 0, 100000000ull), mbar_wait(bar_sig, 1, 100000000ull);
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, Cfg::TCOLS);
+    if (warp == 0) tmem_dealloc(tmem, ST_TCOLS);
 }
 
-template <int NV>
-kda_status_t launch_state(const StateArgs &sa, int B, int H, cudaStream_t st) {
-    using Cfg = StateCfg<NV>;
-    cudaFuncSetAttribute(chunk_state_kernel<NV>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM);
-    chunk_state_kernel<NV><<<dim3(DD / NV, H, B), 128, Cfg::SMEM, st>>>(sa);
+kda_status_t launch_state(const CUtensorMap &tmo, const StateArgs &sa, int B, int H, cudaStream_t st) {
+    cudaFuncSetAttribute(chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
+    chunk_state_kernel<<<dim3(H, B), ST_THREADS, STATE_SMEM, st>>>(tmo, sa);
     return check_launch("chunk_state_kernel");
 }
 
@@ -881,12 +1051,6 @@ kda_status_t make_tmap_tokens(CUtensorMap *m, const void *base, int H, int64_t S
                         CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-int pick_nv(int64_t BH) {
-    if (BH >= 148) return 64;
-    if (BH >= 74) return 32;
-    return 16;
-}
-
 }  // namespace
 
 bool chunk_tc_supported(const kda_chunk_args &a, int chunk) {
@@ -896,24 +1060,30 @@ bool chunk_tc_supported(const kda_chunk_args &a, int chunk) {
 
 bool chunk_tc_aligned(const kda_chunk_args &a) {
     auto al = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
-    bool okp = al(a.q) && al(a.k) && al(a.v) && al(a.o) && al(a.initial_state) && al(a.final_state);
+    bool okp = al(a.q) && al(a.k) && al(a.v) && al(a.o) && al(a.initial_state) && al(a.final_state) &&
+               al(a.gate_logits);
     if (!a.log_decay) okp = okp && al(a.z);
     return okp;
 }
 
 size_t chunk_tc_workspace(const kda_chunk_args &a) {
     const int64_t Nc = (a.S + CH - 1) / CH;
-    return (size_t)a.B * a.H * Nc * REC_BYTES;
+    return (size_t)a.B * a.H * Nc * (REC_BYTES + SIG_BYTES);
 }
 
 kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
     const int64_t Nc = (a.S + CH - 1) / CH;
-    const int nv = pick_nv((int64_t)a.B * a.H);
     unsigned int *timeouts = device_timeout_counter();
+    CUtensorMap to;
+    memset(&to, 0, sizeof(to));  // (no chunks: never read)
+    // sigmoid(gate) per chunk, after the records
+    __half *sig = reinterpret_cast<__half *>((uint8_t *)a.workspace + (size_t)a.B * a.H * Nc * REC_BYTES);
     if (Nc > 0) {
         CUtensorMap tq, tk, tv, tz;
         const uint64_t rs = (uint64_t)DD, ss = (uint64_t)a.H * DD, bs = (uint64_t)a.S * a.H * DD;
         kda_status_t s;
+        s = make_tmap_tokens(&to, a.o, a.H, a.S, a.B, rs, ss, bs);
+        if (s != KDA_OK) return s;
         s = make_tmap_tokens(&tq, a.q, a.H, a.S, a.B, rs, ss, bs);
         if (s != KDA_OK) return s;
         s = make_tmap_tokens(&tk, a.k, a.H, a.S, a.B, rs, ss, bs);
@@ -930,12 +1100,13 @@ kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
         pa.S = (int)a.S;
         pa.H = a.H;
         pa.Nc = (int)Nc;
-        pa.Nv = nv;
         pa.units = Nc * a.H * a.B;
         pa.g_min = a.g_min;
         pa.beta = (const __nv_bfloat16 *)a.beta;
         pa.log_decay = a.log_decay;
         pa.ws = (uint8_t *)a.workspace;
+        pa.gate = (const __nv_bfloat16 *)a.gate_logits;
+        pa.sig = sig;
         pa.timeouts = timeouts;
         pa.dev_status = a.dev_status;
         int dev = 0, sms = 148;
@@ -954,19 +1125,11 @@ kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
     sa.ws = (const uint8_t *)a.workspace;
     sa.S0 = a.initial_state;
     sa.Sf = a.final_state;
-    sa.o = (__nv_bfloat16 *)a.o;
+    sa.sig = a.gate_logits ? sig : nullptr;
+    sa.eps = a.eps;
     sa.timeouts = timeouts;
     sa.dev_status = a.dev_status;
-    kda_status_t s;
-    switch (nv) {
-        case 16: s = launch_state<16>(sa, (int)a.B, a.H, st); break;
-        case 32: s = launch_state<32>(sa, (int)a.B, a.H, st); break;
-        default: s = launch_state<64>(sa, (int)a.B, a.H, st); break;
-    }
-    if (s != KDA_OK) return s;
-    if (a.gate_logits && a.S > 0)
-        return launch_norm_gate(a.o, a.gate_logits, a.B * a.S, a.H, DD, a.eps, a.o, KDA_BF16, st);
-    return KDA_OK;
+    return launch_state(to, sa, (int)a.B, a.H, st);
 }
 
 }  // namespace kda

@@ -11,7 +11,8 @@ from kda_testlib import (assert_bf16_outputs, assert_bf16_state, oracle_layer, r
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
-REC = 74240  # workspace bytes per (b, h, chunk)
+REC = 74240  # workspace record bytes per (b, h, chunk)
+SIG = 16384  # plus the f16 sigmoid of the gate logits per (b, h, chunk)
 
 
 @pytest.fixture(scope="module")
@@ -48,6 +49,17 @@ def _kmajor_image(buf, rows=64):
     return out
 
 
+def _atom_image(buf, rows):
+    """One 128-byte-swizzled atom column [rows][128 B] of bf16 -> (rows, 64)."""
+    u = np.frombuffer(buf, dtype=np.uint16)
+    out = np.zeros((rows, 64))
+    for r in range(rows):
+        for c in range(64):
+            off = r * 128 + (((c // 8) ^ (r % 8)) * 16) + (c % 8) * 2
+            out[r, c] = _bf(u[off // 2:off // 2 + 1])[0]
+    return out
+
+
 def _mt_image(buf):
     u = np.frombuffer(buf, dtype=np.uint16)
     out = np.zeros((64, 64))
@@ -69,14 +81,13 @@ def test_workspace_intermediates_match_chunk_mirror(K):
     inp = ki.make_inputs(w)
     d = upload(inp, w)
     nb = K.chunk_workspace_bytes(1, 100, 2, 128, 128)
-    assert nb == 1 * 2 * 2 * REC
+    assert nb == 1 * 2 * 2 * (REC + SIG)
     ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
     K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=d["z"], engine="tc", workspace=ws)
     torch.cuda.synchronize()
     assert _timeouts(K) == 0
     wsh = ws.cpu().numpy()
     la = oracle.log_decay(inp["z"], w.g_min)
-    nv = 16  # B*H = 2 -> 16-column value slices
     for h in range(2):
         for n in range(2):
             t0, t1 = 64 * n, min(100, 64 * n + 64)
@@ -88,15 +99,12 @@ def test_workspace_intermediates_match_chunk_mirror(K):
             mir = chunk_mirror.matrix_chunk(q, k, v, beta, g, np.zeros((128, 128)))
             G = mir["G"]
             rec = wsh[(h * 2 + n) * REC:(h * 2 + n + 1) * REC]
-            _close(_kmajor_image(rec[0:16384]), q * np.exp(G), f"Qg h{h} n{n}")
-            _close(_kmajor_image(rec[16384:32768]), k * np.exp(G[-1] - G), f"Kt h{h} n{n}")
-            _close(_kmajor_image(rec[32768:49152]), mir["W"], f"W h{h} n{n}")
+            wq = _kmajor_image(rec[0:32768], rows=128)  # stacked [-W; Q e^G]
+            _close(wq[64:], q * np.exp(G), f"Qg h{h} n{n}")
+            _close(-wq[:64], mir["W"], f"W h{h} n{n}")
+            _close(_kmajor_image(rec[32768:49152]), k * np.exp(G[-1] - G), f"Kt h{h} n{n}")
             _close(_mt_image(rec[49152:57344]), mir["M"].T, f"M h{h} n{n}")
-            U = np.zeros((64, 128))
-            uu = _bf(np.frombuffer(rec[57344:73728].tobytes(), dtype=np.uint16))
-            for s in range(128 // nv):
-                U[:, s * nv:(s + 1) * nv] = uu[s * 64 * nv:(s + 1) * 64 * nv].reshape(64, nv)
-            _close(U, mir["U"], f"U h{h} n{n}")
+            _close(_atom_image(rec[57344:73728], 128).T, mir["U"], f"U h{h} n{n}")  # stored as U^T
             gam = np.frombuffer(rec[73728:74240].tobytes(), dtype=np.float32)
             np.testing.assert_allclose(gam, np.exp(G[-1]), rtol=1e-4, atol=1e-30)
 
