@@ -680,10 +680,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
 // Records stream in by bulk copies, two stages deep.
 struct StateArgs {
     int S, H, Nc;
+    int L, G;              // chunks per segment, segments per sequence
     const uint8_t *ws;
-    const __half *sig;  // sigmoid of the output-gate logits per chunk (tile layout), or null: write o~
+    const __half *sig;     // sigmoid of the output-gate logits per chunk (tile layout), or null: write o~
     const float *S0;
     float *Sf;
+    const float *seg_init; // state entering segment g >= 1, [B*H][G][128][128] (after the combine pass)
+    uint8_t *xt;           // map pass: A_g^T as bf16 operand images [B*H][G-1][32 KB]
+    float *yt;             // map pass: Y_g [B*H][G-1][128][128]
     float eps;
     unsigned int *timeouts;
     int *dev_status;
@@ -712,6 +716,10 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// kMap = false: the chain over segment blockIdx.z from its entering state, with outputs.
+// kMap = true:  the map of segment blockIdx.z / 2 over its chunks, S_end = A_g S_start + Y_g:
+//               even z runs from S = I without U (-> A_g), odd z from S = 0 with U (-> Y_g); no outputs.
+template <bool kMap>
 __global__ void __launch_bounds__(ST_THREADS, 1)
 chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
     extern __shared__ uint8_t smraw[];
@@ -720,6 +728,10 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
     const int q4 = warp & 3, hf = (warp >> 2) & 1;  // TMEM lane quarter, column half (warps 0-7)
     const int h = blockIdx.x, b = blockIdx.y;
     const int bh = b * p.H + h;
+    const int g = kMap ? (int)(blockIdx.z >> 1) : (int)blockIdx.z;
+    const bool ident = kMap && (blockIdx.z & 1) == 0;  // map from the identity (no U)
+    const int n0 = g * p.L;
+    const int nc = max(0, min(p.L, p.Nc - n0));  // chunks of this segment
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ST_BAR);
     uint64_t *full = bars;           // [2] record stage landed
     uint64_t *bar_p = bars + 2;      // PO group done
@@ -733,7 +745,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
     float *sgam = reinterpret_cast<float *>(sm + ST_GAM);
     float *red = reinterpret_cast<float *>(sm + ST_RED);
-    const uint8_t *rec0 = p.ws + (size_t)bh * p.Nc * REC_BYTES;
+    const uint8_t *rec0 = p.ws + ((size_t)bh * p.Nc + n0) * REC_BYTES;
     __shared__ volatile int s_fail;
 
     if (tid == 0) {
@@ -790,9 +802,9 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
                 mma_commit(bar_t);
                 return true;
             };
-            for (int n = 0; n < 2 && n < p.Nc; ++n) issue_record(n);
+            for (int n = 0; n < 2 && n < nc; ++n) issue_record(n);
             int n = 0;
-            for (; n < p.Nc; ++n) {
+            for (; n < nc; ++n) {
                 if (s_fail) { ok = false; break; }
                 const uint32_t sgo = (n & 1) * ST_STAGE;
                 const uint32_t po = tmem + T_PO + (uint32_t)(n & 1) * 128;
@@ -808,11 +820,11 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
                 }
                 mma_commit(bar_p);
                 // record n - 1 is consumed once its last group is done: refill its stage
-                if (n >= 1 && n + 1 < p.Nc) {
+                if (n >= 1 && n + 1 < nc) {
                     if (!mbar_wait(bar_o, (n - 1) & 1)) { ok = false; break; }
                     issue_record(n + 1);
                 }
-                if (n >= 1 && !transpose_o(n - 1)) { ok = false; break; }
+                if (!kMap && n >= 1 && !transpose_o(n - 1)) { ok = false; break; }
                 // S^T += V'^T K~, then PO[:, 64:] += V'^T M^T
                 if (!mbar_wait(bar_vimg, n & 1)) { ok = false; break; }
                 tc_fence_after();
@@ -820,24 +832,32 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
                 for (int s4 = 0; s4 < 4; ++s4)
                     mma_f16_ts(tmem + T_S32, tmem + T_V16 + 8 * s4, dadd(d_mn, sgo + REC_KT + s4 * 2048), id_s, 1);
                 mma_commit(bar_s);
+                if (!kMap) {
 #pragma unroll
-                for (int s4 = 0; s4 < 4; ++s4)
-                    mma_f16_ts(po + 64, tmem + T_V16 + 8 * s4, dadd(d_mn, sgo + REC_MT + s4 * 2048), id_o, 1);
+                    for (int s4 = 0; s4 < 4; ++s4)
+                        mma_f16_ts(po + 64, tmem + T_V16 + 8 * s4, dadd(d_mn, sgo + REC_MT + s4 * 2048), id_o, 1);
+                }
                 mma_commit(bar_o);
             }
-            if (ok && p.Nc > 0 && !transpose_o(p.Nc - 1)) ok = false;
+            if (!kMap && ok && nc > 0 && !transpose_o(nc - 1)) ok = false;
             if (!ok) s_fail = 1;
         }
     } else {
         // ======================================== register work (warps 0-7)
         const uint32_t lrow = (uint32_t)(32 * q4) << 16;
         const int j = 32 * q4 + lane;  // value column (TMEM lane) of this thread
-        {   // initial state -> TMEM (S^T[j, c] = S0[c, j]: a warp reads 128 contiguous bytes per c)
+        {   // entering state -> TMEM (S^T[j, c] = S[c, j]: a warp reads 128 contiguous bytes per c)
+            const float *s_in = kMap ? nullptr
+                                     : (g == 0 ? (p.S0 ? p.S0 + (size_t)bh * DD * DD : nullptr)
+                                               : p.seg_init + ((size_t)bh * p.G + g) * DD * DD);
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t su[32];
-                if (p.S0) {
-                    const float *src = p.S0 + (size_t)bh * DD * DD + (size_t)(64 * hf + 32 * hh) * DD + j;
+                if (ident) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) su[e] = (64 * hf + 32 * hh + e == j) ? 0x3F800000u : 0u;
+                } else if (s_in) {
+                    const float *src = s_in + (size_t)(64 * hf + 32 * hh) * DD + j;
 #pragma unroll
                     for (int e = 0; e < 32; ++e) su[e] = __float_as_uint(src[(size_t)e * DD]);
                 } else {
@@ -849,9 +869,9 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
             tmem_wait_st();
         }
         auto load_sig = [&](int m) {  // sigmoid tile of chunk m -> shared memory (thread 0)
-            if (tid == 0 && p.sig && m < p.Nc) {
+            if (!kMap && tid == 0 && p.sig && m < nc) {
                 mbar_arrive_expect_tx(bar_sig, SIG_BYTES);
-                bulk_load(sm + ST_SIGT, p.sig + ((size_t)bh * p.Nc + m) * (CH * DD), SIG_BYTES, bar_sig);
+                bulk_load(sm + ST_SIGT, p.sig + ((size_t)bh * p.Nc + n0 + m) * (CH * DD), SIG_BYTES, bar_sig);
             }
         };
         // O^T of chunk m (PO[m & 1][j, 64 + r]) -> bf16 operand image (all warps; after bar_o(m))
@@ -925,8 +945,8 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
             fence_proxy_async_smem();
             named_sync(1, 256);
             if (tid == 0) {  // rows past the end of the sequence are clipped by the tensor map
-                tma_store_4d(&tmo, sm + ST_OIMG, 0, h, m * CH, b);
-                tma_store_4d(&tmo, sm + ST_OIMG + 8192, 64, h, m * CH, b);
+                tma_store_4d(&tmo, sm + ST_OIMG, 0, h, (n0 + m) * CH, b);
+                tma_store_4d(&tmo, sm + ST_OIMG + 8192, 64, h, (n0 + m) * CH, b);
                 bulk_commit();
             }
             load_sig(m + 1);  // every reader is past the barrier above
@@ -934,7 +954,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
         };
         load_sig(0);
 
-        for (int n = 0; n < p.Nc; ++n) {
+        for (int n = 0; n < nc; ++n) {
             if (s_fail) { ok = false; break; }
             const uint32_t po = tmem + lrow + T_PO + (uint32_t)(n & 1) * 128;
             // ---------- S_n^T (after the previous chunk's update) -> bf16 copy; S^T <- S^T Diag(e^{G_C})
@@ -967,7 +987,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_simg);
             // ---------- O^T of the previous chunk -> operand image (turned back into rows by the MMA warp)
-            if (n >= 1) {
+            if (!kMap && n >= 1) {
                 if (!mbar_wait(bar_o, (n - 1) & 1)) { ok = false; break; }
                 tc_fence_after();
                 write_ot(n - 1);
@@ -989,8 +1009,10 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
                     unpack8(uu[k], u);
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        pk[4 * k + e] = pack_bf16x2(u[2 * e] + __uint_as_float(pv[8 * k + 2 * e]),
-                                                    u[2 * e + 1] + __uint_as_float(pv[8 * k + 2 * e + 1]));
+                        pk[4 * k + e] = ident ? pack_bf16x2(__uint_as_float(pv[8 * k + 2 * e]),
+                                                        __uint_as_float(pv[8 * k + 2 * e + 1]))
+                                          : pack_bf16x2(u[2 * e] + __uint_as_float(pv[8 * k + 2 * e]),
+                                                        u[2 * e + 1] + __uint_as_float(pv[8 * k + 2 * e + 1]));
                 }
                 tmem_st_32x32b_x16(tmem + lrow + T_V16 + 16 * hf, pk);
                 tmem_wait_st();
@@ -999,15 +1021,43 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_vimg);
             // ---------- the previous chunk's output tile, while this chunk's state update runs
-            if (n >= 1 && !store_o(n - 1)) { ok = false; break; }
+            if (!kMap && n >= 1 && !store_o(n - 1)) { ok = false; break; }
         }
-        if (ok && p.Nc > 0) {
-            if (!mbar_wait(bar_s, (p.Nc - 1) & 1) || !mbar_wait(bar_o, (p.Nc - 1) & 1)) ok = false;
+        if (ok && nc > 0) {
+            if (!mbar_wait(bar_s, (nc - 1) & 1) || !mbar_wait(bar_o, (nc - 1) & 1)) ok = false;
             tc_fence_after();
-            if (ok) write_ot(p.Nc - 1);
-            if (ok && !store_o(p.Nc - 1)) ok = false;
+            if (!kMap) {
+                if (ok) write_ot(nc - 1);
+                if (ok && !store_o(nc - 1)) ok = false;
+            }
         }
-        if (ok && p.Sf) {  // (with no chunks TMEM still holds the initial state)
+        if (ok && kMap && !ident) {  // Y_g, laid out like a state
+            float *dst0 = p.yt + ((size_t)bh * (p.G - 1) + g) * DD * DD;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t sv[32];
+                tmem_ld_32x32b_x32(tmem + lrow + T_S32 + 64 * hf + 32 * hh, sv);
+                tmem_wait_ld();
+                float *dst = dst0 + (size_t)(64 * hf + 32 * hh) * DD + j;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) dst[(size_t)e * DD] = __uint_as_float(sv[e]);
+            }
+        } else if (ok && ident) {  // A_g^T as the combine pass's MN-major B operand: image row j = lane j
+            uint8_t *img = p.xt + ((size_t)bh * (p.G - 1) + g) * 32768;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t sv[32];
+                tmem_ld_32x32b_x32(tmem + lrow + T_S32 + 64 * hf + 32 * hh, sv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(sv[8 * k + e]);
+                    *reinterpret_cast<uint4 *>(img + hf * 16384 + sw128(j, 4 * hh + k)) = pack8(f);
+                }
+            }
+        } else if (ok && p.Sf && g == p.G - 1) {  // (with no chunks TMEM still holds the entering state)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t sv[32];
@@ -1027,15 +1077,161 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
         // let the bulk copies already issued land before the CTA exits
         for (int m = landed; m < issued; ++m) mbar_wait(&full[m & 1], (m >> 1) & 1, 100000000ull);
     }
-    if (tid == 0 && s_fail && p.sig) mbar_wait(bar_sig, 0, 100000000ull), mbar_wait(bar_sig, 1, 100000000ull);
+    if (!kMap && tid == 0 && s_fail && p.sig) mbar_wait(bar_sig, 0, 100000000ull), mbar_wait(bar_sig, 1, 100000000ull);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, ST_TCOLS);
 }
 
+// ================================================================ K2c: chunk_combine_kernel
+// The segment maps chained in order, one CTA per (head, batch):
+//   S_{g+1} = A_g S_g + Y_g,   g = 0 .. G-2,
+// with the state transposed in TMEM (lane j): S_{g+1}^T = S_g^T A_g^T + Y_g^T, one M = 128 MMA per
+// segment (A = bf16 copy of S_g^T in TMEM, B = the A_g^T image).  Writes every S_g (g >= 1) for the
+// segment chains.
+struct CombineArgs {
+    int H, G;
+    const float *S0;
+    const uint8_t *xt;
+    const float *yt;
+    float *seg_init;
+    unsigned int *timeouts;
+    int *dev_status;
+};
+
+constexpr size_t COMB_SMEM = 2 * 32768 + 64 + 1024;
+
+__global__ void __launch_bounds__(128, 1) chunk_combine_kernel(CombineArgs p) {
+    extern __shared__ uint8_t smraw[];
+    uint8_t *sm = align1024(smraw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.y * p.H + blockIdx.x;
+    const int j = tid;
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + 65536);  // [2]
+    uint64_t *bar_m = full + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full + 3);
+    const int nseg = p.G - 1;
+    auto issue = [&](int g) {
+        mbar_arrive_expect_tx(&full[g & 1], 32768);
+        bulk_load(sm + (g & 1) * 32768, p.xt + ((size_t)bh * nseg + g) * 32768, 32768, &full[g & 1]);
+    };
+    if (tid == 0) {
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        mbar_init(bar_m, 1);
+        fence_barrier_init();
+        for (int g = 0; g < 2 && g < nseg; ++g) issue(g);
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lrow = (uint32_t)(32 * warp) << 16;
+    constexpr uint32_t C_S32 = 0, C_S16 = 128, C_D = 256;
+    float sv[128];
+    {
+        const float *src = p.S0 ? p.S0 + (size_t)bh * DD * DD + j : nullptr;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) sv[c] = src ? src[(size_t)c * DD] : 0.f;
+    }
+    bool ok = true;
+    int g = 0;
+    for (; g < nseg; ++g) {
+        // bf16 copy of S_g^T (A operand)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(sv[32 * q + 2 * e], sv[32 * q + 2 * e + 1]);
+            tmem_st_32x32b_x16(tmem + lrow + C_S16 + 16 * q, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            ok = mbar_wait(&full[g & 1], (g >> 1) & 1);
+            if (ok) {
+                tc_fence_after();
+                constexpr uint32_t id = idesc_f16(128, 128, 0, 1);
+                const uint64_t d = smem_desc(smem_u32(sm + (g & 1) * 32768), 16384, 1024, LAYOUT_SW128);
+#pragma unroll
+                for (int s8 = 0; s8 < 8; ++s8) mma_f16_ts(tmem + C_D, tmem + C_S16 + 8 * s8, dadd(d, s8 * 2048), id, s8 > 0);
+                mma_commit(bar_m);
+            }
+        }
+        ok = __syncthreads_and(ok) && mbar_wait(bar_m, g & 1);
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
+        tc_fence_after();
+        if (tid == 0 && g + 2 < nseg) issue(g + 2);  // the image just used has been read
+        // S_{g+1}^T = D + Y_g^T (all of Y's column loaded before any store: the two may not be reordered)
+        const float *y = p.yt + ((size_t)bh * nseg + g) * DD * DD + j;
+        float *dst = p.seg_init + ((size_t)bh * p.G + g + 1) * DD * DD + j;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) sv[c] = y[(size_t)c * DD];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            uint32_t dv[32];
+            tmem_ld_32x32b_x32(tmem + lrow + C_D + 32 * q, dv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) sv[32 * q + e] += __uint_as_float(dv[e]);
+        }
+#pragma unroll
+        for (int c = 0; c < 128; ++c) dst[(size_t)c * DD] = sv[c];
+        tc_fence_before();
+        __syncthreads();
+    }
+    if (!ok && tid == 0) {
+        report_timeout(p.timeouts, p.dev_status);
+        for (int m = g; m < nseg && m < g + 2; ++m) mbar_wait(&full[m & 1], (m >> 1) & 1, 100000000ull);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// Segments per sequence: enough that the map pass fills the GPU once (two CTAs per segment
+// map), with at least 4 chunks per segment; 1 when (batch x heads) alone fills it.
+int pick_segments(int64_t BH, int64_t Nc, int sms) {
+    int64_t G = 1 + sms / (2 * BH);
+    if (G > Nc / 4) G = Nc / 4;
+    return (int)(G < 1 ? 1 : G);
+}
+
+int device_sms() {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms;
+}
+
 kda_status_t launch_state(const CUtensorMap &tmo, const StateArgs &sa, int B, int H, cudaStream_t st) {
-    cudaFuncSetAttribute(chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
-    chunk_state_kernel<<<dim3(H, B), ST_THREADS, STATE_SMEM, st>>>(tmo, sa);
+    if (sa.G > 1) {
+        cudaFuncSetAttribute(chunk_state_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
+        chunk_state_kernel<true><<<dim3(H, B, 2 * (sa.G - 1)), ST_THREADS, STATE_SMEM, st>>>(tmo, sa);
+        kda_status_t s = check_launch("chunk_state_kernel (segment maps)");
+        if (s != KDA_OK) return s;
+        CombineArgs ca;
+        ca.H = H;
+        ca.G = sa.G;
+        ca.S0 = sa.S0;
+        ca.xt = sa.xt;
+        ca.yt = sa.yt;
+        ca.seg_init = const_cast<float *>(sa.seg_init);
+        ca.timeouts = sa.timeouts;
+        ca.dev_status = sa.dev_status;
+        cudaFuncSetAttribute(chunk_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)COMB_SMEM);
+        chunk_combine_kernel<<<dim3(H, B), 128, COMB_SMEM, st>>>(ca);
+        s = check_launch("chunk_combine_kernel");
+        if (s != KDA_OK) return s;
+    }
+    cudaFuncSetAttribute(chunk_state_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
+    chunk_state_kernel<false><<<dim3(H, B, sa.G), ST_THREADS, STATE_SMEM, st>>>(tmo, sa);
     return check_launch("chunk_state_kernel");
 }
 
@@ -1066,18 +1262,38 @@ bool chunk_tc_aligned(const kda_chunk_args &a) {
     return okp;
 }
 
-size_t chunk_tc_workspace(const kda_chunk_args &a) {
-    const int64_t Nc = (a.S + CH - 1) / CH;
-    return (size_t)a.B * a.H * Nc * (REC_BYTES + SIG_BYTES);
+// Workspace: records and gate tiles per chunk, then (with several segments) the segment maps
+// A_g^T (bf16 images) and Y_g, and the segments' entering states.
+struct TcLayout {
+    int G, L;
+    size_t sig, xt, yt, seg, total;
+};
+
+TcLayout tc_layout(const kda_chunk_args &a) {
+    TcLayout t;
+    const int64_t Nc = (a.S + CH - 1) / CH, BH = (int64_t)a.B * a.H;
+    t.G = pick_segments(BH, Nc, device_sms());
+    t.L = (int)((Nc + t.G - 1) / t.G);
+    if (Nc > 0) t.G = (int)((Nc + t.L - 1) / t.L);  // no empty segment
+    t.sig = (size_t)BH * Nc * REC_BYTES;
+    t.xt = t.sig + (size_t)BH * Nc * SIG_BYTES;
+    const size_t nmap = t.G > 1 ? (size_t)BH * (t.G - 1) : 0;
+    t.yt = t.xt + nmap * 32768;
+    t.seg = t.yt + nmap * DD * DD * 4;
+    t.total = t.seg + (t.G > 1 ? (size_t)BH * t.G * DD * DD * 4 : 0);
+    return t;
 }
+
+size_t chunk_tc_workspace(const kda_chunk_args &a) { return tc_layout(a).total; }
 
 kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
     const int64_t Nc = (a.S + CH - 1) / CH;
     unsigned int *timeouts = device_timeout_counter();
     CUtensorMap to;
     memset(&to, 0, sizeof(to));  // (no chunks: never read)
-    // sigmoid(gate) per chunk, after the records
-    __half *sig = reinterpret_cast<__half *>((uint8_t *)a.workspace + (size_t)a.B * a.H * Nc * REC_BYTES);
+    const TcLayout lay = tc_layout(a);
+    uint8_t *ws = (uint8_t *)a.workspace;
+    __half *sig = reinterpret_cast<__half *>(ws + lay.sig);
     if (Nc > 0) {
         CUtensorMap tq, tk, tv, tz;
         const uint64_t rs = (uint64_t)DD, ss = (uint64_t)a.H * DD, bs = (uint64_t)a.S * a.H * DD;
@@ -1109,9 +1325,7 @@ kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
         pa.sig = sig;
         pa.timeouts = timeouts;
         pa.dev_status = a.dev_status;
-        int dev = 0, sms = 148;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int sms = device_sms();
         const int64_t grid = pa.units < sms ? pa.units : sms;
         cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PREP_SMEM);
         chunk_prep_kernel<<<(unsigned)grid, 256, PREP_SMEM, st>>>(tq, tk, tv, tz, pa);
@@ -1126,6 +1340,11 @@ kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
     sa.S0 = a.initial_state;
     sa.Sf = a.final_state;
     sa.sig = a.gate_logits ? sig : nullptr;
+    sa.L = Nc > 0 ? lay.L : 1;
+    sa.G = Nc > 0 ? lay.G : 1;
+    sa.xt = ws + lay.xt;
+    sa.yt = reinterpret_cast<float *>(ws + lay.yt);
+    sa.seg_init = reinterpret_cast<const float *>(ws + lay.seg);
     sa.eps = a.eps;
     sa.timeouts = timeouts;
     sa.dev_status = a.dev_status;

@@ -124,6 +124,26 @@ def test_tc_core_matches_oracle(K, B, S, H):
     assert_bf16_state(to_np(sf), s_ref, "final_state")
 
 
+@pytest.mark.parametrize("B,S,H,g_min", [(1, 2560, 2, -5.0), (2, 1999, 1, -5.0), (1, 2048, 1, -0.5)])
+def test_tc_segmented_state_pass(K, B, S, H, g_min):
+    """Sequences long enough for the state pass to be split into segments (each segment's affine
+    map computed in parallel, the maps chained by the combine pass, the segments then run from
+    their entering states); g_min = -0.5 keeps a long memory across segment boundaries."""
+    w = small("seg", B, S, H, 128, 128, 16, "bf16", seed=S + 7 * H, s0_std=0.02, g_min=g_min)
+    inp = ki.make_inputs(w)
+    d = upload(inp, w)
+    nc = (S + 63) // 64
+    assert K.chunk_workspace_bytes(B, S, H, 128, 128) > B * H * nc * (REC + SIG)  # segments in use
+    o, sf = K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=d["z"], g_min=g_min, initial_state=d["S0"],
+                        engine="tc")
+    torch.cuda.synchronize()
+    assert _timeouts(K) == 0
+    o_ref, s_ref = oracle.recurrence(inp["q"], inp["k"], inp["v"], inp["beta"], z=inp["z"], g_min=g_min,
+                                     initial_state=inp["S0"])
+    assert_bf16_outputs(to_np(o), o_ref, "o~")
+    assert_bf16_state(to_np(sf), s_ref, "final_state")
+
+
 def test_tc_matches_simt_engine(K):
     w = small("ts", 2, 333, 4, 128, 128, 16, "bf16", seed=5, s0_std=0.02, z_std=2.0)
     inp = ki.make_inputs(w)
