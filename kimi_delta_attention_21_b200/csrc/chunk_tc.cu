@@ -133,18 +133,19 @@ __device__ __forceinline__ void report_timeout(unsigned int *timeouts, int *dev_
 
 // ================================================================ K2a: chunk_prep_kernel
 // Persistent: one CTA per SM walks (chunk, head, batch) units.  The next unit's
-// q, k and z tiles are loaded by TMA as soon as this unit's copies of them are
-// dead (after the A/M MMAs), v after the W/U MMA, and the workspace bulk
-// stores drain while the next unit is computed.
+// q and k tiles are loaded by TMA as soon as this unit's copies of them are
+// dead (after the A/M MMAs), z and v after the W/U MMAs, and the workspace
+// bulk stores drain while the next unit is computed.
 // Shared-memory map (bytes from a 1024-aligned base).
 constexpr uint32_t P_QI = 0;         // q image; becomes Q e^G (stored as soon as P2 ends)
 constexpr uint32_t P_KI = 16384;     // k image; becomes K e^{G_C - G}
-constexpr uint32_t P_VI = 32768;     // v image; becomes beta V (MN-major B operand of the W|U MMA)
-constexpr uint32_t P_ZI = 49152;     // z image; becomes lo part of the q row operand
-constexpr uint32_t P_KC = 65536;     // column operands, 4 versions packed [2 atoms][160 rows][128 B]; later W, U
-constexpr uint32_t P_KR = 106496;    // row operand from k [2 atoms][64 rows][128 B]; later the M^T image
-constexpr uint32_t P_QR = 122880;    // row operand from q; later the T image
-constexpr uint32_t P_RH = 139264;    // beta K e^G image (MN-major B) + lo part of the diagonal column operand
+constexpr uint32_t P_VI = 32768;     // v image; becomes beta V (operand of the W and U^T MMAs)
+constexpr uint32_t P_ZI = 49152;     // z image; becomes beta K e^G (MN-major B operand of the W MMA)
+constexpr uint32_t P_A = 65536;      // A operand of the A/M MMAs [2 atoms][224 rows][128 B]: the column operand
+                                     // in its 4 block versions (rows 0-159) and the low part of the diagonal
+                                     // one (rows 160-223); later -W, U^T and the M^T image
+constexpr uint32_t P_B = 122880;     // B operand [2 atoms][192 rows][128 B]: row operands from k, q and the low
+                                     // part of the q one; later the T image and the diagonal residues
 constexpr uint32_t P_SG = 172032;    // G fp32 [64][132]; later A [64][65] and T [64][68] fp32
 constexpr uint32_t P_TAB = 206080;   // per-channel block constants [26][128] fp32
 constexpr uint32_t P_XS = 219392;    // scratch for the blocked inverse [3][256] fp32
@@ -153,12 +154,14 @@ constexpr uint32_t P_GAM = 222720;   // e^{G_C} [128] fp32
 constexpr uint32_t P_BAR = 223232;   // 3 mbarriers + TMEM slot
 constexpr uint32_t P_END = 223312;
 constexpr size_t PREP_SMEM = P_END + 1024;
-constexpr uint32_t P_MT = P_KR, P_TI = P_QR;
-constexpr uint32_t P_KLO = P_RH + 16384;
+constexpr uint32_t P_RH = P_ZI;
+constexpr uint32_t P_WI = P_A, P_UI = P_A + 16384, P_MT = P_A + 32768;
+constexpr uint32_t P_TI = P_B, P_LOHI = P_B + 8192;  // LOHI: [64][16] fp32
 constexpr uint32_t P_SA = P_SG, P_ST = P_SG + 16640;
-constexpr uint32_t P_WI = P_KC, P_UI = P_KC + 16384;
 constexpr int SG_LD = 132, SA_LD = 65, ST_LD = 68;
-constexpr uint32_t KC_ATOM = 160 * 128;  // bytes per atom column of the packed column operand
+constexpr uint32_t A_ATOM = 224 * 128;  // bytes per atom column of the A/M MMAs' A operand
+constexpr uint32_t B_ATOM = 192 * 128;  // ... and of their B operand
+constexpr uint32_t A_KLO = 160;         // first row of the low part of the diagonal column operand
 
 // table rows: b_R (0-3), F_R = e^{b_{R-1} - m_R} (4-7), E_R = e^{b_{R-1}} (8-11),
 // D_R = e^{b_3 - b_R} (12-15), C_{V,R} = e^{m_V - b_R} for R <= V (16 + V(V+1)/2 + R)
@@ -200,20 +203,49 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         h = (int)(bh % p.H);
         b = (int)(bh / p.H);
     };
-    auto load_qkz = [&](int64_t u) {  // arms bar_in for the whole unit
+    auto load_qk = [&](int64_t u) {  // arms bar_in for the whole unit
         int n, h, b;
         unit_coords(u, n, h, b);
         mbar_arrive_expect_tx(bar_in, in_bytes);
         for (int a = 0; a < 2; ++a) {
             tma_load_4d(sm + P_QI + a * 8192, &tq, bar_in, 64 * a, h, n * CH, b);
             tma_load_4d(sm + P_KI + a * 8192, &tk, bar_in, 64 * a, h, n * CH, b);
-            if (!p.log_decay) tma_load_4d(sm + P_ZI + a * 8192, &tz, bar_in, 64 * a, h, n * CH, b);
         }
     };
-    auto load_v = [&](int64_t u) {
+    auto load_zv = [&](int64_t u) {
         int n, h, b;
         unit_coords(u, n, h, b);
-        for (int a = 0; a < 2; ++a) tma_load_4d(sm + P_VI + a * 8192, &tv, bar_in, 64 * a, h, n * CH, b);
+        for (int a = 0; a < 2; ++a) {
+            if (!p.log_decay) tma_load_4d(sm + P_ZI + a * 8192, &tz, bar_in, 64 * a, h, n * CH, b);
+            tma_load_4d(sm + P_VI + a * 8192, &tv, bar_in, 64 * a, h, n * CH, b);
+        }
+    };
+
+    // sigmoid of the output-gate logits (full fp32, stored as f16) for the state kernel's output stage,
+    // in its tile layout [2 atoms (j / 64)][64 rows r][128 B], 128-byte swizzled: one row x 32 value
+    // columns per thread
+    auto gate_sigmoid = [&](int n, int h, int b, int t0, int len) {
+        const int row = tid >> 2, c0 = 32 * (tid & 3);
+        if (!p.gate || row >= len) return;
+        const uint4 *src =
+            reinterpret_cast<const uint4 *>(p.gate + (((int64_t)b * p.S + t0 + row) * p.H + h) * DD + c0);
+        uint8_t *dst = reinterpret_cast<uint8_t *>(p.sig + ((size_t)(b * p.H + h) * p.Nc + n) * (CH * DD)) +
+                       (c0 >> 6) * 8192;
+        uint4 gv[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) gv[k] = src[k];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            float g[8];
+            unpack8(gv[k], g);
+            uint4 o;
+            __half2 *oh = reinterpret_cast<__half2 *>(&o);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                oh[e] = __floats2half2_rn(__fdividef(1.0f, 1.0f + __expf(-g[2 * e])),
+                                          __fdividef(1.0f, 1.0f + __expf(-g[2 * e + 1])));
+            *reinterpret_cast<uint4 *>(dst + sw128(row, (c0 & 63) / 8 + k)) = o;
+        }
     };
 
     if (tid == 0) {
@@ -222,12 +254,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         mbar_init(bar_wu, 1);
         fence_barrier_init();
         if ((int64_t)blockIdx.x < p.units) {
-            load_qkz(blockIdx.x);
-            load_v(blockIdx.x);
+            load_qk(blockIdx.x);
+            load_zv(blockIdx.x);
         }
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -319,6 +351,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 const int j = grp + 4 * mi;
                 const int atom = j >> 3, jj = j & 7, c0 = 8 * j;
                 const uint32_t img = atom * 8192 + sw128(r, jj);
+                const uint32_t bimg = P_B + atom * B_ATOM, aimg = P_A + atom * A_ATOM;
                 float qv[8], kv[8], vv[8], G[8], bR[8], bRm1[8], F[8], E[8], Dd[8];
                 unpack8(*reinterpret_cast<const uint4 *>(sm + P_QI + img), qv);
                 unpack8(*reinterpret_cast<const uint4 *>(sm + P_KI + img), kv);
@@ -342,17 +375,17 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 }
 #pragma unroll
                 for (int e = 0; e < 8; ++e) t[e] = kv[e] * e1[e] * F[e];
-                *reinterpret_cast<uint4 *>(sm + P_KR + img) = pack8(t);
+                *reinterpret_cast<uint4 *>(sm + bimg + sw128(r, jj)) = pack8(t);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) t[e] = qv[e] * e1[e] * F[e];
                 {
                     const uint4 hi = pack8(t);
-                    *reinterpret_cast<uint4 *>(sm + P_QR + img) = hi;
+                    *reinterpret_cast<uint4 *>(sm + bimg + sw128(64 + r, jj)) = hi;
                     float hf[8], lo[8];
                     unpack8(hi, hf);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) lo[e] = t[e] - hf[e];
-                    *reinterpret_cast<uint4 *>(sm + P_ZI + img) = pack8(lo);  // z image is dead
+                    *reinterpret_cast<uint4 *>(sm + bimg + sw128(128 + r, jj)) = pack8(lo);
                 }
                 for (int V = R; V < 4; ++V) {
                     float Cv[8];
@@ -360,13 +393,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
 #pragma unroll
                     for (int e = 0; e < 8; ++e) t[e] = kv[e] * e3[e] * Cv[e];
                     const uint4 hi = pack8(t);
-                    *reinterpret_cast<uint4 *>(sm + P_KC + atom * KC_ATOM + sw128(kc_row0(V) + r, jj)) = hi;
+                    *reinterpret_cast<uint4 *>(sm + aimg + sw128(kc_row0(V) + r, jj)) = hi;
                     if (V == R) {  // diagonal block: keep the rounding residue
                         float hf[8], lo[8];
                         unpack8(hi, hf);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) lo[e] = t[e] - hf[e];
-                        *reinterpret_cast<uint4 *>(sm + P_KLO + img) = pack8(lo);
+                        *reinterpret_cast<uint4 *>(sm + aimg + sw128(A_KLO + r, jj)) = pack8(lo);
                     }
                 }
 #pragma unroll
@@ -397,107 +430,109 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             bulk_store(rec + REC_KT, sm + P_KI, 16384);
             bulk_commit();
             tc_fence_after();
-            constexpr uint32_t id = idesc_f16(64, 16, 0, 0);
-            const uint64_t kc = smem_desc(smem_u32(sm + P_KC), 16, 1024, LAYOUT_SW128);
-            const uint64_t kr = smem_desc(smem_u32(sm + P_KR), 16, 1024, LAYOUT_SW128);
-            const uint64_t qr = smem_desc(smem_u32(sm + P_QR), 16, 1024, LAYOUT_SW128);
-            const uint64_t klo = smem_desc(smem_u32(sm + P_KLO), 16, 1024, LAYOUT_SW128);
-            const uint64_t qlo = smem_desc(smem_u32(sm + P_ZI), 16, 1024, LAYOUT_SW128);
-            // lo(k) * hi(q) for all four diagonal blocks at once: rows i of the residue image
-            // carry the scaling of their own block, so the products are right wherever i and
-            // r share a block (the only entries read)
-            constexpr uint32_t id64 = idesc_f16(64, 64, 0, 0);
+            // all block versions at once: D1 = rows 0-127 of the A operand, D2 = rows 96-223 (version 3 and
+            // the low part of the diagonal operand), each against [k rows | q rows | low q rows]; every
+            // entry read afterwards pairs a row of version V with a column of block V
+            constexpr uint32_t id = idesc_f16(128, 192, 0, 0);
+            const uint64_t da = smem_desc(smem_u32(sm + P_A), 16, 1024, LAYOUT_SW128);
+            const uint64_t db = smem_desc(smem_u32(sm + P_B), 16, 1024, LAYOUT_SW128);
 #pragma unroll
             for (int s8 = 0; s8 < 8; ++s8) {
-                const uint32_t ko = (s8 >> 2), kb = (s8 & 3) * 32;
-                mma_f16_ss(tmem + 128, dadd(klo, ko * 8192 + kb), dadd(qr, ko * 8192 + kb), id64, s8 > 0);
-            }
-#pragma unroll
-            for (int V = 0; V < 4; ++V) {
-#pragma unroll
-                for (int s8 = 0; s8 < 8; ++s8) {
-                    const uint32_t ko = (s8 >> 2), kb = (s8 & 3) * 32;
-                    const uint64_t a = dadd(kc, ko * KC_ATOM + kc_row0(V) * 128 + kb);
-                    const uint64_t bk = dadd(kr, ko * 8192 + V * 2048 + kb);
-                    const uint64_t bq = dadd(qr, ko * 8192 + V * 2048 + kb);
-                    mma_f16_ss(tmem + 16 * V, a, bk, id, s8 > 0);
-                    mma_f16_ss(tmem + 64 + 16 * V, a, bq, id, s8 > 0);
-                    // hi(k) * lo(q) on block V's columns, added to the residue above
-                    mma_f16_ss(tmem + 128 + 16 * V, a, dadd(qlo, ko * 8192 + V * 2048 + kb), id, 1);
-                }
+                const uint32_t ko = s8 >> 2, kb = (s8 & 3) * 32;
+                mma_f16_ss(tmem, dadd(da, ko * A_ATOM + kb), dadd(db, ko * B_ATOM + kb), id, s8 > 0);
+                mma_f16_ss(tmem + 192, dadd(da, ko * A_ATOM + 96 * 128 + kb), dadd(db, ko * B_ATOM + kb), id, s8 > 0);
             }
             mma_commit(bar_am);
         }
-        // while the MMAs run: sigmoid of the output-gate logits (full fp32, stored as f16) for the state
-        // kernel's output stage, in its tile layout [2 atoms (j / 64)][64 rows r][128 B], 128-byte swizzled
-        if (p.gate) {
-            const int row = tid >> 2, part = tid & 3;
-            if (row < len) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(
-                    p.gate + (((int64_t)b * p.S + t0 + row) * p.H + h) * DD + part * 32);
-                uint8_t *dst = reinterpret_cast<uint8_t *>(p.sig + ((size_t)(b * p.H + h) * p.Nc + n) * (CH * DD)) +
-                               (part >> 1) * 8192;
-                uint4 gv[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) gv[k] = src[k];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    float g[8];
-                    unpack8(gv[k], g);
-                    uint4 o;
-                    __half2 *oh = reinterpret_cast<__half2 *>(&o);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        oh[e] = __floats2half2_rn(__fdividef(1.0f, 1.0f + __expf(-g[2 * e])),
-                                                  __fdividef(1.0f, 1.0f + __expf(-g[2 * e + 1])));
-                    *reinterpret_cast<uint4 *>(dst + sw128(row, 4 * (part & 1) + k)) = o;
-                }
-            }
-        }
+        // while the MMAs run: the sigmoid of the output-gate logits
+        gate_sigmoid(n, h, b, t0, len);
         ok = mbar_wait(bar_am, par);
         ok = __syncthreads_and(ok);
         tc_fence_after();
         if (!ok) break;
-        // q, k, z images are dead (their stores have read them once the group drains): prefetch
-        if (tid == 0) {
-            if (u_next < p.units) {
-                bulk_wait_read_all();
-                load_qkz(u_next);
-            }
+        // q and k images are dead (their stores have read them once the group drains): prefetch
+        if (tid == 0 && u_next < p.units) {
+            bulk_wait_read_all();
+            load_qk(u_next);
         }
 
-        // ---------------- P3: A (masked, beta-weighted, fp32) and the M^T image
+        // ---------------- P3: A (masked, beta-weighted, fp32) and the M^T image.
+        // Lanes of D1 (warps 0-2) and D2 (warps 4-7) are rows of the A operand: version V, row i gives
+        // A[r, i] and M[r, i] for r in block V; rows 160-223 (warps 6-7) give the low-part products for
+        // the diagonal blocks, handed over through shared memory.
         {
-            const int q4 = warp & 3, role = warp >> 2;
-            const int i = 16 * q4 + lane;
-            uint32_t va[32], vb[32], vd[16];
-            const uint32_t taddr = tmem + ((uint32_t)(32 * q4) << 16) + 64 * role;
-            tmem_ld_32x32b_x32(taddr, va);
-            tmem_ld_32x32b_x32(taddr + 32, vb);
-            tmem_ld_32x32b_x16(tmem + ((uint32_t)(32 * q4) << 16) + 128 + 16 * q4, vd);
-            tmem_wait_ld();
-            if (lane < 16) {
-                if (role == 0) {
-                    float *sA = reinterpret_cast<float *>(sm + P_SA);
+            const int q4 = warp & 3;
+            const uint32_t lq = (uint32_t)(32 * q4) << 16;
+            float *lohi = reinterpret_cast<float *>(sm + P_LOHI);
+            if (warp >= 6) {  // low part of the diagonal column operand x q: row i, block R = i / 16
+                const int i = 32 * (warp - 6) + lane, R = i >> 4;
+                uint32_t v[16];
+                // lanes of one warp span two blocks: load both candidate column blocks, keep the own one
+                uint32_t w0[16], w1[16];
+                tmem_ld_32x32b_x16(tmem + lq + 192 + 64 + 32 * (warp - 6), w0);
+                tmem_ld_32x32b_x16(tmem + lq + 192 + 64 + 32 * (warp - 6) + 16, w1);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int r = 0; r < 64; ++r) {
-                        const float v = __uint_as_float(r < 32 ? va[r] : vb[r - 32]);
-                        sA[r * SA_LD + i] = (i < r) ? sbeta[r] * v : 0.f;
-                    }
-                } else {
+                for (int e = 0; e < 16; ++e) v[e] = (R & 1) ? w1[e] : w0[e];
 #pragma unroll
-                    for (int cc = 0; cc < 8; ++cc) {
-                        float t[8];
+                for (int e = 0; e < 16; e += 4)
+                    *reinterpret_cast<float4 *>(lohi + i * 16 + e) =
+                        make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
+                                    __uint_as_float(v[e + 3]));
+            }
+            __syncthreads();
+            if (warp != 3 && warp < 6) {
+                const int prow = warp < 3 ? 32 * warp + lane : 96 + 32 * (warp - 4) + lane;
+                const int V = prow < 16 ? 0 : (prow < 48 ? 1 : (prow < 96 ? 2 : 3));
+                const int i = prow - kc_row0(V);
+                const bool diag = (i >> 4) == V;
+                const uint32_t cb = tmem + lq + (warp < 3 ? 0u : 192u);
+                // column block V differs between lanes of a warp: each warp's rows span at most two
+                // versions, so load the block of every version present and select
+                uint32_t a_[16], m_[16], r_[16];
+                const int Vlo = (warp < 3 ? (32 * warp < 16 ? 0 : (32 * warp < 48 ? 1 : 2)) : 3);
+                const int Vhi = (warp < 3 ? ((32 * warp + 31) < 16 ? 0 : ((32 * warp + 31) < 48 ? 1 : 2)) : 3);
+                {
+                    uint32_t x[16], y[16], z[16];
+                    tmem_ld_32x32b_x16(cb + 16 * Vlo, x);
+                    tmem_ld_32x32b_x16(cb + 64 + 16 * Vlo, y);
+                    tmem_ld_32x32b_x16(cb + 128 + 16 * Vlo, z);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int r = 8 * cc + e;
-                            float v = __uint_as_float(r < 32 ? va[r] : vb[r - 32]);
-                            if ((r >> 4) == q4) v += __uint_as_float(vd[r & 15]);
-                            t[e] = (i <= r) ? v : 0.f;
-                        }
-                        *reinterpret_cast<uint4 *>(sm + P_MT + sw128(i, cc)) = pack8(t);
+                    for (int e = 0; e < 16; ++e) { a_[e] = x[e]; m_[e] = y[e]; r_[e] = z[e]; }
+                }
+                if (Vhi != Vlo) {
+                    uint32_t x[16], y[16], z[16];
+                    tmem_ld_32x32b_x16(cb + 16 * Vhi, x);
+                    tmem_ld_32x32b_x16(cb + 64 + 16 * Vhi, y);
+                    tmem_ld_32x32b_x16(cb + 128 + 16 * Vhi, z);
+                    tmem_wait_ld();
+                    if (V == Vhi) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) { a_[e] = x[e]; m_[e] = y[e]; r_[e] = z[e]; }
                     }
                 }
+                float *sA = reinterpret_cast<float *>(sm + P_SA);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int r = 16 * V + e;
+                    sA[r * SA_LD + i] = (i < r) ? sbeta[r] * __uint_as_float(a_[e]) : 0.f;
+                }
+#pragma unroll
+                for (int hc = 0; hc < 2; ++hc) {
+                    float t[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int ee = 8 * hc + e, r = 16 * V + ee;
+                        float v = __uint_as_float(m_[ee]);
+                        if (diag) v += __uint_as_float(r_[ee]) + lohi[i * 16 + ee];
+                        t[e] = (i <= r) ? v : 0.f;
+                    }
+                    *reinterpret_cast<uint4 *>(sm + P_MT + sw128(i, 2 * V + hc)) = pack8(t);
+                }
+                if (diag)  // columns of earlier blocks: masked (i > r)
+                    for (int cc = 0; cc < 2 * V; ++cc)
+                        *reinterpret_cast<uint4 *>(sm + P_MT + sw128(i, cc)) = make_uint4(0u, 0u, 0u, 0u);
             }
         }
         tc_fence_before();
@@ -597,7 +632,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         ok = __syncthreads_and(ok);
         tc_fence_after();
         if (!ok) break;
-        if (tid == 0 && u_next < p.units) load_v(u_next);  // beta V has been consumed
+        if (tid == 0 && u_next < p.units) load_zv(u_next);  // beta K e^G and beta V have been consumed
 
         // ---------------- P5: -W image (warps 0-3, M = 64 accumulator rows) and U^T image (warps 4-7,
         // one value column j per lane)
@@ -657,7 +692,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 256);
+    if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 // ================================================================ K2b: chunk_state_kernel
