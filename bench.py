@@ -46,7 +46,10 @@ REF_SAMPLE_TOKENS = 512   # tokens (all heads) per reference-arm step
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
 # the committed ncu summaries under profiles/, keyed by kernel and workload,
 # valid only while the kernel's source file is unchanged (sha256 prefix).
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # prefill_4k_chunk_engine.md: prep 130.7 + segment maps 64.2 + combine 6.3 + segment chains 102.5 MB
+    "chunk_engine@prefill_4k": {"bytes": 303637760, "src_sha": "100718e5c32d9d72"},
+}
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -296,7 +299,7 @@ def run_ours(args, rank, world, local):
     if t_chunk >= t_proj:
         roof = {"kernel": "kda_chunk_fwd (chunk engine)", "bound": "hbm", "achieved": round(chunk_ach, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(chunk_frac, 4),
-                "traffic": traffic_for("chunk_engine", PREFILL, "kimi_delta_attention_21_b200/csrc/chunk_simt.cu"),
+                "traffic": traffic_for("chunk_engine", PREFILL, "kimi_delta_attention_21_b200/csrc/chunk_tc.cu"),
                 "algorithmic_bytes": chunk_bytes, "ms": round(t_chunk * 1e3, 4)}
     else:
         roof = {"kernel": "kda_out_proj", "bound": "tensor", "achieved": round(proj_ach, 1),
