@@ -1134,7 +1134,7 @@ struct CombineArgs {
     int *dev_status;
 };
 
-constexpr size_t COMB_SMEM = 2 * 32768 + 64 + 1024;
+constexpr size_t COMB_SMEM = 2 * (32768 + 65536) + 64 + 1024;  // 2 stages of [A_g^T image | Y_g]
 
 __global__ void __launch_bounds__(128, 1) chunk_combine_kernel(CombineArgs p) {
     extern __shared__ uint8_t smraw[];
@@ -1142,13 +1142,15 @@ __global__ void __launch_bounds__(128, 1) chunk_combine_kernel(CombineArgs p) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.y * p.H + blockIdx.x;
     const int j = tid;
-    uint64_t *full = reinterpret_cast<uint64_t *>(sm + 65536);  // [2]
+    constexpr uint32_t CST = 32768 + 65536;                         // stage: A_g^T image, then Y_g fp32
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + 2 * CST);  // [2]
     uint64_t *bar_m = full + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full + 3);
     const int nseg = p.G - 1;
     auto issue = [&](int g) {
-        mbar_arrive_expect_tx(&full[g & 1], 32768);
-        bulk_load(sm + (g & 1) * 32768, p.xt + ((size_t)bh * nseg + g) * 32768, 32768, &full[g & 1]);
+        mbar_arrive_expect_tx(&full[g & 1], CST);
+        bulk_load(sm + (g & 1) * CST, p.xt + ((size_t)bh * nseg + g) * 32768, 32768, &full[g & 1]);
+        bulk_load(sm + (g & 1) * CST + 32768, p.yt + ((size_t)bh * nseg + g) * DD * DD, 65536, &full[g & 1]);
     };
     if (tid == 0) {
         mbar_init(&full[0], 1);
@@ -1192,22 +1194,21 @@ __global__ void __launch_bounds__(128, 1) chunk_combine_kernel(CombineArgs p) {
             if (ok) {
                 tc_fence_after();
                 constexpr uint32_t id = idesc_f16(128, 128, 0, 1);
-                const uint64_t d = smem_desc(smem_u32(sm + (g & 1) * 32768), 16384, 1024, LAYOUT_SW128);
+                const uint64_t d = smem_desc(smem_u32(sm + (g & 1) * CST), 16384, 1024, LAYOUT_SW128);
 #pragma unroll
                 for (int s8 = 0; s8 < 8; ++s8) mma_f16_ts(tmem + C_D, tmem + C_S16 + 8 * s8, dadd(d, s8 * 2048), id, s8 > 0);
                 mma_commit(bar_m);
             }
         }
-        ok = __syncthreads_and(ok) && mbar_wait(bar_m, g & 1);
+        ok = __syncthreads_and(ok) && mbar_wait(bar_m, g & 1) && mbar_wait(&full[g & 1], (g >> 1) & 1);
         ok = __syncthreads_and(ok);
         if (!ok) break;
         tc_fence_after();
-        if (tid == 0 && g + 2 < nseg) issue(g + 2);  // the image just used has been read
-        // S_{g+1}^T = D + Y_g^T (all of Y's column loaded before any store: the two may not be reordered)
-        const float *y = p.yt + ((size_t)bh * nseg + g) * DD * DD + j;
+        // S_{g+1}^T = D + Y_g^T (Y_g in shared memory, [c][j])
+        const float *y = reinterpret_cast<const float *>(sm + (g & 1) * CST + 32768) + j;
         float *dst = p.seg_init + ((size_t)bh * p.G + g + 1) * DD * DD + j;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) sv[c] = y[(size_t)c * DD];
+        for (int c = 0; c < 128; ++c) sv[c] = y[c * DD];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             uint32_t dv[32];
@@ -1220,6 +1221,7 @@ __global__ void __launch_bounds__(128, 1) chunk_combine_kernel(CombineArgs p) {
         for (int c = 0; c < 128; ++c) dst[(size_t)c * DD] = sv[c];
         tc_fence_before();
         __syncthreads();
+        if (tid == 0 && g + 2 < nseg) issue(g + 2);  // this stage has been read
     }
     if (!ok && tid == 0) {
         report_timeout(p.timeouts, p.dev_status);
