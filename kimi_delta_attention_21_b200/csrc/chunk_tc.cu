@@ -181,7 +181,9 @@ struct PrepArgs {
     int *dev_status;
 };
 
-__global__ void __launch_bounds__(256, 1)
+constexpr int PREP_THREADS = 512;
+
+__global__ void __launch_bounds__(PREP_THREADS, 1)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tz, PrepArgs p) {
     extern __shared__ uint8_t smraw[];
@@ -222,20 +224,20 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     };
 
     // sigmoid of the output-gate logits (full fp32, stored as f16) for the state kernel's output stage,
-    // in its tile layout [2 atoms (j / 64)][64 rows r][128 B], 128-byte swizzled: one row x 32 value
+    // in its tile layout [2 atoms (j / 64)][64 rows r][128 B], 128-byte swizzled: one row x 16 value
     // columns per thread
     auto gate_sigmoid = [&](int n, int h, int b, int t0, int len) {
-        const int row = tid >> 2, c0 = 32 * (tid & 3);
+        const int row = tid >> 3, c0 = 16 * (tid & 7);
         if (!p.gate || row >= len) return;
         const uint4 *src =
             reinterpret_cast<const uint4 *>(p.gate + (((int64_t)b * p.S + t0 + row) * p.H + h) * DD + c0);
         uint8_t *dst = reinterpret_cast<uint8_t *>(p.sig + ((size_t)(b * p.H + h) * p.Nc + n) * (CH * DD)) +
                        (c0 >> 6) * 8192;
-        uint4 gv[4];
+        uint4 gv[2];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) gv[k] = src[k];
+        for (int k = 0; k < 2; ++k) gv[k] = src[k];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < 2; ++k) {
             float g[8];
             unpack8(gv[k], g);
             uint4 o;
@@ -285,37 +287,38 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         if (!ok) break;
 
         // ---------------- P1: G = in-chunk cumulative log-decay (rows past the sequence end: no decay)
-        {
-            const int c = tid & 127, half = tid >> 7;
-            float g[32];
+        {   // one thread per channel c and 16 rows (quarter qt); quarter sums through the inverse scratch
+            const int c = tid & 127, qt = tid >> 7;
+            float *qsum = reinterpret_cast<float *>(sm + P_XS);
+            float g[16];
             if (p.log_decay) {
 #pragma unroll
-                for (int rr = 0; rr < 32; ++rr) {
-                    const int r = half * 32 + rr;
+                for (int rr = 0; rr < 16; ++rr) {
+                    const int r = qt * 16 + rr;
                     g[rr] = (r < len) ? p.log_decay[(((int64_t)b * p.S + t0 + r) * p.H + h) * DD + c] : 0.f;
                 }
             } else {
                 const uint8_t *zc = sm + P_ZI + (c >> 6) * 8192 + (c & 7) * 2;
                 const uint32_t ch = (c & 63) >> 3;
 #pragma unroll
-                for (int rr = 0; rr < 32; ++rr) {
-                    const int r = half * 32 + rr;
+                for (int rr = 0; rr < 16; ++rr) {
+                    const int r = qt * 16 + rr;
                     const float zv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(zc + sw128(r, ch)));
                     g[rr] = (r < len) ? log_alpha_fast(zv, p.g_min) : 0.f;
                 }
             }
             float acc = 0.f;
 #pragma unroll
-            for (int rr = 0; rr < 32; ++rr) {
+            for (int rr = 0; rr < 16; ++rr) {
                 acc += g[rr];
                 g[rr] = acc;
             }
-            if (half == 0) sG[31 * SG_LD + c] = acc;
+            qsum[qt * 128 + c] = acc;
             __syncthreads();
-            const float base = half ? sG[31 * SG_LD + c] : 0.f;
-            __syncthreads();
+            float base = 0.f;
+            for (int q = 0; q < qt; ++q) base += qsum[q * 128 + c];
 #pragma unroll
-            for (int rr = 0; rr < 32; ++rr) sG[(half * 32 + rr) * SG_LD + c] = g[rr] + base;
+            for (int rr = 0; rr < 16; ++rr) sG[(qt * 16 + rr) * SG_LD + c] = g[rr] + base;
         }
         __syncthreads();
         // ---------------- per-channel block constants
@@ -342,13 +345,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             sgam[c] = fexp(bb[3]);
         }
         __syncthreads();
-        // ---------------- P2: decay-scaled operands (one thread per row r and 4 chunks of 8 channels)
+        // ---------------- P2: decay-scaled operands (one thread per row r and 2 chunks of 8 channels)
         {
             const int r = tid & 63, grp = tid >> 6, R = r >> 4;
             const float beta_r = sbeta[r];
 #pragma unroll 1
-            for (int mi = 0; mi < 4; ++mi) {
-                const int j = grp + 4 * mi;
+            for (int mi = 0; mi < 2; ++mi) {
+                const int j = grp + 8 * mi;
                 const int atom = j >> 3, jj = j & 7, c0 = 8 * j;
                 const uint32_t img = atom * 8192 + sw128(r, jj);
                 const uint32_t bimg = P_B + atom * B_ATOM, aimg = P_A + atom * A_ATOM;
@@ -464,7 +467,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             const int q4 = warp & 3;
             const uint32_t lq = (uint32_t)(32 * q4) << 16;
             float *lohi = reinterpret_cast<float *>(sm + P_LOHI);
-            if (warp >= 6) {  // low part of the diagonal column operand x q: row i, block R = i / 16
+            if (warp == 6 || warp == 7) {  // low part of the diagonal column operand x q: row i, block R = i / 16
                 const int i = 32 * (warp - 6) + lane, R = i >> 4;
                 uint32_t v[16];
                 // lanes of one warp span two blocks: load both candidate column blocks, keep the own one
@@ -543,7 +546,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             const float *sA = reinterpret_cast<const float *>(sm + P_SA);
             float *sT = reinterpret_cast<float *>(sm + P_ST);
             float *xs = reinterpret_cast<float *>(sm + P_XS);
-            for (int e = tid; e < 64 * ST_LD / 4; e += 256)
+            for (int e = tid; e < 64 * ST_LD / 4; e += PREP_THREADS)
                 reinterpret_cast<float4 *>(sT)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
             __syncthreads();
             if (tid < 64) {  // diagonal block R, column jc: forward substitution
@@ -596,16 +599,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 }
                 __syncthreads();
             }
-            {  // T image (K-major, 64 rows x 64 cols)
-                const int r = tid >> 2, part = tid & 3;
+            {  // T image (K-major, 64 rows x 64 cols), one 8-column chunk per thread
+                const int r = tid >> 3, cc = tid & 7;
+                float t[8];
 #pragma unroll
-                for (int uu = 0; uu < 2; ++uu) {
-                    const int cc = 2 * part + uu;
-                    float t[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) t[e] = sT[r * ST_LD + 8 * cc + e];
-                    *reinterpret_cast<uint4 *>(sm + P_TI + sw128(r, cc)) = pack8(t);
-                }
+                for (int e = 0; e < 8; ++e) t[e] = sT[r * ST_LD + 8 * cc + e];
+                *reinterpret_cast<uint4 *>(sm + P_TI + sw128(r, cc)) = pack8(t);
             }
             fence_proxy_async_smem();
         }
@@ -634,16 +633,16 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         if (!ok) break;
         if (tid == 0 && u_next < p.units) load_zv(u_next);  // beta K e^G and beta V have been consumed
 
-        // ---------------- P5: -W image (warps 0-3, M = 64 accumulator rows) and U^T image (warps 4-7,
-        // one value column j per lane)
+        // ---------------- P5: -W image (warp groups 0 and 2: M = 64 accumulator rows, half the columns
+        // each) and U^T image (warp groups 1 and 3: one value column j per lane, half the rows each)
         {
-            const int q4 = warp & 3;
-            if (warp < 4) {
+            const int q4 = warp & 3, wg = warp >> 2;
+            if ((wg & 1) == 0) {
                 const int r = 16 * q4 + lane;
 #pragma unroll 1
-                for (int cb = 0; cb < 4; ++cb) {
+                for (int cb = 0; cb < 2; ++cb) {
                     uint32_t v[32];
-                    tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q4) << 16) + 32 * cb, v);
+                    tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q4) << 16) + 64 * (wg >> 1) + 32 * cb, v);
                     tmem_wait_ld();
                     if (lane < 16) {
 #pragma unroll
@@ -651,25 +650,22 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                             float t[8];
 #pragma unroll
                             for (int e = 0; e < 8; ++e) t[e] = -__uint_as_float(v[8 * g + e]);
-                            const int j = 4 * cb + g;  // 8-column group
+                            const int j = 8 * (wg >> 1) + 4 * cb + g;  // 8-column group
                             *reinterpret_cast<uint4 *>(sm + P_WI + (j >> 3) * 8192 + sw128(r, j & 7)) = pack8(t);
                         }
                     }
                 }
             } else {
                 const int jv = 32 * q4 + lane;
-#pragma unroll 1
-                for (int cb = 0; cb < 2; ++cb) {
-                    uint32_t v[32];
-                    tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q4) << 16) + 128 + 32 * cb, v);
-                    tmem_wait_ld();
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q4) << 16) + 128 + 32 * (wg >> 1), v);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int g = 0; g < 4; ++g) {
-                        float t[8];
+                for (int g = 0; g < 4; ++g) {
+                    float t[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) t[e] = __uint_as_float(v[8 * g + e]);
-                        *reinterpret_cast<uint4 *>(sm + P_UI + sw128(jv, 4 * cb + g)) = pack8(t);
-                    }
+                    for (int e = 0; e < 8; ++e) t[e] = __uint_as_float(v[8 * g + e]);
+                    *reinterpret_cast<uint4 *>(sm + P_UI + sw128(jv, 4 * (wg >> 1) + g)) = pack8(t);
                 }
             }
         }
@@ -1365,7 +1361,7 @@ kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
         const int sms = device_sms();
         const int64_t grid = pa.units < sms ? pa.units : sms;
         cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PREP_SMEM);
-        chunk_prep_kernel<<<(unsigned)grid, 256, PREP_SMEM, st>>>(tq, tk, tv, tz, pa);
+        chunk_prep_kernel<<<(unsigned)grid, PREP_THREADS, PREP_SMEM, st>>>(tq, tk, tv, tz, pa);
         s = check_launch("chunk_prep_kernel");
         if (s != KDA_OK) return s;
     }
