@@ -251,7 +251,7 @@ def test_prefill_4k_layer(K, engine):
 
 
 @pytest.mark.parametrize("N,K,Dm", [(1, 8, 8), (128, 64, 256), (129, 64, 264), (300, 200, 96), (4096, 2048, 2048),
-                                    (256, 4096, 4096), (77, 4096, 520)])
+                                    (256, 4096, 4096), (77, 4096, 520), (100, 1024, 2048)])
 def test_projection_tensor_core_shapes(K, N, Dm):
     rng = np.random.default_rng(N * 3 + K)
     x = ki.round_bf16(rng.standard_normal((N, K)).astype(np.float32))
