@@ -726,7 +726,7 @@ struct StateArgs {
 
 constexpr int ST_THREADS = 288;                // warps 0-7 register work, warp 8 MMA + copies
 constexpr uint32_t ST_STAGE = REC_GAM;         // the image part of a record (73728 B)
-constexpr uint32_t ST_GAM = 2 * ST_STAGE;      // e^{G_C} [2 stages][128] fp32
+constexpr uint32_t ST_GAM = 2 * ST_STAGE;      // e^{G_C} [2 stages][128] fp32 (the maps: 3 stages, into OIMG)
 constexpr uint32_t ST_OIMG = ST_GAM + 1024;    // output tile [2 atoms (j / 64)][64 rows r][128 B]
 constexpr uint32_t ST_SIGT = ST_OIMG + 16384;  // sigmoid(gate) tile, same layout, f16
 constexpr uint32_t ST_OT = ST_SIGT + 16384;    // O^T image, K-major B [128 rows j][128 B: 64 r]
@@ -763,17 +763,25 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
     const bool ident = kMap && (blockIdx.z & 1) == 0;  // map from the identity (no U)
     const int n0 = g * p.L;
     const int nc = max(0, min(p.L, p.Nc - n0));  // chunks of this segment
+    // Record stages: the chains use whole records, two deep; the maps only -W, K~ and U^T (48 KB),
+    // three deep.  The e^{G_C} of each stage sits after the stages.
+    constexpr int STG = kMap ? 3 : 2;
+    constexpr uint32_t STB = kMap ? 49152u : ST_STAGE;
+    constexpr uint32_t O_W_ATOM = kMap ? 8192u : 16384u;  // atom stride of the [-W; Q e^G] (or -W) B operand
+    constexpr uint32_t O_KT = kMap ? 16384u : REC_KT;
+    constexpr uint32_t O_U = kMap ? 32768u : REC_U;
+    static_assert(STG * STB == ST_GAM, "record stages end where e^{G_C} starts");
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ST_BAR);
-    uint64_t *full = bars;           // [2] record stage landed
-    uint64_t *bar_p = bars + 2;      // PO group done
-    uint64_t *bar_s = bars + 3;      // S^T += V'^T K~ done (and every earlier group)
-    uint64_t *bar_o = bars + 4;      // PO += V'^T M^T done
-    uint64_t *bar_t = bars + 5;      // transposition of O done
-    uint64_t *bar_simg = bars + 6;   // bf16 copy of S^T written (8 warps)
-    uint64_t *bar_vimg = bars + 7;   // bf16 copy of V'^T written (8 warps)
-    uint64_t *bar_ot = bars + 8;     // O^T image written (8 warps)
-    uint64_t *bar_sig = bars + 9;    // sigmoid tile landed
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 10);
+    uint64_t *full = bars;           // [STG] record stage landed
+    uint64_t *bar_p = bars + 3;      // PO group done
+    uint64_t *bar_s = bars + 4;      // S^T += V'^T K~ done (and every earlier group)
+    uint64_t *bar_o = bars + 5;      // PO += V'^T M^T done
+    uint64_t *bar_t = bars + 6;      // transposition of O done
+    uint64_t *bar_simg = bars + 7;   // bf16 copy of S^T written (8 warps)
+    uint64_t *bar_vimg = bars + 8;   // bf16 copy of V'^T written (8 warps)
+    uint64_t *bar_ot = bars + 9;     // O^T image written (8 warps)
+    uint64_t *bar_sig = bars + 10;   // sigmoid tile landed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 11);
     float *sgam = reinterpret_cast<float *>(sm + ST_GAM);
     float *red = reinterpret_cast<float *>(sm + ST_RED);
     const uint8_t *rec0 = p.ws + ((size_t)bh * p.Nc + n0) * REC_BYTES;
@@ -781,7 +789,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
 
     if (tid == 0) {
         s_fail = 0;
-        for (int i = 0; i < 6; ++i) mbar_init(&bars[i], 1);
+        for (int i = 0; i < 7; ++i) mbar_init(&bars[i], 1);
         mbar_init(bar_simg, 8);
         mbar_init(bar_vimg, 8);
         mbar_init(bar_ot, 8);
@@ -815,10 +823,18 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
             const uint64_t d_k = smem_desc(smem_u32(sm), 16, 1024, LAYOUT_SW128);     // K-major images
             const uint64_t d_mn = smem_desc(smem_u32(sm), 8192, 1024, LAYOUT_SW128);  // K~ and M^T images
             auto issue_record = [&](int n) {
-                const int stg = n & 1;
-                mbar_arrive_expect_tx(&full[stg], ST_STAGE + 512);
+                const int stg = n % STG;
+                uint8_t *dst = sm + stg * STB;
                 const uint8_t *src = rec0 + (size_t)n * REC_BYTES;
-                bulk_load(sm + stg * ST_STAGE, src, ST_STAGE, &full[stg]);
+                mbar_arrive_expect_tx(&full[stg], STB + 512);
+                if (kMap) {  // -W rows of both atoms, K~, U^T
+                    bulk_load(dst, src + REC_WQ, 8192, &full[stg]);
+                    bulk_load(dst + 8192, src + REC_WQ + 16384, 8192, &full[stg]);
+                    bulk_load(dst + O_KT, src + REC_KT, 16384, &full[stg]);
+                    bulk_load(dst + O_U, src + REC_U, 16384, &full[stg]);
+                } else {
+                    bulk_load(dst, src, ST_STAGE, &full[stg]);
+                }
                 bulk_load(sgam + stg * 128, src + REC_GAM, 512, &full[stg]);
                 ++issued;
             };
@@ -833,35 +849,36 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
                 mma_commit(bar_t);
                 return true;
             };
-            for (int n = 0; n < 2 && n < nc; ++n) issue_record(n);
+            for (int n = 0; n < STG && n < nc; ++n) issue_record(n);
             int n = 0;
             for (; n < nc; ++n) {
                 if (s_fail) { ok = false; break; }
-                const uint32_t sgo = (n & 1) * ST_STAGE;
+                // the stage of record n - 1 is free once its last group is done: refill it, STG - 1 ahead
+                if (n >= 1 && n + STG - 1 < nc) {
+                    if (!mbar_wait(bar_o, (n - 1) & 1)) { ok = false; break; }
+                    issue_record(n + STG - 1);
+                }
+                const uint32_t sgo = (n % STG) * STB;
                 const uint32_t po = tmem + T_PO + (uint32_t)(n & 1) * 128;
-                if (!mbar_wait(&full[n & 1], (n >> 1) & 1)) { ok = false; break; }
+                if (!mbar_wait(&full[n % STG], (n / STG) & 1)) { ok = false; break; }
                 landed = n + 1;
-                // PO = S_n^T [-W; Q e^G]^T
+                // PO = S_n^T [-W; Q e^G]^T (the maps: S_n^T (-W)^T)
                 if (!mbar_wait(bar_simg, n & 1)) { ok = false; break; }
                 tc_fence_after();
+                constexpr uint32_t id_po = kMap ? idesc_f16(128, 64, 0, 0) : id_kk;
 #pragma unroll
                 for (int s8 = 0; s8 < 8; ++s8) {
                     const uint32_t ko = s8 >> 2, kb = (s8 & 3) * 32;
-                    mma_f16_ts(po, tmem + T_S16 + 8 * s8, dadd(d_k, sgo + REC_WQ + ko * 16384 + kb), id_kk, s8 > 0);
+                    mma_f16_ts(po, tmem + T_S16 + 8 * s8, dadd(d_k, sgo + ko * O_W_ATOM + kb), id_po, s8 > 0);
                 }
                 mma_commit(bar_p);
-                // record n - 1 is consumed once its last group is done: refill its stage
-                if (n >= 1 && n + 1 < nc) {
-                    if (!mbar_wait(bar_o, (n - 1) & 1)) { ok = false; break; }
-                    issue_record(n + 1);
-                }
                 if (!kMap && n >= 1 && !transpose_o(n - 1)) { ok = false; break; }
                 // S^T += V'^T K~, then PO[:, 64:] += V'^T M^T
                 if (!mbar_wait(bar_vimg, n & 1)) { ok = false; break; }
                 tc_fence_after();
 #pragma unroll
                 for (int s4 = 0; s4 < 4; ++s4)
-                    mma_f16_ts(tmem + T_S32, tmem + T_V16 + 8 * s4, dadd(d_mn, sgo + REC_KT + s4 * 2048), id_s, 1);
+                    mma_f16_ts(tmem + T_S32, tmem + T_V16 + 8 * s4, dadd(d_mn, sgo + O_KT + s4 * 2048), id_s, 1);
                 mma_commit(bar_s);
                 if (!kMap) {
 #pragma unroll
@@ -990,10 +1007,10 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
             const uint32_t po = tmem + lrow + T_PO + (uint32_t)(n & 1) * 128;
             // ---------- S_n^T (after the previous chunk's update) -> bf16 copy; S^T <- S^T Diag(e^{G_C})
             if (n >= 1 && !mbar_wait(bar_s, (n - 1) & 1)) { ok = false; break; }
-            if (!mbar_wait(&full[n & 1], (n >> 1) & 1)) { ok = false; break; }
+            if (!mbar_wait(&full[n % STG], (n / STG) & 1)) { ok = false; break; }
             tc_fence_after();
             {
-                const float4 *g4 = reinterpret_cast<const float4 *>(sgam + (n & 1) * 128 + 64 * hf);
+                const float4 *g4 = reinterpret_cast<const float4 *>(sgam + (n % STG) * 128 + 64 * hf);
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     uint32_t sv[32], pk[16];
@@ -1025,7 +1042,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
             }
             // ---------- V'^T = U^T - (W S_n)^T -> bf16 copy in TMEM
             {
-                const uint8_t *ut = sm + (n & 1) * ST_STAGE + REC_U;
+                const uint8_t *ut = sm + (n % STG) * STB + O_U;
                 uint4 uu[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) uu[k] = *reinterpret_cast<const uint4 *>(ut + sw128(j, 4 * hf + k));
@@ -1106,7 +1123,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
     if (warp == 8 && lane == 0 && s_fail) {
         report_timeout(p.timeouts, p.dev_status);
         // let the bulk copies already issued land before the CTA exits
-        for (int m = landed; m < issued; ++m) mbar_wait(&full[m & 1], (m >> 1) & 1, 100000000ull);
+        for (int m = landed; m < issued; ++m) mbar_wait(&full[m % STG], (m / STG) & 1, 100000000ull);
     }
     if (!kMap && tid == 0 && s_fail && p.sig) mbar_wait(bar_sig, 0, 100000000ull), mbar_wait(bar_sig, 1, 100000000ull);
     tc_fence_before();
