@@ -186,6 +186,8 @@ constexpr int PREP_THREADS = 512;
 __global__ void __launch_bounds__(PREP_THREADS, 1)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tz, PrepArgs p) {
+    pdl_trigger();
+    pdl_wait();
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = align1024(smraw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -753,6 +755,8 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
 template <bool kMap>
 __global__ void __launch_bounds__(ST_THREADS, 1)
 chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
+    pdl_trigger();
+    pdl_wait();
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = align1024(smraw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1150,6 +1154,8 @@ struct CombineArgs {
 constexpr size_t COMB_SMEM = 2 * (32768 + 65536) + 64 + 1024;  // 2 stages of [A_g^T image | Y_g]
 
 __global__ void __launch_bounds__(128, 1) chunk_combine_kernel(CombineArgs p) {
+    pdl_trigger();
+    pdl_wait();
     extern __shared__ uint8_t smraw[];
     uint8_t *sm = align1024(smraw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1263,7 +1269,9 @@ int device_sms() {
 kda_status_t launch_state(const CUtensorMap &tmo, const StateArgs &sa, int B, int H, cudaStream_t st) {
     if (sa.G > 1) {
         cudaFuncSetAttribute(chunk_state_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
-        chunk_state_kernel<true><<<dim3(H, B, 2 * (sa.G - 1)), ST_THREADS, STATE_SMEM, st>>>(tmo, sa);
+        cudaError_t e = launch_pdl(chunk_state_kernel<true>, dim3(H, B, 2 * (sa.G - 1)), dim3(ST_THREADS),
+                                   STATE_SMEM, st, tmo, sa);
+        if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "chunk_state_kernel (segment maps): %s", cudaGetErrorString(e));
         kda_status_t s = check_launch("chunk_state_kernel (segment maps)");
         if (s != KDA_OK) return s;
         CombineArgs ca;
@@ -1276,12 +1284,14 @@ kda_status_t launch_state(const CUtensorMap &tmo, const StateArgs &sa, int B, in
         ca.timeouts = sa.timeouts;
         ca.dev_status = sa.dev_status;
         cudaFuncSetAttribute(chunk_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)COMB_SMEM);
-        chunk_combine_kernel<<<dim3(H, B), 128, COMB_SMEM, st>>>(ca);
+        e = launch_pdl(chunk_combine_kernel, dim3(H, B), dim3(128), COMB_SMEM, st, ca);
+        if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "chunk_combine_kernel: %s", cudaGetErrorString(e));
         s = check_launch("chunk_combine_kernel");
         if (s != KDA_OK) return s;
     }
     cudaFuncSetAttribute(chunk_state_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
-    chunk_state_kernel<false><<<dim3(H, B, sa.G), ST_THREADS, STATE_SMEM, st>>>(tmo, sa);
+    cudaError_t e = launch_pdl(chunk_state_kernel<false>, dim3(H, B, sa.G), dim3(ST_THREADS), STATE_SMEM, st, tmo, sa);
+    if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "chunk_state_kernel: %s", cudaGetErrorString(e));
     return check_launch("chunk_state_kernel");
 }
 
@@ -1378,7 +1388,9 @@ kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
         const int sms = device_sms();
         const int64_t grid = pa.units < sms ? pa.units : sms;
         cudaFuncSetAttribute(chunk_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PREP_SMEM);
-        chunk_prep_kernel<<<(unsigned)grid, PREP_THREADS, PREP_SMEM, st>>>(tq, tk, tv, tz, pa);
+        cudaError_t e = launch_pdl(chunk_prep_kernel, dim3((unsigned)grid), dim3(PREP_THREADS), PREP_SMEM, st, tq, tk,
+                                   tv, tz, pa);
+        if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "chunk_prep_kernel: %s", cudaGetErrorString(e));
         s = check_launch("chunk_prep_kernel");
         if (s != KDA_OK) return s;
     }

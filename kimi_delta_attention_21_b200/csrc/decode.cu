@@ -129,6 +129,8 @@ decode128_stream_kernel(int nbh, const __nv_bfloat16 *__restrict__ q, const __nv
                         float *__restrict__ state, const __nv_bfloat16 *__restrict__ gate, float eps,
                         __nv_bfloat16 *__restrict__ o, unsigned int *timeouts) {
     using namespace sm100;
+    pdl_trigger();
+    pdl_wait();
     extern __shared__ __align__(128) uint8_t dsm[];
     __shared__ uint64_t fullS[DSTAGES], fullV[DSTAGES];
     __shared__ float s_a[DK], s_qk;
@@ -323,10 +325,12 @@ kda_status_t launch_typed(const kda_decode_args &a, cudaStream_t st) {
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         const int grid = (int)(nbh < sms ? nbh : sms);
         cudaFuncSetAttribute(decode128_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DS_SMEM);
-        decode128_stream_kernel<<<grid, 256, DS_SMEM, st>>>(
-            (int)nbh, (const __nv_bfloat16 *)q, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v,
-            (const __nv_bfloat16 *)z, a.log_decay, a.g_min, (const __nv_bfloat16 *)beta, a.state,
-            (const __nv_bfloat16 *)gate, a.eps, (__nv_bfloat16 *)o, device_timeout_counter());
+        cudaError_t e = launch_pdl(
+            decode128_stream_kernel, dim3(grid), dim3(256), DS_SMEM, st, (int)nbh, (const __nv_bfloat16 *)q,
+            (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, (const __nv_bfloat16 *)z, a.log_decay, a.g_min,
+            (const __nv_bfloat16 *)beta, a.state, (const __nv_bfloat16 *)gate, a.eps, (__nv_bfloat16 *)o,
+            device_timeout_counter());
+        if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "decode128_stream_kernel: %s", cudaGetErrorString(e));
         return check_launch("decode128_stream_kernel");
     }
     if (a.D_k == DK && a.D_v == DV && (reinterpret_cast<uintptr_t>(a.state) & 15u) == 0) {

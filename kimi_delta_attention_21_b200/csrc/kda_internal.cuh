@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "kda.h"
 
 namespace kda {
@@ -62,5 +64,23 @@ kda_status_t launch_proj_simt(const void *x, const void *W, int64_t N, int K, in
 bool proj_tc_supported(int64_t N, int K, int Dm, kda_dtype_t dt);
 kda_status_t launch_proj_tc(const void *x, const void *W, int64_t N, int K, int Dm, void *y,
                             cudaStream_t st);
+
+// Launch with programmatic stream serialisation (the kernel starts early and waits in device code
+// for the previous kernel of the stream before it touches global memory).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 }  // namespace kda

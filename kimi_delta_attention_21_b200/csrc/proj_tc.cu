@@ -36,6 +36,8 @@ template <int BN>
 __global__ void __launch_bounds__(192, 1)
 proj_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M, int N,
                int K, __nv_bfloat16 *__restrict__ y, unsigned int *timeouts) {
+    pdl_trigger();
+    pdl_wait();
     using Cfg = ProjCfg<BN>;
     constexpr int ST = Cfg::STAGES;
     extern __shared__ uint8_t smraw[];
@@ -195,8 +197,9 @@ kda_status_t launch_proj_tc_bn(const CUtensorMap &ta, const void *W, int64_t N, 
     cudaFuncSetAttribute(proj_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM_BYTES);
     const int64_t tiles = ((N + BM - 1) / BM) * ((Dm + BN - 1) / BN);
     const int grid = (int)(tiles < sms ? tiles : sms);
-    proj_tc_kernel<BN><<<grid, 192, Cfg::SMEM_BYTES, st>>>(ta, tb, (int)N, Dm, K, (__nv_bfloat16 *)y,
-                                                          device_timeout_counter());
+    cudaError_t e = launch_pdl(proj_tc_kernel<BN>, dim3(grid), dim3(192), Cfg::SMEM_BYTES, st, ta, tb, (int)N, Dm, K,
+                               (__nv_bfloat16 *)y, device_timeout_counter());
+    if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "proj_tc_kernel: %s", cudaGetErrorString(e));
     return check_launch("proj_tc_kernel");
 }
 
