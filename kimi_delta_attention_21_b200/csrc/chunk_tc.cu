@@ -38,12 +38,13 @@
 // no intermediate underflows unless the true value does.
 //
 // Precision of M.  Rounding the decay-scaled q and k to bf16 costs ~2^-9 of
-// sum_c |q_c k_c| in every product; on the diagonal 16x16 blocks of M (no
-// decay to shrink the terms) that error can be a large part of a small
-// q_r . k_i, and the per-head RMS normalisation then turns it into a large
-// output error for tokens whose o~ is small.  The diagonal blocks of M are
-// therefore computed with split operands, x = hi + lo (both bf16): the MMA
-// adds hi*lo + lo*hi on top of hi*hi, which leaves ~2^-17 relative error.
+// sum_c |q_c k_c| in every product, which can be a large part of a token's
+// o~ when o~ is small (the state decayed away, small writes), and the per-head
+// RMS normalisation then turns it into a large output error.  M is therefore
+// computed with split operands, x = hi + lo (both bf16): every block adds
+// hi(k) lo(q) (the low q rows are part of the stacked B operand), and the
+// diagonal 16x16 blocks, where no decay shrinks the terms, add lo(k) hi(q)
+// too (the low part of the diagonal column operand is part of the A operand).
 #include <cstring>
 
 #include <cuda_fp16.h>
@@ -529,8 +530,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int ee = 8 * hc + e, r = 16 * V + ee;
-                        float v = __uint_as_float(m_[ee]);
-                        if (diag) v += __uint_as_float(r_[ee]) + lohi[i * 16 + ee];
+                        // hi(k) lo(q) for every block; lo(k) hi(q) on the diagonal block
+                        float v = __uint_as_float(m_[ee]) + __uint_as_float(r_[ee]);
+                        if (diag) v += lohi[i * 16 + ee];
                         t[e] = (i <= r) ? v : 0.f;
                     }
                     *reinterpret_cast<uint4 *>(sm + P_MT + sw128(i, 2 * V + hc)) = pack8(t);

@@ -194,6 +194,45 @@ def test_tc_state_handoff_in_place(K):
     assert rel_fro(to_np(st), to_np(s_all)) <= 1e-2
 
 
+def test_tc_segmented_variants(K):
+    """The segmented state pass with precomputed log-decay input, several batch rows and heads,
+    and an in-place split-sequence handoff whose parts are themselves segmented, with the fused
+    norm and gate (checked on the projected layer output)."""
+    w = small("segv", 2, 1536, 3, 128, 128, 256, "bf16", seed=91, s0_std=0.02)
+    inp = ki.make_inputs(w)
+    d = upload(inp, w)
+    nc = (w.S + 63) // 64
+    assert K.chunk_workspace_bytes(w.B, w.S, w.H, 128, 128) > w.B * w.H * nc * (REC + SIG)
+    la = oracle.log_decay(inp["z"], w.g_min)
+    ld = torch.from_numpy(np.ascontiguousarray(la, dtype=np.float32)).cuda()
+    o_ref, s_ref = oracle.recurrence(inp["q"], inp["k"], inp["v"], inp["beta"], z=inp["z"], g_min=w.g_min,
+                                     initial_state=inp["S0"])
+    # precomputed log-decay (fp32) instead of z
+    o, sf = K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], log_decay=ld, g_min=w.g_min,
+                        initial_state=d["S0"], engine="tc")
+    torch.cuda.synchronize()
+    assert _timeouts(K) == 0
+    assert_bf16_outputs(to_np(o), o_ref, "o~ (log-decay input)")
+    assert_bf16_state(to_np(sf), s_ref, "final_state (log-decay input)")
+    # split-sequence handoff in place, with the fused gate; each part is long enough to be segmented
+    st = d["S0"].clone()
+    outs = []
+    for a, b in ((0, 640), (640, 1536)):
+        sl = lambda t: t[:, a:b].contiguous()
+        og, _ = K.chunk_fwd(sl(d["q"]), sl(d["k"]), sl(d["v"]), sl(d["beta"]), z=sl(d["z"]), initial_state=st,
+                            final_state=st, gate_logits=sl(d["gate"]), eps=w.eps, engine="tc")
+        outs.append(og)
+    torch.cuda.synchronize()
+    assert _timeouts(K) == 0
+    # the tolerance is stated on the layer output: project the normalised, gated rows (a row whose
+    # o~ has a small norm is amplified by the normalisation, and the projection averages it)
+    x = torch.cat(outs, 1).reshape(w.B * w.S, w.H * w.Dv)
+    y = K.out_proj(x, d["W_o"])
+    want = oracle.project(oracle.norm_gate(o_ref, inp["gate"], w.eps), inp["W_o"])
+    assert_bf16_outputs(to_np(y).reshape(want.shape), want, "layer outputs (handoff)")
+    assert_bf16_state(to_np(st), s_ref, "final_state (handoff)")
+
+
 def test_tc_layer_with_fused_gate(K):
     w = ki.custom("lay", 2, 500, 4, 128, 128, 256, "bf16", seed=77)
     inp = ki.make_inputs(w)
