@@ -47,8 +47,10 @@ REF_SAMPLE_TOKENS = 512   # tokens (all heads) per reference-arm step
 # the committed ncu summaries under profiles/, keyed by kernel and workload,
 # valid only while the kernel's source file is unchanged (sha256 prefix).
 NCU_TRAFFIC = {
-    # prefill_4k_chunk_engine.md: prep 130.7 + segment maps 64.2 + combine 6.3 + segment chains 102.5 MB
-    "chunk_engine@prefill_4k": {"bytes": 303637760, "src_sha": "100718e5c32d9d72"},
+    # prefill_4k_chunk_engine.md: prep 126.5 + segment maps 41.5 + combine 6.3 + segment chains 103.3 MB
+    "chunk_engine@prefill_4k": {"bytes": 277645824, "src_sha": "5d03b3c2324a1d10"},
+    # decode_256_step.md: decode128_stream_kernel, 547.4 MB read + 479.8 MB written
+    "decode@decode_256": {"bytes": 1027173120, "src_sha": "079db3bd726bd665"},
 }
 
 
@@ -207,6 +209,9 @@ def run_ours(args, rank, world, local):
     init_dist(world, "nccl")
     lib = K.load_library()
     peaks, peak_src = load_peaks()
+    if args.only == "decode":
+        dec = run_decode(args, rank, world, local, K, dev, peaks)
+        return {"metric": METRIC, "decode": dec, "n_gpus": world} if rank == 0 else None
 
     # ---------------- prefill inputs, resident in HBM
     w = rank_workload(PREFILL, rank)
@@ -256,9 +261,6 @@ def run_ours(args, rank, world, local):
     t_step = t_chunk + t_proj
     t_step_max, t_chunk_max, t_proj_max = reduce_max([t_step, t_chunk, t_proj], world, dev)
 
-    if args.only == "decode":
-        dec = run_decode(args, rank, world, local, K, dev, peaks)
-        return {"metric": METRIC, "decode": dec, "n_gpus": world} if rank == 0 else None
     if args.only == "prefill":
         return {"metric": METRIC, "value": round(N * world / t_step_max, 1), "unit": "tokens/s",
                 "kernels_ms": {"chunk_engine": round(t_chunk * 1e3, 4), "out_proj": round(t_proj * 1e3, 4)},
