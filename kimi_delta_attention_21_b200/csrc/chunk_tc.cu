@@ -13,17 +13,19 @@
 //   O      = (Q * e^G) S + M V'        (o_t = S_t^T q_t, read after the update)
 //   S     <- Diag(e^{G_C}) S + (K * e^{G_C - G})^T V'
 //
-// Two kernels:
-//  * chunk_prep_kernel, one CTA per (chunk, head, batch), all chunks in
-//    parallel: TMA loads of q, k, v, z; the cumulative log-decay; decay-scaled
-//    operands; A^T and M^T on tcgen05; the blocked inverse T in fp32 SIMT;
-//    [W | U] = T [beta K e^G | beta V] on tcgen05.  It writes one workspace
-//    record per chunk holding Q*e^G, K*e^{G_C-G}, W and M^T as ready-made
-//    128-byte-swizzled shared-memory images, U split by value-column slice,
-//    and e^{G_C}.
-//  * chunk_state_kernel, one CTA per (value-column slice, head, batch), walks
-//    the chunks in order with the state slice resident in TMEM, streaming the
-//    records with bulk copies (two stages), and writes o~ and the final state.
+// Kernels:
+//  * chunk_prep_kernel, persistent (one CTA per SM walks the (chunk, head,
+//    batch) units; all chunks are independent): TMA loads of q, k, v; the
+//    cumulative log-decay (from z or the log-decay input, read directly);
+//    decay-scaled operands; A^T and M^T on tcgen05; the inverse T in fp32 SIMT;
+//    [W | U^T] = T [beta K e^G | beta V] on tcgen05; the sigmoid of the output
+//    gate.  It writes one workspace record per chunk holding [-W; Q*e^G],
+//    K*e^{G_C-G}, M^T and U^T as ready-made 128-byte-swizzled shared-memory
+//    images, and e^{G_C}.
+//  * chunk_state_kernel, one CTA per (head, batch, segment of the sequence),
+//    walks the chunks in order with the state resident in TMEM, streaming the
+//    records with bulk copies, and writes the gated, normalised output and
+//    the final state; chunk_combine_kernel chains the segments (below).
 //
 // Decay factors as GEMM operands.  exp(G_r - G_i) is split into a row factor
 // and a column factor around a reference point.  G spans up to |g_min| * 64
@@ -127,6 +129,10 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
 
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
 __device__ __forceinline__ void report_timeout(unsigned int *timeouts, int *dev_status) {
     if (timeouts) atomicAdd(timeouts, 1u);
     if (dev_status) atomicExch(dev_status, (int)KDA_ERR_TIMEOUT);
@@ -134,29 +140,32 @@ __device__ __forceinline__ void report_timeout(unsigned int *timeouts, int *dev_
 
 // ================================================================ K2a: chunk_prep_kernel
 // Persistent: one CTA per SM walks (chunk, head, batch) units.  The next unit's
-// q and k tiles are loaded by TMA as soon as this unit's copies of them are
-// dead (after the A/M MMAs), z and v after the W/U MMAs, and the workspace
-// bulk stores drain while the next unit is computed.
+// q and k tiles are loaded by TMA as soon as the record stores have read this
+// unit's copies (while the A/M MMAs run), its z tile once the A/M MMAs have
+// read their operands, v after the W/U MMAs; the workspace bulk stores drain
+// while the next unit is computed.
 // Shared-memory map (bytes from a 1024-aligned base).
 constexpr uint32_t P_QI = 0;         // q image; becomes Q e^G (stored as soon as P2 ends)
 constexpr uint32_t P_KI = 16384;     // k image; becomes K e^{G_C - G}
 constexpr uint32_t P_VI = 32768;     // v image; becomes beta V (operand of the W and U^T MMAs)
-constexpr uint32_t P_ZI = 49152;     // z image; becomes beta K e^G (MN-major B operand of the W MMA)
+constexpr uint32_t P_ZI = 49152;     // beta K e^G (MN-major B operand of the W MMA)
 constexpr uint32_t P_A = 65536;      // A operand of the A/M MMAs [2 atoms][224 rows][128 B]: the column operand
                                      // in its 4 block versions (rows 0-159) and the low part of the diagonal
                                      // one (rows 160-223); later -W, U^T and the M^T image
 constexpr uint32_t P_B = 122880;     // B operand [2 atoms][192 rows][128 B]: row operands from k, q and the low
                                      // part of the q one; later the T image and the diagonal residues
 constexpr uint32_t P_SG = 172032;    // G fp32 [64][132]; later A [64][65] and T [64][68] fp32
-constexpr uint32_t P_TAB = 206080;   // per-channel block constants [26][128] fp32
-constexpr uint32_t P_XS = 219392;    // scratch for the blocked inverse [3][256] fp32
+constexpr uint32_t P_TAB = 206080;   // per-channel block constants [26][128] fp32; then inverse scratch
+constexpr uint32_t P_XS = 219392;    // quarter sums of the cumulative log-decay [4][128] fp32
 constexpr uint32_t P_BETA = 222464;  // beta [64] fp32
 constexpr uint32_t P_GAM = 222720;   // e^{G_C} [128] fp32
-constexpr uint32_t P_BAR = 223232;   // 3 mbarriers + TMEM slot
+constexpr uint32_t P_BAR = 223232;   // mbarriers: inputs, A/M MMAs, W/U MMAs; TMEM slot (+24); z tile (+32)
 constexpr uint32_t P_END = 223312;
 constexpr size_t PREP_SMEM = P_END + 1024;
 constexpr uint32_t P_RH = P_ZI;
 constexpr uint32_t P_WI = P_A, P_UI = P_A + 16384, P_MT = P_A + 32768;
+constexpr uint32_t P_ZT = P_A + 40960;  // the next unit's z tile [2 atoms][64 rows][128 B], between the A/M MMAs
+                                        // and the next unit's P2 (nothing else uses these 16 KB then)
 constexpr uint32_t P_TI = P_B, P_LOHI = P_B + 8192;  // LOHI: [64][16] fp32
 constexpr uint32_t P_SA = P_SG, P_ST = P_SG + 16640;
 constexpr int SG_LD = 132, SA_LD = 65, ST_LD = 68;
@@ -196,11 +205,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     uint64_t *bar_am = bar_in + 1;
     uint64_t *bar_wu = bar_in + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + P_BAR + 24);
+    uint64_t *bar_z = reinterpret_cast<uint64_t *>(sm + P_BAR + 32);
     float *sG = reinterpret_cast<float *>(sm + P_SG);
     float *tab = reinterpret_cast<float *>(sm + P_TAB);
     float *sbeta = reinterpret_cast<float *>(sm + P_BETA);
     float *sgam = reinterpret_cast<float *>(sm + P_GAM);
-    const uint32_t in_bytes = (p.log_decay ? 6u : 8u) * 8192u;
+    const uint32_t in_bytes = 6u * 8192u;  // q, k, v
 
     auto unit_coords = [&](int64_t u, int &n, int &h, int &b) {
         n = (int)(u % p.Nc);
@@ -217,30 +227,38 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             tma_load_4d(sm + P_KI + a * 8192, &tk, bar_in, 64 * a, h, n * CH, b);
         }
     };
-    auto load_zv = [&](int64_t u) {
+    auto load_z = [&](int64_t u) {  // z tile of unit u -> P_ZT (bf16 decay logits only)
         int n, h, b;
         unit_coords(u, n, h, b);
-        for (int a = 0; a < 2; ++a) {
-            if (!p.log_decay) tma_load_4d(sm + P_ZI + a * 8192, &tz, bar_in, 64 * a, h, n * CH, b);
-            tma_load_4d(sm + P_VI + a * 8192, &tv, bar_in, 64 * a, h, n * CH, b);
-        }
+        mbar_arrive_expect_tx(bar_z, 16384u);
+        for (int a = 0; a < 2; ++a) tma_load_4d(sm + P_ZT + a * 8192, &tz, bar_z, 64 * a, h, n * CH, b);
+    };
+    auto load_v = [&](int64_t u) {
+        int n, h, b;
+        unit_coords(u, n, h, b);
+        for (int a = 0; a < 2; ++a) tma_load_4d(sm + P_VI + a * 8192, &tv, bar_in, 64 * a, h, n * CH, b);
     };
 
     // sigmoid of the output-gate logits (full fp32, stored as f16) for the state kernel's output stage,
-    // in its tile layout [2 atoms (j / 64)][64 rows r][128 B], 128-byte swizzled: one row x 16 value
-    // columns per thread
+    // in its tile layout [2 atoms (j / 64)][64 rows r][128 B], 128-byte swizzled.  Warps 4-15 take the
+    // 1024 groups of 8 values while warps 0-3 invert (I + A); the logits were prefetched into L2 one
+    // unit ahead.
+    constexpr int SIG_T = PREP_THREADS - 128;
     auto gate_sigmoid = [&](int n, int h, int b, int t0, int len) {
-        const int row = tid >> 3, c0 = 16 * (tid & 7);
-        if (!p.gate || row >= len) return;
-        const uint4 *src =
-            reinterpret_cast<const uint4 *>(p.gate + (((int64_t)b * p.S + t0 + row) * p.H + h) * DD + c0);
-        uint8_t *dst = reinterpret_cast<uint8_t *>(p.sig + ((size_t)(b * p.H + h) * p.Nc + n) * (CH * DD)) +
-                       (c0 >> 6) * 8192;
-        uint4 gv[2];
+        if (!p.gate || tid < 128) return;
+        const __nv_bfloat16 *src = p.gate + (((int64_t)b * p.S + t0) * p.H + h) * DD;
+        uint8_t *dst = reinterpret_cast<uint8_t *>(p.sig + ((size_t)(b * p.H + h) * p.Nc + n) * (CH * DD));
+        uint4 gv[3] = {};
 #pragma unroll
-        for (int k = 0; k < 2; ++k) gv[k] = src[k];
+        for (int k = 0; k < 3; ++k) {
+            const int gi = tid - 128 + SIG_T * k, row = gi >> 4;
+            if (gi < CH * DD / 8 && row < len)
+                gv[k] = *reinterpret_cast<const uint4 *>(src + (int64_t)row * p.H * DD + (gi & 15) * 8);
+        }
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
+        for (int k = 0; k < 3; ++k) {
+            const int gi = tid - 128 + SIG_T * k, row = gi >> 4, c8 = (gi & 15) * 8;
+            if (gi >= CH * DD / 8 || row >= len) continue;
             float g[8];
             unpack8(gv[k], g);
             uint4 o;
@@ -249,59 +267,41 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             for (int e = 0; e < 4; ++e)
                 oh[e] = __floats2half2_rn(__fdividef(1.0f, 1.0f + __expf(-g[2 * e])),
                                           __fdividef(1.0f, 1.0f + __expf(-g[2 * e + 1])));
-            *reinterpret_cast<uint4 *>(dst + sw128(row, (c0 & 63) / 8 + k)) = o;
+            *reinterpret_cast<uint4 *>(dst + (c8 >> 6) * 8192 + sw128(row, (c8 & 63) >> 3)) = o;
         }
     };
 
-    if (tid == 0) {
-        mbar_init(bar_in, 1);
-        mbar_init(bar_am, 1);
-        mbar_init(bar_wu, 1);
-        fence_barrier_init();
-        if ((int64_t)blockIdx.x < p.units) {
-            load_qk(blockIdx.x);
-            load_zv(blockIdx.x);
-        }
-    }
-    if (warp == 0) {
-        tmem_alloc(tmem_slot, 512);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = *tmem_slot;
-    bool ok = true;
-
-    int it = 0;
-    for (int64_t u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++it) {
+    // P1 and the per-channel tables of unit u: beta, G = in-chunk cumulative log-decay (rows past the
+    // sequence end: no decay, beta 0), the block constants and e^{G_C}.  The decay input is z (the tile
+    // at P_ZT, loaded one unit ahead, landed on bar_z with parity zpar) or the log-decay (read from
+    // global memory, prefetched into L2 one unit ahead); beta_row is row tid's beta, loaded one unit
+    // ahead.  Called by all threads; returns false if the z tile never landed.
+    auto load_beta = [&](int64_t u) -> float {  // beta of row tid (< 64) of unit u; 0 past the end
         int n, h, b;
         unit_coords(u, n, h, b);
         const int t0 = n * CH;
-        const int len = min(CH, p.S - t0);
-        const int64_t u_next = u + gridDim.x;
-        const uint32_t par = it & 1;
-        // the previous unit's bulk stores must have read their shared sources
-        if (tid == 0) bulk_wait_read_all();
-        if (tid < CH)
-            sbeta[tid] = (tid < len) ? __bfloat162float(p.beta[((int64_t)b * p.S + t0 + tid) * p.H + h]) : 0.f;
-        ok = mbar_wait(bar_in, par);
-        ok = __syncthreads_and(ok);
-        if (!ok) break;
-
-        // ---------------- P1: G = in-chunk cumulative log-decay (rows past the sequence end: no decay)
-        {   // one thread per channel c and 16 rows (quarter qt); quarter sums through the inverse scratch
+        return (t0 + tid < p.S) ? __bfloat162float(p.beta[((int64_t)b * p.S + t0 + tid) * p.H + h]) : 0.f;
+    };
+    auto decay_tables = [&](int64_t u, uint32_t zpar, float beta_row) -> bool {
+        int n, h, b;
+        unit_coords(u, n, h, b);
+        const int t0 = n * CH, len = min(CH, p.S - t0);
+        bool landed = true;
+        if (tid < CH) sbeta[tid] = beta_row;
+        {   // one thread per channel c and 16 rows (quarter qt); quarter sums through a scratch
             const int c = tid & 127, qt = tid >> 7;
             float *qsum = reinterpret_cast<float *>(sm + P_XS);
+            const int64_t i0 = (((int64_t)b * p.S + t0) * p.H + h) * DD + c, rstr = (int64_t)p.H * DD;
             float g[16];
             if (p.log_decay) {
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr) {
                     const int r = qt * 16 + rr;
-                    g[rr] = (r < len) ? p.log_decay[(((int64_t)b * p.S + t0 + r) * p.H + h) * DD + c] : 0.f;
+                    g[rr] = (r < len) ? p.log_decay[i0 + r * rstr] : 0.f;
                 }
             } else {
-                const uint8_t *zc = sm + P_ZI + (c >> 6) * 8192 + (c & 7) * 2;
+                if (!mbar_wait(bar_z, zpar)) landed = false;
+                const uint8_t *zc = sm + P_ZT + (c >> 6) * 8192 + (c & 7) * 2;
                 const uint32_t ch = (c & 63) >> 3;
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr) {
@@ -324,8 +324,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             for (int rr = 0; rr < 16; ++rr) sG[(qt * 16 + rr) * SG_LD + c] = g[rr] + base;
         }
         __syncthreads();
-        // ---------------- per-channel block constants
-        if (tid < 128) {
+        if (tid < 128) {  // per-channel block constants
             const int c = tid;
             float bb[4], mm[4];
 #pragma unroll
@@ -347,15 +346,74 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 for (int R = 0; R <= V; ++R) tab[tab_c(V, R) * 128 + c] = fexp(mm[V] - bb[R]);
             sgam[c] = fexp(bb[3]);
         }
-        __syncthreads();
-        // ---------------- P2: decay-scaled operands (one thread per row r and 2 chunks of 8 channels)
+        return landed;
+    };
+
+    if (tid == 0) {
+        mbar_init(bar_in, 1);
+        mbar_init(bar_am, 1);
+        mbar_init(bar_wu, 1);
+        mbar_init(bar_z, 1);
+        fence_barrier_init();
+        if ((int64_t)blockIdx.x < p.units) {
+            load_qk(blockIdx.x);
+            load_v(blockIdx.x);
+            if (!p.log_decay) load_z(blockIdx.x);
+        }
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = true;
+    float beta_cur = (tid < CH && (int64_t)blockIdx.x < p.units) ? load_beta(blockIdx.x) : 0.f;
+
+    int it = 0;
+    for (int64_t u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++it) {
+        int n, h, b;
+        unit_coords(u, n, h, b);
+        const int t0 = n * CH;
+        const int len = min(CH, p.S - t0);
+        const int64_t u_next = u + gridDim.x;
+        const uint32_t par = it & 1;
+        // the next unit's beta, consumed by its tables (issued now, so its latency stays hidden)
+        const float beta_next = (tid < CH && u_next < p.units) ? load_beta(u_next) : 0.f;
+        if (u_next < p.units && tid < 256) {  // the next unit's gate and log-decay inputs -> L2
+            int n2, h2, b2;
+            unit_coords(u_next, n2, h2, b2);
+            const int64_t row0 = ((int64_t)b2 * p.S + n2 * CH) * p.H + h2;
+            if (tid < 128) {
+                const int row = tid >> 1;
+                if (p.gate && n2 * CH + row < p.S)
+                    prefetch_l2(p.gate + (row0 + (int64_t)row * p.H) * DD + (tid & 1) * 64);
+            }
+            const int row = tid >> 2;
+            if (p.log_decay && n2 * CH + row < p.S)
+                prefetch_l2(p.log_decay + (row0 + (int64_t)row * p.H) * DD + (tid & 3) * 32);
+        }
+        // the previous unit's bulk stores must have read their shared sources
+        if (tid == 0) bulk_wait_read_all();
+        // the decay and tables need neither q, k nor v: they run while v is still landing
+        ok = decay_tables(u, par, beta_cur);
+        beta_cur = beta_next;
+        ok = mbar_wait(bar_in, par) && ok;
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
+
+        // ---------------- P2: decay-scaled operands.  A thread takes one row and 8 channels in block R0 =
+        // warp % 4 and one in block 3 - R0, so that every warp writes 4 - R0 + 1 + R0 = 5 block versions
+        // of the column operand (and no warp diverges on the version count).
         {
-            const int r = tid & 63, grp = tid >> 6, R = r >> 4;
-            const float beta_r = sbeta[r];
+            const int R0 = warp & 3, jj = 2 * (warp >> 2) + (lane >> 4);
 #pragma unroll 1
             for (int mi = 0; mi < 2; ++mi) {
-                const int j = grp + 8 * mi;
-                const int atom = j >> 3, jj = j & 7, c0 = 8 * j;
+                const int R = mi ? 3 - R0 : R0, r = 16 * R + (lane & 15);
+                const float beta_r = sbeta[r];
+                const int j = jj + 8 * mi, atom = mi, c0 = 8 * j;
                 const uint32_t img = atom * 8192 + sw128(r, jj);
                 const uint32_t bimg = P_B + atom * B_ATOM, aimg = P_A + atom * A_ATOM;
                 float qv[8], kv[8], vv[8], G[8], bR[8], bRm1[8], F[8], E[8], Dd[8];
@@ -427,14 +485,18 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         __syncthreads();
 
         uint8_t *rec = p.ws + ((size_t)(b * p.H + h) * p.Nc + n) * REC_BYTES;
-        // ---------------- Q e^G and K e^{G_C - G} leave now; tcgen05: A^T (cols 0-63), M^T (64-127),
-        // residues of M's diagonal blocks (128-191)
-        if (tid == 0) {
+        // ---------------- tcgen05: A^T (cols 0-63), M^T (64-127), residues of M's diagonal blocks (128-191);
+        // meanwhile Q e^G, K e^{G_C - G} and e^{G_C} leave (thread 96; once the stores have read them,
+        // during P3, the next unit's q and k tiles take their place: they are not operands of these MMAs)
+        if (tid == 96) {
             // Q e^G fills rows 64-127 of each atom of the stacked [W; Q e^G] image
             bulk_store(rec + REC_WQ + 8192, sm + P_QI, 8192);
             bulk_store(rec + REC_WQ + 16384 + 8192, sm + P_QI + 8192, 8192);
             bulk_store(rec + REC_KT, sm + P_KI, 16384);
+            bulk_store(rec + REC_GAM, sgam, 512);
             bulk_commit();
+        }
+        if (tid == 0) {
             tc_fence_after();
             // all block versions at once: D1 = rows 0-127 of the A operand, D2 = rows 96-223 (version 3 and
             // the low part of the diagonal operand), each against [k rows | q rows | low q rows]; every
@@ -450,16 +512,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             }
             mma_commit(bar_am);
         }
-        // while the MMAs run: the sigmoid of the output-gate logits
-        gate_sigmoid(n, h, b, t0, len);
         ok = mbar_wait(bar_am, par);
         ok = __syncthreads_and(ok);
         tc_fence_after();
         if (!ok) break;
-        // q and k images are dead (their stores have read them once the group drains): prefetch
-        if (tid == 0 && u_next < p.units) {
+        if (tid == 0 && !p.log_decay && u_next < p.units) load_z(u_next);  // the A/M MMAs have read P_A
+        if (tid == 96) {
             bulk_wait_read_all();
-            load_qk(u_next);
+            if (u_next < p.units) load_qk(u_next);
         }
 
         // ---------------- P3: A (masked, beta-weighted, fp32) and the M^T image.
@@ -545,14 +605,15 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         tc_fence_before();
         __syncthreads();
 
-        // ---------------- P4: T = (I + A)^{-1} by blocks of 16 (fp32)
-        {
+        // ---------------- P4: T = (I + A)^{-1} (fp32) by block doubling: the four diagonal 16x16 blocks by
+        // forward substitution, then T_{R,R-1} = -T_RR A_{R,R-1} T_{R-1,R-1} for R = 1, 3, then the lower-left
+        // 32x32 block the same way from the two diagonal 32x32 blocks.  Blocks above the diagonal are written
+        // as zeros where a later product reads them; the T image zero-fills the upper-right 32x32 block.
+        // Warps 0-3 only (named barrier 1); warps 4-15 compute the gate sigmoid meanwhile.
+        if (warp < 4) {
             const float *sA = reinterpret_cast<const float *>(sm + P_SA);
             float *sT = reinterpret_cast<float *>(sm + P_ST);
-            float *xs = reinterpret_cast<float *>(sm + P_XS);
-            for (int e = tid; e < 64 * ST_LD / 4; e += PREP_THREADS)
-                reinterpret_cast<float4 *>(sT)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-            __syncthreads();
+            float *xs = reinterpret_cast<float *>(sm + P_TAB);  // the tables are dead after P2
             if (tid < 64) {  // diagonal block R, column jc: forward substitution
                 const int R = tid >> 4, jc = tid & 15, o = 16 * R;
                 float col[16];
@@ -567,50 +628,89 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
 #pragma unroll
                 for (int a = 0; a < 16; ++a) sT[(o + a) * ST_LD + o + jc] = col[a];
             }
-            __syncthreads();
-            // blocks below the diagonal, one distance d = R - I at a time, 4 columns per thread:
-            //   X = A[16R+a, 16I:16R] T[16I:16R, 16I+bc..+3],  T_RI = -T_RR X
+            named_sync(1, 128);
+            // The products below give each thread rows (p, p + h) and four adjacent columns, so that one
+            // float4 of the right operand feeds eight FMAs (shared-memory wavefronts, not FMAs, bound them).
+            if (tid < 64) {  // 16 -> 32: X = A_{R,R-1} T_{R-1,R-1}, R = 1 + 2 hb
+                const int hb = tid >> 5, R = 1 + 2 * hb, pr = (tid >> 2) & 7, c4 = 4 * (tid & 3), o = 16 * (R - 1);
+                const float *a0 = sA + (16 * R + pr) * SA_LD + o, *a1 = a0 + 8 * SA_LD;
+                const float *tb = sT + o * ST_LD + o + c4;
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
 #pragma unroll
-            for (int d = 1; d < 4; ++d) {
-                const int e = tid;
-                const bool act = e < (4 - d) * 64;
-                const int blk = e >> 6, R = d + blk, I = R - d, a = (e >> 2) & 15, bc = (e & 3) * 4;
-                if (act) {
-                    const float *arow = sA + (16 * R + a) * SA_LD + 16 * I;
-                    const float *tblk = sT + 16 * I * ST_LD + 16 * I + bc;
-                    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                    for (int k = 0; k < 16 * d; ++k) {
-                        const float av = arow[k];
-                        const float4 tv = *reinterpret_cast<const float4 *>(tblk + k * ST_LD);
-                        x.x += av * tv.x; x.y += av * tv.y; x.z += av * tv.z; x.w += av * tv.w;
-                    }
-                    *reinterpret_cast<float4 *>(xs + blk * 256 + a * 16 + bc) = x;
+                for (int m = 0; m < 16; ++m) {
+                    const float u = a0[m], v = a1[m];
+                    const float4 t = *reinterpret_cast<const float4 *>(tb + m * ST_LD);
+                    x.x += u * t.x; x.y += u * t.y; x.z += u * t.z; x.w += u * t.w;
+                    y.x += v * t.x; y.y += v * t.y; y.z += v * t.z; y.w += v * t.w;
                 }
-                __syncthreads();
-                if (act) {
-                    const float *trow = sT + (16 * R + a) * ST_LD + 16 * R;
-                    const float *xb = xs + blk * 256 + bc;
-                    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                    for (int m = 0; m < 16; ++m) {
-                        const float tv = trow[m];  // zero above the diagonal
-                        const float4 xv = *reinterpret_cast<const float4 *>(xb + m * 16);
-                        y.x += tv * xv.x; y.y += tv * xv.y; y.z += tv * xv.z; y.w += tv * xv.w;
-                    }
-                    *reinterpret_cast<float4 *>(sT + (16 * R + a) * ST_LD + 16 * I + bc) =
-                        make_float4(-y.x, -y.y, -y.z, -y.w);
-                }
-                __syncthreads();
+                *reinterpret_cast<float4 *>(xs + hb * 256 + pr * 16 + c4) = x;
+                *reinterpret_cast<float4 *>(xs + hb * 256 + (pr + 8) * 16 + c4) = y;
             }
-            {  // T image (K-major, 64 rows x 64 cols), one 8-column chunk per thread
-                const int r = tid >> 3, cc = tid & 7;
-                float t[8];
+            named_sync(1, 128);
+            if (tid < 64) {  //       T_{R,R-1} = -T_RR X  (T_RR is zero above its diagonal); zero block (R-1, R)
+                const int hb = tid >> 5, R = 1 + 2 * hb, pr = (tid >> 2) & 7, c4 = 4 * (tid & 3);
+                const float *t0 = sT + (16 * R + pr) * ST_LD + 16 * R, *t1 = t0 + 8 * ST_LD;
+                const float *xb = xs + hb * 256 + c4;
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) t[e] = sT[r * ST_LD + 8 * cc + e];
+                for (int m = 0; m < 16; ++m) {
+                    const float u = t0[m], v = t1[m];
+                    const float4 t = *reinterpret_cast<const float4 *>(xb + m * 16);
+                    x.x += u * t.x; x.y += u * t.y; x.z += u * t.z; x.w += u * t.w;
+                    y.x += v * t.x; y.y += v * t.y; y.z += v * t.z; y.w += v * t.w;
+                }
+                float *d0 = sT + (16 * R + pr) * ST_LD + 16 * (R - 1) + c4;
+                *reinterpret_cast<float4 *>(d0) = make_float4(-x.x, -x.y, -x.z, -x.w);
+                *reinterpret_cast<float4 *>(d0 + 8 * ST_LD) = make_float4(-y.x, -y.y, -y.z, -y.w);
+                float *z0 = sT + (16 * (R - 1) + pr) * ST_LD + 16 * R + c4;
+                *reinterpret_cast<float4 *>(z0) = make_float4(0.f, 0.f, 0.f, 0.f);
+                *reinterpret_cast<float4 *>(z0 + 8 * ST_LD) = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            named_sync(1, 128);
+            if (tid < 128) {  // 32 -> 64: X = A[32:64, 0:32] T[0:32, 0:32]
+                const int pr = tid >> 3, c4 = 4 * (tid & 7);
+                const float *a0 = sA + (32 + pr) * SA_LD, *a1 = a0 + 16 * SA_LD;
+                const float *tb = sT + c4;
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
+#pragma unroll
+                for (int m = 0; m < 32; ++m) {
+                    const float u = a0[m], v = a1[m];
+                    const float4 t = *reinterpret_cast<const float4 *>(tb + m * ST_LD);
+                    x.x += u * t.x; x.y += u * t.y; x.z += u * t.z; x.w += u * t.w;
+                    y.x += v * t.x; y.y += v * t.y; y.z += v * t.z; y.w += v * t.w;
+                }
+                *reinterpret_cast<float4 *>(xs + pr * 32 + c4) = x;
+                *reinterpret_cast<float4 *>(xs + (pr + 16) * 32 + c4) = y;
+            }
+            named_sync(1, 128);
+            if (tid < 128) {  //       T[32:64, 0:32] = -T[32:64, 32:64] X
+                const int pr = tid >> 3, c4 = 4 * (tid & 7);
+                const float *t0 = sT + (32 + pr) * ST_LD + 32, *t1 = t0 + 16 * ST_LD;
+                const float *xb = xs + c4;
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
+#pragma unroll
+                for (int m = 0; m < 32; ++m) {
+                    const float u = t0[m], v = t1[m];
+                    const float4 t = *reinterpret_cast<const float4 *>(xb + m * 32);
+                    x.x += u * t.x; x.y += u * t.y; x.z += u * t.z; x.w += u * t.w;
+                    y.x += v * t.x; y.y += v * t.y; y.z += v * t.z; y.w += v * t.w;
+                }
+                float *d0 = sT + (32 + pr) * ST_LD + c4;
+                *reinterpret_cast<float4 *>(d0) = make_float4(-x.x, -x.y, -x.z, -x.w);
+                *reinterpret_cast<float4 *>(d0 + 16 * ST_LD) = make_float4(-y.x, -y.y, -y.z, -y.w);
+            }
+            named_sync(1, 128);
+            for (int k = 0; k < 4; ++k) {  // T image (K-major, 64 rows x 64 cols), 8-column chunks
+                const int r = (tid >> 3) + 16 * k, cc = tid & 7;
+                float t[8];
+                const bool upper = r < 32 && cc >= 4;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) t[e] = upper ? 0.f : sT[r * ST_LD + 8 * cc + e];
                 *reinterpret_cast<uint4 *>(sm + P_TI + sw128(r, cc)) = pack8(t);
             }
             fence_proxy_async_smem();
+        } else {
+            gate_sigmoid(n, h, b, t0, len);
         }
         tc_fence_before();
         __syncthreads();
@@ -631,11 +731,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             }
             mma_commit(bar_wu);
         }
-        ok = mbar_wait(bar_wu, par);
+        ok = mbar_wait(bar_wu, par) && ok;
         ok = __syncthreads_and(ok);
         tc_fence_after();
         if (!ok) break;
-        if (tid == 0 && u_next < p.units) load_zv(u_next);  // beta K e^G and beta V have been consumed
+        if (tid == 0 && u_next < p.units) load_v(u_next);  // beta K e^G and beta V have been consumed
 
         // ---------------- P5: -W image (warp groups 0 and 2: M = 64 accumulator rows, half the columns
         // each) and U^T image (warp groups 1 and 3: one value column j per lane, half the rows each)
@@ -681,15 +781,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             bulk_store(rec + REC_WQ + 16384, sm + P_WI + 8192, 8192);
             bulk_store(rec + REC_MT, sm + P_MT, 8192);
             bulk_store(rec + REC_U, sm + P_UI, 16384);
-            bulk_store(rec + REC_GAM, sgam, 512);
             bulk_commit();
         }
     }
 
-    if (tid == 0) {
-        bulk_wait_all();
-        if (!ok) report_timeout(p.timeouts, p.dev_status);
-    }
+    if (tid == 0 || tid == 96) bulk_wait_all();
+    if (tid == 0 && !ok) report_timeout(p.timeouts, p.dev_status);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 512);
@@ -746,10 +843,6 @@ constexpr uint32_t T_S16 = 128;   // S^T bf16 pairs (A operand, K = c)
 constexpr uint32_t T_PO = 192;    // two [128][128] accumulators
 constexpr uint32_t T_V16 = 448;   // V'^T bf16 pairs (A operand, K = r)
 constexpr uint32_t ST_TCOLS = 512;
-
-__device__ __forceinline__ void named_sync(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 // kMap = false: the chain over segment blockIdx.z from its entering state, with outputs.
 // kMap = true:  the map of segment blockIdx.z / 2 over its chunks, S_end = A_g S_start + Y_g:
