@@ -212,11 +212,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     float *sgam = reinterpret_cast<float *>(sm + P_GAM);
     const uint32_t in_bytes = 6u * 8192u;  // q, k, v
 
-    auto unit_coords = [&](int64_t u, int &n, int &h, int &b) {
-        n = (int)(u % p.Nc);
-        const int64_t bh = u / p.Nc;
-        h = (int)(bh % p.H);
-        b = (int)(bh / p.H);
+    auto unit_coords = [&](int64_t u, int &n, int &h, int &b) {  // 32-bit: units < 2^31 (host check)
+        const uint32_t uu = (uint32_t)u, nc = (uint32_t)p.Nc, hh = (uint32_t)p.H;
+        const uint32_t bh = uu / nc;
+        n = (int)(uu - bh * nc);
+        b = (int)(bh / hh);
+        h = (int)(bh - (uint32_t)b * hh);
     };
     auto load_qk = [&](int64_t u) {  // arms bar_in for the whole unit
         int n, h, b;
@@ -324,27 +325,36 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             for (int rr = 0; rr < 16; ++rr) sG[(qt * 16 + rr) * SG_LD + c] = g[rr] + base;
         }
         __syncthreads();
-        if (tid < 128) {  // per-channel block constants
-            const int c = tid;
+        {  // per-channel block constants, four threads per channel (8, 6, 5 and 4 exponentials)
+            const int c = tid & 127, part = tid >> 7;
             float bb[4], mm[4];
 #pragma unroll
             for (int R = 0; R < 4; ++R) {
                 bb[R] = sG[(16 * R + 15) * SG_LD + c];
                 mm[R] = sG[(16 * R + 7) * SG_LD + c];
             }
+            if (part == 0) {
 #pragma unroll
-            for (int R = 0; R < 4; ++R) {
-                const float bm1 = R ? bb[R - 1] : 0.f;
-                tab[R * 128 + c] = bb[R];
-                tab[(4 + R) * 128 + c] = fexp(bm1 - mm[R]);
-                tab[(8 + R) * 128 + c] = fexp(bm1);
-                tab[(12 + R) * 128 + c] = fexp(bb[3] - bb[R]);
+                for (int R = 0; R < 4; ++R) {
+                    const float bm1 = R ? bb[R - 1] : 0.f;
+                    tab[R * 128 + c] = bb[R];
+                    tab[(4 + R) * 128 + c] = fexp(bm1 - mm[R]);
+                    tab[(8 + R) * 128 + c] = fexp(bm1);
+                }
+            } else if (part == 1) {
+#pragma unroll
+                for (int R = 0; R < 4; ++R) tab[(12 + R) * 128 + c] = fexp(bb[3] - bb[R]);
+                tab[tab_c(0, 0) * 128 + c] = fexp(mm[0] - bb[0]);
+                sgam[c] = fexp(bb[3]);
+            } else if (part == 2) {
+#pragma unroll
+                for (int R = 0; R <= 1; ++R) tab[tab_c(1, R) * 128 + c] = fexp(mm[1] - bb[R]);
+#pragma unroll
+                for (int R = 0; R <= 2; ++R) tab[tab_c(2, R) * 128 + c] = fexp(mm[2] - bb[R]);
+            } else {
+#pragma unroll
+                for (int R = 0; R <= 3; ++R) tab[tab_c(3, R) * 128 + c] = fexp(mm[3] - bb[R]);
             }
-#pragma unroll
-            for (int V = 0; V < 4; ++V)
-#pragma unroll
-                for (int R = 0; R <= V; ++R) tab[tab_c(V, R) * 128 + c] = fexp(mm[V] - bb[R]);
-            sgam[c] = fexp(bb[3]);
         }
         return landed;
     };
@@ -395,11 +405,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             if (p.log_decay && n2 * CH + row < p.S)
                 prefetch_l2(p.log_decay + (row0 + (int64_t)row * p.H) * DD + (tid & 3) * 32);
         }
-        // the previous unit's bulk stores must have read their shared sources
-        if (tid == 0) bulk_wait_read_all();
         // the decay and tables need neither q, k nor v: they run while v is still landing
         ok = decay_tables(u, par, beta_cur);
         beta_cur = beta_next;
+        // the previous unit's bulk stores must have read their shared sources (P2 overwrites them)
+        if (tid == 0) bulk_wait_read_all();
         ok = mbar_wait(bar_in, par) && ok;
         ok = __syncthreads_and(ok);
         if (!ok) break;
@@ -431,17 +441,21 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 load8f(tab + (4 + R) * 128 + c0, F);
                 load8f(tab + (8 + R) * 128 + c0, E);
                 load8f(tab + (12 + R) * 128 + c0, Dd);
-                float e1[8], e3[8], t[8];
+                // fr = e^{G - m_R} (row factor), fg = e^G, ke3 = k e^{b_R - G} (column factors follow from
+                // it by per-channel constants)
+                float fr[8], fg[8], ke3[8], t[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    e1[e] = fexp(G[e] - bRm1[e]);
-                    e3[e] = fexp(bR[e] - G[e]);
+                    const float e1 = fexp(G[e] - bRm1[e]);
+                    fr[e] = e1 * F[e];
+                    fg[e] = e1 * E[e];
+                    ke3[e] = kv[e] * fexp(bR[e] - G[e]);
                 }
 #pragma unroll
-                for (int e = 0; e < 8; ++e) t[e] = kv[e] * e1[e] * F[e];
+                for (int e = 0; e < 8; ++e) t[e] = kv[e] * fr[e];
                 *reinterpret_cast<uint4 *>(sm + bimg + sw128(r, jj)) = pack8(t);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) t[e] = qv[e] * e1[e] * F[e];
+                for (int e = 0; e < 8; ++e) t[e] = qv[e] * fr[e];
                 {
                     const uint4 hi = pack8(t);
                     *reinterpret_cast<uint4 *>(sm + bimg + sw128(64 + r, jj)) = hi;
@@ -455,7 +469,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                     float Cv[8];
                     load8f(tab + tab_c(V, R) * 128 + c0, Cv);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) t[e] = kv[e] * e3[e] * Cv[e];
+                    for (int e = 0; e < 8; ++e) t[e] = ke3[e] * Cv[e];
                     const uint4 hi = pack8(t);
                     *reinterpret_cast<uint4 *>(sm + aimg + sw128(kc_row0(V) + r, jj)) = hi;
                     if (V == R) {  // diagonal block: keep the rounding residue
@@ -467,13 +481,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                     }
                 }
 #pragma unroll
-                for (int e = 0; e < 8; ++e) t[e] = qv[e] * e1[e] * E[e];
+                for (int e = 0; e < 8; ++e) t[e] = qv[e] * fg[e];
                 *reinterpret_cast<uint4 *>(sm + P_QI + img) = pack8(t);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) t[e] = kv[e] * e3[e] * Dd[e];
+                for (int e = 0; e < 8; ++e) t[e] = ke3[e] * Dd[e];
                 *reinterpret_cast<uint4 *>(sm + P_KI + img) = pack8(t);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) t[e] = beta_r * kv[e] * e1[e] * E[e];
+                for (int e = 0; e < 8; ++e) t[e] = (beta_r * kv[e]) * fg[e];
                 *reinterpret_cast<uint4 *>(sm + P_RH + img) = pack8(t);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) t[e] = beta_r * vv[e];
@@ -614,19 +628,19 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             const float *sA = reinterpret_cast<const float *>(sm + P_SA);
             float *sT = reinterpret_cast<float *>(sm + P_ST);
             float *xs = reinterpret_cast<float *>(sm + P_TAB);  // the tables are dead after P2
-            if (tid < 64) {  // diagonal block R, column jc: forward substitution
+            if (tid < 64) {  // diagonal block R, column jc: (I + A_RR) x = e_jc, right-looking
                 const int R = tid >> 4, jc = tid & 15, o = 16 * R;
-                float col[16];
+                float x[16];
 #pragma unroll
-                for (int a = 0; a < 16; ++a) {
-                    float part[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int a = 0; a < 16; ++a) x[a] = (a == jc) ? 1.f : 0.f;
+                // once x[m] is final, every later row subtracts its term: one FMA per step on the
+                // critical path (entries above jc stay exact zeros)
 #pragma unroll
-                    for (int m = 0; m < a; ++m) part[m & 3] += sA[(o + a) * SA_LD + o + m] * col[m];
-                    const float x = ((a == jc) ? 1.f : 0.f) - ((part[0] + part[1]) + (part[2] + part[3]));
-                    col[a] = (a < jc) ? 0.f : x;
-                }
+                for (int m = 0; m < 15; ++m)
 #pragma unroll
-                for (int a = 0; a < 16; ++a) sT[(o + a) * ST_LD + o + jc] = col[a];
+                    for (int a = m + 1; a < 16; ++a) x[a] = fmaf(-sA[(o + a) * SA_LD + o + m], x[m], x[a]);
+#pragma unroll
+                for (int a = 0; a < 16; ++a) sT[(o + a) * ST_LD + o + jc] = x[a];
             }
             named_sync(1, 128);
             // The products below give each thread rows (p, p + h) and four adjacent columns, so that one
@@ -1314,15 +1328,21 @@ __global__ void __launch_bounds__(128, 1) chunk_combine_kernel(CombineArgs p) {
                 mma_commit(bar_m);
             }
         }
-        ok = __syncthreads_and(ok) && mbar_wait(bar_m, g & 1) && mbar_wait(&full[g & 1], (g >> 1) & 1);
-        ok = __syncthreads_and(ok);
+        // while the MMA runs: S_g leaves for its segment chain (g >= 1) and Y_g comes into registers
+        if (g > 0) {
+            float *dst = p.seg_init + ((size_t)bh * p.G + g) * DD * DD + j;
+#pragma unroll
+            for (int c = 0; c < 128; ++c) dst[(size_t)c * DD] = sv[c];
+        }
+        ok = __syncthreads_and(ok) && mbar_wait(&full[g & 1], (g >> 1) & 1);
+        if (ok) {  // S_{g+1}^T = D + Y_g^T (Y_g in shared memory, [c][j])
+            const float *y = reinterpret_cast<const float *>(sm + (g & 1) * CST + 32768) + j;
+#pragma unroll
+            for (int c = 0; c < 128; ++c) sv[c] = y[c * DD];
+        }
+        ok = __syncthreads_and(ok && mbar_wait(bar_m, g & 1));
         if (!ok) break;
         tc_fence_after();
-        // S_{g+1}^T = D + Y_g^T (Y_g in shared memory, [c][j])
-        const float *y = reinterpret_cast<const float *>(sm + (g & 1) * CST + 32768) + j;
-        float *dst = p.seg_init + ((size_t)bh * p.G + g + 1) * DD * DD + j;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) sv[c] = y[c * DD];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             uint32_t dv[32];
@@ -1331,11 +1351,14 @@ __global__ void __launch_bounds__(128, 1) chunk_combine_kernel(CombineArgs p) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) sv[32 * q + e] += __uint_as_float(dv[e]);
         }
-#pragma unroll
-        for (int c = 0; c < 128; ++c) dst[(size_t)c * DD] = sv[c];
         tc_fence_before();
         __syncthreads();
         if (tid == 0 && g + 2 < nseg) issue(g + 2);  // this stage has been read
+    }
+    if (ok && nseg > 0) {  // the last entering state
+        float *dst = p.seg_init + ((size_t)bh * p.G + nseg) * DD * DD + j;
+#pragma unroll
+        for (int c = 0; c < 128; ++c) dst[(size_t)c * DD] = sv[c];
     }
     if (!ok && tid == 0) {
         report_timeout(p.timeouts, p.dev_status);
@@ -1472,6 +1495,7 @@ kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
         pa.H = a.H;
         pa.Nc = (int)Nc;
         pa.units = Nc * a.H * a.B;
+        if (pa.units > 0x7fffffffLL) return fail(KDA_ERR_UNSUPPORTED, "chunk engine: more than 2^31 chunks");
         pa.g_min = a.g_min;
         pa.beta = (const __nv_bfloat16 *)a.beta;
         pa.log_decay = a.log_decay;
