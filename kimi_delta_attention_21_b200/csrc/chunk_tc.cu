@@ -859,8 +859,9 @@ constexpr uint32_t T_V16 = 448;   // V'^T bf16 pairs (A operand, K = r)
 constexpr uint32_t ST_TCOLS = 512;
 
 // kMap = false: the chain over segment blockIdx.z from its entering state, with outputs.
-// kMap = true:  the map of segment blockIdx.z / 2 over its chunks, S_end = A_g S_start + Y_g:
-//               even z runs from S = I without U (-> A_g), odd z from S = 0 with U (-> Y_g); no outputs.
+// kMap = true:  no outputs; z = 0 runs segment 0 from the initial state (its end state is S_1, the
+//               entering state of segment 1); for g >= 1 the map S_end = A_g S_start + Y_g of segment
+//               g = (z + 1) / 2: odd z from S = I without U (-> A_g), even z from S = 0 with U (-> Y_g).
 template <bool kMap>
 __global__ void __launch_bounds__(ST_THREADS, 1)
 chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
@@ -872,8 +873,8 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
     const int q4 = warp & 3, hf = (warp >> 2) & 1;  // TMEM lane quarter, column half (warps 0-7)
     const int h = blockIdx.x, b = blockIdx.y;
     const int bh = b * p.H + h;
-    const int g = kMap ? (int)(blockIdx.z >> 1) : (int)blockIdx.z;
-    const bool ident = kMap && (blockIdx.z & 1) == 0;  // map from the identity (no U)
+    const int g = kMap ? (int)((blockIdx.z + 1) >> 1) : (int)blockIdx.z;
+    const bool ident = kMap && (blockIdx.z & 1) == 1;  // map from the identity (no U)
     const int n0 = g * p.L;
     const int nc = max(0, min(p.L, p.Nc - n0));  // chunks of this segment
     // Record stages: the chains use whole records, two deep; the maps only -W, K~ and U^T (48 KB),
@@ -1008,9 +1009,8 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
         const uint32_t lrow = (uint32_t)(32 * q4) << 16;
         const int j = 32 * q4 + lane;  // value column (TMEM lane) of this thread
         {   // entering state -> TMEM (S^T[j, c] = S[c, j]: a warp reads 128 contiguous bytes per c)
-            const float *s_in = kMap ? nullptr
-                                     : (g == 0 ? (p.S0 ? p.S0 + (size_t)bh * DD * DD : nullptr)
-                                               : p.seg_init + ((size_t)bh * p.G + g) * DD * DD);
+            const float *s_in = (g == 0) ? (p.S0 ? p.S0 + (size_t)bh * DD * DD : nullptr)
+                                         : (kMap ? nullptr : p.seg_init + ((size_t)bh * p.G + g) * DD * DD);
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t su[32];
@@ -1192,7 +1192,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
                 if (ok && !store_o(nc - 1)) ok = false;
             }
         }
-        if (ok && kMap && !ident) {  // Y_g, laid out like a state
+        if (ok && kMap && !ident) {  // Y_g (S_1 for segment 0), laid out like a state
             float *dst0 = p.yt + ((size_t)bh * (p.G - 1) + g) * DD * DD;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
@@ -1245,14 +1245,14 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
 }
 
 // ================================================================ K2c: chunk_combine_kernel
-// The segment maps chained in order, one CTA per (head, batch):
-//   S_{g+1} = A_g S_g + Y_g,   g = 0 .. G-2,
+// The segment maps chained in order, one CTA per (head, batch): S_1 is segment 0's end state (the map
+// pass ran it from the initial state, its Y slot), then
+//   S_{g+1} = A_g S_g + Y_g,   g = 1 .. G-2,
 // with the state transposed in TMEM (lane j): S_{g+1}^T = S_g^T A_g^T + Y_g^T, one M = 128 MMA per
 // segment (A = bf16 copy of S_g^T in TMEM, B = the A_g^T image).  Writes every S_g (g >= 1) for the
 // segment chains.
 struct CombineArgs {
     int H, G;
-    const float *S0;
     const uint8_t *xt;
     const float *yt;
     float *seg_init;
@@ -1274,18 +1274,19 @@ __global__ void __launch_bounds__(128, 1) chunk_combine_kernel(CombineArgs p) {
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + 2 * CST);  // [2]
     uint64_t *bar_m = full + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(full + 3);
-    const int nseg = p.G - 1;
-    auto issue = [&](int g) {
-        mbar_arrive_expect_tx(&full[g & 1], CST);
-        bulk_load(sm + (g & 1) * CST, p.xt + ((size_t)bh * nseg + g) * 32768, 32768, &full[g & 1]);
-        bulk_load(sm + (g & 1) * CST + 32768, p.yt + ((size_t)bh * nseg + g) * DD * DD, 65536, &full[g & 1]);
+    const int nseg = p.G - 1;  // entering states S_1 .. S_{G-1}
+    auto issue = [&](int g) {   // A_g^T image and Y_g (g >= 1) -> stage (g - 1) & 1
+        const int k = (g - 1) & 1;
+        mbar_arrive_expect_tx(&full[k], CST);
+        bulk_load(sm + k * CST, p.xt + ((size_t)bh * nseg + g) * 32768, 32768, &full[k]);
+        bulk_load(sm + k * CST + 32768, p.yt + ((size_t)bh * nseg + g) * DD * DD, 65536, &full[k]);
     };
     if (tid == 0) {
         mbar_init(&full[0], 1);
         mbar_init(&full[1], 1);
         mbar_init(bar_m, 1);
         fence_barrier_init();
-        for (int g = 0; g < 2 && g < nseg; ++g) issue(g);
+        for (int g = 1; g < 3 && g < nseg; ++g) issue(g);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 512);
@@ -1298,14 +1299,16 @@ __global__ void __launch_bounds__(128, 1) chunk_combine_kernel(CombineArgs p) {
     const uint32_t lrow = (uint32_t)(32 * warp) << 16;
     constexpr uint32_t C_S32 = 0, C_S16 = 128, C_D = 256;
     float sv[128];
-    {
-        const float *src = p.S0 ? p.S0 + (size_t)bh * DD * DD + j : nullptr;
+    {   // S_1 (segment 0's end state, in Y slot 0)
+        const float *src = p.yt + (size_t)bh * nseg * DD * DD + j;
 #pragma unroll
-        for (int c = 0; c < 128; ++c) sv[c] = src ? src[(size_t)c * DD] : 0.f;
+        for (int c = 0; c < 128; ++c) sv[c] = src[(size_t)c * DD];
     }
     bool ok = true;
-    int g = 0;
+    int g = 1;
     for (; g < nseg; ++g) {
+        const int k = (g - 1) & 1;
+        const uint32_t kph = ((g - 1) >> 1) & 1;
         // bf16 copy of S_g^T (A operand)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -1318,29 +1321,29 @@ __global__ void __launch_bounds__(128, 1) chunk_combine_kernel(CombineArgs p) {
         tc_fence_before();
         __syncthreads();
         if (tid == 0) {
-            ok = mbar_wait(&full[g & 1], (g >> 1) & 1);
+            ok = mbar_wait(&full[k], kph);
             if (ok) {
                 tc_fence_after();
                 constexpr uint32_t id = idesc_f16(128, 128, 0, 1);
-                const uint64_t d = smem_desc(smem_u32(sm + (g & 1) * CST), 16384, 1024, LAYOUT_SW128);
+                const uint64_t d = smem_desc(smem_u32(sm + k * CST), 16384, 1024, LAYOUT_SW128);
 #pragma unroll
                 for (int s8 = 0; s8 < 8; ++s8) mma_f16_ts(tmem + C_D, tmem + C_S16 + 8 * s8, dadd(d, s8 * 2048), id, s8 > 0);
                 mma_commit(bar_m);
             }
         }
-        // while the MMA runs: S_g leaves for its segment chain (g >= 1) and Y_g comes into registers
-        if (g > 0) {
+        // while the MMA runs: S_g leaves for its segment chain and Y_g comes into registers
+        {
             float *dst = p.seg_init + ((size_t)bh * p.G + g) * DD * DD + j;
 #pragma unroll
             for (int c = 0; c < 128; ++c) dst[(size_t)c * DD] = sv[c];
         }
-        ok = __syncthreads_and(ok) && mbar_wait(&full[g & 1], (g >> 1) & 1);
+        ok = __syncthreads_and(ok) && mbar_wait(&full[k], kph);
         if (ok) {  // S_{g+1}^T = D + Y_g^T (Y_g in shared memory, [c][j])
-            const float *y = reinterpret_cast<const float *>(sm + (g & 1) * CST + 32768) + j;
+            const float *y = reinterpret_cast<const float *>(sm + k * CST + 32768) + j;
 #pragma unroll
             for (int c = 0; c < 128; ++c) sv[c] = y[c * DD];
         }
-        ok = __syncthreads_and(ok && mbar_wait(bar_m, g & 1));
+        ok = __syncthreads_and(ok && mbar_wait(bar_m, (g - 1) & 1));
         if (!ok) break;
         tc_fence_after();
 #pragma unroll
@@ -1362,17 +1365,19 @@ __global__ void __launch_bounds__(128, 1) chunk_combine_kernel(CombineArgs p) {
     }
     if (!ok && tid == 0) {
         report_timeout(p.timeouts, p.dev_status);
-        for (int m = g; m < nseg && m < g + 2; ++m) mbar_wait(&full[m & 1], (m >> 1) & 1, 100000000ull);
+        for (int m = g; m < nseg && m < g + 2; ++m) mbar_wait(&full[(m - 1) & 1], ((m - 1) >> 1) & 1, 100000000ull);
     }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-// Segments per sequence: enough that the map pass fills the GPU once (two CTAs per segment
-// map), with at least 4 chunks per segment; 1 when (batch x heads) alone fills it.
+// Segments per sequence: as many as let the map pass (one CTA for segment 0, two for every later
+// segment but the last: BH (2G - 3) CTAs) and the chain pass (BH G CTAs) each run in one wave, with at
+// least 4 chunks per segment; 1 when (batch x heads) alone fills the GPU.
 int pick_segments(int64_t BH, int64_t Nc, int sms) {
-    int64_t G = 1 + sms / (2 * BH);
+    int64_t G = (sms / BH + 3) / 2;
+    if (G > sms / BH) G = sms / BH;
     if (G > Nc / 4) G = Nc / 4;
     return (int)(G < 1 ? 1 : G);
 }
@@ -1387,7 +1392,7 @@ int device_sms() {
 kda_status_t launch_state(const CUtensorMap &tmo, const StateArgs &sa, int B, int H, cudaStream_t st) {
     if (sa.G > 1) {
         cudaFuncSetAttribute(chunk_state_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
-        cudaError_t e = launch_pdl(chunk_state_kernel<true>, dim3(H, B, 2 * (sa.G - 1)), dim3(ST_THREADS),
+        cudaError_t e = launch_pdl(chunk_state_kernel<true>, dim3(H, B, 2 * sa.G - 3), dim3(ST_THREADS),
                                    STATE_SMEM, st, tmo, sa);
         if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "chunk_state_kernel (segment maps): %s", cudaGetErrorString(e));
         kda_status_t s = check_launch("chunk_state_kernel (segment maps)");
@@ -1395,7 +1400,6 @@ kda_status_t launch_state(const CUtensorMap &tmo, const StateArgs &sa, int B, in
         CombineArgs ca;
         ca.H = H;
         ca.G = sa.G;
-        ca.S0 = sa.S0;
         ca.xt = sa.xt;
         ca.yt = sa.yt;
         ca.seg_init = const_cast<float *>(sa.seg_init);
