@@ -1010,7 +1010,9 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
         const int j = 32 * q4 + lane;  // value column (TMEM lane) of this thread
         {   // entering state -> TMEM (S^T[j, c] = S[c, j]: a warp reads 128 contiguous bytes per c)
             const float *s_in = (g == 0) ? (p.S0 ? p.S0 + (size_t)bh * DD * DD : nullptr)
-                                         : (kMap ? nullptr : p.seg_init + ((size_t)bh * p.G + g) * DD * DD);
+                              : kMap     ? nullptr
+                              : (g == 1) ? p.yt + (size_t)bh * (p.G - 1) * DD * DD  // S_1: segment 0's end state
+                                         : p.seg_init + ((size_t)bh * p.G + g) * DD * DD;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t su[32];
@@ -1246,10 +1248,10 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
 
 // ================================================================ K2c: chunk_combine_kernel
 // The segment maps chained in order, one CTA per (head, batch): S_1 is segment 0's end state (the map
-// pass ran it from the initial state, its Y slot), then
+// pass ran it from the initial state, its Y slot; segment 1's chain reads it there), then
 //   S_{g+1} = A_g S_g + Y_g,   g = 1 .. G-2,
 // with the state transposed in TMEM (lane j): S_{g+1}^T = S_g^T A_g^T + Y_g^T, one M = 128 MMA per
-// segment (A = bf16 copy of S_g^T in TMEM, B = the A_g^T image).  Writes every S_g (g >= 1) for the
+// segment (A = bf16 copy of S_g^T in TMEM, B = the A_g^T image).  Writes S_2 .. S_{G-1} for the
 // segment chains.
 struct CombineArgs {
     int H, G;
@@ -1331,8 +1333,9 @@ __global__ void __launch_bounds__(128, 1) chunk_combine_kernel(CombineArgs p) {
                 mma_commit(bar_m);
             }
         }
-        // while the MMA runs: S_g leaves for its segment chain and Y_g comes into registers
-        {
+        // while the MMA runs: S_g leaves for its segment chain (S_1 is read where the map pass left it)
+        // and Y_g comes into registers
+        if (g > 1) {
             float *dst = p.seg_init + ((size_t)bh * p.G + g) * DD * DD + j;
 #pragma unroll
             for (int c = 0; c < 128; ++c) dst[(size_t)c * DD] = sv[c];
@@ -1397,6 +1400,8 @@ kda_status_t launch_state(const CUtensorMap &tmo, const StateArgs &sa, int B, in
         if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "chunk_state_kernel (segment maps): %s", cudaGetErrorString(e));
         kda_status_t s = check_launch("chunk_state_kernel (segment maps)");
         if (s != KDA_OK) return s;
+    }
+    if (sa.G > 2) {  // (with two segments, segment 1 starts from S_1 itself)
         CombineArgs ca;
         ca.H = H;
         ca.G = sa.G;
@@ -1406,9 +1411,9 @@ kda_status_t launch_state(const CUtensorMap &tmo, const StateArgs &sa, int B, in
         ca.timeouts = sa.timeouts;
         ca.dev_status = sa.dev_status;
         cudaFuncSetAttribute(chunk_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)COMB_SMEM);
-        e = launch_pdl(chunk_combine_kernel, dim3(H, B), dim3(128), COMB_SMEM, st, ca);
+        cudaError_t e = launch_pdl(chunk_combine_kernel, dim3(H, B), dim3(128), COMB_SMEM, st, ca);
         if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "chunk_combine_kernel: %s", cudaGetErrorString(e));
-        s = check_launch("chunk_combine_kernel");
+        kda_status_t s = check_launch("chunk_combine_kernel");
         if (s != KDA_OK) return s;
     }
     cudaFuncSetAttribute(chunk_state_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);

@@ -124,7 +124,9 @@ def test_tc_core_matches_oracle(K, B, S, H):
     assert_bf16_state(to_np(sf), s_ref, "final_state")
 
 
-@pytest.mark.parametrize("B,S,H,g_min", [(1, 2560, 2, -5.0), (2, 1999, 1, -5.0), (1, 2048, 1, -0.5)])
+# segment counts 10, 8, 8, 2 (no combine step) and 3 (one combine step)
+@pytest.mark.parametrize("B,S,H,g_min", [(1, 2560, 2, -5.0), (2, 1999, 1, -5.0), (1, 2048, 1, -0.5),
+                                         (1, 600, 1, -5.0), (1, 768, 2, -5.0)])
 def test_tc_segmented_state_pass(K, B, S, H, g_min):
     """Sequences long enough for the state pass to be split into segments (each segment's affine
     map computed in parallel, the maps chained by the combine pass, the segments then run from
