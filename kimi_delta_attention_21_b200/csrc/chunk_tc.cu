@@ -544,32 +544,19 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             const int q4 = warp & 3;
             const uint32_t lq = (uint32_t)(32 * q4) << 16;
             float *lohi = reinterpret_cast<float *>(sm + P_LOHI);
-            if (warp == 6 || warp == 7) {  // low part of the diagonal column operand x q: row i, block R = i / 16
-                const int i = 32 * (warp - 6) + lane, R = i >> 4;
-                uint32_t v[16];
-                // lanes of one warp span two blocks: load both candidate column blocks, keep the own one
-                uint32_t w0[16], w1[16];
-                tmem_ld_32x32b_x16(tmem + lq + 192 + 64 + 32 * (warp - 6), w0);
-                tmem_ld_32x32b_x16(tmem + lq + 192 + 64 + 32 * (warp - 6) + 16, w1);
-                tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] = (R & 1) ? w1[e] : w0[e];
-#pragma unroll
-                for (int e = 0; e < 16; e += 4)
-                    *reinterpret_cast<float4 *>(lohi + i * 16 + e) =
-                        make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
-                                    __uint_as_float(v[e + 3]));
-            }
-            __syncthreads();
-            if (warp != 3 && warp < 6) {
-                const int prow = warp < 3 ? 32 * warp + lane : 96 + 32 * (warp - 4) + lane;
-                const int V = prow < 16 ? 0 : (prow < 48 ? 1 : (prow < 96 ? 2 : 3));
-                const int i = prow - kc_row0(V);
-                const bool diag = (i >> 4) == V;
+            // the readout warps load their accumulator rows and write A first (neither needs the
+            // low-part hand-off below); only the M^T image waits for it
+            const bool rd = warp != 3 && warp < 6;
+            const int prow = warp < 3 ? 32 * warp + lane : 96 + 32 * (warp - 4) + lane;
+            const int V = prow < 16 ? 0 : (prow < 48 ? 1 : (prow < 96 ? 2 : 3));
+            const int i = prow - kc_row0(V);
+            const bool diag = (i >> 4) == V;
+            uint32_t m_[16], r_[16];
+            if (rd) {
                 const uint32_t cb = tmem + lq + (warp < 3 ? 0u : 192u);
                 // column block V differs between lanes of a warp: each warp's rows span at most two
                 // versions, so load the block of every version present and select
-                uint32_t a_[16], m_[16], r_[16];
+                uint32_t a_[16];
                 const int Vlo = (warp < 3 ? (32 * warp < 16 ? 0 : (32 * warp < 48 ? 1 : 2)) : 3);
                 const int Vhi = (warp < 3 ? ((32 * warp + 31) < 16 ? 0 : ((32 * warp + 31) < 48 ? 1 : 2)) : 3);
                 {
@@ -598,6 +585,25 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                     const int r = 16 * V + e;
                     sA[r * SA_LD + i] = (i < r) ? sbeta[r] * __uint_as_float(a_[e]) : 0.f;
                 }
+            }
+            if (warp == 6 || warp == 7) {  // low part of the diagonal column operand x q: row i, block R = i / 16
+                const int il = 32 * (warp - 6) + lane, R = il >> 4;
+                uint32_t v[16];
+                // lanes of one warp span two blocks: load both candidate column blocks, keep the own one
+                uint32_t w0[16], w1[16];
+                tmem_ld_32x32b_x16(tmem + lq + 192 + 64 + 32 * (warp - 6), w0);
+                tmem_ld_32x32b_x16(tmem + lq + 192 + 64 + 32 * (warp - 6) + 16, w1);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) v[e] = (R & 1) ? w1[e] : w0[e];
+#pragma unroll
+                for (int e = 0; e < 16; e += 4)
+                    *reinterpret_cast<float4 *>(lohi + il * 16 + e) =
+                        make_float4(__uint_as_float(v[e]), __uint_as_float(v[e + 1]), __uint_as_float(v[e + 2]),
+                                    __uint_as_float(v[e + 3]));
+            }
+            __syncthreads();
+            if (rd) {
 #pragma unroll
                 for (int hc = 0; hc < 2; ++hc) {
                     float t[8];
@@ -645,6 +651,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             named_sync(1, 128);
             // The products below give each thread rows (p, p + h) and four adjacent columns, so that one
             // float4 of the right operand feeds eight FMAs (shared-memory wavefronts, not FMAs, bound them).
+            float *x2 = xs + 512;  // X = A[32:64, 0:32] T[0:32, 0:32] for the 32 -> 64 step, [32][32]
             if (tid < 64) {  // 16 -> 32: X = A_{R,R-1} T_{R-1,R-1}, R = 1 + 2 hb
                 const int hb = tid >> 5, R = 1 + 2 * hb, pr = (tid >> 2) & 7, c4 = 4 * (tid & 3), o = 16 * (R - 1);
                 const float *a0 = sA + (16 * R + pr) * SA_LD + o, *a1 = a0 + 8 * SA_LD;
@@ -659,6 +666,26 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 }
                 *reinterpret_cast<float4 *>(xs + hb * 256 + pr * 16 + c4) = x;
                 *reinterpret_cast<float4 *>(xs + hb * 256 + (pr + 8) * 16 + c4) = y;
+            } else {  // meanwhile the part of the 32 -> 64 product that needs only the diagonal blocks:
+                      // X[:, 16 B + c] = A[32:64, 16 B : 16 B + 16] T_BB  (B = 0, 1)
+                const int t2 = tid - 64, pr = t2 >> 2, c8 = 8 * (t2 & 3), blk = c8 >> 4;
+                const float *a0 = sA + (32 + pr) * SA_LD + 16 * blk, *a1 = a0 + 16 * SA_LD;
+                const float *tb = sT + 16 * blk * ST_LD + c8;
+                float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0, y0 = x0, y1 = x0;
+#pragma unroll
+                for (int m = 0; m < 16; ++m) {
+                    const float u = a0[m], v = a1[m];
+                    const float4 t0 = *reinterpret_cast<const float4 *>(tb + m * ST_LD);
+                    const float4 t1 = *reinterpret_cast<const float4 *>(tb + m * ST_LD + 4);
+                    x0.x += u * t0.x; x0.y += u * t0.y; x0.z += u * t0.z; x0.w += u * t0.w;
+                    x1.x += u * t1.x; x1.y += u * t1.y; x1.z += u * t1.z; x1.w += u * t1.w;
+                    y0.x += v * t0.x; y0.y += v * t0.y; y0.z += v * t0.z; y0.w += v * t0.w;
+                    y1.x += v * t1.x; y1.y += v * t1.y; y1.z += v * t1.z; y1.w += v * t1.w;
+                }
+                *reinterpret_cast<float4 *>(x2 + pr * 32 + c8) = x0;
+                *reinterpret_cast<float4 *>(x2 + pr * 32 + c8 + 4) = x1;
+                *reinterpret_cast<float4 *>(x2 + (pr + 16) * 32 + c8) = y0;
+                *reinterpret_cast<float4 *>(x2 + (pr + 16) * 32 + c8 + 4) = y1;
             }
             named_sync(1, 128);
             if (tid < 64) {  //       T_{R,R-1} = -T_RR X  (T_RR is zero above its diagonal); zero block (R-1, R)
@@ -681,32 +708,39 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 *reinterpret_cast<float4 *>(z0 + 8 * ST_LD) = make_float4(0.f, 0.f, 0.f, 0.f);
             }
             named_sync(1, 128);
-            if (tid < 128) {  // 32 -> 64: X = A[32:64, 0:32] T[0:32, 0:32]
-                const int pr = tid >> 3, c4 = 4 * (tid & 7);
-                const float *a0 = sA + (32 + pr) * SA_LD, *a1 = a0 + 16 * SA_LD;
-                const float *tb = sT + c4;
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
+            if (tid < 64) {  // 32 -> 64: the rest of X, X[:, 0:16] += A[32:64, 16:32] T_10
+                const int pr = tid >> 2, c4 = 4 * (tid & 3);
+                const float *a0 = sA + (32 + pr) * SA_LD + 16, *a1 = a0 + 16 * SA_LD;
+                const float *tb = sT + 16 * ST_LD + c4;
+                float4 x = *reinterpret_cast<const float4 *>(x2 + pr * 32 + c4);
+                float4 y = *reinterpret_cast<const float4 *>(x2 + (pr + 16) * 32 + c4);
 #pragma unroll
-                for (int m = 0; m < 32; ++m) {
+                for (int m = 0; m < 16; ++m) {
                     const float u = a0[m], v = a1[m];
                     const float4 t = *reinterpret_cast<const float4 *>(tb + m * ST_LD);
                     x.x += u * t.x; x.y += u * t.y; x.z += u * t.z; x.w += u * t.w;
                     y.x += v * t.x; y.y += v * t.y; y.z += v * t.z; y.w += v * t.w;
                 }
-                *reinterpret_cast<float4 *>(xs + pr * 32 + c4) = x;
-                *reinterpret_cast<float4 *>(xs + (pr + 16) * 32 + c4) = y;
+                *reinterpret_cast<float4 *>(x2 + pr * 32 + c4) = x;
+                *reinterpret_cast<float4 *>(x2 + (pr + 16) * 32 + c4) = y;
             }
             named_sync(1, 128);
-            if (tid < 128) {  //       T[32:64, 0:32] = -T[32:64, 32:64] X
+            if (tid < 128) {  //       T[32:64, 0:32] = -T[32:64, 32:64] X  (rows 32-47: T_22 only, T_23 = 0)
                 const int pr = tid >> 3, c4 = 4 * (tid & 7);
                 const float *t0 = sT + (32 + pr) * ST_LD + 32, *t1 = t0 + 16 * ST_LD;
-                const float *xb = xs + c4;
+                const float *xb = x2 + c4;
                 float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
 #pragma unroll
-                for (int m = 0; m < 32; ++m) {
+                for (int m = 0; m < 16; ++m) {
                     const float u = t0[m], v = t1[m];
                     const float4 t = *reinterpret_cast<const float4 *>(xb + m * 32);
                     x.x += u * t.x; x.y += u * t.y; x.z += u * t.z; x.w += u * t.w;
+                    y.x += v * t.x; y.y += v * t.y; y.z += v * t.z; y.w += v * t.w;
+                }
+#pragma unroll
+                for (int m = 16; m < 32; ++m) {
+                    const float v = t1[m];
+                    const float4 t = *reinterpret_cast<const float4 *>(xb + m * 32);
                     y.x += v * t.x; y.y += v * t.y; y.z += v * t.z; y.w += v * t.w;
                 }
                 float *d0 = sT + (32 + pr) * ST_LD + c4;
