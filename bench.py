@@ -47,8 +47,8 @@ REF_SAMPLE_TOKENS = 512   # tokens (all heads) per reference-arm step
 # the committed ncu summaries under profiles/, keyed by kernel and workload,
 # valid only while the kernel's source file is unchanged (sha256 prefix).
 NCU_TRAFFIC = {
-    # prefill_4k_chunk_engine.md: prep 128.4 + segment maps 44.0 + combine 7.4 + segment chains 102.6 MB
-    "chunk_engine@prefill_4k": {"bytes": 282365184, "src_sha": "deb0b7709dbd0b02"},
+    # prefill_4k_chunk_engine.md: prep 129.4 + segment maps 43.9 + combine 7.4 + segment chains 104.6 MB
+    "chunk_engine@prefill_4k": {"bytes": 285193728, "src_sha": "062ca38e894c9ecc"},
     # decode_256_step.md: decode128_stream_kernel, 547.4 MB read + 479.8 MB written
     "decode@decode_256": {"bytes": 1027173120, "src_sha": "079db3bd726bd665"},
 }
