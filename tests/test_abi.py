@@ -154,3 +154,33 @@ def test_workspace_query_needs_no_device():
     a = _args(shape=(2, 100, 3, 32, 32))
     n = ctypes.c_size_t(123)
     assert _lib.load().kda_chunk_workspace_size(ctypes.byref(a), ctypes.byref(n)) == _lib.KDA_OK
+
+
+def _expected_tc_workspace(B, S, H, sms=148):
+    """Workspace of the tensor-core chunk engine, from the rule it follows: per-chunk records and gate
+    tiles, and, with G segments, BH (G - 1) map slots (A image + Y) and BH G entering states, G the
+    largest count for which the map pass (BH (2G - 3) CTAs) and the chain pass (BH G CTAs) each fit
+    in one wave, at least 4 chunks per segment, and no empty segment."""
+    rec, sig = 74240, 64 * 128 * 2
+    bh, nc = B * H, (S + 63) // 64
+    per_sm = sms // bh
+    g = min((per_sm + 3) // 2, per_sm, nc // 4)
+    g = max(g, 1)
+    L = (nc + g - 1) // g
+    g = (nc + L - 1) // L
+    ws = bh * nc * (rec + sig)
+    if g > 1:
+        ws += bh * (g - 1) * (32768 + 65536) + bh * g * 128 * 128 * 4
+    return ws, g
+
+
+@pytest.mark.parametrize("B,S,H,G", [(1, 4096, 16, 6),      # prefill_4k: 6 segments of 11 chunks
+                                     (8, 8192, 32, 1),      # batch_8x8k: one segment
+                                     (1, 600, 1, 2), (1, 768, 2, 3), (1, 2560, 2, 10)])
+def test_tc_workspace_and_segment_count(B, S, H, G):
+    a = _args(shape=(B, S, H, 128, 128))
+    n = ctypes.c_size_t(0)
+    assert _lib.load().kda_chunk_workspace_size(ctypes.byref(a), ctypes.byref(n)) == _lib.KDA_OK
+    want, g = _expected_tc_workspace(B, S, H)
+    assert g == G
+    assert n.value == want
