@@ -244,3 +244,37 @@ def test_tc_layer_with_fused_gate(K):
     want = oracle_layer(inp, w)
     assert_bf16_outputs(to_np(out["outputs"]), want["outputs"], "outputs")
     assert_bf16_state(to_np(out["final_state"]), want["final_state"], "final_state")
+
+
+def _random_case(seed):
+    import random
+    r = random.Random(seed)
+    return dict(B=r.choice([1, 1, 2, 3]), S=r.randint(1, 3000), H=r.choice([1, 2, 3, 4]),
+                g_min=r.choice([-5.0, -1.0, -0.3]), gated=r.random() < 0.5, s0=r.choice([0.0, 0.02]))
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_tc_random_shapes(K, seed):
+    """Seeded random batch sizes, lengths (ragged tails, one to many segments), head counts, decay
+    bounds, initial states and with or without the fused gate.  Gated rows are checked on the
+    projected layer output, where the tolerance is stated (a row whose o~ is close to zero is
+    amplified by the normalisation before the projection averages it); o~ otherwise."""
+    c = _random_case(seed)
+    B, S, H = c["B"], c["S"], c["H"]
+    w = small("rnd", B, S, H, 128, 128, 256, "bf16", seed=4000 + seed, s0_std=c["s0"], g_min=c["g_min"])
+    inp = ki.make_inputs(w)
+    d = upload(inp, w)
+    o, sf = K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=d["z"], g_min=w.g_min, initial_state=d["S0"],
+                        gate_logits=d["gate"] if c["gated"] else None, eps=w.eps, engine="tc")
+    torch.cuda.synchronize()
+    assert _timeouts(K) == 0
+    o_ref, s_ref = oracle.recurrence(inp["q"], inp["k"], inp["v"], inp["beta"], z=inp["z"], g_min=w.g_min,
+                                     initial_state=inp["S0"])
+    what = f"B{B} S{S} H{H} g_min {w.g_min} gated {c['gated']}"
+    if c["gated"]:
+        y = K.out_proj(o.reshape(B * S, H * w.Dv), d["W_o"])
+        want = oracle.project(oracle.norm_gate(o_ref, inp["gate"], w.eps), inp["W_o"])
+        assert_bf16_outputs(to_np(y).reshape(want.shape), want, "layer outputs, " + what)
+    else:
+        assert_bf16_outputs(to_np(o), o_ref, "o~, " + what)
+    assert_bf16_state(to_np(sf), s_ref, "final_state, " + what)
