@@ -1,20 +1,28 @@
 #!/usr/bin/env python
-"""Throughput of the KDA layer forward on B200: chunkwise prefill (headline)
-and the single-token decode step, with roofline fractions.
+"""Throughput of the KDA layer forward on B200: chunkwise prefill and the
+single-token decode step, with roofline fractions.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     torchrun --nproc-per-node N bench.py --gpus N ...      (one process per GPU)
 
-One step = one whole layer forward (gate, chunk engine with the fused
-RMSNorm and sigmoid gate, output projection) over one batch of the
-``prefill_4k`` workload (B1 S4096 H16 D128, D_model 2048, bf16, fp32 state),
-inputs resident in HBM, L2 flushed between steps.  Each rank runs its own
-independent sequence (weak scaling, no collective on the data path).  The
-decode engine is timed in the same run on the ``decode_256`` workload and
-reported under "decode".  Rank 0 prints one JSON line.
+Without a launcher, ``--gpus N`` (N > 1) starts the N rank processes itself.
+
+One step = one whole layer forward (chunk engine with the gate, the fused
+RMSNorm and sigmoid gate, then the output projection) over one batch of a
+workload, inputs resident in HBM, a 256 MiB L2 flush between steps.  The
+headline (top-level ``value``) is the largest single-GPU prefill workload,
+``long_1m`` (B1 S1,048,576 H16 D128, D_model 2048, bf16, fp32 state from
+S0 ~ N(0, 0.02)); ``batch_8x8k``, ``prefill_4k`` and the decode engine on
+``decode_256`` are timed in the same run and reported under ``workloads``.
+Each rank runs its own independently seeded batch (weak scaling, no
+collective on the data path).  Rank 0 prints one JSON line.
+
+Rooflines follow the layer's arithmetic: the chunk engine's fraction is
+max(FLOPs / peak FLOP/s, bytes / peak bandwidth) / time with algorithmic
+FLOPs and bytes; the layer's adds the projection's FLOPs and output bytes.
 
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
-same workload instead (rank 0 only).
+headline workload instead (rank 0 only).
 """
 from __future__ import annotations
 
@@ -23,6 +31,7 @@ import datetime
 import hashlib
 import json
 import os
+import socket
 import statistics
 import sys
 import threading
@@ -37,20 +46,23 @@ if ROOT not in sys.path:
 import kda_inputs as ki  # noqa: E402
 
 METRIC = "KDA tokens/s (chunk prefill, decode) on 1 B200; % of tensor/HBM roofline"
-PREFILL = "prefill_4k"
+HEADLINE = "long_1m"
+PREFILL_EXTRA = ("batch_8x8k", "prefill_4k")
 DECODE = "decode_256"
+ALL_WORKLOADS = (HEADLINE,) + PREFILL_EXTRA + (DECODE,)
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 REF_SAMPLE_TOKENS = 512   # tokens (all heads) per reference-arm step
+CHUNK = 64
 
-# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) from
-# the committed ncu summaries under profiles/, keyed by kernel and workload,
-# valid only while the kernel's source file is unchanged (sha256 prefix).
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one chunk-engine
+# call or one decode step, from an ncu capture of the named kernels on the
+# named workload, valid only while the kernel source is unchanged (sha256
+# prefix of the listed files).  "scale" marks a figure taken on a smaller
+# workload and scaled by the number of (batch, head, chunk) units.
 NCU_TRAFFIC = {
-    # prefill_4k_chunk_engine.md: prep 129.4 + segment maps 43.9 + combine 7.4 + segment chains 104.6 MB
-    "chunk_engine@prefill_4k": {"bytes": 285193728, "src_sha": "062ca38e894c9ecc"},
-    # decode_256_step.md: decode128_stream_kernel, 547.4 MB read + 479.8 MB written
-    "decode@decode_256": {"bytes": 1027173120, "src_sha": "079db3bd726bd665"},
+    "decode@decode_256": {"bytes": 1027173120, "src_sha": {"kimi_delta_attention_21_b200/csrc/decode.cu":
+                                                              "079db3bd726bd665"}},
 }
 
 
@@ -61,11 +73,14 @@ def src_sha(relpath):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def traffic_for(kernel, workload, src):
-    rec = NCU_TRAFFIC.get(f"{kernel}@{workload}")
-    if rec and rec["src_sha"] == src_sha(src):
-        return rec["bytes"]
-    return None
+def traffic_for(key, units=None):
+    """Per-call DRAM bytes for `key` if its sources are unchanged since the capture, else None."""
+    rec = NCU_TRAFFIC.get(key)
+    if not rec or any(src_sha(p) != h for p, h in rec["src_sha"].items()):
+        return None
+    if "units" in rec and units is not None:
+        return int(round(rec["bytes"] * units / rec["units"]))
+    return rec["bytes"]
 
 
 def load_peaks():
@@ -77,27 +92,41 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def n_chunks(w):
+    return (w.S + CHUNK - 1) // CHUNK
+
+
 def prefill_bytes(w):
     """Algorithmic HBM bytes of the chunk engine for a whole workload: read q, k,
     z (D_k each), v, gate (D_v each) and beta per token-head, write the gated
-    output (D_v) per token-head, write the fp32 final state per (b, h)."""
+    output (D_v) per token-head; read the fp32 initial state (when there is one)
+    and write the fp32 final state per (b, h)."""
     es = 2 if w.dtype == "bf16" else 4
     per_tok_head = es * (3 * w.Dk + 3 * w.Dv + 1)
-    return w.B * w.S * w.H * per_tok_head + w.B * w.H * w.Dk * w.Dv * 4
+    n_states = 2 if w.s0_std > 0 else 1
+    return w.B * w.S * w.H * per_tok_head + n_states * w.B * w.H * w.Dk * w.Dv * 4
 
 
-def chunk_flops(w, C=64):
+def chunk_flops(w, C=CHUNK):
     """Algorithmic tensor FLOPs of the chunkwise prefill (2 per multiply-add), per chunk of C tokens:
     the causal intra-chunk products A = (beta K) K^T and M = Q K^T, the UT-transform products
     W = T (beta K e^G) and U = T (beta V) and the intra-chunk output M V' (lower triangles: C^2 D
     each), and the three state products W S, (Q e^G) S and K~^T V' (2 C D_k D_v each).  The
     triangular solve itself is not counted."""
     per_chunk = C * C * (2 * w.Dk + w.Dk + 2 * w.Dv) + 3 * 2 * C * w.Dk * w.Dv
-    return w.B * w.H * ((w.S + C - 1) // C) * per_chunk
+    return w.B * w.H * n_chunks(w) * per_chunk
 
 
 def proj_flops(n_rows, w):
     return 2.0 * n_rows * w.H * w.Dv * w.D_model
+
+
+def layer_bytes(w):
+    """Algorithmic HBM bytes of the whole layer: the chunk engine's inputs and
+    states, W_o once, and the projected output y (N x D_model)."""
+    es = 2 if w.dtype == "bf16" else 4
+    core = prefill_bytes(w) - w.B * w.S * w.H * w.Dv * es   # o is an intermediate of the layer
+    return core + w.D_model * w.H * w.Dv * es + w.B * w.S * w.D_model * es
 
 
 def decode_bytes(w):
@@ -106,6 +135,28 @@ def decode_bytes(w):
     es = 2 if w.dtype == "bf16" else 4
     per_bh = 2 * w.Dk * w.Dv * 4 + es * (3 * w.Dk + 3 * w.Dv + 1)
     return w.B * w.H * per_bh
+
+
+def roofline(flops, nbytes, seconds, peaks, tensor_peak_key="bf16_tflops"):
+    """max(flop time, byte time) at the peaks over the measured time.  `bound` is
+    the roof that sets the floor; `achieved` is in that roof's unit."""
+    t_flop = flops / (peaks[tensor_peak_key] * 1e12)
+    t_byte = nbytes / (peaks["hbm_gbs"] * 1e9)
+    if t_byte >= t_flop:
+        out = {"bound": "hbm", "achieved": round(nbytes / seconds / 1e9, 1), "peak": peaks["hbm_gbs"],
+               "unit": "GB/s"}
+    else:
+        out = {"bound": "tensor", "achieved": round(flops / seconds / 1e12, 2), "peak": peaks[tensor_peak_key],
+               "unit": "TFLOP/s"}
+    out["frac"] = round(max(t_flop, t_byte) / seconds, 4)
+    out.update({"algorithmic_flops": int(flops), "algorithmic_bytes": int(nbytes),
+                "flop_time_ms": round(t_flop * 1e3, 4), "byte_time_ms": round(t_byte * 1e3, 4),
+                "ms": round(seconds * 1e3, 4),
+                "tensor_achieved_tflops": round(flops / seconds / 1e12, 2),
+                "tensor_frac": round(flops / seconds / 1e12 / peaks[tensor_peak_key], 4),
+                "hbm_achieved_gbs": round(nbytes / seconds / 1e9, 1),
+                "hbm_frac": round(nbytes / seconds / 1e9 / peaks["hbm_gbs"], 4)})
+    return out
 
 
 class ClockSampler:
@@ -208,7 +259,258 @@ def rank_workload(name, rank):
     return dataclasses.replace(w, seed=w.seed + 7919 * rank)
 
 
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _rank_entry(rank, argv, world, port):
+    os.environ.update(RANK=str(rank), LOCAL_RANK=str(rank), WORLD_SIZE=str(world), LOCAL_WORLD_SIZE=str(world),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    rc = main(argv)
+    if rc:
+        raise SystemExit(rc)
+
+
+def launch_ranks(argv, world):
+    """Start `world` rank processes on this node (one per GPU), each running
+    main(argv) with RANK / LOCAL_RANK / WORLD_SIZE set, and wait for all of
+    them; a failing rank fails the launch."""
+    import torch.multiprocessing as mp
+    mp.start_processes(_rank_entry, args=(list(argv), world, _free_port()), nprocs=world, join=True,
+                       start_method="spawn")
+    return 0
+
+
 # ----------------------------------------------------------------------------- our arm
+
+class Timer:
+    """CUDA events around the chunk-engine call and the projection of each step."""
+
+    def __init__(self, torch, n):
+        self.ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+
+    def means(self):
+        n = len(self.ev)
+        a = sum(e[0].elapsed_time(e[1]) for e in self.ev) / n * 1e-3
+        b = sum(e[1].elapsed_time(e[2]) for e in self.ev) / n * 1e-3
+        return a, b
+
+
+def time_prefill(K, torch, w, d, steps, warmup, world, dev, flush, lib, sampler=None):
+    """Times `steps` layer forwards of workload `w` (device inputs `d`).  Returns
+    per-step seconds (chunk engine, projection; max over ranks) and launches."""
+    B, S, H = w.B, w.S, w.H
+    N = B * S
+    x = torch.empty((B, S, H, w.Dv), dtype=d["v"].dtype, device=dev)
+    y = torch.empty((N, w.D_model), dtype=d["v"].dtype, device=dev)
+    sf = torch.empty((B, H, w.Dk, w.Dv), dtype=torch.float32, device=dev)
+    ws = torch.empty(K.chunk_workspace_bytes(B, S, H, w.Dk, w.Dv), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def chunk():
+        K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=d["z"], g_min=w.g_min, initial_state=d["S0"],
+                    gate_logits=d["gate"], eps=w.eps, out=x, final_state=sf, workspace=ws)
+
+    def proj():
+        K.out_proj(x.view(N, H * w.Dv), d["W_o"], out=y)
+
+    for _ in range(warmup):
+        flush.fill_(1.0)
+        chunk()
+        proj()
+    torch.cuda.synchronize(dev)
+    tm = Timer(torch, steps)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    n0 = lib.kda_launch_count()
+    t_wall0 = time.perf_counter()
+    if sampler is not None:
+        sampler.__enter__()
+    for i in range(steps):
+        flush.fill_(float(i))
+        tm.ev[i][0].record(stream)
+        chunk()
+        tm.ev[i][1].record(stream)
+        proj()
+        tm.ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    if sampler is not None:
+        sampler.__exit__(None, None, None)
+    barrier(world)
+    t_wall = time.perf_counter() - t_wall0
+    launches = lib.kda_launch_count() - n0
+    t_chunk, t_proj = tm.means()
+    t_step_max, t_chunk_max, t_proj_max = reduce_max([t_chunk + t_proj, t_chunk, t_proj], world, dev)
+    del x, y, sf, ws
+    return {"t_step": t_step_max, "t_chunk": t_chunk_max, "t_proj": t_proj_max, "launches": launches,
+            "wall": t_wall}
+
+
+def prefill_record(w, tm, peaks, world, traffic_key):
+    N = w.B * w.S
+    units = w.B * w.H * n_chunks(w)
+    chunk = roofline(chunk_flops(w), prefill_bytes(w), tm["t_chunk"], peaks)
+    chunk["kernel"] = "kda_chunk_fwd (chunk engine: prep, segment maps, combine, segment chains)"
+    chunk["traffic"] = traffic_for(traffic_key, units)
+    layer = roofline(chunk_flops(w) + proj_flops(N, w), layer_bytes(w), tm["t_step"], peaks)
+    layer_s = roofline(chunk_flops(w) + proj_flops(N, w), layer_bytes(w), tm["t_step"], peaks,
+                       "bf16_tflops_sustained")
+    layer["kernel"] = "layer forward (kda_chunk_fwd + kda_out_proj)"
+    layer["frac_vs_sustained_tensor_peak"] = layer_s["frac"]
+    proj_t = proj_flops(N, w) / tm["t_proj"] / 1e12
+    return {
+        "workload": w.name, "value": round(N * world / tm["t_step"], 1), "unit": "tokens/s",
+        "ms_per_step": round(tm["t_step"] * 1e3, 4),
+        "config": {"B": w.B, "S": w.S, "H": w.H, "D_k": w.Dk, "D_v": w.Dv, "D_model": w.D_model, "chunk": CHUNK,
+                   "g_min": w.g_min, "z_std": w.z_std, "initial_state": f"N(0, {w.s0_std})" if w.s0_std else "zeros",
+                   "state": "fp32", "units_b_h_chunk": units},
+        "kernels_ms": {"chunk_engine": round(tm["t_chunk"] * 1e3, 4), "out_proj": round(tm["t_proj"] * 1e3, 4)},
+        "roofline": chunk,
+        "layer_roofline": layer,
+        "out_proj": {"achieved_tflops": round(proj_t, 1), "frac": round(proj_t / peaks["bf16_tflops"], 4)},
+        "chunk_engine_tokens_per_s": round(N * world / tm["t_chunk"], 1),
+    }
+
+
+def cpu_baseline_prefill(w, d, target_s):
+    """The oracle as it stands, on this host's cores, on the first n tokens of
+    batch row 0 (all heads) of the same device-generated inputs: fp64
+    recurrence + norm/gate + projection.  n is calibrated so that the timed
+    call takes about `target_s` seconds."""
+    import oracle
+    cores = oracle.default_threads()
+
+    def run(n):
+        h = ki.host_rows(d, 0, 0, n)
+        t0 = time.perf_counter()
+        oracle.forward(h["q"], h["k"], h["v"], h["z"], h["beta"], h["gate"], h["W_o"], h["S0"],
+                       g_min=w.g_min, eps=w.eps, threads=cores)
+        return time.perf_counter() - t0
+
+    n = min(w.S, 256)
+    dt = run(n)
+    n = int(min(w.S, max(n, n * target_s / max(dt, 1e-3))))
+    dt = run(n)
+    return {"value": round(n / dt, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {n} of {w.S} tokens x {w.H} heads of batch row 0 of {w.name} (same device-generated "
+                      f"inputs, copied to the host): fp64 recurrence + norm/gate + projection, {dt:.2f} s"}
+
+
+def cpu_baseline_decode(w, d, target_s):
+    """The oracle on the first m sequences (all heads, all decode steps) of the
+    decode workload: its recurrence over the steps from each sequence's state."""
+    import oracle
+    cores = oracle.default_threads()
+
+    def run(m):
+        h = {n: d[n][:m].float().cpu().numpy() for n in ("q", "k", "z", "v", "gate", "beta")}
+        s0 = d["S0"][:m].float().cpu().numpy()
+        W = d["W_o"].float().cpu().numpy()
+        t0 = time.perf_counter()
+        oracle.forward(h["q"], h["k"], h["v"], h["z"], h["beta"], h["gate"], W, s0, g_min=w.g_min, eps=w.eps,
+                       threads=cores)
+        return time.perf_counter() - t0
+
+    m = 2
+    dt = run(m)
+    m = int(min(w.B, max(m, m * target_s / max(dt, 1e-3))))
+    dt = run(m)
+    return {"value": round(m * w.S / dt, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{m} of {w.B} sequences x {w.H} heads x {w.S} decode steps of {w.name} (same device-generated "
+                      f"inputs): fp64 recurrence + norm/gate + projection, {dt:.2f} s"}
+
+
+def run_e2e(K, torch, w, d, steps, world, dev):
+    """The headline metric through the public API with HOST buffers: every step
+    copies the step's inputs from pinned host memory to the device, runs the
+    layer and copies the outputs and the final state back (kda_forward)."""
+    names = ("q", "k", "v", "z", "beta", "gate")
+    hin = {}
+    for n in names:
+        t = torch.empty(d[n].shape, dtype=d[n].dtype, pin_memory=True)
+        t.copy_(d[n])
+        hin[n] = t
+    s0 = None
+    if d["S0"] is not None:
+        s0 = torch.empty(d["S0"].shape, dtype=torch.float32, pin_memory=True)
+        s0.copy_(d["S0"])
+    W = d["W_o"]
+    for n in names:
+        d[n] = None   # the device copies of the timing run are not needed any more
+    torch.cuda.empty_cache()
+    y_h = torch.empty((w.B, w.S, w.D_model), dtype=hin["q"].dtype, pin_memory=True)
+    s_h = torch.empty((w.B, w.H, w.Dk, w.Dv), dtype=torch.float32, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in hin.values()) + (0 if s0 is None else s0.numel() * 4)
+    d2h = y_h.numel() * y_h.element_size() + s_h.numel() * 4
+
+    def one():
+        K.kda_forward(hin["q"], hin["k"], hin["v"], hin["z"], hin["beta"], hin["gate"], W, s0, g_min=w.g_min,
+                      eps=w.eps, state_dtype=torch.float32, outputs=y_h, final_state_out=s_h)
+
+    one()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        one()
+    torch.cuda.synchronize(dev)
+    t = (time.perf_counter() - t0) / steps
+    (t_max,) = reduce_max([t], world, dev)
+    return {"value": round(w.B * w.S * world / t_max, 1), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": steps, "ms_per_step": round(t_max * 1e3, 2),
+            "api": "kimi_delta_attention_21_b200.kda_forward (pinned host tensors in and out)"}
+
+
+def run_decode(K, torch, w, d, warmup, world, dev, peaks, lib):
+    dt = d["q"].dtype
+    T = w.decode_steps
+    steps = {n: d[n].transpose(0, 1).contiguous() for n in ("q", "k", "v", "z", "beta", "gate")}
+    state = d["S0"].clone()
+    x = torch.empty((w.B, w.H, w.Dv), dtype=dt, device=dev)
+    y = torch.empty((w.B, w.D_model), dtype=dt, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def one(t):
+        K.decode_step(steps["q"][t], steps["k"][t], steps["v"][t], steps["beta"][t], state, z=steps["z"][t],
+                      g_min=w.g_min, gate_logits=steps["gate"][t], eps=w.eps, out=x)
+
+    for t in range(min(warmup, T)):
+        one(t)
+        K.out_proj(x.view(w.B, w.H * w.Dv), d["W_o"], out=y)
+    state.copy_(d["S0"])
+    torch.cuda.synchronize(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(T)]
+    barrier(world)
+    n0 = lib.kda_launch_count()
+    for t in range(T):
+        ev[t][0].record(stream)
+        one(t)
+        ev[t][1].record(stream)
+        K.out_proj(x.view(w.B, w.H * w.Dv), d["W_o"], out=y)
+        ev[t][2].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    launches = lib.kda_launch_count() - n0
+    t_dec = sum(e[0].elapsed_time(e[1]) for e in ev) / T * 1e-3
+    t_prj = sum(e[1].elapsed_time(e[2]) for e in ev) / T * 1e-3
+    t_dec_m, t_prj_m = reduce_max([t_dec, t_prj], world, dev)
+    nb = decode_bytes(w)
+    ach = nb / t_dec_m / 1e9
+    return {"workload": w.name, "value": round(w.B * world / (t_dec_m + t_prj_m), 1), "unit": "tokens/s",
+            "steps": T, "ms_per_step": round((t_dec_m + t_prj_m) * 1e3, 4),
+            "config": {"B": w.B, "H": w.H, "D_k": w.Dk, "D_v": w.Dv, "D_model": w.D_model,
+                       "initial_state": f"N(0, {w.s0_std}) fp32, {w.B * w.H * w.Dk * w.Dv * 4 >> 20} MiB"},
+            "kernels_ms": {"decode_step": round(t_dec_m * 1e3, 4), "out_proj": round(t_prj_m * 1e3, 4)},
+            "roofline": {"kernel": "kda_decode_step", "bound": "hbm", "achieved": round(ach, 1),
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
+                         "traffic": traffic_for(f"decode@{DECODE}"), "algorithmic_bytes": nb},
+            "gpu_launches": int(launches),
+            "l2": "state (512 MiB) larger than L2"}
+
 
 def run_ours(args, rank, world, local):
     import torch
@@ -219,203 +521,70 @@ def run_ours(args, rank, world, local):
     init_dist(world, "nccl")
     lib = K.load_library()
     peaks, peak_src = load_peaks()
-    if args.only == "decode":
-        dec = run_decode(args, rank, world, local, K, dev, peaks)
-        return {"metric": METRIC, "decode": dec, "n_gpus": world} if rank == 0 else None
-
-    # ---------------- prefill inputs, resident in HBM
-    w = rank_workload(PREFILL, rank)
-    inp = ki.make_inputs(w)
-    dt = torch.bfloat16
-    dv = {n: torch.from_numpy(inp[n]).to(dev).to(dt).contiguous() for n in ("q", "k", "v", "z", "beta", "gate", "W_o")}
-    B, S, H = w.B, w.S, w.H
-    N = B * S
-    x = torch.empty((B, S, H, w.Dv), dtype=dt, device=dev)
-    y = torch.empty((N, w.D_model), dtype=dt, device=dev)
-    sf = torch.empty((B, H, w.Dk, w.Dv), dtype=torch.float32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
+    only = set(ALL_WORKLOADS) if args.only == "all" else {args.only}
+    records, baselines = {}, {}
+    head_tm, e2e, sampler = None, None, ClockSampler(local)
 
-    def step():
-        K.chunk_fwd(dv["q"], dv["k"], dv["v"], dv["beta"], z=dv["z"], g_min=w.g_min, gate_logits=dv["gate"],
-                    eps=w.eps, out=x, final_state=sf)
-        K.out_proj(x.view(N, H * w.Dv), dv["W_o"], out=y)
-
-    for _ in range(args.warmup):
-        flush.fill_(1.0)
-        step()
-    torch.cuda.synchronize(dev)
-
-    n_ev = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_ev)]
-    sampler = ClockSampler(local)
-    launches0 = lib.kda_launch_count()
-    with sampler:
-        barrier(world)
+    for name in (HEADLINE,) + PREFILL_EXTRA:
+        if name not in only:
+            continue
+        w = rank_workload(name, rank)
+        d = ki.device_inputs(w, dev)
         torch.cuda.synchronize(dev)
-        t_wall0 = time.perf_counter()
-        for i in range(n_ev):
-            flush.fill_(float(i))
-            ev[i][0].record(stream)
-            K.chunk_fwd(dv["q"], dv["k"], dv["v"], dv["beta"], z=dv["z"], g_min=w.g_min,
-                        gate_logits=dv["gate"], eps=w.eps, out=x, final_state=sf)
-            ev[i][1].record(stream)
-            K.out_proj(x.view(N, H * w.Dv), dv["W_o"], out=y)
-            ev[i][2].record(stream)
-        torch.cuda.synchronize(dev)
-        barrier(world)
-        t_wall = time.perf_counter() - t_wall0
-    launches = lib.kda_launch_count() - launches0
-    t_chunk = sum(e[0].elapsed_time(e[1]) for e in ev) / n_ev * 1e-3
-    t_proj = sum(e[1].elapsed_time(e[2]) for e in ev) / n_ev * 1e-3
-    t_step = t_chunk + t_proj
-    t_step_max, t_chunk_max, t_proj_max = reduce_max([t_step, t_chunk, t_proj], world, dev)
+        tm = time_prefill(K, torch, w, d, args.steps, args.warmup, world, dev, flush, lib,
+                          sampler if name == HEADLINE else None)
+        records[name] = prefill_record(w, tm, peaks, world, f"chunk_engine@{name}")
+        records[name]["gpu_launches"] = int(tm["launches"])
+        if name == HEADLINE:
+            head_tm = tm
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            baselines[name] = cpu_baseline_prefill(w, d, 12.0 if name == HEADLINE else 5.0)
+        if name == HEADLINE and not args.no_e2e:
+            e2e = run_e2e(K, torch, w, d, max(2, min(args.steps, 3)), world, dev)
+        del d
+        torch.cuda.empty_cache()
 
-    if args.only == "prefill":
-        return {"metric": METRIC, "value": round(N * world / t_step_max, 1), "unit": "tokens/s",
-                "kernels_ms": {"chunk_engine": round(t_chunk * 1e3, 4), "out_proj": round(t_proj * 1e3, 4)},
-                "gpu_launches": int(launches)} if rank == 0 else None
-
-    # ---------------- end to end through the public API, host buffers
-    hin = {n: torch.from_numpy(inp[n]).to(dt).pin_memory() for n in ("q", "k", "v", "z", "beta", "gate")}
-    h2d = sum(t.numel() * t.element_size() for t in hin.values())
-    for _ in range(2):
-        out = K.kda_forward(hin["q"], hin["k"], hin["v"], hin["z"], hin["beta"], hin["gate"], dv["W_o"],
-                            None, g_min=w.g_min, eps=w.eps, state_dtype=torch.float32)
-    d2h = out["outputs"].numel() * out["outputs"].element_size() + \
-        out["final_state"].numel() * out["final_state"].element_size()
-    e2e_steps = max(3, min(args.steps, 20))
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    t0 = time.perf_counter()
-    for _ in range(e2e_steps):
-        out = K.kda_forward(hin["q"], hin["k"], hin["v"], hin["z"], hin["beta"], hin["gate"], dv["W_o"],
-                            None, g_min=w.g_min, eps=w.eps, state_dtype=torch.float32)
-    torch.cuda.synchronize(dev)
-    t_e2e = (time.perf_counter() - t0) / e2e_steps
-    (t_e2e_max,) = reduce_max([t_e2e], world, dev)
-
-    # ---------------- decode engine (decode_256), state larger than L2
-    dec = run_decode(args, rank, world, local, K, dev, peaks)
+    if DECODE in only:
+        w = rank_workload(DECODE, rank)
+        d = ki.device_inputs(w, dev)
+        records[DECODE] = run_decode(K, torch, w, d, args.warmup, world, dev, peaks, lib)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            baselines[DECODE] = cpu_baseline_decode(w, d, 5.0)
+        del d
+        torch.cuda.empty_cache()
 
     if rank != 0:
         return None
-    tokens_all = N * world
-    value = tokens_all / t_step_max
-    chunk_bytes = prefill_bytes(w)
-    cflops = chunk_flops(w)
-    pflops = proj_flops(N, w)
-    chunk_ach = chunk_bytes / t_chunk / 1e9
-    chunk_tach = cflops / t_chunk / 1e12
-    proj_ach = pflops / t_proj / 1e12
-    chunk_frac = chunk_ach / peaks["hbm_gbs"]
-    chunk_tfrac = chunk_tach / peaks["bf16_tflops"]
-    proj_frac = proj_ach / peaks["bf16_tflops"]
-    if t_chunk >= t_proj:
-        # the chunk products are the path's dense contractions: tensor-pipe roofline, with the HBM view
-        # (algorithmic bytes, DRAM traffic from the ncu capture) beside it
-        roof = {"kernel": "kda_chunk_fwd (chunk engine)", "bound": "tensor", "achieved": round(chunk_tach, 2),
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(chunk_tfrac, 4),
-                "traffic": traffic_for("chunk_engine", PREFILL, "kimi_delta_attention_21_b200/csrc/chunk_tc.cu"),
-                "algorithmic_flops": cflops, "algorithmic_bytes": chunk_bytes,
-                "hbm_achieved_gbs": round(chunk_ach, 1), "hbm_frac": round(chunk_frac, 4),
-                "ms": round(t_chunk * 1e3, 4)}
-    else:
-        roof = {"kernel": "kda_out_proj", "bound": "tensor", "achieved": round(proj_ach, 1),
-                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": round(proj_frac, 4),
-                "traffic": traffic_for("proj", PREFILL, "kimi_delta_attention_21_b200/csrc/proj_tc.cu"),
-                "algorithmic_flops": pflops, "ms": round(t_proj * 1e3, 4)}
-    roof["peak_source"] = f"{peak_src} (burst)"
+    for name, b in baselines.items():
+        records[name]["cpu_baseline"] = b
+    if head_tm is None:   # a partial run for profiling: print what ran
+        return {"metric": METRIC, "partial": True, "n_gpus": world, "workloads": records}
+    w = ki.WORKLOADS[HEADLINE]
+    rec = records.pop(HEADLINE)
     line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(t_step_max * 1e3, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": PREFILL, "B": w.B, "S": w.S, "H": w.H, "D_k": w.Dk, "D_v": w.Dv,
-                   "D_model": w.D_model, "chunk": 64, "g_min": w.g_min, "state": "fp32",
-                   "global_batch": w.B * world, "seq_len": w.S, "parallelism": f"dp{world} (independent sequences)",
-                   "l2": f"flushed between steps ({L2_FLUSH_BYTES >> 20} MiB write, untimed)"},
-        "roofline": roof,
-        "kernels_ms": {"chunk_engine": round(t_chunk * 1e3, 4), "out_proj": round(t_proj * 1e3, 4),
-                       "chunk_engine_tensor_frac": round(chunk_tfrac, 4), "chunk_engine_hbm_frac": round(chunk_frac, 4),
-                       "out_proj_tensor_frac": round(proj_frac, 4)},
-        "e2e": {"value": round(tokens_all / t_e2e_max, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "api": "kimi_delta_attention_21_b200.kda_forward (pinned host tensors)"},
-        "gpu_launches": int(launches),
+        "metric": METRIC, "value": rec["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded, generated on the device)",
+        "config": dict(rec["config"], workload=HEADLINE, global_batch=w.B * world, seq_len=w.S,
+                       parallelism=f"dp{world} (independent sequences)",
+                       l2=f"inputs ({prefill_bytes(w) / 1e9:.1f} GB) larger than L2, and a {L2_FLUSH_BYTES >> 20} "
+                          f"MiB write between steps (untimed)"),
+        "roofline": dict(rec["roofline"], peak_source=f"{peak_src} (burst)"),
+        "layer_roofline": rec["layer_roofline"],
+        "kernels_ms": rec["kernels_ms"],
+        "out_proj": rec["out_proj"],
+        "chunk_engine_tokens_per_s": rec["chunk_engine_tokens_per_s"],
+        "e2e": e2e,
+        "gpu_launches": rec["gpu_launches"],
         "clocks": sampler.summary(),
-        "wall_s_timed_region": round(t_wall, 4),
-        "decode": dec,
+        "wall_s_timed_region": round(head_tm["wall"], 4),
+        "workloads": records,
     }
-    if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_baseline(w, inp)
+    if "cpu_baseline" in rec:
+        line["cpu_baseline"] = rec["cpu_baseline"]
     return line
-
-
-def run_decode(args, rank, world, local, K, dev, peaks):
-    import torch
-    w = rank_workload(DECODE, rank)
-    inp = ki.make_inputs(w)
-    dt = torch.bfloat16
-    T = w.decode_steps
-    dv = {n: torch.from_numpy(inp[n]).to(dev).to(dt) for n in ("q", "k", "v", "z", "beta", "gate", "W_o")}
-    # per-step contiguous inputs (B, H, D) laid out step-major
-    steps = {n: dv[n].transpose(0, 1).contiguous() for n in ("q", "k", "v", "z", "beta", "gate")}
-    state0 = torch.from_numpy(inp["S0"]).to(dev)
-    state = state0.clone()
-    x = torch.empty((w.B, w.H, w.Dv), dtype=dt, device=dev)
-    y = torch.empty((w.B, w.D_model), dtype=dt, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    def one(t):
-        K.decode_step(steps["q"][t], steps["k"][t], steps["v"][t], steps["beta"][t], state, z=steps["z"][t],
-                      g_min=w.g_min, gate_logits=steps["gate"][t], eps=w.eps, out=x)
-
-    for t in range(min(args.warmup, T)):
-        one(t)
-        K.out_proj(x.view(w.B, w.H * w.Dv), dv["W_o"], out=y)
-    state.copy_(state0)
-    torch.cuda.synchronize(dev)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(T)]
-    barrier(world)
-    for t in range(T):
-        ev[t][0].record(stream)
-        one(t)
-        ev[t][1].record(stream)
-        K.out_proj(x.view(w.B, w.H * w.Dv), dv["W_o"], out=y)
-        ev[t][2].record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(world)
-    t_dec = sum(e[0].elapsed_time(e[1]) for e in ev) / T * 1e-3
-    t_prj = sum(e[1].elapsed_time(e[2]) for e in ev) / T * 1e-3
-    t_dec_m, t_prj_m = reduce_max([t_dec, t_prj], world, dev)
-    nb = decode_bytes(w)
-    ach = nb / t_dec / 1e9
-    return {"workload": DECODE, "value": round(w.B * world / (t_dec_m + t_prj_m), 1), "unit": "tokens/s",
-            "steps": T, "ms_per_step": round((t_dec_m + t_prj_m) * 1e3, 4),
-            "kernels_ms": {"decode_step": round(t_dec * 1e3, 4), "out_proj": round(t_prj * 1e3, 4)},
-            "roofline": {"kernel": "kda_decode_step", "bound": "hbm", "achieved": round(ach, 1),
-                         "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4),
-                         "traffic": traffic_for("decode", DECODE, "kimi_delta_attention_21_b200/csrc/decode.cu"),
-                         "algorithmic_bytes": nb},
-            "l2": "state (512 MiB) larger than L2"}
-
-
-def cpu_baseline(w, inp, max_seconds=20.0):
-    """The oracle as it stands on this host's cores, on a bounded sample: the
-    first n tokens (all heads) of the same workload, whole layer forward."""
-    import oracle
-    cores = oracle.default_threads()
-    n = min(w.S, 512)
-    while True:
-        t0 = time.perf_counter()
-        oracle.forward(inp["q"][:, :n], inp["k"][:, :n], inp["v"][:, :n], inp["z"][:, :n], inp["beta"][:, :n],
-                       inp["gate"][:, :n], inp["W_o"], None, g_min=w.g_min, eps=w.eps, threads=cores)
-        dt = time.perf_counter() - t0
-        if n >= w.S or dt * (w.S / n) > max_seconds:
-            break
-        n = w.S
-    return {"value": round(w.B * n / dt, 1), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"first {n} of {w.S} tokens x {w.H} heads of {w.name}, fp64 recurrence + norm/gate + "
-                      f"projection, {dt:.2f} s"}
 
 
 # ----------------------------------------------------------------------------- reference arm (the oracle)
@@ -424,13 +593,13 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     import oracle
-    w = ki.WORKLOADS[PREFILL]
+    w = ki.WORKLOADS[HEADLINE]
     n = min(REF_SAMPLE_TOKENS, w.S)
-    inp = ki.make_inputs(ki.custom("ref_sample", w.B, n, w.H, w.Dk, w.Dv, w.D_model, w.dtype, seed=w.seed))
+    inp = ki.make_inputs_prefix(w, n)
     cores = oracle.default_threads()
 
     def one():
-        oracle.forward(inp["q"], inp["k"], inp["v"], inp["z"], inp["beta"], inp["gate"], inp["W_o"], None,
+        oracle.forward(inp["q"], inp["k"], inp["v"], inp["z"], inp["beta"], inp["gate"], inp["W_o"], inp["S0"],
                        g_min=w.g_min, eps=w.eps, threads=cores)
 
     for _ in range(args.warmup):
@@ -440,11 +609,12 @@ def run_reference(args, rank, world):
         one()
     dt = (time.perf_counter() - t0) / args.steps
     value = round(w.B * n / dt, 1)
-    sample = f"{n} tokens x {w.H} heads of {PREFILL} per step (fp64 oracle, whole layer)"
+    sample = (f"the first {n} tokens x {w.H} heads of {HEADLINE} per step, from its initial state "
+              f"(fp64 oracle, whole layer)")
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt * 1e3, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": PREFILL, "B": w.B, "S": w.S, "H": w.H, "D_k": w.Dk,
+            "data": "synthetic", "config": {"workload": HEADLINE, "B": w.B, "S": w.S, "H": w.H, "D_k": w.Dk,
                                             "D_v": w.Dv, "D_model": w.D_model, "sample_tokens": n},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": sample},
@@ -452,20 +622,31 @@ def run_reference(args, rank, world):
 
 
 def main(argv=None):
+    argv = sys.argv[1:] if argv is None else list(argv)
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
-                    help="run one engine only (for profiling); the default runs both plus e2e")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", choices=("all",) + ALL_WORKLOADS, default="all",
+                    help="time one workload only (for profiling); the default runs all of them")
+    ap.add_argument("--ranks-log", default=None, help="append one line per rank (rank world pid) to this file")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ and args.gpus > 1:
+        return launch_ranks(argv, args.gpus)
     rank, world, local = dist_env()
-    if world != args.gpus and "WORLD_SIZE" in os.environ:
-        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    if world != args.gpus:
+        print(f"bench.py: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+        return 2
+    if args.ranks_log:
+        with open(args.ranks_log, "a") as f:
+            f.write(f"{rank} {world} {os.getpid()}\n")
     if args.impl == "reference":
         line = run_reference(args, rank, world)
     else:

@@ -195,14 +195,17 @@ def out_norm_gate_proj(o, gate_logits, W_o, eps=1e-6, out=None):
 
 
 def kda_forward(query, key, value, decay_logits, write_strength, output_gate_logits, output_projection,
-                initial_state=None, g_min=-5.0, eps=1e-6, *, state_dtype=None, chunk=64, engine="auto"):
+                initial_state=None, g_min=-5.0, eps=1e-6, *, state_dtype=None, chunk=64, engine="auto",
+                outputs=None, final_state_out=None):
     """The KDA layer forward with the "KDA Recurrence" page's interface.
 
     Returns {"outputs": (B,S,D_model), "final_state": (B,H,D_k,D_v)}, both in the
     input dtype (``state_dtype`` overrides the state's dtype, e.g. torch.float32 to
     keep the library's fp32 state) and on the inputs' device.  CPU inputs are
     copied to the current CUDA device and the results copied back; no input is
-    modified.
+    modified.  ``outputs`` / ``final_state_out`` optionally receive the results
+    (tensors of the right shape and dtype on the inputs' device, e.g. reused
+    pinned host buffers).
     """
     dt = query.dtype
     cpu = not query.is_cuda
@@ -228,13 +231,26 @@ def kda_forward(query, key, value, decay_logits, write_strength, output_gate_log
                       chunk=chunk, engine=engine)
     y = out_proj(x.view(B, S, H * v.shape[-1]), W)
     sf = sf.to(state_dtype or dt)
+
+    def dest(given, like, name):
+        if given is None:
+            return torch.empty(like.shape, dtype=like.dtype, pin_memory=True) if cpu else None
+        if tuple(given.shape) != tuple(like.shape) or given.dtype != like.dtype or given.is_cuda == cpu:
+            raise ValueError(f"{name} must be a {like.dtype} tensor of shape {tuple(like.shape)} on the inputs' device")
+        return given
+
+    y_o, s_o = dest(outputs, y, "outputs"), dest(final_state_out, sf, "final_state_out")
     if cpu:
-        y_h = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
-        s_h = torch.empty(sf.shape, dtype=sf.dtype, pin_memory=True)
-        y_h.copy_(y, non_blocking=True)
-        s_h.copy_(sf, non_blocking=True)
+        y_o.copy_(y, non_blocking=True)
+        s_o.copy_(sf, non_blocking=True)
         torch.cuda.current_stream(dev).synchronize()
-        return {"outputs": y_h, "final_state": s_h}
+        return {"outputs": y_o, "final_state": s_o}
+    if y_o is not None:
+        y_o.copy_(y)
+        y = y_o
+    if s_o is not None:
+        s_o.copy_(sf)
+        sf = s_o
     return {"outputs": y, "final_state": sf}
 
 

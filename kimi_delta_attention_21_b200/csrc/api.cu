@@ -11,6 +11,8 @@ namespace kda {
 
 static thread_local char g_err[512];
 
+void clear_error() { g_err[0] = 0; }
+
 void set_error(const char *fmt, ...) {
     va_list ap;
     va_start(ap, fmt);

@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(NT) chunk_simt_kernel(SimtParams p) {
                 const int64_t off = (row0 + r) * strideK + (int64_t)h * Dk + c;
                 kv = load_elem(k, off);
                 qv = load_elem(q, off);
-                g = p.log_decay ? (GT)p.log_decay[off] : log_alpha_gt((GT)load_elem(z, off), p.g_min, GT(0));
+                g = p.log_decay ? (GT)clamp_log_decay(p.log_decay[off], p.g_min) : log_alpha_gt((GT)load_elem(z, off), p.g_min, GT(0));
             }
             sK[r * LD + c] = kv;
             sQ[r * LD + c] = qv;

@@ -298,7 +298,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr) {
                     const int r = qt * 16 + rr;
-                    g[rr] = (r < len) ? p.log_decay[i0 + r * rstr] : 0.f;
+                    g[rr] = (r < len) ? clamp_log_decay(p.log_decay[i0 + r * rstr], p.g_min) : 0.f;
                 }
             } else {
                 if (!mbar_wait(bar_z, zpar)) landed = false;

@@ -46,7 +46,7 @@ decode128_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__re
         const int64_t off = (int64_t)bh * DK + tid;
         s_q[tid] = load_elem(q, off);
         s_k[tid] = load_elem(k, off);
-        const float g = log_decay ? log_decay[off] : log_alpha_of(load_elem(z, off), g_min);
+        const float g = log_decay ? clamp_log_decay(log_decay[off], g_min) : log_alpha_of(load_elem(z, off), g_min);
         s_a[tid] = expf(g);
     }
     __syncthreads();
@@ -179,7 +179,7 @@ decode128_stream_kernel(int nbh, const __nv_bfloat16 *__restrict__ q, const __nv
         const __nv_bfloat16 *sk = sq + 128, *sv = sq + 256, *sz = sq + 384;
         const float *sld = reinterpret_cast<const float *>(vecs + stg * DS_VEC + 1024);
         const __nv_bfloat16 *sg = sq + 768;
-        if (tid < DK) s_a[tid] = expf(log_decay ? sld[tid] : log_alpha_of(__bfloat162float(sz[tid]), g_min));
+        if (tid < DK) s_a[tid] = expf(log_decay ? clamp_log_decay(sld[tid], g_min) : log_alpha_of(__bfloat162float(sz[tid]), g_min));
         if (w == 0) {
             float tq = 0.f;
 #pragma unroll
@@ -277,7 +277,7 @@ decode_generic_kernel(int Dk, int Dv, const T *__restrict__ q, const T *__restri
         const int64_t off = (int64_t)bh * Dk + j;
         s_q[j] = load_elem(q, off);
         s_k[j] = load_elem(k, off);
-        const float g = log_decay ? log_decay[off] : log_alpha_of(load_elem(z, off), g_min);
+        const float g = log_decay ? clamp_log_decay(log_decay[off], g_min) : log_alpha_of(load_elem(z, off), g_min);
         s_a[j] = expf(g);
     }
     __syncthreads();

@@ -12,6 +12,7 @@
 namespace kda {
 
 // ----------------------------------------------------------------- host-side error state
+void clear_error();
 void set_error(const char *fmt, ...);
 kda_status_t fail(kda_status_t s, const char *fmt, ...);
 kda_status_t check_launch(const char *what);
@@ -34,6 +35,11 @@ template <> struct AccT<float> { using type = double; };
 
 // sigmoid in full fp32 precision (expf, not the fast approximation)
 __device__ __forceinline__ float sigmoid_precise(float x) { return 1.0f / (1.0f + expf(-x)); }
+
+// A caller-supplied log(alpha), clamped to the documented range [g_min, 0]
+// (a NaN becomes g_min).  Values outside it would leave the layer's
+// definition and, on the tensor-core path, the range its decay factors cover.
+__device__ __forceinline__ float clamp_log_decay(float g, float g_min) { return fminf(0.0f, fmaxf(g, g_min)); }
 
 // log(alpha) from the decay logits: g_min * sigmoid(z)
 __device__ __forceinline__ float log_alpha_of(float z, float g_min) {

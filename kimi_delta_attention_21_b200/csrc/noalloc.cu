@@ -68,16 +68,19 @@ extern "C" kda_status_t kda_out_norm_gate_proj_noalloc(const void *o, const void
                                                        int64_t N, int32_t H, int32_t D_v, int32_t D_model,
                                                        float eps, void *y, kda_dtype_t dtype, void *stream) {
     using namespace kda;
+    clear_error();
     if (dtype != KDA_F32 && dtype != KDA_BF16) return fail(KDA_ERR_UNSUPPORTED, "dtype %d not supported", (int)dtype);
     if (N < 0 || H < 1 || D_v < 1 || D_model < 1) return fail(KDA_ERR_INVALID_ARG, "bad sizes");
     if (!(isfinite(eps) && eps >= 0.0f)) return fail(KDA_ERR_INVALID_ARG, "eps must be finite and >= 0");
     const size_t es = dtype == KDA_F32 ? 4 : 2;
-    const size_t nx = (size_t)N * H * D_v * es;
-    if (nx > NOALLOC_SCRATCH_BYTES)
+    // the limit is checked on N before any product that could wrap
+    const size_t row_bytes = (size_t)H * (size_t)D_v * es;
+    if (row_bytes > NOALLOC_SCRATCH_BYTES || (uint64_t)N > NOALLOC_SCRATCH_BYTES / row_bytes)
         return fail(KDA_ERR_UNSUPPORTED,
-                    "N*H*D_v*element_size = %zu bytes exceeds the fixed %zu-byte scratch of the no-allocation "
-                    "entry point; use kda_out_norm_gate_proj with a workspace",
-                    nx, NOALLOC_SCRATCH_BYTES);
+                    "N*H*D_v*element_size (N = %lld, %zu bytes per row) exceeds the fixed %zu-byte scratch of the "
+                    "no-allocation entry point; use kda_out_norm_gate_proj with a workspace",
+                    (long long)N, row_bytes, NOALLOC_SCRATCH_BYTES);
+    const size_t nx = (size_t)N * row_bytes;
     if (N == 0) return KDA_OK;
     const void *ptrs[] = {o, gate_logits, W_o, y};
     const char *names[] = {"o", "gate_logits", "W_o", "y"};

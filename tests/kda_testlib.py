@@ -107,3 +107,25 @@ def oracle_head(w, b, h, t_rec=None, threads=1):
                               z=sl(hd["z"]), g_min=w.g_min, initial_state=s0, t_rec=t_rec, threads=threads)
     gate = hd["gate"][b, t_rec if t_rec is not None else slice(None)]
     return o[0, :, 0], sf[0, 0], gate
+
+
+def oracle_head_dev(w, d, b, h, t_rec=None, threads=1):
+    """Oracle o~ (at t_rec tokens), final state and gate logits for one (b, h) of
+    device-generated inputs ``d`` (kda_inputs.device_inputs): the device's own
+    input bytes are copied to the host and run through the fp64 recurrence."""
+    hs = ki.host_slice(d, b, h)
+    o, sf = oracle.recurrence(hs["q"], hs["k"], hs["v"], hs["beta"], z=hs["z"], g_min=w.g_min,
+                              initial_state=hs["S0"], t_rec=t_rec, threads=threads)
+    gate = hs["gate"][0, t_rec if t_rec is not None else slice(None), 0]
+    return o[0, :, 0], sf[0, 0], gate
+
+
+def oracle_heads_dev(w, d, pairs, t_rec=None, workers=None):
+    """oracle_head_dev over several (b, h) pairs in parallel host threads (the
+    oracle's C recurrence runs without the interpreter lock)."""
+    import concurrent.futures as cf
+    import os
+    workers = workers or max(1, min(len(pairs), len(os.sched_getaffinity(0))))
+    with cf.ThreadPoolExecutor(workers) as ex:
+        futs = {bh: ex.submit(oracle_head_dev, w, d, bh[0], bh[1], t_rec) for bh in pairs}
+        return {bh: f.result() for bh, f in futs.items()}

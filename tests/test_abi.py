@@ -184,3 +184,18 @@ def test_tc_workspace_and_segment_count(B, S, H, G):
     want, g = _expected_tc_workspace(B, S, H)
     assert g == G
     assert n.value == want
+
+
+def test_noalloc_size_check_cannot_be_wrapped():
+    """A row count whose byte size wraps 64 bits is rejected on the host before
+    any CUDA call (fake, aligned, non-NULL pointers: nothing is dereferenced)."""
+    lib = _lib.load()
+    H, Dv, Dm = 16, 128, 64
+    N = (1 << 64) // (H * Dv * 2) + 1            # N * H * Dv * 2 wraps to 4096
+    fake = [ctypes.c_void_p(0x100000 * (i + 1)) for i in range(4)]
+    n0 = lib.kda_launch_count()
+    st = lib.kda_out_norm_gate_proj_noalloc(fake[0], fake[1], fake[2], N, H, Dv, Dm, 1e-6, fake[3], _lib.KDA_BF16,
+                                            None)
+    assert st == _lib.KDA_ERR_UNSUPPORTED
+    assert "scratch" in lib.kda_last_error().decode()
+    assert lib.kda_launch_count() == n0

@@ -1,6 +1,8 @@
 """bench.py's multi-rank host logic (one process per GPU on a real run) with
 world_size 2 over gloo on CPU: rank-specific inputs, max-over-ranks timing,
-barrier, and the reference arm running on rank 0 only."""
+barrier, the reference arm running on rank 0 only, and the launcher that
+``--gpus N`` starts when no WORLD_SIZE is set."""
+import json
 import os
 import socket
 import sys
@@ -32,7 +34,7 @@ def _worker(rank, world, port, q):
         t = [1.0 + rank, 10.0 - rank]
         m = bench.reduce_max(t, wsz)
         bench.barrier(wsz)
-        w = bench.rank_workload(bench.PREFILL, rank)
+        w = bench.rank_workload(bench.HEADLINE, rank)
         q.put((rank, m, w.seed, None))
     finally:
         dist.destroy_process_group()
@@ -65,3 +67,31 @@ def test_reference_arm_runs_on_rank0_only(monkeypatch):
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0
     assert line["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_gpus_flag_launches_that_many_ranks(tmp_path, capfd, monkeypatch):
+    """`bench.py --gpus 2` without a launcher starts two rank processes itself;
+    rank 0 prints the one JSON line with n_gpus 2."""
+    sys.path.insert(0, ROOT)
+    import bench
+    for v in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(v, raising=False)
+    log = tmp_path / "ranks.txt"
+    rc = bench.main(["--gpus", "2", "--impl", "reference", "--steps", "1", "--warmup", "3",
+                     "--ranks-log", str(log)])
+    assert rc == 0
+    lines = sorted(log.read_text().split("\n")[:-1])
+    assert [ln.split()[:2] for ln in lines] == [["0", "2"], ["1", "2"]]
+    assert len({ln.split()[2] for ln in lines}) == 2          # two processes
+    out = [ln for ln in capfd.readouterr().out.splitlines() if ln.startswith("{")]
+    assert len(out) == 1                                       # rank 0 alone prints
+    rec = json.loads(out[0])
+    assert rec["n_gpus"] == 2 and rec["impl"] == "reference"
+
+
+def test_gpus_flag_disagreeing_with_launcher_fails(monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setenv("RANK", "0")
+    assert bench.main(["--gpus", "2", "--impl", "reference", "--steps", "1", "--warmup", "3"]) == 2

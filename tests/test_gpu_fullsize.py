@@ -1,13 +1,14 @@
 """Parity at the full workload sizes, in the launch configuration bench.py
-times (default engine choice), on outputs the oracle can compute one head at a
-time, plus properties that hold at any size."""
+times (default engine choice, device-generated inputs), on outputs the oracle
+can compute one head at a time from the device's own input bytes, plus
+properties that hold at any size."""
 import numpy as np
 import pytest
 
 import kda_inputs as ki
 import oracle
-from kda_testlib import (BF16_OUT_ATOL, assert_bf16_outputs, assert_bf16_state, oracle_head, rel_fro, to_np,
-                         upload_by_head)
+from kda_testlib import (BF16_OUT_ATOL, assert_bf16_outputs, assert_bf16_state, oracle_heads_dev, rel_fro,
+                         to_np)
 
 torch = pytest.importorskip("torch")
 pytestmark = [pytest.mark.gpu, pytest.mark.slow]
@@ -28,27 +29,49 @@ def _check_projection_rows(x, y, W, rows):
     assert_bf16_outputs(to_np(y.reshape(-1, y.shape[-1]).index_select(0, idx)), want, "projection rows")
 
 
-def _check_heads(w, x, sf, heads, t_rec):
-    for b, h in heads:
-        o_ref, s_ref, gate = oracle_head(w, b, h, t_rec=t_rec)
-        x_ref = oracle.norm_gate(o_ref, gate, w.eps)
-        idx = torch.as_tensor(np.asarray(t_rec), device=x.device)
-        assert_bf16_outputs(to_np(x[b, :, h].index_select(0, idx)), x_ref, f"x (b={b}, h={h})")
+def _check_heads(w, d, x, sf, pairs, t_rec, states_only=()):
+    """x[b, t_rec, h] and sf[b, h] against the oracle for every (b, h) in pairs
+    (final state only for the pairs in states_only)."""
+    ref = oracle_heads_dev(w, d, list(pairs) + list(states_only), t_rec=t_rec)
+    idx = torch.as_tensor(np.asarray(t_rec), device=x.device)
+    for (b, h), (o_ref, s_ref, gate) in ref.items():
         assert_bf16_state(to_np(sf[b, h]), s_ref, f"final state (b={b}, h={h})")
+        if (b, h) in pairs:
+            x_ref = oracle.norm_gate(o_ref, gate, w.eps)
+            assert_bf16_outputs(to_np(x[b, :, h].index_select(0, idx)), x_ref, f"x (b={b}, h={h})")
 
 
-@pytest.mark.parametrize("name", ["prefill_4k", "batch_8x8k"])
-def test_full_size_prefill(K, name):
-    w = ki.WORKLOADS[name]
-    d = upload_by_head(w)
+def _tokens(S, n, seed):
+    rng = np.random.default_rng(seed)
+    edge = [0, 1, 63, 64, 65, S // 2, S - 65, S - 64, S - 1]
+    return np.unique(np.concatenate([[t for t in edge if 0 <= t < S], rng.integers(0, S, n)]))
+
+
+def test_full_size_prefill_4k(K):
+    w = ki.WORKLOADS["prefill_4k"]
+    d = ki.device_inputs(w, "cuda")
     x, sf = K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=d["z"], g_min=w.g_min, initial_state=d["S0"],
                         gate_logits=d["gate"], eps=w.eps)
     y = K.out_proj(x.view(w.B, w.S, w.H * w.Dv), d["W_o"])
     torch.cuda.synchronize()
-    rng = np.random.default_rng(0)
-    t_rec = np.unique(np.concatenate([[0, 1, 63, 64, w.S - 1], rng.integers(0, w.S, 40)]))
-    heads = [(0, 0), (w.B - 1, w.H - 1), (w.B // 2, w.H // 2)]
-    _check_heads(w, x, sf, heads, t_rec)
+    t_rec = _tokens(w.S, 120, 0)
+    _check_heads(w, d, x, sf, [(0, h) for h in range(w.H)], t_rec)          # every head
+    rows = np.unique(np.concatenate([[0, w.S - 1], np.random.default_rng(1).integers(0, w.S, 200)]))
+    _check_projection_rows(x, y, d["W_o"], rows)
+
+
+def test_full_size_batch_8x8k(K):
+    w = ki.WORKLOADS["batch_8x8k"]
+    d = ki.device_inputs(w, "cuda")
+    x, sf = K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=d["z"], g_min=w.g_min, initial_state=d["S0"],
+                        gate_logits=d["gate"], eps=w.eps)
+    y = K.out_proj(x.view(w.B, w.S, w.H * w.Dv), d["W_o"])
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(2)
+    pairs = {(0, 0), (w.B - 1, w.H - 1), (w.B // 2, w.H // 2)}
+    while len(pairs) < 16:
+        pairs.add((int(rng.integers(0, w.B)), int(rng.integers(0, w.H))))
+    _check_heads(w, d, x, sf, sorted(pairs), _tokens(w.S, 64, 3))
     rows = np.unique(np.concatenate([[0, w.B * w.S - 1], rng.integers(0, w.B * w.S, 200)]))
     _check_projection_rows(x, y, d["W_o"], rows)
     assert np.isfinite(to_np(y.float().view(-1)[:: 9973])).all()
@@ -56,12 +79,14 @@ def test_full_size_prefill(K, name):
 
 def test_full_size_long_context(K):
     w = ki.WORKLOADS["long_1m"]
-    d = upload_by_head(w)
+    d = ki.device_inputs(w, "cuda")
     x, sf = K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=d["z"], g_min=w.g_min, initial_state=d["S0"],
                         gate_logits=d["gate"], eps=w.eps)
     torch.cuda.synchronize()
-    t_rec = np.array([0, 1, 4095, 500000, w.S - 65, w.S - 1])
-    _check_heads(w, x, sf, [(0, 5)], t_rec)
+    # every head's final state; o~ on 72+ tokens of four heads
+    t_rec = _tokens(w.S, 64, 4)
+    out_heads = [(0, 0), (0, 5), (0, 10), (0, 15)]
+    _check_heads(w, d, x, sf, out_heads, t_rec, states_only=[(0, h) for h in range(w.H) if (0, h) not in out_heads])
     # property at full size: a split at an unaligned token with the state handed over
     cut = 700001
     sl = lambda t, a, b: t[:, a:b].contiguous()
@@ -78,7 +103,7 @@ def test_full_size_long_context(K):
 
 def test_full_size_decode(K):
     w = ki.WORKLOADS["decode_256"]
-    d = upload_by_head(w)
+    d = ki.device_inputs(w, "cuda")
     steps = {n: d[n].transpose(0, 1).contiguous() for n in ("q", "k", "v", "z", "beta", "gate")}
     state = d["S0"].clone()
     xs = []
@@ -88,6 +113,9 @@ def test_full_size_decode(K):
     y_last = K.out_proj(xs[-1].view(w.B, w.H * w.Dv), d["W_o"])
     torch.cuda.synchronize()
     x = torch.stack(xs, 1)  # (B, T, H, Dv)
-    t_rec = np.arange(w.decode_steps)
-    _check_heads(w, x, state, [(0, 0), (255, 31), (100, 7), (17, 20)], t_rec)
+    rng = np.random.default_rng(5)
+    pairs = {(0, 0), (255, 31), (100, 7), (17, 20)}
+    while len(pairs) < 16:
+        pairs.add((int(rng.integers(0, w.B)), int(rng.integers(0, w.H))))
+    _check_heads(w, d, x, state, sorted(pairs), np.arange(w.decode_steps))
     _check_projection_rows(x[:, -1:], y_last, d["W_o"], np.arange(0, 256, 17))
