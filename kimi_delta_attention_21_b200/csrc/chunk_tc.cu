@@ -76,7 +76,7 @@ constexpr uint32_t REC_MT = 49152;    // M^T            [64 rows i][128 B: r]; w
 constexpr uint32_t REC_U = 57344;     // U^T            [128 rows j][128 B: r]
 constexpr uint32_t REC_GAM = 73728;   // e^{G_C}        128 fp32
 constexpr uint32_t REC_BYTES = 74240;
-constexpr uint32_t SIG_BYTES = CH * 128 * 2;  // per chunk: sigmoid of the output-gate logits, [64][128] f16
+constexpr uint32_t GATE_TILE_BYTES = CH * 128 * 2;  // one chunk of output-gate logits, [2 atoms][64 rows][128 B] bf16
 
 __device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
     return row * 128u + ((chunk ^ (row & 7u)) << 4);
@@ -184,9 +184,7 @@ struct PrepArgs {
     float g_min;
     const __nv_bfloat16 *beta;
     const float *log_decay;
-    const __nv_bfloat16 *gate;  // output-gate logits (B, S, H, 128), or null
     uint8_t *ws;
-    __half *sig;                // sigmoid(gate) per (b, h, chunk): [2 atoms (j / 64)][64 rows r][128 B] f16, swizzled
     unsigned int *timeouts;
     int *dev_status;
 };
@@ -238,38 +236,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         int n, h, b;
         unit_coords(u, n, h, b);
         for (int a = 0; a < 2; ++a) tma_load_4d(sm + P_VI + a * 8192, &tv, bar_in, 64 * a, h, n * CH, b);
-    };
-
-    // sigmoid of the output-gate logits (full fp32, stored as f16) for the state kernel's output stage,
-    // in its tile layout [2 atoms (j / 64)][64 rows r][128 B], 128-byte swizzled.  Warps 4-15 take the
-    // 1024 groups of 8 values while warps 0-3 invert (I + A); the logits were prefetched into L2 one
-    // unit ahead.
-    constexpr int SIG_T = PREP_THREADS - 128;
-    auto gate_sigmoid = [&](int n, int h, int b, int t0, int len) {
-        if (!p.gate || tid < 128) return;
-        const __nv_bfloat16 *src = p.gate + (((int64_t)b * p.S + t0) * p.H + h) * DD;
-        uint8_t *dst = reinterpret_cast<uint8_t *>(p.sig + ((size_t)(b * p.H + h) * p.Nc + n) * (CH * DD));
-        uint4 gv[3] = {};
-#pragma unroll
-        for (int k = 0; k < 3; ++k) {
-            const int gi = tid - 128 + SIG_T * k, row = gi >> 4;
-            if (gi < CH * DD / 8 && row < len)
-                gv[k] = *reinterpret_cast<const uint4 *>(src + (int64_t)row * p.H * DD + (gi & 15) * 8);
-        }
-#pragma unroll
-        for (int k = 0; k < 3; ++k) {
-            const int gi = tid - 128 + SIG_T * k, row = gi >> 4, c8 = (gi & 15) * 8;
-            if (gi >= CH * DD / 8 || row >= len) continue;
-            float g[8];
-            unpack8(gv[k], g);
-            uint4 o;
-            __half2 *oh = reinterpret_cast<__half2 *>(&o);
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                oh[e] = __floats2half2_rn(__fdividef(1.0f, 1.0f + __expf(-g[2 * e])),
-                                          __fdividef(1.0f, 1.0f + __expf(-g[2 * e + 1])));
-            *reinterpret_cast<uint4 *>(dst + (c8 >> 6) * 8192 + sw128(row, (c8 & 63) >> 3)) = o;
-        }
     };
 
     // P1 and the per-channel tables of unit u: beta, G = in-chunk cumulative log-decay (rows past the
@@ -386,21 +352,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     for (int64_t u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++it) {
         int n, h, b;
         unit_coords(u, n, h, b);
-        const int t0 = n * CH;
-        const int len = min(CH, p.S - t0);
         const int64_t u_next = u + gridDim.x;
         const uint32_t par = it & 1;
         // the next unit's beta, consumed by its tables (issued now, so its latency stays hidden)
         const float beta_next = (tid < CH && u_next < p.units) ? load_beta(u_next) : 0.f;
-        if (u_next < p.units && tid < 256) {  // the next unit's gate and log-decay inputs -> L2
+        if (u_next < p.units && tid < 256 && p.log_decay) {  // the next unit's log-decay input -> L2
             int n2, h2, b2;
             unit_coords(u_next, n2, h2, b2);
             const int64_t row0 = ((int64_t)b2 * p.S + n2 * CH) * p.H + h2;
-            if (tid < 128) {
-                const int row = tid >> 1;
-                if (p.gate && n2 * CH + row < p.S)
-                    prefetch_l2(p.gate + (row0 + (int64_t)row * p.H) * DD + (tid & 1) * 64);
-            }
             const int row = tid >> 2;
             if (p.log_decay && n2 * CH + row < p.S)
                 prefetch_l2(p.log_decay + (row0 + (int64_t)row * p.H) * DD + (tid & 3) * 32);
@@ -629,7 +588,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         // forward substitution, then T_{R,R-1} = -T_RR A_{R,R-1} T_{R-1,R-1} for R = 1, 3, then the lower-left
         // 32x32 block the same way from the two diagonal 32x32 blocks.  Blocks above the diagonal are written
         // as zeros where a later product reads them; the T image zero-fills the upper-right 32x32 block.
-        // Warps 0-3 only (named barrier 1); warps 4-15 compute the gate sigmoid meanwhile.
+        // Warps 0-3 only (named barrier 1).
         if (warp < 4) {
             const float *sA = reinterpret_cast<const float *>(sm + P_SA);
             float *sT = reinterpret_cast<float *>(sm + P_ST);
@@ -757,8 +716,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 *reinterpret_cast<uint4 *>(sm + P_TI + sw128(r, cc)) = pack8(t);
             }
             fence_proxy_async_smem();
-        } else {
-            gate_sigmoid(n, h, b, t0, len);
         }
         tc_fence_before();
         __syncthreads();
@@ -862,7 +819,7 @@ struct StateArgs {
     int S, H, Nc;
     int L, G;              // chunks per segment, segments per sequence
     const uint8_t *ws;
-    const __half *sig;     // sigmoid of the output-gate logits per chunk (tile layout), or null: write o~
+    bool gated;            // apply RMSNorm and sigmoid(gate logits) (tensor map tgl); else write o~
     const float *S0;
     float *Sf;
     const float *seg_init; // state entering segment g >= 1, [B*H][G][128][128] (after the combine pass)
@@ -877,7 +834,7 @@ constexpr int ST_THREADS = 288;                // warps 0-7 register work, warp 
 constexpr uint32_t ST_STAGE = REC_GAM;         // the image part of a record (73728 B)
 constexpr uint32_t ST_GAM = 2 * ST_STAGE;      // e^{G_C} [2 stages][128] fp32 (the maps: 3 stages, into OIMG)
 constexpr uint32_t ST_OIMG = ST_GAM + 1024;    // output tile [2 atoms (j / 64)][64 rows r][128 B]
-constexpr uint32_t ST_SIGT = ST_OIMG + 16384;  // sigmoid(gate) tile, same layout, f16
+constexpr uint32_t ST_SIGT = ST_OIMG + 16384;  // output-gate logits tile (TMA), same layout, bf16
 constexpr uint32_t ST_OT = ST_SIGT + 16384;    // O^T image, K-major B [128 rows j][128 B: 64 r]
 constexpr uint32_t ST_ID = ST_OT + 16384;      // [I_64; I_64], K-major A [128 rows][128 B: 64 k]
 constexpr uint32_t ST_RED = ST_ID + 16384;     // per-row partial sums of squares [64][4] fp32
@@ -898,7 +855,7 @@ constexpr uint32_t ST_TCOLS = 512;
 //               g = (z + 1) / 2: odd z from S = I without U (-> A_g), even z from S = 0 with U (-> Y_g).
 template <bool kMap>
 __global__ void __launch_bounds__(ST_THREADS, 1)
-chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
+chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constant__ CUtensorMap tgl, StateArgs p) {
     pdl_trigger();
     pdl_wait();
     extern __shared__ uint8_t smraw[];
@@ -928,7 +885,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
     uint64_t *bar_simg = bars + 7;   // bf16 copy of S^T written (8 warps)
     uint64_t *bar_vimg = bars + 8;   // bf16 copy of V'^T written (8 warps)
     uint64_t *bar_ot = bars + 9;     // O^T image written (8 warps)
-    uint64_t *bar_sig = bars + 10;   // sigmoid tile landed
+    uint64_t *bar_sig = bars + 10;   // gate-logits tile landed
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 11);
     float *sgam = reinterpret_cast<float *>(sm + ST_GAM);
     float *red = reinterpret_cast<float *>(sm + ST_RED);
@@ -1065,10 +1022,11 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
             }
             tmem_wait_st();
         }
-        auto load_sig = [&](int m) {  // sigmoid tile of chunk m -> shared memory (thread 0)
-            if (!kMap && tid == 0 && p.sig && m < nc) {
-                mbar_arrive_expect_tx(bar_sig, SIG_BYTES);
-                bulk_load(sm + ST_SIGT, p.sig + ((size_t)bh * p.Nc + n0 + m) * (CH * DD), SIG_BYTES, bar_sig);
+        auto load_sig = [&](int m) {  // gate-logits tile of chunk m -> shared memory (thread 0)
+            if (!kMap && tid == 0 && p.gated && m < nc) {
+                mbar_arrive_expect_tx(bar_sig, GATE_TILE_BYTES);
+                tma_load_4d(sm + ST_SIGT, &tgl, bar_sig, 0, h, (n0 + m) * CH, b);
+                tma_load_4d(sm + ST_SIGT + 8192, &tgl, bar_sig, 64, h, (n0 + m) * CH, b);
             }
         };
         // O^T of chunk m (PO[m & 1][j, 64 + r]) -> bf16 operand image (all warps; after bar_o(m))
@@ -1100,7 +1058,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
             tc_fence_after();
             bool okw = true;
             float inv = 1.f;
-            if (p.sig) {
+            if (p.gated) {
                 uint32_t ov[32];
                 tmem_ld_32x32b_x32(ocol, ov);
                 tmem_wait_ld();
@@ -1111,7 +1069,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
             }
             if (tid == 0) bulk_wait_read_all();  // the previous tile's store has left shared memory
             named_sync(1, 256);
-            if (p.sig) {
+            if (p.gated) {
                 const float4 rr = *reinterpret_cast<const float4 *>(red + r * 4);
                 inv = rsqrtf(((rr.x + rr.y) + (rr.z + rr.w)) * (1.0f / 128.0f) + p.eps);
                 okw = mbar_wait(bar_sig, m & 1);
@@ -1126,15 +1084,11 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
                     float f[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(ov[8 * k + e]);
-                    if (p.sig) {
-                        const uint4 g8 = *reinterpret_cast<const uint4 *>(sm + ST_SIGT + off);
-                        const __half2 *gh = reinterpret_cast<const __half2 *>(&g8);
+                    if (p.gated) {  // RMSNorm, then the sigmoid of the gate logits (fp32)
+                        float gl[8];
+                        unpack8(*reinterpret_cast<const uint4 *>(sm + ST_SIGT + off), gl);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 g = __half22float2(gh[e]);
-                            f[2 * e] *= inv * g.x;
-                            f[2 * e + 1] *= inv * g.y;
-                        }
+                        for (int e = 0; e < 8; ++e) f[e] *= inv * __fdividef(1.0f, 1.0f + __expf(-gl[e]));
                     }
                     *reinterpret_cast<uint4 *>(sm + ST_OIMG + off) = pack8(f);
                 }
@@ -1274,7 +1228,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, StateArgs p) {
         // let the bulk copies already issued land before the CTA exits
         for (int m = landed; m < issued; ++m) mbar_wait(&full[m % STG], (m / STG) & 1, 100000000ull);
     }
-    if (!kMap && tid == 0 && s_fail && p.sig) mbar_wait(bar_sig, 0, 100000000ull), mbar_wait(bar_sig, 1, 100000000ull);
+    if (!kMap && tid == 0 && s_fail && p.gated) mbar_wait(bar_sig, 0, 100000000ull), mbar_wait(bar_sig, 1, 100000000ull);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, ST_TCOLS);
@@ -1426,11 +1380,12 @@ int device_sms() {
     return sms;
 }
 
-kda_status_t launch_state(const CUtensorMap &tmo, const StateArgs &sa, int B, int H, cudaStream_t st) {
+kda_status_t launch_state(const CUtensorMap &tmo, const CUtensorMap &tgl, const StateArgs &sa, int B, int H,
+                          cudaStream_t st) {
     if (sa.G > 1) {
         cudaFuncSetAttribute(chunk_state_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
         cudaError_t e = launch_pdl(chunk_state_kernel<true>, dim3(H, B, 2 * sa.G - 3), dim3(ST_THREADS),
-                                   STATE_SMEM, st, tmo, sa);
+                                   STATE_SMEM, st, tmo, tgl, sa);
         if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "chunk_state_kernel (segment maps): %s", cudaGetErrorString(e));
         kda_status_t s = check_launch("chunk_state_kernel (segment maps)");
         if (s != KDA_OK) return s;
@@ -1451,7 +1406,8 @@ kda_status_t launch_state(const CUtensorMap &tmo, const StateArgs &sa, int B, in
         if (s != KDA_OK) return s;
     }
     cudaFuncSetAttribute(chunk_state_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
-    cudaError_t e = launch_pdl(chunk_state_kernel<false>, dim3(H, B, sa.G), dim3(ST_THREADS), STATE_SMEM, st, tmo, sa);
+    cudaError_t e = launch_pdl(chunk_state_kernel<false>, dim3(H, B, sa.G), dim3(ST_THREADS), STATE_SMEM, st, tmo, tgl,
+                               sa);
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "chunk_state_kernel: %s", cudaGetErrorString(e));
     return check_launch("chunk_state_kernel");
 }
@@ -1483,11 +1439,11 @@ bool chunk_tc_aligned(const kda_chunk_args &a) {
     return okp;
 }
 
-// Workspace: records and gate tiles per chunk, then (with several segments) the segment maps
+// Workspace: one record per chunk, then (with several segments) the segment maps
 // A_g^T (bf16 images) and Y_g, and the segments' entering states.
 struct TcLayout {
     int G, L;
-    size_t sig, xt, yt, seg, total;
+    size_t xt, yt, seg, total;
 };
 
 TcLayout tc_layout(const kda_chunk_args &a) {
@@ -1496,8 +1452,7 @@ TcLayout tc_layout(const kda_chunk_args &a) {
     t.G = pick_segments(BH, Nc, device_sms());
     t.L = (int)((Nc + t.G - 1) / t.G);
     if (Nc > 0) t.G = (int)((Nc + t.L - 1) / t.L);  // no empty segment
-    t.sig = (size_t)BH * Nc * REC_BYTES;
-    t.xt = t.sig + (size_t)BH * Nc * SIG_BYTES;
+    t.xt = (size_t)BH * Nc * REC_BYTES;
     const size_t nmap = t.G > 1 ? (size_t)BH * (t.G - 1) : 0;
     t.yt = t.xt + nmap * 32768;
     t.seg = t.yt + nmap * DD * DD * 4;
@@ -1510,17 +1465,21 @@ size_t chunk_tc_workspace(const kda_chunk_args &a) { return tc_layout(a).total; 
 kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
     const int64_t Nc = (a.S + CH - 1) / CH;
     unsigned int *timeouts = device_timeout_counter();
-    CUtensorMap to;
+    CUtensorMap to, tgl;
     memset(&to, 0, sizeof(to));  // (no chunks: never read)
+    memset(&tgl, 0, sizeof(tgl));  // (no gate: never read)
     const TcLayout lay = tc_layout(a);
     uint8_t *ws = (uint8_t *)a.workspace;
-    __half *sig = reinterpret_cast<__half *>(ws + lay.sig);
     if (Nc > 0) {
         CUtensorMap tq, tk, tv, tz;
         const uint64_t rs = (uint64_t)DD, ss = (uint64_t)a.H * DD, bs = (uint64_t)a.S * a.H * DD;
         kda_status_t s;
         s = make_tmap_tokens(&to, a.o, a.H, a.S, a.B, rs, ss, bs);
         if (s != KDA_OK) return s;
+        if (a.gate_logits) {
+            s = make_tmap_tokens(&tgl, a.gate_logits, a.H, a.S, a.B, rs, ss, bs);
+            if (s != KDA_OK) return s;
+        }
         s = make_tmap_tokens(&tq, a.q, a.H, a.S, a.B, rs, ss, bs);
         if (s != KDA_OK) return s;
         s = make_tmap_tokens(&tk, a.k, a.H, a.S, a.B, rs, ss, bs);
@@ -1543,8 +1502,6 @@ kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
         pa.beta = (const __nv_bfloat16 *)a.beta;
         pa.log_decay = a.log_decay;
         pa.ws = (uint8_t *)a.workspace;
-        pa.gate = (const __nv_bfloat16 *)a.gate_logits;
-        pa.sig = sig;
         pa.timeouts = timeouts;
         pa.dev_status = a.dev_status;
         const int sms = device_sms();
@@ -1563,7 +1520,7 @@ kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
     sa.ws = (const uint8_t *)a.workspace;
     sa.S0 = a.initial_state;
     sa.Sf = a.final_state;
-    sa.sig = a.gate_logits ? sig : nullptr;
+    sa.gated = a.gate_logits != nullptr && Nc > 0;
     sa.L = Nc > 0 ? lay.L : 1;
     sa.G = Nc > 0 ? lay.G : 1;
     sa.xt = ws + lay.xt;
@@ -1572,7 +1529,7 @@ kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
     sa.eps = a.eps;
     sa.timeouts = timeouts;
     sa.dev_status = a.dev_status;
-    return launch_state(to, sa, (int)a.B, a.H, st);
+    return launch_state(to, tgl, sa, (int)a.B, a.H, st);
 }
 
 }  // namespace kda

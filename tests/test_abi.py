@@ -157,18 +157,18 @@ def test_workspace_query_needs_no_device():
 
 
 def _expected_tc_workspace(B, S, H, sms=148):
-    """Workspace of the tensor-core chunk engine, from the rule it follows: per-chunk records and gate
-    tiles, and, with G segments, BH (G - 1) map slots (A image + Y) and BH G entering states, G the
+    """Workspace of the tensor-core chunk engine, from the rule it follows: per-chunk records, and,
+    with G segments, BH (G - 1) map slots (A image + Y) and BH G entering states, G the
     largest count for which the map pass (BH (2G - 3) CTAs) and the chain pass (BH G CTAs) each fit
     in one wave, at least 4 chunks per segment, and no empty segment."""
-    rec, sig = 74240, 64 * 128 * 2
+    rec = 74240
     bh, nc = B * H, (S + 63) // 64
     per_sm = sms // bh
     g = min((per_sm + 3) // 2, per_sm, nc // 4)
     g = max(g, 1)
     L = (nc + g - 1) // g
     g = (nc + L - 1) // L
-    ws = bh * nc * (rec + sig)
+    ws = bh * nc * rec
     if g > 1:
         ws += bh * (g - 1) * (32768 + 65536) + bh * g * 128 * 128 * 4
     return ws, g
