@@ -798,23 +798,27 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
 }
 
 // ================================================================ K2b: chunk_state_kernel
-// One CTA per (head, batch) walks the chunks in order.  The state is kept
-// transposed in TMEM: lane j (value column) holds S[:, j] in fp32, so every
-// per-chunk product takes its A operand straight from TMEM and the register
-// work of the chain is spread over all 128 lanes.  Warp 8 issues the MMAs and
-// the record copies; warps 0-7 (lane quarter = warp % 4, column half =
-// warp / 4) do the register work.  Per chunk n:
-//   warps:    S^T -> bf16 copy in TMEM; S^T <- S^T Diag(e^{G_C})
-//   MMA:      PO  = S^T [-W; Q e^G]^T           PO[j, r] = -(W S)[r, j],  PO[j, 64 + r] = (Q e^G S)[r, j]
-//   warps:    V'^T = U^T + PO[:, 0:64] -> bf16 copy in TMEM
-//   MMA:      S^T += V'^T K~,  PO[:, 64:128] += V'^T M^T      (= O^T of chunk n)
-// and, one chunk behind, the output: the warps write O^T (bf16) as an operand
-// image, one MMA with [I; I] turns it back into token rows (into the PO
-// buffer, now free; lanes 64-127 repeat lanes 0-63), and the eight warps, 32
-// rows x 32 columns each, apply the RMS normalisation over the head and the
-// sigmoid output gate (precomputed by the prep kernel) and store the tile with
-// a TMA tensor store.
-// Records stream in by bulk copies, two stages deep.
+// One CTA per (head, batch, segment) walks the chunks in order.  The state is
+// kept transposed in TMEM: lane j (value column) holds S[:, j] in fp32, so
+// every per-chunk product takes its A operand straight from TMEM and the
+// register work of the chain is spread over all 128 lanes.  Warp roles:
+//   warps 0-7   the chain's register work (lane quarter = warp % 4, column
+//               half = warp / 4);
+//   warp 8      issues the MMAs and the record copies (one thread);
+//   warps 9-12  the output stage (chains only; the maps have no output).
+// Per chunk n:
+//   chain warps:  S^T -> bf16 copy in TMEM; S^T <- S^T Diag(e^{G_C})
+//   MMA:          PO  = S^T [-W; Q e^G]^T        PO[j, r] = -(W S)[r, j],  PO[j, 64 + r] = (Q e^G S)[r, j]
+//   chain warps:  V'^T = U^T + PO[:, 0:64] -> bf16 copy in TMEM
+//   MMA:          S^T += V'^T K~,  PO[:, 64:128] += V'^T M^T      (= O^T of chunk n)
+// and, off the chain's critical path, the output warps write O^T (bf16) as an
+// operand image, one MMA with [I; I] turns it back into token rows (into the
+// same PO buffer; lanes 64-127 repeat lanes 0-63), and the output warps, 32
+// rows x 64 columns each, apply the RMS normalisation over the head and the
+// sigmoid of the output-gate logits (a bf16 tile loaded by TMA one chunk
+// ahead) and store the tile with a TMA tensor store.  PO is double-buffered;
+// a buffer is reused for chunk n + 2 once the output warps have read chunk n.
+// Records stream in by bulk copies, two stages deep (three for the maps).
 struct StateArgs {
     int S, H, Nc;
     int L, G;              // chunks per segment, segments per sequence
@@ -830,14 +834,16 @@ struct StateArgs {
     int *dev_status;
 };
 
-constexpr int ST_THREADS = 288;                // warps 0-7 register work, warp 8 MMA + copies
+constexpr int ST_THREADS_MAP = 288;            // warps 0-7 chain register work, warp 8 MMA + copies
+constexpr int ST_THREADS_CHAIN = 416;          // ... and warps 9-12 the output stage
+constexpr int ST_OUT_WARP0 = 9;
 constexpr uint32_t ST_STAGE = REC_GAM;         // the image part of a record (73728 B)
 constexpr uint32_t ST_GAM = 2 * ST_STAGE;      // e^{G_C} [2 stages][128] fp32 (the maps: 3 stages, into OIMG)
 constexpr uint32_t ST_OIMG = ST_GAM + 1024;    // output tile [2 atoms (j / 64)][64 rows r][128 B]
 constexpr uint32_t ST_SIGT = ST_OIMG + 16384;  // output-gate logits tile (TMA), same layout, bf16
 constexpr uint32_t ST_OT = ST_SIGT + 16384;    // O^T image, K-major B [128 rows j][128 B: 64 r]
 constexpr uint32_t ST_ID = ST_OT + 16384;      // [I_64; I_64], K-major A [128 rows][128 B: 64 k]
-constexpr uint32_t ST_RED = ST_ID + 16384;     // per-row partial sums of squares [64][4] fp32
+constexpr uint32_t ST_RED = ST_ID + 16384;     // per-row partial sums of squares [64][2] fp32
 constexpr uint32_t ST_BAR = ST_RED + 1024;     // mbarriers + TMEM slot
 constexpr uint32_t ST_END = ST_BAR + 128;
 constexpr size_t STATE_SMEM = ST_END + 1024;
@@ -849,12 +855,19 @@ constexpr uint32_t T_PO = 192;    // two [128][128] accumulators
 constexpr uint32_t T_V16 = 448;   // V'^T bf16 pairs (A operand, K = r)
 constexpr uint32_t ST_TCOLS = 512;
 
+// sigmoid(x) = (1 + tanh(x / 2)) / 2 with the hardware tanh approximation (|error| < 2^-11 of the result)
+__device__ __forceinline__ float sigmoid_fast(float x) {
+    float t;
+    asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * x));
+    return fmaf(0.5f, t, 0.5f);
+}
+
 // kMap = false: the chain over segment blockIdx.z from its entering state, with outputs.
 // kMap = true:  no outputs; z = 0 runs segment 0 from the initial state (its end state is S_1, the
 //               entering state of segment 1); for g >= 1 the map S_end = A_g S_start + Y_g of segment
 //               g = (z + 1) / 2: odd z from S = I without U (-> A_g), even z from S = 0 with U (-> Y_g).
 template <bool kMap>
-__global__ void __launch_bounds__(ST_THREADS, 1)
+__global__ void __launch_bounds__(kMap ? ST_THREADS_MAP : ST_THREADS_CHAIN, 1)
 chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constant__ CUtensorMap tgl, StateArgs p) {
     pdl_trigger();
     pdl_wait();
@@ -880,13 +893,19 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
     uint64_t *full = bars;           // [STG] record stage landed
     uint64_t *bar_p = bars + 3;      // PO group done
     uint64_t *bar_s = bars + 4;      // S^T += V'^T K~ done (and every earlier group)
-    uint64_t *bar_o = bars + 5;      // PO += V'^T M^T done
+    uint64_t *bar_o = bars + 5;      // PO += V'^T M^T done, [2] by PO buffer (slots 5 and 13): chunk n on
+                                     // bar_o[n & 1] phase n >> 1, so the output warps, which may trail the
+                                     // chain by a chunk, never see a barrier two phases ahead
     uint64_t *bar_t = bars + 6;      // transposition of O done
-    uint64_t *bar_simg = bars + 7;   // bf16 copy of S^T written (8 warps)
-    uint64_t *bar_vimg = bars + 8;   // bf16 copy of V'^T written (8 warps)
-    uint64_t *bar_ot = bars + 9;     // O^T image written (8 warps)
+    uint64_t *bar_simg = bars + 7;   // bf16 copy of S^T written (8 chain warps)
+    uint64_t *bar_vimg = bars + 8;   // bf16 copy of V'^T written (8 chain warps)
+    uint64_t *bar_ot = bars + 9;     // O^T image written (4 output warps)
     uint64_t *bar_sig = bars + 10;   // gate-logits tile landed
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 11);
+    uint64_t *pofree = bars + 11;    // [2] PO buffer read by the output warps (4 output warps)
+    uint64_t *bar_o1 = bars + 13;
+    auto bar_of = [&](int n) { return (n & 1) ? bar_o1 : bar_o; };
+    auto par_of = [](int n) { return (uint32_t)((n >> 1) & 1); };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 14);
     float *sgam = reinterpret_cast<float *>(sm + ST_GAM);
     float *red = reinterpret_cast<float *>(sm + ST_RED);
     const uint8_t *rec0 = p.ws + ((size_t)bh * p.Nc + n0) * REC_BYTES;
@@ -897,15 +916,18 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
         for (int i = 0; i < 7; ++i) mbar_init(&bars[i], 1);
         mbar_init(bar_simg, 8);
         mbar_init(bar_vimg, 8);
-        mbar_init(bar_ot, 8);
+        mbar_init(bar_ot, 4);
         mbar_init(bar_sig, 1);
+        mbar_init(&pofree[0], 4);
+        mbar_init(&pofree[1], 4);
+        mbar_init(bar_o1, 1);
         fence_barrier_init();
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, ST_TCOLS);
         tmem_relinquish();
     }
-    for (int e = tid; e < 128 * 8; e += ST_THREADS) {  // [I_64; I_64]
+    for (int e = tid; e < 128 * 8; e += blockDim.x) {  // [I_64; I_64]
         const int row = e >> 3, ch = e & 7;
         uint4 v = make_uint4(0u, 0u, 0u, 0u);
         if (((row & 63) >> 3) == ch) reinterpret_cast<uint16_t *>(&v)[row & 7] = 0x3F80;  // bf16 1.0
@@ -944,15 +966,13 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
                 ++issued;
             };
             // O of chunk m back to token rows: PO[m & 1][r, j] = sum_k [I; I][r, k] O^T[j, k]
-            auto transpose_o = [&](int m) -> bool {
-                if (!mbar_wait(bar_ot, m & 1)) return false;
+            auto transpose_o = [&](int m) {
                 tc_fence_after();
                 const uint32_t d = tmem + T_PO + (uint32_t)(m & 1) * 128;
 #pragma unroll
                 for (int s4 = 0; s4 < 4; ++s4)
                     mma_f16_ss(d, dadd(d_k, ST_ID + s4 * 32), dadd(d_k, ST_OT + s4 * 32), id_kk, s4 > 0);
                 mma_commit(bar_t);
-                return true;
             };
             for (int n = 0; n < STG && n < nc; ++n) issue_record(n);
             int n = 0;
@@ -960,15 +980,16 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
                 if (s_fail) { ok = false; break; }
                 // the stage of record n - 1 is free once its last group is done: refill it, STG - 1 ahead
                 if (n >= 1 && n + STG - 1 < nc) {
-                    if (!mbar_wait(bar_o, (n - 1) & 1)) { ok = false; break; }
+                    if (!mbar_wait(bar_of(n - 1), par_of(n - 1))) { ok = false; break; }
                     issue_record(n + STG - 1);
                 }
                 const uint32_t sgo = (n % STG) * STB;
                 const uint32_t po = tmem + T_PO + (uint32_t)(n & 1) * 128;
                 if (!mbar_wait(&full[n % STG], (n / STG) & 1)) { ok = false; break; }
                 landed = n + 1;
-                // PO = S_n^T [-W; Q e^G]^T (the maps: S_n^T (-W)^T)
+                // PO = S_n^T [-W; Q e^G]^T (the maps: S_n^T (-W)^T), once the output warps have read chunk n - 2
                 if (!mbar_wait(bar_simg, n & 1)) { ok = false; break; }
+                if (!kMap && n >= 2 && !mbar_wait(&pofree[n & 1], ((n - 2) >> 1) & 1)) { ok = false; break; }
                 tc_fence_after();
                 constexpr uint32_t id_po = kMap ? idesc_f16(128, 64, 0, 0) : id_kk;
 #pragma unroll
@@ -977,7 +998,13 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
                     mma_f16_ts(po, tmem + T_S16 + 8 * s8, dadd(d_k, sgo + ko * O_W_ATOM + kb), id_po, s8 > 0);
                 }
                 mma_commit(bar_p);
-                if (!kMap && n >= 1 && !transpose_o(n - 1)) { ok = false; break; }
+                // the previous chunk's transposition, if its O^T image is ready (else after this chunk's
+                // state update, which is on the chain's critical path)
+                bool t_pending = !kMap && n >= 1;
+                if (t_pending && mbar_test_wait(bar_ot, (n - 1) & 1)) {
+                    transpose_o(n - 1);
+                    t_pending = false;
+                }
                 // S^T += V'^T K~, then PO[:, 64:] += V'^T M^T
                 if (!mbar_wait(bar_vimg, n & 1)) { ok = false; break; }
                 tc_fence_after();
@@ -990,13 +1017,108 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
                     for (int s4 = 0; s4 < 4; ++s4)
                         mma_f16_ts(po + 64, tmem + T_V16 + 8 * s4, dadd(d_mn, sgo + REC_MT + s4 * 2048), id_o, 1);
                 }
-                mma_commit(bar_o);
+                mma_commit(bar_of(n));
+                if (t_pending) {
+                    if (!mbar_wait(bar_ot, (n - 1) & 1)) { ok = false; break; }
+                    transpose_o(n - 1);
+                }
             }
-            if (!kMap && ok && nc > 0 && !transpose_o(nc - 1)) ok = false;
+            if (!kMap && ok && nc > 0) {
+                if (mbar_wait(bar_ot, (nc - 1) & 1)) transpose_o(nc - 1);
+                else ok = false;
+            }
             if (!ok) s_fail = 1;
         }
+    } else if (warp >= ST_OUT_WARP0) {
+        // ======================================== output stage (warps 9-12, chains only)
+        const int otid = tid - ST_OUT_WARP0 * 32;
+        const int oq = warp & 3;               // TMEM lane quarter of this warp
+        const uint32_t olane = (uint32_t)(32 * oq) << 16;
+        const int j = 32 * oq + lane;          // value column (O^T image row) of this thread
+        const int r = 32 * (oq & 1) + lane;    // token row (lanes 64-127 repeat lanes 0-63)
+        const int cq2 = oq >> 1;               // value columns 64 cq2 .. 64 cq2 + 63
+        auto load_sig = [&](int m) {           // gate-logits tile of chunk m -> shared memory
+            if (otid == 0 && p.gated && m < nc) {
+                mbar_arrive_expect_tx(bar_sig, GATE_TILE_BYTES);
+                tma_load_4d(sm + ST_SIGT, &tgl, bar_sig, 0, h, (n0 + m) * CH, b);
+                tma_load_4d(sm + ST_SIGT + 8192, &tgl, bar_sig, 64, h, (n0 + m) * CH, b);
+            }
+        };
+        load_sig(0);
+        for (int m = 0; m < nc; ++m) {
+            if (s_fail) { ok = false; break; }
+            const uint32_t pob = tmem + olane + T_PO + (uint32_t)(m & 1) * 128;
+            // O^T of chunk m (PO[m & 1][j, 64 + r]) -> bf16 operand image
+            if (!mbar_wait(bar_of(m), par_of(m))) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t ov[32];
+                tmem_ld_32x32b_x32(pob + 64 + 32 * hh, ov);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    float f[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(ov[8 * k + e]);
+                    *reinterpret_cast<uint4 *>(sm + ST_OT + sw128(j, 4 * hh + k)) = pack8(f);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_ot);
+            // token rows of chunk m (after the [I; I] transposition) -> normalised, gated output tile
+            if (!mbar_wait(bar_t, m & 1)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t ov[64];
+            tmem_ld_32x32b_x32(pob + 64 * cq2, *reinterpret_cast<uint32_t(*)[32]>(&ov[0]));
+            tmem_ld_32x32b_x32(pob + 64 * cq2 + 32, *reinterpret_cast<uint32_t(*)[32]>(&ov[32]));
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pofree[m & 1]);  // this PO buffer may take chunk m + 2
+            if (p.gated) {
+                float ss = 0.f;
+#pragma unroll
+                for (int e = 0; e < 64; ++e) ss = fmaf(__uint_as_float(ov[e]), __uint_as_float(ov[e]), ss);
+                red[r * 2 + cq2] = ss;
+            }
+            if (otid == 0) bulk_wait_read_all();  // the previous tile's store has left shared memory
+            named_sync(2, 128);
+            float inv = 1.f;
+            if (p.gated) {
+                inv = rsqrtf((red[r * 2] + red[r * 2 + 1]) * (1.0f / 128.0f) + p.eps);
+                if (!mbar_wait(bar_sig, m & 1)) ok = false;
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const uint32_t off = cq2 * 8192 + sw128(r, k);
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(ov[8 * k + e]);
+                if (p.gated) {  // RMSNorm, then the sigmoid of the gate logits
+                    float gl[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(sm + ST_SIGT + off), gl);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) f[e] *= inv * sigmoid_fast(gl[e]);
+                }
+                *reinterpret_cast<uint4 *>(sm + ST_OIMG + off) = pack8(f);
+            }
+            fence_proxy_async_smem();
+            named_sync(2, 128);
+            if (otid == 0) {  // rows past the end of the sequence are clipped by the tensor map
+                tma_store_4d(&tmo, sm + ST_OIMG, 0, h, (n0 + m) * CH, b);
+                tma_store_4d(&tmo, sm + ST_OIMG + 8192, 64, h, (n0 + m) * CH, b);
+                bulk_commit();
+            }
+            load_sig(m + 1);  // every reader of the gate tile is past the barrier above
+            if (!ok) break;
+        }
+        if (!ok) s_fail = 1;
+        if (otid == 0) bulk_wait_all();
     } else {
-        // ======================================== register work (warps 0-7)
+        // ======================================== chain register work (warps 0-7)
         const uint32_t lrow = (uint32_t)(32 * q4) << 16;
         const int j = 32 * q4 + lane;  // value column (TMEM lane) of this thread
         {   // entering state -> TMEM (S^T[j, c] = S[c, j]: a warp reads 128 contiguous bytes per c)
@@ -1022,88 +1144,6 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
             }
             tmem_wait_st();
         }
-        auto load_sig = [&](int m) {  // gate-logits tile of chunk m -> shared memory (thread 0)
-            if (!kMap && tid == 0 && p.gated && m < nc) {
-                mbar_arrive_expect_tx(bar_sig, GATE_TILE_BYTES);
-                tma_load_4d(sm + ST_SIGT, &tgl, bar_sig, 0, h, (n0 + m) * CH, b);
-                tma_load_4d(sm + ST_SIGT + 8192, &tgl, bar_sig, 64, h, (n0 + m) * CH, b);
-            }
-        };
-        // O^T of chunk m (PO[m & 1][j, 64 + r]) -> bf16 operand image (all warps; after bar_o(m))
-        auto write_ot = [&](int m) {
-            uint32_t ov[32];
-            tmem_ld_32x32b_x32(tmem + lrow + T_PO + (uint32_t)(m & 1) * 128 + 64 + 32 * hf, ov);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                uint4 u;
-                u.x = pack_bf16x2(__uint_as_float(ov[8 * k]), __uint_as_float(ov[8 * k + 1]));
-                u.y = pack_bf16x2(__uint_as_float(ov[8 * k + 2]), __uint_as_float(ov[8 * k + 3]));
-                u.z = pack_bf16x2(__uint_as_float(ov[8 * k + 4]), __uint_as_float(ov[8 * k + 5]));
-                u.w = pack_bf16x2(__uint_as_float(ov[8 * k + 6]), __uint_as_float(ov[8 * k + 7]));
-                *reinterpret_cast<uint4 *>(sm + ST_OT + sw128(j, 4 * hf + k)) = u;
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_ot);
-        };
-        // token rows of chunk m (PO[m & 1][r, j], lane r and r + 64) -> normalised, gated output tile;
-        // each warp takes rows 32 (q4 & 1) .. +32 and value columns 32 cq .. +32
-        auto store_o = [&](int m) -> bool {
-            const int r = 32 * (q4 & 1) + lane;
-            const int cq = (q4 >> 1) + 2 * hf;
-            const uint32_t ocol = tmem + lrow + T_PO + (uint32_t)(m & 1) * 128 + 32 * cq;
-            if (!mbar_wait(bar_t, m & 1)) return false;
-            tc_fence_after();
-            bool okw = true;
-            float inv = 1.f;
-            if (p.gated) {
-                uint32_t ov[32];
-                tmem_ld_32x32b_x32(ocol, ov);
-                tmem_wait_ld();
-                float ss = 0.f;
-#pragma unroll
-                for (int e = 0; e < 32; ++e) ss += __uint_as_float(ov[e]) * __uint_as_float(ov[e]);
-                red[r * 4 + cq] = ss;
-            }
-            if (tid == 0) bulk_wait_read_all();  // the previous tile's store has left shared memory
-            named_sync(1, 256);
-            if (p.gated) {
-                const float4 rr = *reinterpret_cast<const float4 *>(red + r * 4);
-                inv = rsqrtf(((rr.x + rr.y) + (rr.z + rr.w)) * (1.0f / 128.0f) + p.eps);
-                okw = mbar_wait(bar_sig, m & 1);
-            }
-            {
-                uint32_t ov[32];
-                tmem_ld_32x32b_x32(ocol, ov);
-                tmem_wait_ld();
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const uint32_t off = (cq >> 1) * 8192 + sw128(r, 4 * (cq & 1) + k);
-                    float f[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(ov[8 * k + e]);
-                    if (p.gated) {  // RMSNorm, then the sigmoid of the gate logits (fp32)
-                        float gl[8];
-                        unpack8(*reinterpret_cast<const uint4 *>(sm + ST_SIGT + off), gl);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) f[e] *= inv * __fdividef(1.0f, 1.0f + __expf(-gl[e]));
-                    }
-                    *reinterpret_cast<uint4 *>(sm + ST_OIMG + off) = pack8(f);
-                }
-            }
-            fence_proxy_async_smem();
-            named_sync(1, 256);
-            if (tid == 0) {  // rows past the end of the sequence are clipped by the tensor map
-                tma_store_4d(&tmo, sm + ST_OIMG, 0, h, (n0 + m) * CH, b);
-                tma_store_4d(&tmo, sm + ST_OIMG + 8192, 64, h, (n0 + m) * CH, b);
-                bulk_commit();
-            }
-            load_sig(m + 1);  // every reader is past the barrier above
-            return okw;
-        };
-        load_sig(0);
 
         for (int n = 0; n < nc; ++n) {
             if (s_fail) { ok = false; break; }
@@ -1124,11 +1164,11 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
                     tmem_st_32x32b_x16(tmem + lrow + T_S16 + 32 * hf + 16 * hh, pk);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const float4 g = g4[8 * hh + e];
-                        sv[4 * e] = __float_as_uint(__uint_as_float(sv[4 * e]) * g.x);
-                        sv[4 * e + 1] = __float_as_uint(__uint_as_float(sv[4 * e + 1]) * g.y);
-                        sv[4 * e + 2] = __float_as_uint(__uint_as_float(sv[4 * e + 2]) * g.z);
-                        sv[4 * e + 3] = __float_as_uint(__uint_as_float(sv[4 * e + 3]) * g.w);
+                        const float4 gg = g4[8 * hh + e];
+                        sv[4 * e] = __float_as_uint(__uint_as_float(sv[4 * e]) * gg.x);
+                        sv[4 * e + 1] = __float_as_uint(__uint_as_float(sv[4 * e + 1]) * gg.y);
+                        sv[4 * e + 2] = __float_as_uint(__uint_as_float(sv[4 * e + 2]) * gg.z);
+                        sv[4 * e + 3] = __float_as_uint(__uint_as_float(sv[4 * e + 3]) * gg.w);
                     }
                     tmem_st_32x32b_x32(tmem + lrow + T_S32 + 64 * hf + 32 * hh, sv);
                 }
@@ -1137,12 +1177,6 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_simg);
-            // ---------- O^T of the previous chunk -> operand image (turned back into rows by the MMA warp)
-            if (!kMap && n >= 1) {
-                if (!mbar_wait(bar_o, (n - 1) & 1)) { ok = false; break; }
-                tc_fence_after();
-                write_ot(n - 1);
-            }
             // ---------- V'^T = U^T - (W S_n)^T -> bf16 copy in TMEM
             {
                 const uint8_t *ut = sm + (n % STG) * STB + O_U;
@@ -1161,9 +1195,9 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         pk[4 * k + e] = ident ? pack_bf16x2(__uint_as_float(pv[8 * k + 2 * e]),
-                                                        __uint_as_float(pv[8 * k + 2 * e + 1]))
-                                          : pack_bf16x2(u[2 * e] + __uint_as_float(pv[8 * k + 2 * e]),
-                                                        u[2 * e + 1] + __uint_as_float(pv[8 * k + 2 * e + 1]));
+                                                            __uint_as_float(pv[8 * k + 2 * e + 1]))
+                                              : pack_bf16x2(u[2 * e] + __uint_as_float(pv[8 * k + 2 * e]),
+                                                            u[2 * e + 1] + __uint_as_float(pv[8 * k + 2 * e + 1]));
                 }
                 tmem_st_32x32b_x16(tmem + lrow + T_V16 + 16 * hf, pk);
                 tmem_wait_st();
@@ -1171,16 +1205,10 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_vimg);
-            // ---------- the previous chunk's output tile, while this chunk's state update runs
-            if (!kMap && n >= 1 && !store_o(n - 1)) { ok = false; break; }
         }
         if (ok && nc > 0) {
-            if (!mbar_wait(bar_s, (nc - 1) & 1) || !mbar_wait(bar_o, (nc - 1) & 1)) ok = false;
+            if (!mbar_wait(bar_s, (nc - 1) & 1) || !mbar_wait(bar_of(nc - 1), par_of(nc - 1))) ok = false;
             tc_fence_after();
-            if (!kMap) {
-                if (ok) write_ot(nc - 1);
-                if (ok && !store_o(nc - 1)) ok = false;
-            }
         }
         if (ok && kMap && !ident) {  // Y_g (S_1 for segment 0), laid out like a state
             float *dst0 = p.yt + ((size_t)bh * (p.G - 1) + g) * DD * DD;
@@ -1220,7 +1248,6 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
             }
         }
         if (!ok) s_fail = 1;
-        if (tid == 0) bulk_wait_all();
     }
     __syncthreads();
     if (warp == 8 && lane == 0 && s_fail) {
@@ -1228,7 +1255,8 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
         // let the bulk copies already issued land before the CTA exits
         for (int m = landed; m < issued; ++m) mbar_wait(&full[m % STG], (m / STG) & 1, 100000000ull);
     }
-    if (!kMap && tid == 0 && s_fail && p.gated) mbar_wait(bar_sig, 0, 100000000ull), mbar_wait(bar_sig, 1, 100000000ull);
+    if (!kMap && tid == ST_OUT_WARP0 * 32 && s_fail && p.gated)
+        mbar_wait(bar_sig, 0, 100000000ull), mbar_wait(bar_sig, 1, 100000000ull);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, ST_TCOLS);
@@ -1384,7 +1412,7 @@ kda_status_t launch_state(const CUtensorMap &tmo, const CUtensorMap &tgl, const 
                           cudaStream_t st) {
     if (sa.G > 1) {
         cudaFuncSetAttribute(chunk_state_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
-        cudaError_t e = launch_pdl(chunk_state_kernel<true>, dim3(H, B, 2 * sa.G - 3), dim3(ST_THREADS),
+        cudaError_t e = launch_pdl(chunk_state_kernel<true>, dim3(H, B, 2 * sa.G - 3), dim3(ST_THREADS_MAP),
                                    STATE_SMEM, st, tmo, tgl, sa);
         if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "chunk_state_kernel (segment maps): %s", cudaGetErrorString(e));
         kda_status_t s = check_launch("chunk_state_kernel (segment maps)");
@@ -1406,7 +1434,7 @@ kda_status_t launch_state(const CUtensorMap &tmo, const CUtensorMap &tgl, const 
         if (s != KDA_OK) return s;
     }
     cudaFuncSetAttribute(chunk_state_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
-    cudaError_t e = launch_pdl(chunk_state_kernel<false>, dim3(H, B, sa.G), dim3(ST_THREADS), STATE_SMEM, st, tmo, tgl,
+    cudaError_t e = launch_pdl(chunk_state_kernel<false>, dim3(H, B, sa.G), dim3(ST_THREADS_CHAIN), STATE_SMEM, st, tmo, tgl,
                                sa);
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "chunk_state_kernel: %s", cudaGetErrorString(e));
     return check_launch("chunk_state_kernel");
