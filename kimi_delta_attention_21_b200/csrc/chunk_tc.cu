@@ -166,11 +166,20 @@ constexpr uint32_t P_RH = P_ZI;
 constexpr uint32_t P_WI = P_A, P_UI = P_A + 16384, P_MT = P_A + 32768;
 constexpr uint32_t P_ZT = P_A + 40960;  // the next unit's z tile [2 atoms][64 rows][128 B], between the A/M MMAs
                                         // and the next unit's P2 (nothing else uses these 16 KB then)
-constexpr uint32_t P_TI = P_B, P_LOHI = P_B + 8192;  // LOHI: [64][16] fp32
-constexpr uint32_t P_SA = P_SG, P_ST = P_SG + 16640;
-constexpr int SG_LD = 132, SA_LD = 65, ST_LD = 68;
 constexpr uint32_t A_ATOM = 224 * 128;  // bytes per atom column of the A/M MMAs' A operand
 constexpr uint32_t B_ATOM = 192 * 128;  // ... and of their B operand
+constexpr uint32_t B_ATOM_BYTES = B_ATOM;
+// During P3 and P4 the A/M operands are dead: the T image, A and T (fp32) live in the B operand's
+// space, the low-part hand-off and the inverse's scratch in the first 10 KB of the A operand's (the
+// W and U^T images only take it in P5), so that G, the tables, beta and e^{G_C} are free for the next
+// unit's decay, which runs beside the inverse.
+constexpr uint32_t P_TI = P_B;                        // T image (bf16)
+constexpr uint32_t P_SA = P_B + 8192;                 // A [64][65] fp32
+constexpr uint32_t P_ST = P_SA + 16640;               // T [64][68] fp32
+constexpr uint32_t P_LOHI = P_A;                      // [64][16] fp32
+constexpr uint32_t P_IX = P_A + 4096;                 // inverse scratch [512 + 1024] fp32
+static_assert(P_ST + 64 * 68 * 4 <= P_B + 2 * B_ATOM_BYTES, "A and T fit in the B operand's space");
+constexpr int SG_LD = 132, SA_LD = 65, ST_LD = 68;
 constexpr uint32_t A_KLO = 160;         // first row of the low part of the diagonal column operand
 
 // table rows: b_R (0-3), F_R = e^{b_{R-1} - m_R} (4-7), E_R = e^{b_{R-1}} (8-11),
@@ -241,29 +250,33 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     // P1 and the per-channel tables of unit u: beta, G = in-chunk cumulative log-decay (rows past the
     // sequence end: no decay, beta 0), the block constants and e^{G_C}.  The decay input is z (the tile
     // at P_ZT, loaded one unit ahead, landed on bar_z with parity zpar) or the log-decay (read from
-    // global memory, prefetched into L2 one unit ahead); beta_row is row tid's beta, loaded one unit
-    // ahead.  Called by all threads; returns false if the z tile never landed.
-    auto load_beta = [&](int64_t u) -> float {  // beta of row tid (< 64) of unit u; 0 past the end
+    // global memory, prefetched into L2 one unit ahead); beta_row is row t's beta (t < 64), loaded one
+    // unit ahead.  Run by the decay group, warps 4-11 (t = tid - 128, named barrier 3): for the first
+    // unit before the loop, for every later one beside the previous unit's inverse.  Returns false if
+    // the z tile never landed.
+    constexpr int DT0 = 128, DTN = 256;
+    auto load_beta = [&](int64_t u, int row) -> float {  // beta of row `row` of unit u; 0 past the end
         int n, h, b;
         unit_coords(u, n, h, b);
         const int t0 = n * CH;
-        return (t0 + tid < p.S) ? __bfloat162float(p.beta[((int64_t)b * p.S + t0 + tid) * p.H + h]) : 0.f;
+        return (t0 + row < p.S) ? __bfloat162float(p.beta[((int64_t)b * p.S + t0 + row) * p.H + h]) : 0.f;
     };
     auto decay_tables = [&](int64_t u, uint32_t zpar, float beta_row) -> bool {
         int n, h, b;
         unit_coords(u, n, h, b);
+        const int t = tid - DT0;
         const int t0 = n * CH, len = min(CH, p.S - t0);
         bool landed = true;
-        if (tid < CH) sbeta[tid] = beta_row;
-        {   // one thread per channel c and 16 rows (quarter qt); quarter sums through a scratch
-            const int c = tid & 127, qt = tid >> 7;
+        if (t < CH) sbeta[t] = beta_row;
+        {   // one thread per channel c and 32 rows (half hv); the half sums through a scratch
+            const int c = t & 127, hv = t >> 7;
             float *qsum = reinterpret_cast<float *>(sm + P_XS);
             const int64_t i0 = (((int64_t)b * p.S + t0) * p.H + h) * DD + c, rstr = (int64_t)p.H * DD;
-            float g[16];
+            float g[32];
             if (p.log_decay) {
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    const int r = qt * 16 + rr;
+                for (int rr = 0; rr < 32; ++rr) {
+                    const int r = hv * 32 + rr;
                     g[rr] = (r < len) ? clamp_log_decay(p.log_decay[i0 + r * rstr], p.g_min) : 0.f;
                 }
             } else {
@@ -271,34 +284,35 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 const uint8_t *zc = sm + P_ZT + (c >> 6) * 8192 + (c & 7) * 2;
                 const uint32_t ch = (c & 63) >> 3;
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    const int r = qt * 16 + rr;
+                for (int rr = 0; rr < 32; ++rr) {
+                    const int r = hv * 32 + rr;
                     const float zv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(zc + sw128(r, ch)));
                     g[rr] = (r < len) ? log_alpha_fast(zv, p.g_min) : 0.f;
                 }
             }
             float acc = 0.f;
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) {
+            for (int rr = 0; rr < 32; ++rr) {
                 acc += g[rr];
                 g[rr] = acc;
             }
-            qsum[qt * 128 + c] = acc;
-            __syncthreads();
-            float base = 0.f;
-            for (int q = 0; q < qt; ++q) base += qsum[q * 128 + c];
+            qsum[hv * 128 + c] = acc;
+            named_sync(3, DTN);
+            const float base = hv ? qsum[c] : 0.f;
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) sG[(qt * 16 + rr) * SG_LD + c] = g[rr] + base;
+            for (int rr = 0; rr < 32; ++rr) sG[(hv * 32 + rr) * SG_LD + c] = g[rr] + base;
         }
-        __syncthreads();
-        {  // per-channel block constants, four threads per channel (8, 6, 5 and 4 exponentials)
-            const int c = tid & 127, part = tid >> 7;
+        named_sync(3, DTN);
+        {  // per-channel block constants, two threads per channel, each two of the four parts
+            const int c = t & 127;
             float bb[4], mm[4];
 #pragma unroll
             for (int R = 0; R < 4; ++R) {
                 bb[R] = sG[(16 * R + 15) * SG_LD + c];
                 mm[R] = sG[(16 * R + 7) * SG_LD + c];
             }
+#pragma unroll
+            for (int part = t >> 7; part < 4; part += 2) {
             if (part == 0) {
 #pragma unroll
                 for (int R = 0; R < 4; ++R) {
@@ -320,6 +334,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             } else {
 #pragma unroll
                 for (int R = 0; R <= 3; ++R) tab[tab_c(3, R) * 128 + c] = fexp(mm[3] - bb[R]);
+            }
             }
         }
         return landed;
@@ -346,7 +361,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
-    float beta_cur = (tid < CH && (int64_t)blockIdx.x < p.units) ? load_beta(blockIdx.x) : 0.f;
+    if (warp >= 4 && warp < 12 && (int64_t)blockIdx.x < p.units) {  // the first unit's decay and tables
+        const int t = tid - DT0;
+        ok = decay_tables(blockIdx.x, 0u, t < CH ? load_beta(blockIdx.x, t) : 0.f);
+    }
 
     int it = 0;
     for (int64_t u = blockIdx.x; u < p.units && ok; u += gridDim.x, ++it) {
@@ -354,8 +372,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         unit_coords(u, n, h, b);
         const int64_t u_next = u + gridDim.x;
         const uint32_t par = it & 1;
-        // the next unit's beta, consumed by its tables (issued now, so its latency stays hidden)
-        const float beta_next = (tid < CH && u_next < p.units) ? load_beta(u_next) : 0.f;
+        // the next unit's beta, consumed by its decay during this unit's inverse
+        const float beta_next = (warp >= 4 && warp < 6 && u_next < p.units) ? load_beta(u_next, tid - DT0) : 0.f;
         if (u_next < p.units && tid < 256 && p.log_decay) {  // the next unit's log-decay input -> L2
             int n2, h2, b2;
             unit_coords(u_next, n2, h2, b2);
@@ -364,9 +382,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             if (p.log_decay && n2 * CH + row < p.S)
                 prefetch_l2(p.log_decay + (row0 + (int64_t)row * p.H) * DD + (tid & 3) * 32);
         }
-        // the decay and tables need neither q, k nor v: they run while v is still landing
-        ok = decay_tables(u, par, beta_cur);
-        beta_cur = beta_next;
+        // (this unit's decay and tables ran beside the previous unit's inverse)
         // the previous unit's bulk stores must have read their shared sources (P2 overwrites them)
         if (tid == 0) bulk_wait_read_all();
         ok = mbar_wait(bar_in, par) && ok;
@@ -588,11 +604,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         // forward substitution, then T_{R,R-1} = -T_RR A_{R,R-1} T_{R-1,R-1} for R = 1, 3, then the lower-left
         // 32x32 block the same way from the two diagonal 32x32 blocks.  Blocks above the diagonal are written
         // as zeros where a later product reads them; the T image zero-fills the upper-right 32x32 block.
-        // Warps 0-3 only (named barrier 1).
+        // Warps 0-3 only (named barrier 1); warps 4-11 meanwhile compute the next unit's decay and tables.
         if (warp < 4) {
             const float *sA = reinterpret_cast<const float *>(sm + P_SA);
             float *sT = reinterpret_cast<float *>(sm + P_ST);
-            float *xs = reinterpret_cast<float *>(sm + P_TAB);  // the tables are dead after P2
+            float *xs = reinterpret_cast<float *>(sm + P_IX);
             if (tid < 64) {  // diagonal block R, column jc: (I + A_RR) x = e_jc, right-looking
                 const int R = tid >> 4, jc = tid & 15, o = 16 * R;
                 float x[16];
@@ -716,9 +732,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 *reinterpret_cast<uint4 *>(sm + P_TI + sw128(r, cc)) = pack8(t);
             }
             fence_proxy_async_smem();
+        } else if (warp < 12 && u_next < p.units) {
+            ok = decay_tables(u_next, (uint32_t)(it + 1) & 1u, beta_next) && ok;
         }
         tc_fence_before();
-        __syncthreads();
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
 
         // ---------------- tcgen05: W = T (beta K e^G)            (M=64, N=128, K=64: A = T, B MN-major)
         //                   U^T = (beta V)^T T^T              (M=128, N=64, K=64: A MN-major, B = T K-major)
@@ -804,8 +823,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
 // register work of the chain is spread over all 128 lanes.  Warp roles:
 //   warps 0-7   the chain's register work (lane quarter = warp % 4, column
 //               half = warp / 4);
-//   warp 8      issues the MMAs and the record copies (one thread);
-//   warps 9-12  the output stage (chains only; the maps have no output).
+//   warp 8      issues the chain's MMAs and the record copies (one thread);
+//   warps 9-12  the output stage (chains only; the maps have no output); its
+//               first thread issues the output's transposition MMA itself, so
+//               the output never waits on the chain's MMA issue order.
 // Per chunk n:
 //   chain warps:  S^T -> bf16 copy in TMEM; S^T <- S^T Diag(e^{G_C})
 //   MMA:          PO  = S^T [-W; Q e^G]^T        PO[j, r] = -(W S)[r, j],  PO[j, 64 + r] = (Q e^G S)[r, j]
@@ -965,24 +986,10 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
                 bulk_load(sgam + stg * 128, src + REC_GAM, 512, &full[stg]);
                 ++issued;
             };
-            // O of chunk m back to token rows: PO[m & 1][r, j] = sum_k [I; I][r, k] O^T[j, k]
-            auto transpose_o = [&](int m) {
-                tc_fence_after();
-                const uint32_t d = tmem + T_PO + (uint32_t)(m & 1) * 128;
-#pragma unroll
-                for (int s4 = 0; s4 < 4; ++s4)
-                    mma_f16_ss(d, dadd(d_k, ST_ID + s4 * 32), dadd(d_k, ST_OT + s4 * 32), id_kk, s4 > 0);
-                mma_commit(bar_t);
-            };
             for (int n = 0; n < STG && n < nc; ++n) issue_record(n);
             int n = 0;
             for (; n < nc; ++n) {
                 if (s_fail) { ok = false; break; }
-                // the stage of record n - 1 is free once its last group is done: refill it, STG - 1 ahead
-                if (n >= 1 && n + STG - 1 < nc) {
-                    if (!mbar_wait(bar_of(n - 1), par_of(n - 1))) { ok = false; break; }
-                    issue_record(n + STG - 1);
-                }
                 const uint32_t sgo = (n % STG) * STB;
                 const uint32_t po = tmem + T_PO + (uint32_t)(n & 1) * 128;
                 if (!mbar_wait(&full[n % STG], (n / STG) & 1)) { ok = false; break; }
@@ -998,12 +1005,10 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
                     mma_f16_ts(po, tmem + T_S16 + 8 * s8, dadd(d_k, sgo + ko * O_W_ATOM + kb), id_po, s8 > 0);
                 }
                 mma_commit(bar_p);
-                // the previous chunk's transposition, if its O^T image is ready (else after this chunk's
-                // state update, which is on the chain's critical path)
-                bool t_pending = !kMap && n >= 1;
-                if (t_pending && mbar_test_wait(bar_ot, (n - 1) & 1)) {
-                    transpose_o(n - 1);
-                    t_pending = false;
+                // the stage of record n - 1 is free once its last group is done: refill it, STG - 1 ahead
+                if (n >= 1 && n + STG - 1 < nc) {
+                    if (!mbar_wait(bar_of(n - 1), par_of(n - 1))) { ok = false; break; }
+                    issue_record(n + STG - 1);
                 }
                 // S^T += V'^T K~, then PO[:, 64:] += V'^T M^T
                 if (!mbar_wait(bar_vimg, n & 1)) { ok = false; break; }
@@ -1018,14 +1023,6 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
                         mma_f16_ts(po + 64, tmem + T_V16 + 8 * s4, dadd(d_mn, sgo + REC_MT + s4 * 2048), id_o, 1);
                 }
                 mma_commit(bar_of(n));
-                if (t_pending) {
-                    if (!mbar_wait(bar_ot, (n - 1) & 1)) { ok = false; break; }
-                    transpose_o(n - 1);
-                }
-            }
-            if (!kMap && ok && nc > 0) {
-                if (mbar_wait(bar_ot, (nc - 1) & 1)) transpose_o(nc - 1);
-                else ok = false;
             }
             if (!ok) s_fail = 1;
         }
@@ -1068,6 +1065,22 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_ot);
+            // O of chunk m back to token rows, PO[m & 1][r, j] = sum_k [I; I][r, k] O^T[j, k], issued by
+            // this group's first thread (its commit tracks only its own MMAs)
+            if (otid == 0) {
+                if (mbar_wait(bar_ot, m & 1)) {
+                    tc_fence_after();
+                    constexpr uint32_t id_t = idesc_f16(128, 128, 0, 0);
+                    const uint64_t d_k = smem_desc(smem_u32(sm), 16, 1024, LAYOUT_SW128);
+                    const uint32_t d = tmem + T_PO + (uint32_t)(m & 1) * 128;
+#pragma unroll
+                    for (int s4 = 0; s4 < 4; ++s4)
+                        mma_f16_ss(d, dadd(d_k, ST_ID + s4 * 32), dadd(d_k, ST_OT + s4 * 32), id_t, s4 > 0);
+                    mma_commit(bar_t);
+                } else {
+                    s_fail = 1;
+                }
+            }
             // token rows of chunk m (after the [I; I] transposition) -> normalised, gated output tile
             if (!mbar_wait(bar_t, m & 1)) { ok = false; break; }
             tc_fence_after();
@@ -1152,31 +1165,36 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
             if (n >= 1 && !mbar_wait(bar_s, (n - 1) & 1)) { ok = false; break; }
             if (!mbar_wait(&full[n % STG], (n / STG) & 1)) { ok = false; break; }
             tc_fence_after();
-            {
+            {   // the bf16 copy goes out first (the PO MMA waits for it); the decay is applied after
                 const float4 *g4 = reinterpret_cast<const float4 *>(sgam + (n % STG) * 128 + 64 * hf);
+                uint32_t sv[64];
+                tmem_ld_32x32b_x32(tmem + lrow + T_S32 + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                tmem_ld_32x32b_x32(tmem + lrow + T_S32 + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+                tmem_wait_ld();
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    uint32_t sv[32], pk[16];
-                    tmem_ld_32x32b_x32(tmem + lrow + T_S32 + 64 * hf + 32 * hh, sv);
-                    tmem_wait_ld();
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(sv[2 * e]), __uint_as_float(sv[2 * e + 1]));
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack_bf16x2(__uint_as_float(sv[32 * hh + 2 * e]), __uint_as_float(sv[32 * hh + 2 * e + 1]));
                     tmem_st_32x32b_x16(tmem + lrow + T_S16 + 32 * hf + 16 * hh, pk);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float4 gg = g4[8 * hh + e];
-                        sv[4 * e] = __float_as_uint(__uint_as_float(sv[4 * e]) * gg.x);
-                        sv[4 * e + 1] = __float_as_uint(__uint_as_float(sv[4 * e + 1]) * gg.y);
-                        sv[4 * e + 2] = __float_as_uint(__uint_as_float(sv[4 * e + 2]) * gg.z);
-                        sv[4 * e + 3] = __float_as_uint(__uint_as_float(sv[4 * e + 3]) * gg.w);
-                    }
-                    tmem_st_32x32b_x32(tmem + lrow + T_S32 + 64 * hf + 32 * hh, sv);
                 }
                 tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar_simg);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float4 gg = g4[e];
+                    sv[4 * e] = __float_as_uint(__uint_as_float(sv[4 * e]) * gg.x);
+                    sv[4 * e + 1] = __float_as_uint(__uint_as_float(sv[4 * e + 1]) * gg.y);
+                    sv[4 * e + 2] = __float_as_uint(__uint_as_float(sv[4 * e + 2]) * gg.z);
+                    sv[4 * e + 3] = __float_as_uint(__uint_as_float(sv[4 * e + 3]) * gg.w);
+                }
+                tmem_st_32x32b_x32(tmem + lrow + T_S32 + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                tmem_st_32x32b_x32(tmem + lrow + T_S32 + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+                tmem_wait_st();
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_simg);
             // ---------- V'^T = U^T - (W S_n)^T -> bf16 copy in TMEM
             {
                 const uint8_t *ut = sm + (n % STG) * STB + O_U;
