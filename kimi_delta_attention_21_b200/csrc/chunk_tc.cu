@@ -159,7 +159,7 @@ constexpr uint32_t P_TAB = 206080;   // per-channel block constants [26][128] fp
 constexpr uint32_t P_XS = 219392;    // quarter sums of the cumulative log-decay [4][128] fp32
 constexpr uint32_t P_BETA = 222464;  // beta [64] fp32
 constexpr uint32_t P_GAM = 222720;   // e^{G_C} [128] fp32
-constexpr uint32_t P_BAR = 223232;   // mbarriers: inputs, A/M MMAs, W/U MMAs; TMEM slot (+24); z tile (+32)
+constexpr uint32_t P_BAR = 223232;   // mbarriers: q/k, A/M MMAs, W/U MMAs; TMEM slot (+24); z tile (+32); v (+40)
 constexpr uint32_t P_END = 223312;
 constexpr size_t PREP_SMEM = P_END + 1024;
 constexpr uint32_t P_RH = P_ZI;
@@ -213,11 +213,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     uint64_t *bar_wu = bar_in + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + P_BAR + 24);
     uint64_t *bar_z = reinterpret_cast<uint64_t *>(sm + P_BAR + 32);
+    uint64_t *bar_v = reinterpret_cast<uint64_t *>(sm + P_BAR + 40);
     float *sG = reinterpret_cast<float *>(sm + P_SG);
     float *tab = reinterpret_cast<float *>(sm + P_TAB);
     float *sbeta = reinterpret_cast<float *>(sm + P_BETA);
     float *sgam = reinterpret_cast<float *>(sm + P_GAM);
-    const uint32_t in_bytes = 6u * 8192u;  // q, k, v
+    const uint32_t in_bytes = 4u * 8192u;  // q, k
 
     auto unit_coords = [&](int64_t u, int &n, int &h, int &b) {  // 32-bit: units < 2^31 (host check)
         const uint32_t uu = (uint32_t)u, nc = (uint32_t)p.Nc, hh = (uint32_t)p.H;
@@ -226,7 +227,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         b = (int)(bh / hh);
         h = (int)(bh - (uint32_t)b * hh);
     };
-    auto load_qk = [&](int64_t u) {  // arms bar_in for the whole unit
+    auto load_qk = [&](int64_t u) {
         int n, h, b;
         unit_coords(u, n, h, b);
         mbar_arrive_expect_tx(bar_in, in_bytes);
@@ -244,7 +245,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     auto load_v = [&](int64_t u) {
         int n, h, b;
         unit_coords(u, n, h, b);
-        for (int a = 0; a < 2; ++a) tma_load_4d(sm + P_VI + a * 8192, &tv, bar_in, 64 * a, h, n * CH, b);
+        mbar_arrive_expect_tx(bar_v, 16384u);
+        for (int a = 0; a < 2; ++a) tma_load_4d(sm + P_VI + a * 8192, &tv, bar_v, 64 * a, h, n * CH, b);
     };
 
     // P1 and the per-channel tables of unit u: beta, G = in-chunk cumulative log-decay (rows past the
@@ -345,6 +347,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         mbar_init(bar_am, 1);
         mbar_init(bar_wu, 1);
         mbar_init(bar_z, 1);
+        mbar_init(bar_v, 1);
         fence_barrier_init();
         if ((int64_t)blockIdx.x < p.units) {
             load_qk(blockIdx.x);
@@ -383,8 +386,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 prefetch_l2(p.log_decay + (row0 + (int64_t)row * p.H) * DD + (tid & 3) * 32);
         }
         // (this unit's decay and tables ran beside the previous unit's inverse)
-        // the previous unit's bulk stores must have read their shared sources (P2 overwrites them)
-        if (tid == 0) bulk_wait_read_all();
         ok = mbar_wait(bar_in, par) && ok;
         ok = __syncthreads_and(ok);
         if (!ok) break;
@@ -394,17 +395,17 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         // of the column operand (and no warp diverges on the version count).
         {
             const int R0 = warp & 3, jj = 2 * (warp >> 2) + (lane >> 4);
-#pragma unroll 1
+            float ke3s[2][8];  // k e^{b_R - G} of both items, for the column versions written last
+#pragma unroll
             for (int mi = 0; mi < 2; ++mi) {
                 const int R = mi ? 3 - R0 : R0, r = 16 * R + (lane & 15);
                 const float beta_r = sbeta[r];
                 const int j = jj + 8 * mi, atom = mi, c0 = 8 * j;
                 const uint32_t img = atom * 8192 + sw128(r, jj);
-                const uint32_t bimg = P_B + atom * B_ATOM, aimg = P_A + atom * A_ATOM;
-                float qv[8], kv[8], vv[8], G[8], bR[8], bRm1[8], F[8], E[8], Dd[8];
+                const uint32_t bimg = P_B + atom * B_ATOM;
+                float qv[8], kv[8], G[8], bR[8], bRm1[8], F[8], E[8], Dd[8];
                 unpack8(*reinterpret_cast<const uint4 *>(sm + P_QI + img), qv);
                 unpack8(*reinterpret_cast<const uint4 *>(sm + P_KI + img), kv);
-                unpack8(*reinterpret_cast<const uint4 *>(sm + P_VI + img), vv);
                 load8f(sG + r * SG_LD + c0, G);
                 load8f(tab + R * 128 + c0, bR);
                 if (R > 0) {
@@ -440,11 +441,45 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                     for (int e = 0; e < 8; ++e) lo[e] = t[e] - hf[e];
                     *reinterpret_cast<uint4 *>(sm + bimg + sw128(128 + r, jj)) = pack8(lo);
                 }
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ke3s[mi][e] = ke3[e];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) t[e] = qv[e] * fg[e];
+                *reinterpret_cast<uint4 *>(sm + P_QI + img) = pack8(t);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) t[e] = ke3[e] * Dd[e];
+                *reinterpret_cast<uint4 *>(sm + P_KI + img) = pack8(t);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) t[e] = (beta_r * kv[e]) * fg[e];
+                *reinterpret_cast<uint4 *>(sm + P_RH + img) = pack8(t);
+            }
+            // beta V last: the v tile is loaded after the previous unit's W/U MMAs and lands meanwhile
+            if (!mbar_wait(bar_v, par)) ok = false;
+#pragma unroll
+            for (int mi = 0; mi < 2; ++mi) {
+                const int R = mi ? 3 - R0 : R0, r = 16 * R + (lane & 15);
+                const uint32_t img = mi * 8192 + sw128(r, jj);
+                const float beta_r = sbeta[r];
+                float vv[8], t[8];
+                unpack8(*reinterpret_cast<const uint4 *>(sm + P_VI + img), vv);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) t[e] = beta_r * vv[e];
+                *reinterpret_cast<uint4 *>(sm + P_VI + img) = pack8(t);
+            }
+            // the column versions go into the A operand's space, which the previous unit's bulk stores
+            // (W, U^T and M^T images) read from: wait for those reads to finish first
+            if (tid == 0) bulk_wait_read_all();
+            __syncthreads();
+#pragma unroll
+            for (int mi = 0; mi < 2; ++mi) {
+                const int R = mi ? 3 - R0 : R0, r = 16 * R + (lane & 15);
+                const int c0 = 8 * (jj + 8 * mi);
+                const uint32_t aimg = P_A + mi * A_ATOM;
                 for (int V = R; V < 4; ++V) {
-                    float Cv[8];
+                    float Cv[8], t[8];
                     load8f(tab + tab_c(V, R) * 128 + c0, Cv);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) t[e] = ke3[e] * Cv[e];
+                    for (int e = 0; e < 8; ++e) t[e] = ke3s[mi][e] * Cv[e];
                     const uint4 hi = pack8(t);
                     *reinterpret_cast<uint4 *>(sm + aimg + sw128(kc_row0(V) + r, jj)) = hi;
                     if (V == R) {  // diagonal block: keep the rounding residue
@@ -455,23 +490,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                         *reinterpret_cast<uint4 *>(sm + aimg + sw128(A_KLO + r, jj)) = pack8(lo);
                     }
                 }
-#pragma unroll
-                for (int e = 0; e < 8; ++e) t[e] = qv[e] * fg[e];
-                *reinterpret_cast<uint4 *>(sm + P_QI + img) = pack8(t);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) t[e] = ke3[e] * Dd[e];
-                *reinterpret_cast<uint4 *>(sm + P_KI + img) = pack8(t);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) t[e] = (beta_r * kv[e]) * fg[e];
-                *reinterpret_cast<uint4 *>(sm + P_RH + img) = pack8(t);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) t[e] = beta_r * vv[e];
-                *reinterpret_cast<uint4 *>(sm + P_VI + img) = pack8(t);
             }
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        ok = __syncthreads_and(ok);
+        if (!ok) break;
 
         uint8_t *rec = p.ws + ((size_t)(b * p.H + h) * p.Nc + n) * REC_BYTES;
         // ---------------- tcgen05: A^T (cols 0-63), M^T (64-127), residues of M's diagonal blocks (128-191);
