@@ -96,13 +96,14 @@ def n_chunks(w):
     return (w.S + CHUNK - 1) // CHUNK
 
 
-def prefill_bytes(w):
+def prefill_bytes(w, scalar_decay=False):
     """Algorithmic HBM bytes of the chunk engine for a whole workload: read q, k,
-    z (D_k each), v, gate (D_v each) and beta per token-head, write the gated
-    output (D_v) per token-head; read the fp32 initial state (when there is one)
-    and write the fp32 final state per (b, h)."""
+    z (D_k each; one value for the scalar-decay GDN case), v, gate (D_v each) and
+    beta per token-head, write the gated output (D_v) per token-head; read the
+    fp32 initial state (when there is one) and write the fp32 final state per
+    (b, h)."""
     es = 2 if w.dtype == "bf16" else 4
-    per_tok_head = es * (3 * w.Dk + 3 * w.Dv + 1)
+    per_tok_head = es * ((2 * w.Dk + (1 if scalar_decay else w.Dk)) + 3 * w.Dv + 1)
     n_states = 2 if w.s0_std > 0 else 1
     return w.B * w.S * w.H * per_tok_head + n_states * w.B * w.H * w.Dk * w.Dv * 4
 
@@ -300,20 +301,23 @@ class Timer:
         return a, b
 
 
-def time_prefill(K, torch, w, d, steps, warmup, world, dev, flush, lib, sampler=None):
+def time_prefill(K, torch, w, d, steps, warmup, world, dev, flush, lib, sampler=None, gdn=False):
     """Times `steps` layer forwards of workload `w` (device inputs `d`).  Returns
-    per-step seconds (chunk engine, projection; max over ranks) and launches."""
+    per-step seconds (chunk engine, projection; max over ranks) and launches.
+    gdn: the scalar-decay (Gated DeltaNet) engine, one decay logit per token and
+    head (the first channel's logit of the same inputs)."""
     B, S, H = w.B, w.S, w.H
     N = B * S
     x = torch.empty((B, S, H, w.Dv), dtype=d["v"].dtype, device=dev)
     y = torch.empty((N, w.D_model), dtype=d["v"].dtype, device=dev)
     sf = torch.empty((B, H, w.Dk, w.Dv), dtype=torch.float32, device=dev)
-    ws = torch.empty(K.chunk_workspace_bytes(B, S, H, w.Dk, w.Dv), dtype=torch.uint8, device=dev)
+    ws = torch.empty(K.chunk_workspace_bytes(B, S, H, w.Dk, w.Dv, scalar_decay=gdn), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    z = d["z"][..., 0].contiguous() if gdn else d["z"]
 
     def chunk():
-        K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=d["z"], g_min=w.g_min, initial_state=d["S0"],
-                    gate_logits=d["gate"], eps=w.eps, out=x, final_state=sf, workspace=ws)
+        K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=z, g_min=w.g_min, initial_state=d["S0"],
+                    gate_logits=d["gate"], eps=w.eps, out=x, final_state=sf, workspace=ws, scalar_decay=gdn)
 
     def proj():
         K.out_proj(x.view(N, H * w.Dv), d["W_o"], out=y)
@@ -345,7 +349,7 @@ def time_prefill(K, torch, w, d, steps, warmup, world, dev, flush, lib, sampler=
     launches = lib.kda_launch_count() - n0
     t_chunk, t_proj = tm.means()
     t_step_max, t_chunk_max, t_proj_max = reduce_max([t_chunk + t_proj, t_chunk, t_proj], world, dev)
-    del x, y, sf, ws
+    del x, y, sf, ws, z
     return {"t_step": t_step_max, "t_chunk": t_chunk_max, "t_proj": t_proj_max, "launches": launches,
             "wall": t_wall}
 
@@ -536,6 +540,16 @@ def run_ours(args, rank, world, local):
                           sampler if name == HEADLINE else None)
         records[name] = prefill_record(w, tm, peaks, world, f"chunk_engine@{name}")
         records[name]["gpu_launches"] = int(tm["launches"])
+        # the scalar-decay (Gated DeltaNet) engine on the same inputs: what the per-channel decay costs
+        tg = time_prefill(K, torch, w, d, max(3, args.steps // 2), args.warmup, world, dev, flush, lib, gdn=True)
+        gr = roofline(chunk_flops(w), prefill_bytes(w, scalar_decay=True), tg["t_chunk"], peaks)
+        records[name]["gdn"] = {
+            "engine": "kda_gdn_chunk_fwd (scalar decay per token and head)",
+            "chunk_engine_ms": round(tg["t_chunk"] * 1e3, 4),
+            "layer_tokens_per_s": round(w.B * w.S * world / tg["t_step"], 1),
+            "chunk_engine_tokens_per_s": round(w.B * w.S * world / tg["t_chunk"], 1),
+            "roofline": {k: gr[k] for k in ("bound", "achieved", "peak", "unit", "frac")},
+            "kda_over_gdn_chunk_time": round(tm["t_chunk"] / tg["t_chunk"], 3)}
         if name == HEADLINE:
             head_tm = tm
         if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -105,7 +105,8 @@ kda_status_t kda_gate(const void *z, kda_dtype_t dtype, int64_t n, float g_min,
  *
  * Layout ("KDA Recurrence" page, problem statement):
  *   q, k, z       (B, S, H, D_k)  dtype
- *   log_decay     (B, S, H, D_k)  fp32 log(alpha) in [g_min, 0], or NULL to use z
+ *   log_decay     (B, S, H, D_k)  fp32 log(alpha) in [g_min, 0] (values outside
+ *                 that range are clamped to it), or NULL to use z
  *   g_min         the lower log-decay bound, finite and < 0 (always required:
  *                 with log_decay it is the caller's bound on those values)
  *   v             (B, S, H, D_v)  dtype
@@ -148,10 +149,35 @@ typedef struct kda_chunk_args {
     void *stream;
 } kda_chunk_args;
 
-/* Workspace bytes kda_chunk_fwd needs for these arguments (pointers unused). */
+/* Workspace bytes kda_chunk_fwd needs for these arguments (pointers unused).
+ * The tensor-core engine's size depends on the current device's SM count (its
+ * segment count does): query it with the device current that will run the
+ * call.  kda_chunk_fwd re-checks the size and returns KDA_ERR_WORKSPACE if the
+ * workspace is smaller. */
 kda_status_t kda_chunk_workspace_size(const kda_chunk_args *args, size_t *bytes);
 
 kda_status_t kda_chunk_fwd(const kda_chunk_args *args);
+
+/*
+ * kda_gdn_chunk_fwd — the Gated DeltaNet special case of the prefill (the
+ * DPLR post's comparison of GDN with KDA: one scalar decay per token and head,
+ *   S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T,
+ * i.e. Eq. 1 with Diag(alpha_t) = alpha_t I), with the same chunkwise
+ * algorithm, output readout (read after the update), optional fused RMSNorm
+ * and sigmoid gate, and state handling as kda_chunk_fwd.  Arguments are those
+ * of kda_chunk_fwd except the decay inputs, which hold one value per token
+ * and head:
+ *   z             (B, S, H)  dtype decay logits, alpha = exp(g_min * sigmoid(z))
+ *   log_decay     (B, S, H)  fp32 log(alpha) in [g_min, 0], or NULL to use z
+ * Because the decay ratio of two tokens is one number, the intra-chunk
+ * products are plain products of the raw keys and queries scaled per token
+ * pair: the tensor-core engine (bf16, D_k = D_v = 128, chunk 64) has no bound
+ * on g_min.  Other shapes run the exact SIMT engine.
+ * Errors: as kda_chunk_fwd.
+ */
+kda_status_t kda_gdn_chunk_workspace_size(const kda_chunk_args *args, size_t *bytes);
+
+kda_status_t kda_gdn_chunk_fwd(const kda_chunk_args *args);
 
 /*
  * kda_decode_step — one token of the Eq. 1 recurrence for B independent

@@ -4,8 +4,8 @@ The compute lives in ``libkda.so`` (hand-written CUDA behind the C ABI of
 ``include/kda.h``); this package only marshals torch tensors into it.
 """
 from ._lib import KDAError, load as load_library  # noqa: F401
-from .api import (chunk_fwd, chunk_workspace_bytes, decode_step, gate, kda_decode, kda_forward,  # noqa: F401
-                  norm_gate, out_norm_gate_proj, out_proj)
+from .api import (chunk_fwd, chunk_workspace_bytes, decode_step, gate, gdn_chunk_fwd, kda_decode,  # noqa: F401
+                  kda_forward, norm_gate, out_norm_gate_proj, out_proj)
 
-__all__ = ["chunk_fwd", "chunk_workspace_bytes", "decode_step", "gate", "kda_decode", "kda_forward",
-           "norm_gate", "out_norm_gate_proj", "out_proj", "KDAError", "load_library"]
+__all__ = ["chunk_fwd", "chunk_workspace_bytes", "decode_step", "gate", "gdn_chunk_fwd", "kda_decode",
+           "kda_forward", "norm_gate", "out_norm_gate_proj", "out_proj", "KDAError", "load_library"]

@@ -60,6 +60,8 @@ SIGNATURES = {
     "kda_gate": (ctypes.c_int, [_p, ctypes.c_int, _i64, _f32, _p, _p]),
     "kda_chunk_workspace_size": (ctypes.c_int, [ctypes.POINTER(ChunkArgs), ctypes.POINTER(ctypes.c_size_t)]),
     "kda_chunk_fwd": (ctypes.c_int, [ctypes.POINTER(ChunkArgs)]),
+    "kda_gdn_chunk_workspace_size": (ctypes.c_int, [ctypes.POINTER(ChunkArgs), ctypes.POINTER(ctypes.c_size_t)]),
+    "kda_gdn_chunk_fwd": (ctypes.c_int, [ctypes.POINTER(ChunkArgs)]),
     "kda_decode_step": (ctypes.c_int, [ctypes.POINTER(DecodeArgs)]),
     "kda_norm_gate": (ctypes.c_int, [_p, _p, _i64, _i32, _i32, _f32, _p, ctypes.c_int, _p]),
     "kda_out_proj": (ctypes.c_int, [_p, _p, _i64, _i32, _i32, _p, ctypes.c_int, _p]),

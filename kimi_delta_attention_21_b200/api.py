@@ -59,13 +59,15 @@ def gate(z: torch.Tensor, g_min: float) -> torch.Tensor:
 
 def chunk_fwd(q, k, v, beta, *, z=None, log_decay=None, g_min=-5.0, initial_state=None,
               gate_logits=None, eps=1e-6, chunk=64, engine="auto", want_final_state=True,
-              out=None, final_state=None, dev_status=None, workspace=None):
+              out=None, final_state=None, dev_status=None, workspace=None, scalar_decay=False):
     """Chunkwise prefill.  Returns (o, final_state):
     o (B,S,H,D_v) in the input dtype holds o~ (gate_logits None) or
     RMSNorm(o~) * sigmoid(gate_logits); final_state (B,H,D_k,D_v) fp32 or None.
     ``final_state`` may be the same tensor as ``initial_state`` (in-place handoff).
     ``workspace`` is an optional uint8 CUDA tensor at least
-    ``chunk_workspace_bytes(...)`` long (allocated per call when omitted)."""
+    ``chunk_workspace_bytes(...)`` long (allocated per call when omitted).
+    ``scalar_decay=True`` runs the Gated DeltaNet case (kda_gdn_chunk_fwd): z
+    and log_decay are then (B,S,H), one decay per token and head."""
     _dev(q, "q")
     dt = q.dtype
     B, S, H, Dk = q.shape
@@ -75,8 +77,9 @@ def chunk_fwd(q, k, v, beta, *, z=None, log_decay=None, g_min=-5.0, initial_stat
     if beta.dim() == 4 and beta.shape[-1] == 1:
         beta = beta.view(B, S, H)
     _dev(beta, "beta", dt, (B, S, H))
-    _dev(z, "z", dt, q.shape)
-    _dev(log_decay, "log_decay", torch.float32, q.shape)
+    dshape = (B, S, H) if scalar_decay else q.shape
+    _dev(z, "z", dt, dshape)
+    _dev(log_decay, "log_decay", torch.float32, dshape)
     _dev(initial_state, "initial_state", torch.float32, (B, H, Dk, Dv))
     _dev(gate_logits, "gate_logits", dt, (B, S, H, Dv))
     _dev(dev_status, "dev_status", torch.int32)
@@ -94,8 +97,10 @@ def chunk_fwd(q, k, v, beta, *, z=None, log_decay=None, g_min=-5.0, initial_stat
                   chunk=int(chunk), engine=ENGINES[engine], dev_status=_ptr(dev_status),
                   stream=_stream(q.device))
     lib = _lib.load()
+    ws_fn, fwd_fn = (("kda_gdn_chunk_workspace_size", "kda_gdn_chunk_fwd") if scalar_decay
+                     else ("kda_chunk_workspace_size", "kda_chunk_fwd"))
     nbytes = ctypes.c_size_t(0)
-    check("kda_chunk_workspace_size", lib.kda_chunk_workspace_size(ctypes.byref(a), ctypes.byref(nbytes)))
+    check(ws_fn, getattr(lib, ws_fn)(ctypes.byref(a), ctypes.byref(nbytes)))
     ws = workspace
     if nbytes.value:
         if ws is None:
@@ -103,16 +108,24 @@ def chunk_fwd(q, k, v, beta, *, z=None, log_decay=None, g_min=-5.0, initial_stat
         _dev(ws, "workspace", torch.uint8)
         a.workspace = _ptr(ws)
         a.workspace_bytes = ws.numel()
-    check("kda_chunk_fwd", lib.kda_chunk_fwd(ctypes.byref(a)))
+    check(fwd_fn, getattr(lib, fwd_fn)(ctypes.byref(a)))
     return out, final_state
 
 
-def chunk_workspace_bytes(B, S, H, Dk, Dv, dtype=torch.bfloat16, chunk=64, engine="auto", g_min=-5.0):
+def chunk_workspace_bytes(B, S, H, Dk, Dv, dtype=torch.bfloat16, chunk=64, engine="auto", g_min=-5.0,
+                          scalar_decay=False):
     a = ChunkArgs(B=B, S=S, H=H, D_k=Dk, D_v=Dv, dtype=_DT[dtype], g_min=float(g_min), eps=1e-6,
                   chunk=chunk, engine=ENGINES[engine])
     n = ctypes.c_size_t(0)
-    check("kda_chunk_workspace_size", _lib.load().kda_chunk_workspace_size(ctypes.byref(a), ctypes.byref(n)))
+    fn = "kda_gdn_chunk_workspace_size" if scalar_decay else "kda_chunk_workspace_size"
+    check(fn, getattr(_lib.load(), fn)(ctypes.byref(a), ctypes.byref(n)))
     return n.value
+
+
+def gdn_chunk_fwd(q, k, v, beta, **kw):
+    """Gated DeltaNet prefill (one scalar decay per token and head): chunk_fwd with
+    z / log_decay of shape (B,S,H).  Returns (o, final_state)."""
+    return chunk_fwd(q, k, v, beta, scalar_decay=True, **kw)
 
 
 def decode_step(q, k, v, beta, state, *, z=None, log_decay=None, g_min=-5.0, gate_logits=None, eps=1e-6,

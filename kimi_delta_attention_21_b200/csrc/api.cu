@@ -97,7 +97,8 @@ static kda_status_t check_gmin(float g_min) {
             return fail(KDA_ERR_INVALID_ARG, "%s is not %d-byte aligned", name, (int)(al));     \
     } while (0)
 
-static kda_status_t chunk_validate(const kda_chunk_args *a, int *chunk_out, bool *use_tc) {
+// gdn: the scalar-decay (Gated DeltaNet) entry points, whose z / log_decay are (B, S, H).
+static kda_status_t chunk_validate(const kda_chunk_args *a, int *chunk_out, bool *use_tc, bool gdn) {
     if (!a) return fail(KDA_ERR_INVALID_ARG, "args is NULL");
     KDA_TRY(check_dtype(a->dtype));
     KDA_TRY(check_gmin(a->g_min));
@@ -112,10 +113,10 @@ static kda_status_t chunk_validate(const kda_chunk_args *a, int *chunk_out, bool
     if (a->engine != KDA_ENGINE_AUTO && a->engine != KDA_ENGINE_SIMT && a->engine != KDA_ENGINE_TC)
         return fail(KDA_ERR_INVALID_ARG, "unknown engine %d", (int)a->engine);
     *chunk_out = chunk;
-    const bool tc_ok = chunk_tc_supported(*a, chunk);
+    const bool tc_ok = gdn ? gdn_tc_supported(*a, chunk) : chunk_tc_supported(*a, chunk);
     if (a->engine == KDA_ENGINE_TC && !tc_ok)
-        return fail(KDA_ERR_UNSUPPORTED,
-                    "tensor-core engine needs bf16, D_k = D_v = 128, chunk 64 and g_min >= -5.5");
+        return fail(KDA_ERR_UNSUPPORTED, gdn ? "tensor-core engine needs bf16, D_k = D_v = 128 and chunk 64"
+                                             : "tensor-core engine needs bf16, D_k = D_v = 128, chunk 64 and g_min >= -5.5");
     *use_tc = (a->engine == KDA_ENGINE_TC) || (a->engine == KDA_ENGINE_AUTO && tc_ok);
     if (a->gate_logits && !(isfinite(a->eps) && a->eps >= 0.0f))
         return fail(KDA_ERR_INVALID_ARG, "eps must be finite and >= 0");
@@ -160,26 +161,25 @@ kda_status_t kda_gate(const void *z, kda_dtype_t dtype, int64_t n, float g_min, 
     return launch_gate(z, dtype, n, g_min, log_alpha, (cudaStream_t)stream);
 }
 
-kda_status_t kda_chunk_workspace_size(const kda_chunk_args *a, size_t *bytes) {
-    g_err[0] = 0;
+static kda_status_t chunk_workspace_impl(const kda_chunk_args *a, size_t *bytes, bool gdn) {
     if (!bytes) return fail(KDA_ERR_INVALID_ARG, "bytes is NULL");
     int chunk;
     bool tc;
-    KDA_TRY(chunk_validate(a, &chunk, &tc));
+    KDA_TRY(chunk_validate(a, &chunk, &tc, gdn));
     *bytes = tc ? chunk_tc_workspace(*a) : chunk_simt_workspace(*a, chunk);
     return KDA_OK;
 }
 
-kda_status_t kda_chunk_fwd(const kda_chunk_args *a) {
-    g_err[0] = 0;
+static kda_status_t chunk_fwd_impl(const kda_chunk_args *a, bool gdn) {
     int chunk;
     bool tc;
-    KDA_TRY(chunk_validate(a, &chunk, &tc));
+    KDA_TRY(chunk_validate(a, &chunk, &tc, gdn));
     if (a->B == 0) return KDA_OK;
     const size_t es = esize(a->dtype);
     const size_t nk = (size_t)a->B * a->S * a->H * a->D_k;
     const size_t nv = (size_t)a->B * a->S * a->H * a->D_v;
     const size_t nb = (size_t)a->B * a->S * a->H;
+    const size_t nz = gdn ? nb : nk;  // decay inputs: one per key channel, or one per (token, head)
     const size_t ns = (size_t)a->B * a->H * a->D_k * a->D_v * 4;
     if (a->S > 0) {
         KDA_REQ_PTR(a->q, "q", es);
@@ -195,9 +195,10 @@ kda_status_t kda_chunk_fwd(const kda_chunk_args *a) {
     KDA_OPT_PTR(a->final_state, "final_state", 4);
     KDA_OPT_PTR(a->workspace, "workspace", 256);
     KDA_OPT_PTR(a->dev_status, "dev_status", 4);
-    if (tc && a->engine == KDA_ENGINE_TC && !chunk_tc_aligned(*a))
+    const bool aligned = gdn ? gdn_tc_aligned(*a) : chunk_tc_aligned(*a);
+    if (tc && a->engine == KDA_ENGINE_TC && !aligned)
         return fail(KDA_ERR_INVALID_ARG, "the tensor-core engine needs 16-byte aligned q, k, v, z, beta, o");
-    if (tc && !chunk_tc_aligned(*a)) tc = false;
+    if (tc && !aligned) tc = false;
     const size_t need = tc ? chunk_tc_workspace(*a) : chunk_simt_workspace(*a, chunk);
     if (need > 0 && (!a->workspace || a->workspace_bytes < need))
         return fail(KDA_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", need,
@@ -206,8 +207,8 @@ kda_status_t kda_chunk_fwd(const kda_chunk_args *a) {
         {a->S ? a->q : nullptr, nk * es, "q"},
         {a->S ? a->k : nullptr, nk * es, "k"},
         {a->S ? a->v : nullptr, nv * es, "v"},
-        {a->S && !a->log_decay ? a->z : nullptr, nk * es, "z"},
-        {a->S ? a->log_decay : nullptr, nk * 4, "log_decay"},
+        {a->S && !a->log_decay ? a->z : nullptr, nz * es, "z"},
+        {a->S ? a->log_decay : nullptr, nz * 4, "log_decay"},
         {a->S ? a->beta : nullptr, nb * es, "beta"},
         {a->S ? a->gate_logits : nullptr, nv * es, "gate_logits"},
         {a->initial_state, ns, "initial_state"},
@@ -221,12 +222,32 @@ kda_status_t kda_chunk_fwd(const kda_chunk_args *a) {
             return fail(KDA_ERR_INVALID_ARG, "final_state overlaps o");
     }
     cudaStream_t st = (cudaStream_t)a->stream;
-    if (tc) return launch_chunk_tc(*a, st);
-    KDA_TRY(launch_chunk_simt(*a, chunk, st));
+    if (tc) return gdn ? launch_gdn_tc(*a, st) : launch_chunk_tc(*a, st);
+    KDA_TRY(launch_chunk_simt(*a, chunk, st, gdn));
     if (a->gate_logits && a->S > 0)
         return launch_norm_gate(a->o, a->gate_logits, a->B * a->S, a->H, a->D_v, a->eps, a->o,
                                 a->dtype, st);
     return KDA_OK;
+}
+
+kda_status_t kda_chunk_workspace_size(const kda_chunk_args *a, size_t *bytes) {
+    g_err[0] = 0;
+    return chunk_workspace_impl(a, bytes, false);
+}
+
+kda_status_t kda_chunk_fwd(const kda_chunk_args *a) {
+    g_err[0] = 0;
+    return chunk_fwd_impl(a, false);
+}
+
+kda_status_t kda_gdn_chunk_workspace_size(const kda_chunk_args *a, size_t *bytes) {
+    g_err[0] = 0;
+    return chunk_workspace_impl(a, bytes, true);
+}
+
+kda_status_t kda_gdn_chunk_fwd(const kda_chunk_args *a) {
+    g_err[0] = 0;
+    return chunk_fwd_impl(a, true);
 }
 
 kda_status_t kda_decode_step(const kda_decode_args *a) {

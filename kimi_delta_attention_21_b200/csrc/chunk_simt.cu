@@ -37,6 +37,7 @@ struct SimtParams {
     const void *q, *k, *v, *z, *beta;
     const float *log_decay;
     float g_min;
+    int scalar_decay;  // 1: z / log_decay hold one value per (token, head) (the GDN case), shared by all channels
     const float *S0;
     void *o;
     float *Sf;
@@ -102,7 +103,9 @@ __global__ void __launch_bounds__(NT) chunk_simt_kernel(SimtParams p) {
                 const int64_t off = (row0 + r) * strideK + (int64_t)h * Dk + c;
                 kv = load_elem(k, off);
                 qv = load_elem(q, off);
-                g = p.log_decay ? (GT)clamp_log_decay(p.log_decay[off], p.g_min) : log_alpha_gt((GT)load_elem(z, off), p.g_min, GT(0));
+                const int64_t doff = p.scalar_decay ? (row0 + r) * p.H + h : off;
+                g = p.log_decay ? (GT)clamp_log_decay(p.log_decay[doff], p.g_min)
+                                : log_alpha_gt((GT)load_elem(z, doff), p.g_min, GT(0));
             }
             sK[r * LD + c] = kv;
             sQ[r * LD + c] = qv;
@@ -212,7 +215,7 @@ __global__ void __launch_bounds__(NT) chunk_simt_kernel(SimtParams p) {
 
 size_t chunk_simt_workspace(const kda_chunk_args &, int) { return 0; }
 
-kda_status_t launch_chunk_simt(const kda_chunk_args &a, int chunk, cudaStream_t st) {
+kda_status_t launch_chunk_simt(const kda_chunk_args &a, int chunk, cudaStream_t st, bool scalar_decay) {
     SimtParams p;
     p.S = a.S;
     p.H = a.H;
@@ -223,6 +226,7 @@ kda_status_t launch_chunk_simt(const kda_chunk_args &a, int chunk, cudaStream_t 
     p.q = a.q; p.k = a.k; p.v = a.v; p.z = a.z; p.beta = a.beta;
     p.log_decay = a.log_decay;
     p.g_min = a.g_min;
+    p.scalar_decay = scalar_decay ? 1 : 0;
     p.S0 = a.initial_state;
     p.o = a.o;
     p.Sf = a.final_state;

@@ -51,92 +51,15 @@
 
 #include <cuda_fp16.h>
 
-#include "kda_internal.cuh"
-#include "sm100_ptx.cuh"
-#include "tma_host.cuh"
+#include "tc_common.cuh"
 
 namespace kda {
 
 namespace {
 
 using namespace sm100;
+using namespace tc;
 
-constexpr int CH = 64;   // chunk length
-constexpr int DD = 128;  // D_k = D_v
-constexpr float TC_GMIN_LIMIT = -5.5f;
-
-// ---------------------------------------------------------------- workspace record (per b, h, chunk)
-// All images are 128-byte-swizzled bf16 tiles in the layout the state kernel's
-// MMAs read them in, so a record is one contiguous bulk copy away from use.
-constexpr uint32_t REC_WQ = 0;        // [2 atoms (c / 64)][128 rows: -W rows 0-63, Q e^G rows 64-127][128 B]
-                                      //   K-major A operand of [-W; Q e^G] S (M = 128)
-constexpr uint32_t REC_KT = 32768;    // K e^{G_C - G}  [2 atoms (c / 64)][64 rows i][128 B], MN-major A of K~^T V'
-constexpr uint32_t REC_MT = 49152;    // M^T            [64 rows i][128 B: r]; with the K~ atom in front of it,
-                                      //   the MN-major A operand of [*; M] V' (M = 128, rows 64-127 = M)
-constexpr uint32_t REC_U = 57344;     // U^T            [128 rows j][128 B: r]
-constexpr uint32_t REC_GAM = 73728;   // e^{G_C}        128 fp32
-constexpr uint32_t REC_BYTES = 74240;
-constexpr uint32_t GATE_TILE_BYTES = CH * 128 * 2;  // one chunk of output-gate logits, [2 atoms][64 rows][128 B] bf16
-
-__device__ __forceinline__ uint32_t sw128(uint32_t row, uint32_t chunk) {
-    return row * 128u + ((chunk ^ (row & 7u)) << 4);
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t *>(&h);
-}
-
-__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
-    uint4 u;
-    u.x = pack_bf16x2(f[0], f[1]);
-    u.y = pack_bf16x2(f[2], f[3]);
-    u.z = pack_bf16x2(f[4], f[5]);
-    u.w = pack_bf16x2(f[6], f[7]);
-    return u;
-}
-
-__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
-    const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float2 x = __bfloat1622float2(h[j]);
-        f[2 * j] = x.x;
-        f[2 * j + 1] = x.y;
-    }
-}
-
-__device__ __forceinline__ void load8f(const float *p, float (&f)[8]) {
-    const float4 a = reinterpret_cast<const float4 *>(p)[0];
-    const float4 b = reinterpret_cast<const float4 *>(p)[1];
-    f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
-    f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
-}
-
-// The tensor-core engine works on bf16 data and every exponent it takes is
-// bounded (|x| <= 8 |g_min| + |g_min| * 64), so the hardware exp2 approximation
-// (a few ulp of fp32) is far below the bf16 rounding it feeds.
-__device__ __forceinline__ float fexp(float x) { return __expf(x); }
-__device__ __forceinline__ float log_alpha_fast(float z, float g_min) {
-    return g_min * __fdividef(1.0f, 1.0f + __expf(-z));
-}
-
-// A descriptor for base + off: the start-address field holds address >> 4 in 14
-// bits, which cannot carry for shared-memory addresses below 256 KB.
-__device__ __forceinline__ uint64_t dadd(uint64_t d, uint32_t off_bytes) { return d + (off_bytes >> 4); }
-
-__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
-    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
-}
-
-__device__ __forceinline__ void named_sync(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-
-__device__ __forceinline__ void report_timeout(unsigned int *timeouts, int *dev_status) {
-    if (timeouts) atomicAdd(timeouts, 1u);
-    if (dev_status) atomicExch(dev_status, (int)KDA_ERR_TIMEOUT);
-}
 
 // ================================================================ K2a: chunk_prep_kernel
 // Persistent: one CTA per SM walks (chunk, head, batch) units.  The next unit's
@@ -179,7 +102,7 @@ constexpr uint32_t P_ST = P_SA + 16640;               // T [64][68] fp32
 constexpr uint32_t P_LOHI = P_A;                      // [64][16] fp32
 constexpr uint32_t P_IX = P_A + 4096;                 // inverse scratch [512 + 1024] fp32
 static_assert(P_ST + 64 * 68 * 4 <= P_B + 2 * B_ATOM_BYTES, "A and T fit in the B operand's space");
-constexpr int SG_LD = 132, SA_LD = 65, ST_LD = 68;
+constexpr int SG_LD = 132;
 constexpr uint32_t A_KLO = 160;         // first row of the low part of the diagonal column operand
 
 // table rows: b_R (0-3), F_R = e^{b_{R-1} - m_R} (4-7), E_R = e^{b_{R-1}} (8-11),
@@ -630,132 +553,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         // as zeros where a later product reads them; the T image zero-fills the upper-right 32x32 block.
         // Warps 0-3 only (named barrier 1); warps 4-11 meanwhile compute the next unit's decay and tables.
         if (warp < 4) {
-            const float *sA = reinterpret_cast<const float *>(sm + P_SA);
-            float *sT = reinterpret_cast<float *>(sm + P_ST);
-            float *xs = reinterpret_cast<float *>(sm + P_IX);
-            if (tid < 64) {  // diagonal block R, column jc: (I + A_RR) x = e_jc, right-looking
-                const int R = tid >> 4, jc = tid & 15, o = 16 * R;
-                float x[16];
-#pragma unroll
-                for (int a = 0; a < 16; ++a) x[a] = (a == jc) ? 1.f : 0.f;
-                // once x[m] is final, every later row subtracts its term: one FMA per step on the
-                // critical path (entries above jc stay exact zeros)
-#pragma unroll
-                for (int m = 0; m < 15; ++m)
-#pragma unroll
-                    for (int a = m + 1; a < 16; ++a) x[a] = fmaf(-sA[(o + a) * SA_LD + o + m], x[m], x[a]);
-#pragma unroll
-                for (int a = 0; a < 16; ++a) sT[(o + a) * ST_LD + o + jc] = x[a];
-            }
-            named_sync(1, 128);
-            // The products below give each thread rows (p, p + h) and four adjacent columns, so that one
-            // float4 of the right operand feeds eight FMAs (shared-memory wavefronts, not FMAs, bound them).
-            float *x2 = xs + 512;  // X = A[32:64, 0:32] T[0:32, 0:32] for the 32 -> 64 step, [32][32]
-            if (tid < 64) {  // 16 -> 32: X = A_{R,R-1} T_{R-1,R-1}, R = 1 + 2 hb
-                const int hb = tid >> 5, R = 1 + 2 * hb, pr = (tid >> 2) & 7, c4 = 4 * (tid & 3), o = 16 * (R - 1);
-                const float *a0 = sA + (16 * R + pr) * SA_LD + o, *a1 = a0 + 8 * SA_LD;
-                const float *tb = sT + o * ST_LD + o + c4;
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float u = a0[m], v = a1[m];
-                    const float4 t = *reinterpret_cast<const float4 *>(tb + m * ST_LD);
-                    x.x += u * t.x; x.y += u * t.y; x.z += u * t.z; x.w += u * t.w;
-                    y.x += v * t.x; y.y += v * t.y; y.z += v * t.z; y.w += v * t.w;
-                }
-                *reinterpret_cast<float4 *>(xs + hb * 256 + pr * 16 + c4) = x;
-                *reinterpret_cast<float4 *>(xs + hb * 256 + (pr + 8) * 16 + c4) = y;
-            } else {  // meanwhile the part of the 32 -> 64 product that needs only the diagonal blocks:
-                      // X[:, 16 B + c] = A[32:64, 16 B : 16 B + 16] T_BB  (B = 0, 1)
-                const int t2 = tid - 64, pr = t2 >> 2, c8 = 8 * (t2 & 3), blk = c8 >> 4;
-                const float *a0 = sA + (32 + pr) * SA_LD + 16 * blk, *a1 = a0 + 16 * SA_LD;
-                const float *tb = sT + 16 * blk * ST_LD + c8;
-                float4 x0 = make_float4(0.f, 0.f, 0.f, 0.f), x1 = x0, y0 = x0, y1 = x0;
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float u = a0[m], v = a1[m];
-                    const float4 t0 = *reinterpret_cast<const float4 *>(tb + m * ST_LD);
-                    const float4 t1 = *reinterpret_cast<const float4 *>(tb + m * ST_LD + 4);
-                    x0.x += u * t0.x; x0.y += u * t0.y; x0.z += u * t0.z; x0.w += u * t0.w;
-                    x1.x += u * t1.x; x1.y += u * t1.y; x1.z += u * t1.z; x1.w += u * t1.w;
-                    y0.x += v * t0.x; y0.y += v * t0.y; y0.z += v * t0.z; y0.w += v * t0.w;
-                    y1.x += v * t1.x; y1.y += v * t1.y; y1.z += v * t1.z; y1.w += v * t1.w;
-                }
-                *reinterpret_cast<float4 *>(x2 + pr * 32 + c8) = x0;
-                *reinterpret_cast<float4 *>(x2 + pr * 32 + c8 + 4) = x1;
-                *reinterpret_cast<float4 *>(x2 + (pr + 16) * 32 + c8) = y0;
-                *reinterpret_cast<float4 *>(x2 + (pr + 16) * 32 + c8 + 4) = y1;
-            }
-            named_sync(1, 128);
-            if (tid < 64) {  //       T_{R,R-1} = -T_RR X  (T_RR is zero above its diagonal); zero block (R-1, R)
-                const int hb = tid >> 5, R = 1 + 2 * hb, pr = (tid >> 2) & 7, c4 = 4 * (tid & 3);
-                const float *t0 = sT + (16 * R + pr) * ST_LD + 16 * R, *t1 = t0 + 8 * ST_LD;
-                const float *xb = xs + hb * 256 + c4;
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float u = t0[m], v = t1[m];
-                    const float4 t = *reinterpret_cast<const float4 *>(xb + m * 16);
-                    x.x += u * t.x; x.y += u * t.y; x.z += u * t.z; x.w += u * t.w;
-                    y.x += v * t.x; y.y += v * t.y; y.z += v * t.z; y.w += v * t.w;
-                }
-                float *d0 = sT + (16 * R + pr) * ST_LD + 16 * (R - 1) + c4;
-                *reinterpret_cast<float4 *>(d0) = make_float4(-x.x, -x.y, -x.z, -x.w);
-                *reinterpret_cast<float4 *>(d0 + 8 * ST_LD) = make_float4(-y.x, -y.y, -y.z, -y.w);
-                float *z0 = sT + (16 * (R - 1) + pr) * ST_LD + 16 * R + c4;
-                *reinterpret_cast<float4 *>(z0) = make_float4(0.f, 0.f, 0.f, 0.f);
-                *reinterpret_cast<float4 *>(z0 + 8 * ST_LD) = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-            named_sync(1, 128);
-            if (tid < 64) {  // 32 -> 64: the rest of X, X[:, 0:16] += A[32:64, 16:32] T_10
-                const int pr = tid >> 2, c4 = 4 * (tid & 3);
-                const float *a0 = sA + (32 + pr) * SA_LD + 16, *a1 = a0 + 16 * SA_LD;
-                const float *tb = sT + 16 * ST_LD + c4;
-                float4 x = *reinterpret_cast<const float4 *>(x2 + pr * 32 + c4);
-                float4 y = *reinterpret_cast<const float4 *>(x2 + (pr + 16) * 32 + c4);
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float u = a0[m], v = a1[m];
-                    const float4 t = *reinterpret_cast<const float4 *>(tb + m * ST_LD);
-                    x.x += u * t.x; x.y += u * t.y; x.z += u * t.z; x.w += u * t.w;
-                    y.x += v * t.x; y.y += v * t.y; y.z += v * t.z; y.w += v * t.w;
-                }
-                *reinterpret_cast<float4 *>(x2 + pr * 32 + c4) = x;
-                *reinterpret_cast<float4 *>(x2 + (pr + 16) * 32 + c4) = y;
-            }
-            named_sync(1, 128);
-            if (tid < 128) {  //       T[32:64, 0:32] = -T[32:64, 32:64] X  (rows 32-47: T_22 only, T_23 = 0)
-                const int pr = tid >> 3, c4 = 4 * (tid & 7);
-                const float *t0 = sT + (32 + pr) * ST_LD + 32, *t1 = t0 + 16 * ST_LD;
-                const float *xb = x2 + c4;
-                float4 x = make_float4(0.f, 0.f, 0.f, 0.f), y = x;
-#pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const float u = t0[m], v = t1[m];
-                    const float4 t = *reinterpret_cast<const float4 *>(xb + m * 32);
-                    x.x += u * t.x; x.y += u * t.y; x.z += u * t.z; x.w += u * t.w;
-                    y.x += v * t.x; y.y += v * t.y; y.z += v * t.z; y.w += v * t.w;
-                }
-#pragma unroll
-                for (int m = 16; m < 32; ++m) {
-                    const float v = t1[m];
-                    const float4 t = *reinterpret_cast<const float4 *>(xb + m * 32);
-                    y.x += v * t.x; y.y += v * t.y; y.z += v * t.z; y.w += v * t.w;
-                }
-                float *d0 = sT + (32 + pr) * ST_LD + c4;
-                *reinterpret_cast<float4 *>(d0) = make_float4(-x.x, -x.y, -x.z, -x.w);
-                *reinterpret_cast<float4 *>(d0 + 16 * ST_LD) = make_float4(-y.x, -y.y, -y.z, -y.w);
-            }
-            named_sync(1, 128);
-            for (int k = 0; k < 4; ++k) {  // T image (K-major, 64 rows x 64 cols), 8-column chunks
-                const int r = (tid >> 3) + 16 * k, cc = tid & 7;
-                float t[8];
-                const bool upper = r < 32 && cc >= 4;
-#pragma unroll
-                for (int e = 0; e < 8; ++e) t[e] = upper ? 0.f : sT[r * ST_LD + 8 * cc + e];
-                *reinterpret_cast<uint4 *>(sm + P_TI + sw128(r, cc)) = pack8(t);
-            }
-            fence_proxy_async_smem();
+            invert_unit_lower64(reinterpret_cast<const float *>(sm + P_SA), reinterpret_cast<float *>(sm + P_ST),
+                                reinterpret_cast<float *>(sm + P_IX), sm + P_TI, tid);
         } else if (warp < 12 && u_next < p.units) {
             ok = decay_tables(u_next, (uint32_t)(it + 1) & 1u, beta_next) && ok;
         }
@@ -1482,19 +1281,16 @@ kda_status_t launch_state(const CUtensorMap &tmo, const CUtensorMap &tgl, const 
     return check_launch("chunk_state_kernel");
 }
 
-// (B, S, H, 128) bf16 tensor seen as 4-D (channel, head, token, batch); a box is
-// 64 channels x 1 head x 64 tokens x 1 batch row, 128-byte swizzled, and tokens
-// past the end of a sequence read as zero.
-kda_status_t make_tmap_tokens(CUtensorMap *m, const void *base, int H, int64_t S, int64_t B, uint64_t rs,
-                              uint64_t ss, uint64_t bs) {
+}  // namespace
+
+kda_status_t tc::make_tmap_tokens(CUtensorMap *m, const void *base, int H, int64_t S, int64_t B, uint64_t rs,
+                                  uint64_t ss, uint64_t bs) {
     const uint64_t dims[4] = {(uint64_t)DD, (uint64_t)H, (uint64_t)S, (uint64_t)B};
     const uint64_t strides[3] = {rs, ss, bs};
     const uint32_t box[4] = {64, 1, CH, 1};
     return make_tmap_nd(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, 4, dims, strides, box,
                         CU_TENSOR_MAP_SWIZZLE_128B);
 }
-
-}  // namespace
 
 bool chunk_tc_supported(const kda_chunk_args &a, int chunk) {
     return a.dtype == KDA_BF16 && a.D_k == DD && a.D_v == DD && chunk == CH && a.g_min >= TC_GMIN_LIMIT &&
@@ -1508,6 +1304,8 @@ bool chunk_tc_aligned(const kda_chunk_args &a) {
     if (!a.log_decay) okp = okp && al(a.z);
     return okp;
 }
+
+namespace {
 
 // Workspace: one record per chunk, then (with several segments) the segment maps
 // A_g^T (bf16 images) and Y_g, and the segments' entering states.
@@ -1530,27 +1328,52 @@ TcLayout tc_layout(const kda_chunk_args &a) {
     return t;
 }
 
+}  // namespace
+
 size_t chunk_tc_workspace(const kda_chunk_args &a) { return tc_layout(a).total; }
 
-kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
+kda_status_t tc::launch_chunk_state_pass(const kda_chunk_args &a, cudaStream_t st) {
     const int64_t Nc = (a.S + CH - 1) / CH;
-    unsigned int *timeouts = device_timeout_counter();
     CUtensorMap to, tgl;
     memset(&to, 0, sizeof(to));  // (no chunks: never read)
     memset(&tgl, 0, sizeof(tgl));  // (no gate: never read)
     const TcLayout lay = tc_layout(a);
     uint8_t *ws = (uint8_t *)a.workspace;
     if (Nc > 0) {
-        CUtensorMap tq, tk, tv, tz;
         const uint64_t rs = (uint64_t)DD, ss = (uint64_t)a.H * DD, bs = (uint64_t)a.S * a.H * DD;
-        kda_status_t s;
-        s = make_tmap_tokens(&to, a.o, a.H, a.S, a.B, rs, ss, bs);
+        kda_status_t s = make_tmap_tokens(&to, a.o, a.H, a.S, a.B, rs, ss, bs);
         if (s != KDA_OK) return s;
         if (a.gate_logits) {
             s = make_tmap_tokens(&tgl, a.gate_logits, a.H, a.S, a.B, rs, ss, bs);
             if (s != KDA_OK) return s;
         }
-        s = make_tmap_tokens(&tq, a.q, a.H, a.S, a.B, rs, ss, bs);
+    }
+    StateArgs sa;
+    sa.S = (int)a.S;
+    sa.H = a.H;
+    sa.Nc = (int)Nc;
+    sa.ws = (const uint8_t *)a.workspace;
+    sa.S0 = a.initial_state;
+    sa.Sf = a.final_state;
+    sa.gated = a.gate_logits != nullptr && Nc > 0;
+    sa.L = Nc > 0 ? lay.L : 1;
+    sa.G = Nc > 0 ? lay.G : 1;
+    sa.xt = ws + lay.xt;
+    sa.yt = reinterpret_cast<float *>(ws + lay.yt);
+    sa.seg_init = reinterpret_cast<const float *>(ws + lay.seg);
+    sa.eps = a.eps;
+    sa.timeouts = device_timeout_counter();
+    sa.dev_status = a.dev_status;
+    return launch_state(to, tgl, sa, (int)a.B, a.H, st);
+}
+
+kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
+    const int64_t Nc = (a.S + CH - 1) / CH;
+    unsigned int *timeouts = device_timeout_counter();
+    if (Nc > 0) {
+        CUtensorMap tq, tk, tv, tz;
+        const uint64_t rs = (uint64_t)DD, ss = (uint64_t)a.H * DD, bs = (uint64_t)a.S * a.H * DD;
+        kda_status_t s = make_tmap_tokens(&tq, a.q, a.H, a.S, a.B, rs, ss, bs);
         if (s != KDA_OK) return s;
         s = make_tmap_tokens(&tk, a.k, a.H, a.S, a.B, rs, ss, bs);
         if (s != KDA_OK) return s;
@@ -1583,23 +1406,7 @@ kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
         s = check_launch("chunk_prep_kernel");
         if (s != KDA_OK) return s;
     }
-    StateArgs sa;
-    sa.S = (int)a.S;
-    sa.H = a.H;
-    sa.Nc = (int)Nc;
-    sa.ws = (const uint8_t *)a.workspace;
-    sa.S0 = a.initial_state;
-    sa.Sf = a.final_state;
-    sa.gated = a.gate_logits != nullptr && Nc > 0;
-    sa.L = Nc > 0 ? lay.L : 1;
-    sa.G = Nc > 0 ? lay.G : 1;
-    sa.xt = ws + lay.xt;
-    sa.yt = reinterpret_cast<float *>(ws + lay.yt);
-    sa.seg_init = reinterpret_cast<const float *>(ws + lay.seg);
-    sa.eps = a.eps;
-    sa.timeouts = timeouts;
-    sa.dev_status = a.dev_status;
-    return launch_state(to, tgl, sa, (int)a.B, a.H, st);
+    return tc::launch_chunk_state_pass(a, st);
 }
 
 }  // namespace kda

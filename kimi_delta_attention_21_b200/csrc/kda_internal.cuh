@@ -52,8 +52,9 @@ kda_status_t launch_gate(const void *z, kda_dtype_t dt, int64_t n, float g_min, 
 
 kda_status_t launch_decode(const kda_decode_args &a, cudaStream_t st);
 
-// SIMT chunk engine: exact fp32 arithmetic, any D_k, D_v <= 128, chunk <= 64.
-kda_status_t launch_chunk_simt(const kda_chunk_args &a, int chunk, cudaStream_t st);
+// SIMT chunk engine: exact fp32 arithmetic, any D_k, D_v <= 128, chunk <= 64.  scalar_decay: z or
+// log_decay hold one value per (token, head) (B, S, H), the decay of every key channel (GDN).
+kda_status_t launch_chunk_simt(const kda_chunk_args &a, int chunk, cudaStream_t st, bool scalar_decay = false);
 size_t chunk_simt_workspace(const kda_chunk_args &a, int chunk);
 
 // tcgen05 chunk engine: bf16, D_k = D_v = 128, chunk 64.
@@ -61,6 +62,12 @@ bool chunk_tc_supported(const kda_chunk_args &a, int chunk);
 bool chunk_tc_aligned(const kda_chunk_args &a);
 size_t chunk_tc_workspace(const kda_chunk_args &a);
 kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st);
+
+// tcgen05 chunk engine for the scalar-decay (GDN) case: bf16, D_k = D_v = 128, chunk 64, any g_min.
+// Same workspace as the KDA engine (chunk_tc_workspace).
+bool gdn_tc_supported(const kda_chunk_args &a, int chunk);
+bool gdn_tc_aligned(const kda_chunk_args &a);
+kda_status_t launch_gdn_tc(const kda_chunk_args &a, cudaStream_t st);
 
 kda_status_t launch_norm_gate(const void *o, const void *gl, int64_t N, int H, int Dv, float eps,
                               void *x, kda_dtype_t dt, cudaStream_t st);

@@ -125,6 +125,20 @@ def recurrence(q, k, v, beta, *, z=None, log_decay=None, g_min=-5.0,
     return o, sf
 
 
+def gdn_recurrence(q, k, v, beta, *, z=None, log_decay=None, g_min=-5.0, initial_state=None, t_rec=None,
+                   want_outputs=True, threads=None):
+    """Gated DeltaNet: the DPLR post's GDN form with one scalar decay per token
+    and head, S_t = alpha_t (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T,
+    which is Eq. 1 with Diag(alpha_t) = alpha_t I.  ``z`` / ``log_decay`` are
+    (B,S,H); every key channel gets the token's value and the Eq. 1 recurrence
+    above runs unchanged (same readout from the updated state).  Returns what
+    ``recurrence`` returns."""
+    Dk = np.asarray(q).shape[-1]
+    widen = lambda a: None if a is None else np.repeat(np.asarray(a, np.float32)[..., None], Dk, axis=-1)
+    return recurrence(q, k, v, beta, z=widen(z), log_decay=widen(log_decay), g_min=g_min,
+                      initial_state=initial_state, t_rec=t_rec, want_outputs=want_outputs, threads=threads)
+
+
 def log_decay(z, g_min):
     """The decay gate in log form, g_min * sigmoid(z) = log(alpha) ("KDA Recurrence"
     page, gate formula), fp64."""
@@ -164,4 +178,5 @@ def forward(query, key, value, decay_logits, write_strength, output_gate_logits,
     return {"outputs": y, "final_state": sf, "o_core": o}
 
 
-__all__ = ["build", "recurrence", "log_decay", "norm_gate", "project", "forward", "default_threads"]
+__all__ = ["build", "recurrence", "gdn_recurrence", "log_decay", "norm_gate", "project", "forward",
+           "default_threads"]

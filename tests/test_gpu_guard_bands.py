@@ -147,3 +147,23 @@ def test_out_norm_gate_proj_writes_stay_inside(K, dtype):
     gy2, y2 = _tensor((N, Dm), dtype)
     assert lib.kda_out_norm_gate_proj_noalloc(p(o), p(gl), p(W), N, H, Dv, Dm, 1e-6, p(y2), code, stream) == 0
     gy2.check("out_norm_gate_proj_noalloc y")
+
+
+@pytest.mark.parametrize("engine,dtype,D", [("tc", "bf16", 128), ("simt", "f32", 24)])
+def test_gdn_chunk_writes_stay_inside(K, engine, dtype, D):
+    w = small(f"gb_gdn{D}", 2, 333, 3, D, D, 32, dtype, seed=640 + D)
+    inp = ki.make_inputs(w)
+    d = upload(inp, w)
+    dt = d["q"].dtype
+    zh = d["z"][..., 0].contiguous()
+    s0 = torch.randn((w.B, w.H, w.Dk, w.Dv), device="cuda") * 0.02
+    go, o = _tensor((w.B, w.S, w.H, w.Dv), dt)
+    gs, sf = _tensor((w.B, w.H, w.Dk, w.Dv), torch.float32)
+    nws = K.chunk_workspace_bytes(w.B, w.S, w.H, w.Dk, w.Dv, dt, engine=engine, scalar_decay=True)
+    gw = Guarded(nws)
+    K.gdn_chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=zh, g_min=w.g_min, initial_state=s0,
+                    gate_logits=d["gate"], eps=w.eps, engine=engine, out=o, final_state=sf,
+                    workspace=gw.bytes_view() if nws else None)
+    go.check(f"GDN o ({engine})")
+    gs.check(f"GDN final_state ({engine})")
+    gw.check(f"GDN workspace ({engine})")

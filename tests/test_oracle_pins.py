@@ -227,6 +227,36 @@ def test_gated_deltanet_when_decay_is_channel_constant():
         np.testing.assert_allclose(sf[0, h], St, rtol=1e-12, atol=1e-13)
 
 
+def test_gdn_recurrence_matches_the_scalar_decay_form():
+    # the GDN oracle (per-head decay inputs) against the DPLR post's scalar form evaluated directly,
+    # for z and for a log-decay input, readouts included (o_t = S_t^T q_t after the update)
+    q, k, v, z, beta, S0 = _problem(2, 11, 3, 5, 4, 21)
+    zh = z[..., 0]
+    o, sf = oracle.gdn_recurrence(q, k, v, beta, z=zh, g_min=-3.0, initial_state=S0)
+    ld = -3.0 / (1.0 + np.exp(-zh.astype(np.float64)))
+    o2, sf2 = oracle.gdn_recurrence(q, k, v, beta, log_decay=ld.astype(np.float32), g_min=-3.0, initial_state=S0)
+    for b in range(2):
+        for h in range(3):
+            St = S0[b, h].astype(np.float64)
+            for t in range(11):
+                kt = k[b, t, h].astype(np.float64)
+                St = np.exp(ld[b, t, h]) * (np.eye(5) - beta[b, t, h] * np.outer(kt, kt)) @ St + \
+                    beta[b, t, h] * np.outer(kt, v[b, t, h])
+                np.testing.assert_allclose(o[b, t, h], St.T @ q[b, t, h], rtol=1e-11, atol=1e-12)
+            np.testing.assert_allclose(sf[b, h], St, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(sf2, sf, rtol=1e-6, atol=1e-7)   # log alpha rounded to fp32 on that path
+
+
+def test_gdn_recurrence_pure_decay_closed_form():
+    # beta = 0: S_t = (prod alpha) S_0 exactly, for a scalar decay as large as g_min = -20 allows
+    q, k, v, z, beta, S0 = _problem(1, 40, 2, 4, 3, 22)
+    beta[:] = 0
+    zh = z[..., 0]
+    _, sf = oracle.gdn_recurrence(q, k, v, beta, z=zh, g_min=-20.0, initial_state=S0)
+    tot = np.sum(-20.0 / (1.0 + np.exp(-zh.astype(np.float64))), axis=1)   # (1, H)
+    np.testing.assert_allclose(sf, np.exp(tot)[..., None, None] * S0, rtol=1e-12, atol=1e-300)
+
+
 # ---------------------------------------------------------------- output head
 
 def test_rms_norm_and_gate():
