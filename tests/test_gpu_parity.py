@@ -279,3 +279,30 @@ def test_unaligned_views_take_exact_paths(K):
     assert_bf16_state(to_np(st), s_ref)
     zz = d["z"].flatten()[3:1000]
     np.testing.assert_allclose(to_np(K.gate(zz, -5.0)), oracle.log_decay(to_np(zz), -5.0), rtol=1e-6, atol=1e-6)
+
+
+# ------------------------------------------------------------------ head-sharded layer
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_head_sharded_layer_on_one_gpu(K, world):
+    """Each rank's share of the head-sharded layer (its heads through the chunk engine and its W_o
+    column block through the projection), run one after another on this GPU; the fp32 sum of the
+    partial outputs is the layer output (checked against the oracle) and each rank keeps its heads'
+    final states.  The ranks never wait on one another, so one GPU can run them in turn."""
+    from kimi_delta_attention_21_b200.tensor_parallel import head_range, kda_forward_tp, shard, wo_columns
+    w = small("tpg", 2, 300, 6, 128, 128, 512, "bf16", seed=77, s0_std=0.02)
+    inp = ki.make_inputs(w)
+    d = upload(inp, w)
+    want = oracle_layer(inp, w)
+    total = 0
+    for rank in range(world):
+        h0, h1 = head_range(w.H, world, rank)
+        c0, c1 = wo_columns(h0, h1, w.Dv)
+        sl = lambda t: shard(t, h0, h1)
+        y_r, s_r = kda_forward_tp(sl(d["q"]), sl(d["k"]), sl(d["v"]), sl(d["z"]), sl(d["beta"]), sl(d["gate"]),
+                                  d["W_o"][:, c0:c1].contiguous(), shard(d["S0"], h0, h1, head_axis=1),
+                                  g_min=w.g_min, eps=w.eps, H=w.H, rank=rank, world=world, out_dtype=torch.float32)
+        torch.cuda.synchronize()
+        total = total + to_np(y_r)
+        assert_bf16_state(to_np(s_r), want["final_state"][:, h0:h1], f"rank {rank} final states")
+    assert_bf16_outputs(total, want["outputs"], f"summed partial outputs ({world} ranks)")
