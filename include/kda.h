@@ -180,6 +180,56 @@ kda_status_t kda_gdn_chunk_workspace_size(const kda_chunk_args *args, size_t *by
 kda_status_t kda_gdn_chunk_fwd(const kda_chunk_args *args);
 
 /*
+ * kda_recurrent_bwd — gradient of the prefill recurrence for training: given
+ * dL/do~_t for every token (o~_t = S_t^T q_t, the core output before any
+ * normalisation) and dL/dS_T, the gradients with respect to q, k, v, beta,
+ * the decay input (z, or log_decay when that is given) and the initial state.
+ * Reverse-mode differentiation of Eq. 1 (Kimi Linear report, section 3) token
+ * by token, exact fp32: the state is checkpointed every 64 tokens on a forward
+ * pass and each chunk's states are recomputed from its checkpoint before its
+ * tokens are differentiated in reverse order.  (The pages motivate the chunk
+ * form by training; this is the recurrent form of its backward pass.)
+ *   q, k, z/log_decay, v, beta, initial_state, g_min : as kda_chunk_fwd
+ *   d_o           (B, S, H, D_v)  dtype: dL/do~
+ *   d_final_state (B, H, D_k, D_v) fp32, or NULL for zero
+ *   dq, dk, dz    (B, S, H, D_k)  fp32 out (dz is d/dz, or d/dlog_decay with
+ *                 a log_decay input: zero where that input was clamped)
+ *   dv            (B, S, H, D_v)  fp32 out;  dbeta (B, S, H) fp32 out
+ *   d_initial_state (B, H, D_k, D_v) fp32 out, or NULL to skip
+ * Outputs are overwritten (zeroed on the stream first).  D_k, D_v <= 128.
+ * The workspace holds the checkpoints and a per-block stash (size query).
+ * Errors: INVALID_ARG, UNSUPPORTED (D_k or D_v > 128), WORKSPACE.
+ */
+typedef struct kda_recurrent_bwd_args {
+    int64_t B, S;
+    int32_t H, D_k, D_v;
+    kda_dtype_t dtype;
+    const void *q;
+    const void *k;
+    const void *v;
+    const void *z;
+    const float *log_decay;
+    float g_min;
+    const void *beta;
+    const float *initial_state;
+    const void *d_o;
+    const float *d_final_state;
+    float *dq;
+    float *dk;
+    float *dv;
+    float *dbeta;
+    float *dz;
+    float *d_initial_state;
+    void *workspace;
+    size_t workspace_bytes;
+    void *stream;
+} kda_recurrent_bwd_args;
+
+kda_status_t kda_recurrent_bwd_workspace_size(const kda_recurrent_bwd_args *args, size_t *bytes);
+
+kda_status_t kda_recurrent_bwd(const kda_recurrent_bwd_args *args);
+
+/*
  * kda_decode_step — one token of the Eq. 1 recurrence for B independent
  * sequences, fused in one pass over the fp32 state (the fused recurrent
  * form: decay the state, predict k^T S, form the residual beta (v - pred),

@@ -5,7 +5,7 @@ The compute lives in ``libkda.so`` (hand-written CUDA behind the C ABI of
 """
 from ._lib import KDAError, load as load_library  # noqa: F401
 from .api import (chunk_fwd, chunk_workspace_bytes, decode_step, gate, gdn_chunk_fwd, kda_decode,  # noqa: F401
-                  kda_forward, norm_gate, out_norm_gate_proj, out_proj)
+                  kda_forward, norm_gate, out_norm_gate_proj, out_proj, recurrent_bwd)
 
 __all__ = ["chunk_fwd", "chunk_workspace_bytes", "decode_step", "gate", "gdn_chunk_fwd", "kda_decode",
-           "kda_forward", "norm_gate", "out_norm_gate_proj", "out_proj", "KDAError", "load_library"]
+           "kda_forward", "norm_gate", "out_norm_gate_proj", "out_proj", "recurrent_bwd", "KDAError", "load_library"]

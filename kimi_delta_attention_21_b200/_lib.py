@@ -36,6 +36,20 @@ class ChunkArgs(ctypes.Structure):
     ]
 
 
+class RecBwdArgs(ctypes.Structure):
+    _fields_ = [
+        ("B", _i64), ("S", _i64),
+        ("H", _i32), ("D_k", _i32), ("D_v", _i32),
+        ("dtype", ctypes.c_int),
+        ("q", _p), ("k", _p), ("v", _p), ("z", _p), ("log_decay", _p),
+        ("g_min", _f32),
+        ("beta", _p), ("initial_state", _p), ("d_o", _p), ("d_final_state", _p),
+        ("dq", _p), ("dk", _p), ("dv", _p), ("dbeta", _p), ("dz", _p), ("d_initial_state", _p),
+        ("workspace", _p), ("workspace_bytes", ctypes.c_size_t),
+        ("stream", _p),
+    ]
+
+
 class DecodeArgs(ctypes.Structure):
     _fields_ = [
         ("B", _i64),
@@ -63,6 +77,8 @@ SIGNATURES = {
     "kda_gdn_chunk_workspace_size": (ctypes.c_int, [ctypes.POINTER(ChunkArgs), ctypes.POINTER(ctypes.c_size_t)]),
     "kda_gdn_chunk_fwd": (ctypes.c_int, [ctypes.POINTER(ChunkArgs)]),
     "kda_decode_step": (ctypes.c_int, [ctypes.POINTER(DecodeArgs)]),
+    "kda_recurrent_bwd_workspace_size": (ctypes.c_int, [ctypes.POINTER(RecBwdArgs), ctypes.POINTER(ctypes.c_size_t)]),
+    "kda_recurrent_bwd": (ctypes.c_int, [ctypes.POINTER(RecBwdArgs)]),
     "kda_norm_gate": (ctypes.c_int, [_p, _p, _i64, _i32, _i32, _f32, _p, ctypes.c_int, _p]),
     "kda_out_proj": (ctypes.c_int, [_p, _p, _i64, _i32, _i32, _p, ctypes.c_int, _p]),
     "kda_out_norm_gate_proj_workspace_size": (ctypes.c_int, [_i64, _i32, _i32, ctypes.c_int,

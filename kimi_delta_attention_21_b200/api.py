@@ -13,7 +13,7 @@ import ctypes
 import torch
 
 from . import _lib
-from ._lib import ChunkArgs, DecodeArgs, check
+from ._lib import ChunkArgs, DecodeArgs, RecBwdArgs, check
 
 _DT = {torch.float32: _lib.KDA_F32, torch.bfloat16: _lib.KDA_BF16}
 ENGINES = {"auto": _lib.ENGINE_AUTO, "simt": _lib.ENGINE_SIMT, "tc": _lib.ENGINE_TC}
@@ -126,6 +126,53 @@ def gdn_chunk_fwd(q, k, v, beta, **kw):
     """Gated DeltaNet prefill (one scalar decay per token and head): chunk_fwd with
     z / log_decay of shape (B,S,H).  Returns (o, final_state)."""
     return chunk_fwd(q, k, v, beta, scalar_decay=True, **kw)
+
+
+def recurrent_bwd(q, k, v, beta, d_o, *, z=None, log_decay=None, g_min=-5.0, initial_state=None,
+                  d_final_state=None, want_d_initial_state=True, workspace=None):
+    """Gradient of the prefill recurrence (kda_recurrent_bwd): given d_o = dL/do~
+    (B,S,H,D_v) and d_final_state = dL/dS_T (B,H,D_k,D_v) or None, returns a dict
+    of fp32 tensors dq, dk, dv, dbeta, dz (d/dz, or d/dlog_decay when log_decay is
+    given) and d_initial_state (or None)."""
+    _dev(q, "q")
+    dt = q.dtype
+    B, S, H, Dk = q.shape
+    Dv = v.shape[-1]
+    _dev(k, "k", dt, q.shape)
+    _dev(v, "v", dt, (B, S, H, Dv))
+    if beta.dim() == 4 and beta.shape[-1] == 1:
+        beta = beta.view(B, S, H)
+    _dev(beta, "beta", dt, (B, S, H))
+    _dev(d_o, "d_o", dt, (B, S, H, Dv))
+    _dev(z, "z", dt, q.shape)
+    _dev(log_decay, "log_decay", torch.float32, q.shape)
+    _dev(initial_state, "initial_state", torch.float32, (B, H, Dk, Dv))
+    _dev(d_final_state, "d_final_state", torch.float32, (B, H, Dk, Dv))
+    f32 = dict(dtype=torch.float32, device=q.device)
+    out = {"dq": torch.empty((B, S, H, Dk), **f32), "dk": torch.empty((B, S, H, Dk), **f32),
+           "dv": torch.empty((B, S, H, Dv), **f32), "dbeta": torch.empty((B, S, H), **f32),
+           "dz": torch.empty((B, S, H, Dk), **f32),
+           "d_initial_state": torch.empty((B, H, Dk, Dv), **f32) if want_d_initial_state else None}
+    a = RecBwdArgs(B=B, S=S, H=H, D_k=Dk, D_v=Dv, dtype=_dtype_code(q), q=_ptr(q), k=_ptr(k), v=_ptr(v),
+                   z=_ptr(z), log_decay=_ptr(log_decay), g_min=float(g_min), beta=_ptr(beta),
+                   initial_state=_ptr(initial_state), d_o=_ptr(d_o), d_final_state=_ptr(d_final_state),
+                   dq=_ptr(out["dq"]), dk=_ptr(out["dk"]), dv=_ptr(out["dv"]), dbeta=_ptr(out["dbeta"]),
+                   dz=_ptr(out["dz"]), d_initial_state=_ptr(out["d_initial_state"]), workspace=None,
+                   workspace_bytes=0, stream=_stream(q.device))
+    lib = _lib.load()
+    n = ctypes.c_size_t(0)
+    check("kda_recurrent_bwd_workspace_size", lib.kda_recurrent_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)))
+    ws = workspace
+    if n.value:
+        if ws is None:
+            ws = torch.empty(n.value, dtype=torch.uint8, device=q.device)
+        _dev(ws, "workspace", torch.uint8)
+        a.workspace = _ptr(ws)
+        a.workspace_bytes = ws.numel()
+    check("kda_recurrent_bwd", lib.kda_recurrent_bwd(ctypes.byref(a)))
+    if log_decay is not None:
+        out["dlog_decay"] = out.pop("dz")
+    return out
 
 
 def decode_step(q, k, v, beta, state, *, z=None, log_decay=None, g_min=-5.0, gate_logits=None, eps=1e-6,

@@ -250,6 +250,77 @@ kda_status_t kda_gdn_chunk_fwd(const kda_chunk_args *a) {
     return chunk_fwd_impl(a, true);
 }
 
+static kda_status_t rec_bwd_validate(const kda_recurrent_bwd_args *a) {
+    if (!a) return fail(KDA_ERR_INVALID_ARG, "args is NULL");
+    KDA_TRY(check_dtype(a->dtype));
+    KDA_TRY(check_gmin(a->g_min));
+    if (a->B < 0 || a->S < 0 || a->H < 1 || a->D_k < 1 || a->D_v < 1)
+        return fail(KDA_ERR_INVALID_ARG, "bad sizes B=%lld S=%lld H=%d D_k=%d D_v=%d", (long long)a->B,
+                    (long long)a->S, a->H, a->D_k, a->D_v);
+    if (a->D_k > 128 || a->D_v > 128)
+        return fail(KDA_ERR_UNSUPPORTED, "D_k and D_v must be <= 128 (got %d, %d)", a->D_k, a->D_v);
+    if ((int64_t)a->B * a->H > 0x7fffffffLL) return fail(KDA_ERR_UNSUPPORTED, "B*H too large");
+    return KDA_OK;
+}
+
+kda_status_t kda_recurrent_bwd_workspace_size(const kda_recurrent_bwd_args *a, size_t *bytes) {
+    g_err[0] = 0;
+    if (!bytes) return fail(KDA_ERR_INVALID_ARG, "bytes is NULL");
+    KDA_TRY(rec_bwd_validate(a));
+    *bytes = rec_bwd_workspace(a->B, a->S, a->H, a->D_k, a->D_v);
+    return KDA_OK;
+}
+
+kda_status_t kda_recurrent_bwd(const kda_recurrent_bwd_args *a) {
+    g_err[0] = 0;
+    KDA_TRY(rec_bwd_validate(a));
+    if (a->B == 0) return KDA_OK;
+    const size_t es = esize(a->dtype);
+    const size_t nk = (size_t)a->B * a->S * a->H * a->D_k, nv = (size_t)a->B * a->S * a->H * a->D_v;
+    const size_t nb = (size_t)a->B * a->S * a->H, ns = (size_t)a->B * a->H * a->D_k * a->D_v * 4;
+    if (a->S > 0) {
+        KDA_REQ_PTR(a->q, "q", es);
+        KDA_REQ_PTR(a->k, "k", es);
+        KDA_REQ_PTR(a->v, "v", es);
+        KDA_REQ_PTR(a->beta, "beta", es);
+        KDA_REQ_PTR(a->d_o, "d_o", es);
+        if (!a->log_decay) KDA_REQ_PTR(a->z, "z (or log_decay)", es);
+        KDA_OPT_PTR(a->log_decay, "log_decay", 4);
+        KDA_REQ_PTR(a->dq, "dq", 4);
+        KDA_REQ_PTR(a->dk, "dk", 4);
+        KDA_REQ_PTR(a->dv, "dv", 4);
+        KDA_REQ_PTR(a->dbeta, "dbeta", 4);
+        KDA_REQ_PTR(a->dz, "dz", 4);
+    }
+    KDA_OPT_PTR(a->initial_state, "initial_state", 4);
+    KDA_OPT_PTR(a->d_final_state, "d_final_state", 4);
+    KDA_OPT_PTR(a->d_initial_state, "d_initial_state", 4);
+    KDA_OPT_PTR(a->workspace, "workspace", 256);
+    const size_t need = rec_bwd_workspace(a->B, a->S, a->H, a->D_k, a->D_v);
+    if (a->S > 0 && need > 0 && (!a->workspace || a->workspace_bytes < need))
+        return fail(KDA_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", need,
+                    a->workspace ? a->workspace_bytes : (size_t)0);
+    const Buf ins[] = {
+        {a->S ? a->q : nullptr, nk * es, "q"}, {a->S ? a->k : nullptr, nk * es, "k"},
+        {a->S ? a->v : nullptr, nv * es, "v"}, {a->S && !a->log_decay ? a->z : nullptr, nk * es, "z"},
+        {a->S ? a->log_decay : nullptr, nk * 4, "log_decay"}, {a->S ? a->beta : nullptr, nb * es, "beta"},
+        {a->S ? a->d_o : nullptr, nv * es, "d_o"}, {a->initial_state, ns, "initial_state"},
+        {a->d_final_state, ns, "d_final_state"}, {a->S && need ? a->workspace : nullptr, need, "workspace"},
+    };
+    const int nin = (int)(sizeof(ins) / sizeof(ins[0]));
+    const Buf outs[] = {{a->S ? a->dq : nullptr, nk * 4, "dq"}, {a->S ? a->dk : nullptr, nk * 4, "dk"},
+                        {a->S ? a->dv : nullptr, nv * 4, "dv"}, {a->S ? a->dbeta : nullptr, nb * 4, "dbeta"},
+                        {a->S ? a->dz : nullptr, nk * 4, "dz"}, {a->d_initial_state, ns, "d_initial_state"}};
+    for (const Buf &o : outs) {
+        if (!o.p) continue;
+        KDA_TRY(check_no_overlap(o, ins, nin));
+        for (const Buf &o2 : outs)
+            if (&o2 != &o && o2.p && overlap(o.p, o.n, o2.p, o2.n))
+                return fail(KDA_ERR_INVALID_ARG, "outputs %s and %s overlap", o.name, o2.name);
+    }
+    return launch_rec_bwd(*a, (cudaStream_t)a->stream);
+}
+
 kda_status_t kda_decode_step(const kda_decode_args *a) {
     g_err[0] = 0;
     if (!a) return fail(KDA_ERR_INVALID_ARG, "args is NULL");

@@ -69,6 +69,10 @@ bool gdn_tc_supported(const kda_chunk_args &a, int chunk);
 bool gdn_tc_aligned(const kda_chunk_args &a);
 kda_status_t launch_gdn_tc(const kda_chunk_args &a, cudaStream_t st);
 
+// Recurrent backward (exact fp32): checkpoints every 64 tokens, per-block stash.
+size_t rec_bwd_workspace(int64_t B, int64_t S, int H, int Dk, int Dv);
+kda_status_t launch_rec_bwd(const kda_recurrent_bwd_args &a, cudaStream_t st);
+
 kda_status_t launch_norm_gate(const void *o, const void *gl, int64_t N, int H, int Dv, float eps,
                               void *x, kda_dtype_t dt, cudaStream_t st);
 

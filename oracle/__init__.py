@@ -33,18 +33,20 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "kda_oracle.c")
+_SRC_BWD = os.path.join(_HERE, "kda_oracle_bwd.c")
 _LIB = os.path.join(_HERE, "libkda_oracle.so")
 _lock = threading.Lock()
 _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile ``kda_oracle.c`` with gcc (IEEE fp64, no fast-math)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    """Compile ``kda_oracle.c`` and ``kda_oracle_bwd.c`` with gcc (IEEE fp64, no fast-math)."""
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_SRC_BWD))
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
         tmp = _LIB + f".tmp{os.getpid()}"
         subprocess.check_call(
             ["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fPIC", "-shared",
-             "-std=c11", "-o", tmp, _SRC, "-lpthread", "-lm"])
+             "-std=c11", "-o", tmp, _SRC, _SRC_BWD, "-lpthread", "-lm"])
         os.replace(tmp, _LIB)
     return _LIB
 
@@ -60,6 +62,10 @@ def _load():
             f.argtypes = [i64, i64, i64, i64, i64, p, p, p, p, p, p,
                           ctypes.c_double, p, p, i64, p, p, ctypes.c_int]
             f.restype = ctypes.c_int
+            g = lib.kda_oracle_recurrence_bwd
+            g.argtypes = [i64, i64, i64, i64, i64, p, p, p, p, p, p, ctypes.c_double, p, p, p,
+                          p, p, p, p, p, p, ctypes.c_int]
+            g.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -125,6 +131,36 @@ def recurrence(q, k, v, beta, *, z=None, log_decay=None, g_min=-5.0,
     return o, sf
 
 
+def recurrence_bwd(q, k, v, beta, d_o, *, z=None, log_decay=None, g_min=-5.0, initial_state=None,
+                   d_final_state=None, threads=None):
+    """Gradient of the Eq. 1 recurrence (outputs o~_t read after the update, and
+    the final state) by reverse-mode differentiation of the token loop, fp64
+    (the steps are listed in kda_oracle_bwd.c).  Given d_o = dL/do~ (B,S,H,Dv)
+    and d_final_state = dL/dS_T (B,H,Dk,Dv) or None, returns a dict of fp64
+    arrays: dq, dk (B,S,H,Dk), dv (B,S,H,Dv), dbeta (B,S,H), dz (d/dz, when z is
+    given) or dlog_decay (when log_decay is given) (B,S,H,Dk), and
+    d_initial_state (B,H,Dk,Dv)."""
+    q, k, v, d_o = _f32(q), _f32(k), _f32(v), _f32(d_o)
+    B, S, H, Dk = q.shape
+    Dv = v.shape[-1]
+    beta = _f32(beta).reshape(B, S, H)
+    z, log_decay = _f32(z), _f32(log_decay)
+    if z is None and log_decay is None:
+        raise ValueError("need z or log_decay")
+    s0, dst = _f32(initial_state), _f32(d_final_state)
+    out = {n: np.zeros(shp, np.float64) for n, shp in
+           (("dq", (B, S, H, Dk)), ("dk", (B, S, H, Dk)), ("dv", (B, S, H, Dv)), ("dbeta", (B, S, H)),
+            ("dg", (B, S, H, Dk)), ("d_initial_state", (B, H, Dk, Dv)))}
+    rc = _load().kda_oracle_recurrence_bwd(
+        B, S, H, Dk, Dv, _ptr(q), _ptr(k), _ptr(v), _ptr(z), _ptr(log_decay), _ptr(beta), float(g_min),
+        _ptr(s0), _ptr(d_o), _ptr(dst), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dbeta"]),
+        _ptr(out["dg"]), _ptr(out["d_initial_state"]), int(threads or default_threads()))
+    if rc != 0:
+        raise RuntimeError(f"oracle backward failed ({rc})")
+    out["dz" if z is not None else "dlog_decay"] = out.pop("dg")
+    return out
+
+
 def gdn_recurrence(q, k, v, beta, *, z=None, log_decay=None, g_min=-5.0, initial_state=None, t_rec=None,
                    want_outputs=True, threads=None):
     """Gated DeltaNet: the DPLR post's GDN form with one scalar decay per token
@@ -178,5 +214,5 @@ def forward(query, key, value, decay_logits, write_strength, output_gate_logits,
     return {"outputs": y, "final_state": sf, "o_core": o}
 
 
-__all__ = ["build", "recurrence", "gdn_recurrence", "log_decay", "norm_gate", "project", "forward",
+__all__ = ["build", "recurrence", "recurrence_bwd", "gdn_recurrence", "log_decay", "norm_gate", "project", "forward",
            "default_threads"]

@@ -9,7 +9,7 @@ import subprocess
 import pytest
 
 from kimi_delta_attention_21_b200 import _lib
-from kimi_delta_attention_21_b200._lib import ChunkArgs, DecodeArgs
+from kimi_delta_attention_21_b200._lib import ChunkArgs, DecodeArgs, RecBwdArgs
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "kda.h")
@@ -34,28 +34,28 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_struct_layout_matches_header(tmp_path):
+    structs = {"c": ("kda_chunk_args", ChunkArgs), "d": ("kda_decode_args", DecodeArgs),
+               "r": ("kda_recurrent_bwd_args", RecBwdArgs)}
     prog = tmp_path / "layout.c"
-    fields_c = [f for f, _ in ChunkArgs._fields_]
-    fields_d = [f for f, _ in DecodeArgs._fields_]
-    lines = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{HEADER}"', "int main(void){",
-             'printf("%zu %zu\\n", sizeof(kda_chunk_args), sizeof(kda_decode_args));']
-    for f in fields_c:
-        lines.append(f'printf("c {f} %zu\\n", offsetof(kda_chunk_args, {f}));')
-    for f in fields_d:
-        lines.append(f'printf("d {f} %zu\\n", offsetof(kda_decode_args, {f}));')
+    lines = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{HEADER}"', "int main(void){"]
+    for tag, (cname, S) in structs.items():
+        lines.append(f'printf("{tag} sizeof %zu\\n", sizeof({cname}));')
+        for f, _ in S._fields_:
+            lines.append(f'printf("{tag} {f} %zu\\n", offsetof({cname}, {f}));')
     lines.append("return 0;}")
     prog.write_text("\n".join(lines))
     exe = tmp_path / "layout"
     subprocess.check_call(["gcc", "-std=c11", "-o", str(exe), str(prog)])
     out = subprocess.check_output([str(exe)], text=True).split("\n")
-    sc, sd = map(int, out[0].split())
-    assert sc == ctypes.sizeof(ChunkArgs) and sd == ctypes.sizeof(DecodeArgs)
-    for line in out[1:]:
+    for line in out:
         if not line:
             continue
-        kind, f, off = line.split()
-        S = ChunkArgs if kind == "c" else DecodeArgs
-        assert getattr(S, f).offset == int(off), (kind, f)
+        tag, f, off = line.split()
+        S = structs[tag][1]
+        if f == "sizeof":
+            assert ctypes.sizeof(S) == int(off), structs[tag][0]
+        else:
+            assert getattr(S, f).offset == int(off), (tag, f)
 
 
 def test_status_strings():
