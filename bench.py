@@ -469,6 +469,38 @@ def run_e2e(K, torch, w, d, steps, world, dev):
             "api": "kimi_delta_attention_21_b200.kda_forward (pinned host tensors in and out)"}
 
 
+def time_backward(K, torch, w, d, warmup, world, dev, flush, lib, steps=3):
+    """The recurrent backward (kda_recurrent_bwd) on the workload: gradients of the
+    core recurrence w.r.t. q, k, v, beta, z and the initial state from a seeded
+    dL/do~ and dL/dS_T.  Exact fp32, token by token (not the chunkwise form)."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + 99)
+    d_o = torch.randn((w.B, w.S, w.H, w.Dv), generator=g, device=dev).to(d["q"].dtype)
+    d_st = torch.randn((w.B, w.H, w.Dk, w.Dv), generator=g, device=dev)
+    ws = None  # (the binding allocates the outputs and the workspace per call)
+
+    def one():
+        return K.recurrent_bwd(d["q"], d["k"], d["v"], d["beta"], d_o, z=d["z"], g_min=w.g_min,
+                               initial_state=d["S0"], d_final_state=d_st, workspace=ws)
+
+    for _ in range(max(1, warmup // 3)):
+        one()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    n0 = lib.kda_launch_count()
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    (t,) = reduce_max([e0.elapsed_time(e1) / steps * 1e-3], world, dev)
+    return {"entry_point": "kda_recurrent_bwd (exact fp32, recurrent form with 64-token checkpoints)",
+            "ms": round(t * 1e3, 3), "tokens_per_s": round(w.B * w.S * world / t, 1),
+            "gpu_launches_per_call": int((lib.kda_launch_count() - n0) // steps)}
+
+
 def run_decode(K, torch, w, d, warmup, world, dev, peaks, lib):
     dt = d["q"].dtype
     T = w.decode_steps
@@ -559,6 +591,14 @@ def run_ours(args, rank, world, local):
         del d
         torch.cuda.empty_cache()
 
+    if "prefill_4k" in only and not args.no_backward:
+        w = rank_workload("prefill_4k", rank)
+        d = ki.device_inputs(w, dev)
+        records.setdefault("prefill_4k", {})["backward"] = time_backward(K, torch, w, d, args.warmup, world, dev,
+                                                                         flush, lib)
+        del d
+        torch.cuda.empty_cache()
+
     if DECODE in only:
         w = rank_workload(DECODE, rank)
         d = ki.device_inputs(w, dev)
@@ -644,6 +684,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward timing on prefill_4k")
     ap.add_argument("--only", choices=("all",) + ALL_WORKLOADS, default="all",
                     help="time one workload only (for profiling); the default runs all of them")
     ap.add_argument("--ranks-log", default=None, help="append one line per rank (rank world pid) to this file")

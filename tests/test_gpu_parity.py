@@ -9,7 +9,7 @@ import pytest
 
 import kda_inputs as ki
 import oracle
-from kda_testlib import (assert_bf16_outputs, assert_bf16_state, assert_f32_close, oracle_layer, small,
+from kda_testlib import (rel_fro, assert_bf16_outputs, assert_bf16_state, assert_f32_close, oracle_layer, small,
                          to_dev, to_np, upload)
 
 torch = pytest.importorskip("torch")
@@ -287,13 +287,18 @@ def test_unaligned_views_take_exact_paths(K):
 def test_head_sharded_layer_on_one_gpu(K, world):
     """Each rank's share of the head-sharded layer (its heads through the chunk engine and its W_o
     column block through the projection), run one after another on this GPU; the fp32 sum of the
-    partial outputs is the layer output (checked against the oracle) and each rank keeps its heads'
-    final states.  The ranks never wait on one another, so one GPU can run them in turn."""
+    partial outputs is the layer output and each rank keeps its heads' final states.  The ranks never
+    wait on one another, so one GPU can run them in turn.  The sum is checked against the oracle at
+    the output tolerance, and against the whole layer through the same engine at the bf16 rounding of
+    one partial per rank (the only arithmetic the split changes).  16 heads, as in the prefill
+    workloads."""
     from kimi_delta_attention_21_b200.tensor_parallel import head_range, kda_forward_tp, shard, wo_columns
-    w = small("tpg", 2, 300, 6, 128, 128, 512, "bf16", seed=77, s0_std=0.02)
+    w = small("tpg", 1, 512, 16, 128, 128, 2048, "bf16", seed=77, s0_std=0.02)
     inp = ki.make_inputs(w)
     d = upload(inp, w)
     want = oracle_layer(inp, w)
+    whole = K.kda_forward(d["q"], d["k"], d["v"], d["z"], d["beta"], d["gate"], d["W_o"], d["S0"], g_min=w.g_min,
+                          eps=w.eps, state_dtype=torch.float32)
     total = 0
     for rank in range(world):
         h0, h1 = head_range(w.H, world, rank)
@@ -305,4 +310,8 @@ def test_head_sharded_layer_on_one_gpu(K, world):
         torch.cuda.synchronize()
         total = total + to_np(y_r)
         assert_bf16_state(to_np(s_r), want["final_state"][:, h0:h1], f"rank {rank} final states")
+        assert rel_fro(to_np(s_r), to_np(whole["final_state"][:, h0:h1])) <= 1e-3   # same engine, same heads
     assert_bf16_outputs(total, want["outputs"], f"summed partial outputs ({world} ranks)")
+    ref = to_np(whole["outputs"])
+    bound = world * 2.0 ** -8 * max(1.0, float(np.max(np.abs(ref))))
+    assert float(np.max(np.abs(total - ref))) <= bound, "split changes more than the partials' rounding"
