@@ -501,6 +501,42 @@ def time_backward(K, torch, w, d, warmup, world, dev, flush, lib, steps=3):
             "gpu_launches_per_call": int((lib.kda_launch_count() - n0) // steps)}
 
 
+def time_dplr(K, torch, w, d, warmup, world, dev, rec, steps=3):
+    """The general DPLR transition (free erase directions; here random unit
+    directions drawn on the device) evaluated token by token on the workload,
+    against the KDA chunk engine's time on the same workload: what KDA's
+    binding, which makes the chunkwise form possible, is worth on this GPU."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + 7)
+    shp = (w.B, w.S, w.H, w.Dk)
+    a = torch.nn.functional.normalize(torch.randn(shp, generator=g, device=dev), dim=-1).to(d["q"].dtype)
+    b = torch.nn.functional.normalize(torch.randn(shp, generator=g, device=dev), dim=-1).to(d["q"].dtype)
+    o = torch.empty((w.B, w.S, w.H, w.Dv), dtype=d["q"].dtype, device=dev)
+    sf = torch.empty((w.B, w.H, w.Dk, w.Dv), dtype=torch.float32, device=dev)
+
+    def one():
+        K.dplr_recurrent_fwd(d["q"], d["k"], d["v"], a, b, z=d["z"], g_min=w.g_min, initial_state=d["S0"], out=o,
+                             final_state=sf)
+
+    for _ in range(max(1, warmup // 3)):
+        one()
+    torch.cuda.synchronize(dev)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    (t,) = reduce_max([e0.elapsed_time(e1) / steps * 1e-3], world, dev)
+    out = {"entry_point": "kda_dplr_recurrent_fwd (general DPLR, token by token, exact fp32)",
+           "ms": round(t * 1e3, 3), "tokens_per_s": round(w.B * w.S * world / t, 1)}
+    if rec and "kernels_ms" in rec:
+        out["dplr_over_kda_chunk_engine_time"] = round(t * 1e3 / rec["kernels_ms"]["chunk_engine"], 2)
+    return out
+
+
 def run_decode(K, torch, w, d, warmup, world, dev, peaks, lib):
     dt = d["q"].dtype
     T = w.decode_steps
@@ -596,6 +632,14 @@ def run_ours(args, rank, world, local):
         d = ki.device_inputs(w, dev)
         records.setdefault("prefill_4k", {})["backward"] = time_backward(K, torch, w, d, args.warmup, world, dev,
                                                                          flush, lib)
+        del d
+        torch.cuda.empty_cache()
+
+    if "prefill_4k" in only and not args.no_backward:
+        w = rank_workload("prefill_4k", rank)
+        d = ki.device_inputs(w, dev)
+        records.setdefault("prefill_4k", {})["dplr_comparator"] = time_dplr(K, torch, w, d, args.warmup, world, dev,
+                                                                            records.get("prefill_4k"))
         del d
         torch.cuda.empty_cache()
 

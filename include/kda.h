@@ -230,6 +230,41 @@ kda_status_t kda_recurrent_bwd_workspace_size(const kda_recurrent_bwd_args *args
 kda_status_t kda_recurrent_bwd(const kda_recurrent_bwd_args *args);
 
 /*
+ * kda_dplr_recurrent_fwd — the general diagonal-plus-low-rank recurrence of the
+ * "Diagonal-Plus-Low-Rank Matrices and Kimi Delta Attention" post (sections 1
+ * and 3), the comparator of the KDA engines:
+ *   S_t = (Diag(alpha_t) - a_t b_t^T) S_{t-1} + k_t v_t^T,   o_t = S_t^T q_t
+ * with free erase directions a_t, b_t and the readout from the updated state
+ * (KDA's).  KDA is the case a_t = beta_t k_t, b_t = k_t * alpha_t with the
+ * write key beta_t k_t; without that binding the chunkwise UT/WY form of
+ * kda_chunk_fwd does not apply, and this entry point evaluates the recurrence
+ * token by token, exact fp32.
+ *   q, k, a, b, z (B, S, H, D_k) dtype;  log_decay (B, S, H, D_k) fp32 or NULL
+ *   v (B, S, H, D_v) dtype;  initial_state (B, H, D_k, D_v) fp32 or NULL
+ *   o (B, S, H, D_v) dtype out;  final_state (B, H, D_k, D_v) fp32 out or NULL
+ * Errors: INVALID_ARG, UNSUPPORTED (D_k or D_v > 128).
+ */
+typedef struct kda_dplr_args {
+    int64_t B, S;
+    int32_t H, D_k, D_v;
+    kda_dtype_t dtype;
+    const void *q;
+    const void *k;
+    const void *v;
+    const void *a;
+    const void *b;
+    const void *z;
+    const float *log_decay;
+    float g_min;
+    const float *initial_state;
+    void *o;
+    float *final_state;
+    void *stream;
+} kda_dplr_args;
+
+kda_status_t kda_dplr_recurrent_fwd(const kda_dplr_args *args);
+
+/*
  * kda_decode_step — one token of the Eq. 1 recurrence for B independent
  * sequences, fused in one pass over the fp32 state (the fused recurrent
  * form: decay the state, predict k^T S, form the residual beta (v - pred),

@@ -50,6 +50,17 @@ class RecBwdArgs(ctypes.Structure):
     ]
 
 
+class DplrArgs(ctypes.Structure):
+    _fields_ = [
+        ("B", _i64), ("S", _i64),
+        ("H", _i32), ("D_k", _i32), ("D_v", _i32),
+        ("dtype", ctypes.c_int),
+        ("q", _p), ("k", _p), ("v", _p), ("a", _p), ("b", _p), ("z", _p), ("log_decay", _p),
+        ("g_min", _f32),
+        ("initial_state", _p), ("o", _p), ("final_state", _p), ("stream", _p),
+    ]
+
+
 class DecodeArgs(ctypes.Structure):
     _fields_ = [
         ("B", _i64),
@@ -79,6 +90,7 @@ SIGNATURES = {
     "kda_decode_step": (ctypes.c_int, [ctypes.POINTER(DecodeArgs)]),
     "kda_recurrent_bwd_workspace_size": (ctypes.c_int, [ctypes.POINTER(RecBwdArgs), ctypes.POINTER(ctypes.c_size_t)]),
     "kda_recurrent_bwd": (ctypes.c_int, [ctypes.POINTER(RecBwdArgs)]),
+    "kda_dplr_recurrent_fwd": (ctypes.c_int, [ctypes.POINTER(DplrArgs)]),
     "kda_norm_gate": (ctypes.c_int, [_p, _p, _i64, _i32, _i32, _f32, _p, ctypes.c_int, _p]),
     "kda_out_proj": (ctypes.c_int, [_p, _p, _i64, _i32, _i32, _p, ctypes.c_int, _p]),
     "kda_out_norm_gate_proj_workspace_size": (ctypes.c_int, [_i64, _i32, _i32, ctypes.c_int,

@@ -13,7 +13,7 @@ import ctypes
 import torch
 
 from . import _lib
-from ._lib import ChunkArgs, DecodeArgs, RecBwdArgs, check
+from ._lib import ChunkArgs, DecodeArgs, DplrArgs, RecBwdArgs, check
 
 _DT = {torch.float32: _lib.KDA_F32, torch.bfloat16: _lib.KDA_BF16}
 ENGINES = {"auto": _lib.ENGINE_AUTO, "simt": _lib.ENGINE_SIMT, "tc": _lib.ENGINE_TC}
@@ -173,6 +173,34 @@ def recurrent_bwd(q, k, v, beta, d_o, *, z=None, log_decay=None, g_min=-5.0, ini
     if log_decay is not None:
         out["dlog_decay"] = out.pop("dz")
     return out
+
+
+def dplr_recurrent_fwd(q, k, v, a, b, *, z=None, log_decay=None, g_min=-5.0, initial_state=None, out=None,
+                       final_state=None):
+    """General DPLR recurrence S_t = (Diag(alpha_t) - a_t b_t^T) S_{t-1} + k_t v_t^T, o_t = S_t^T q_t
+    (kda_dplr_recurrent_fwd).  q, k, a, b, z (B,S,H,D_k); v (B,S,H,D_v).  Returns (o, final_state fp32)."""
+    _dev(q, "q")
+    dt = q.dtype
+    B, S, H, Dk = q.shape
+    Dv = v.shape[-1]
+    for name, t in (("k", k), ("a", a), ("b", b)):
+        _dev(t, name, dt, q.shape)
+    _dev(v, "v", dt, (B, S, H, Dv))
+    _dev(z, "z", dt, q.shape)
+    _dev(log_decay, "log_decay", torch.float32, q.shape)
+    _dev(initial_state, "initial_state", torch.float32, (B, H, Dk, Dv))
+    if out is None:
+        out = torch.empty((B, S, H, Dv), dtype=dt, device=q.device)
+    if final_state is None:
+        final_state = torch.empty((B, H, Dk, Dv), dtype=torch.float32, device=q.device)
+    _dev(out, "out", dt, (B, S, H, Dv))
+    _dev(final_state, "final_state", torch.float32, (B, H, Dk, Dv))
+    args = DplrArgs(B=B, S=S, H=H, D_k=Dk, D_v=Dv, dtype=_dtype_code(q), q=_ptr(q), k=_ptr(k), v=_ptr(v),
+                    a=_ptr(a), b=_ptr(b), z=_ptr(z), log_decay=_ptr(log_decay), g_min=float(g_min),
+                    initial_state=_ptr(initial_state), o=_ptr(out), final_state=_ptr(final_state),
+                    stream=_stream(q.device))
+    check("kda_dplr_recurrent_fwd", _lib.load().kda_dplr_recurrent_fwd(ctypes.byref(args)))
+    return out, final_state
 
 
 def decode_step(q, k, v, beta, state, *, z=None, log_decay=None, g_min=-5.0, gate_logits=None, eps=1e-6,

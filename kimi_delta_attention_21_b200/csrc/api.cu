@@ -321,6 +321,55 @@ kda_status_t kda_recurrent_bwd(const kda_recurrent_bwd_args *a) {
     return launch_rec_bwd(*a, (cudaStream_t)a->stream);
 }
 
+kda_status_t kda_dplr_recurrent_fwd(const kda_dplr_args *a) {
+    g_err[0] = 0;
+    if (!a) return fail(KDA_ERR_INVALID_ARG, "args is NULL");
+    KDA_TRY(check_dtype(a->dtype));
+    KDA_TRY(check_gmin(a->g_min));
+    if (a->B < 0 || a->S < 0 || a->H < 1 || a->D_k < 1 || a->D_v < 1)
+        return fail(KDA_ERR_INVALID_ARG, "bad sizes");
+    if (a->D_k > 128 || a->D_v > 128) return fail(KDA_ERR_UNSUPPORTED, "D_k and D_v must be <= 128");
+    if ((int64_t)a->B * a->H > 0x7fffffffLL) return fail(KDA_ERR_UNSUPPORTED, "B*H too large");
+    if (a->B == 0) return KDA_OK;
+    const size_t es = esize(a->dtype);
+    const size_t nk = (size_t)a->B * a->S * a->H * a->D_k, nv = (size_t)a->B * a->S * a->H * a->D_v;
+    const size_t ns = (size_t)a->B * a->H * a->D_k * a->D_v * 4;
+    if (a->S > 0) {
+        KDA_REQ_PTR(a->q, "q", es);
+        KDA_REQ_PTR(a->k, "k", es);
+        KDA_REQ_PTR(a->v, "v", es);
+        KDA_REQ_PTR(a->a, "a", es);
+        KDA_REQ_PTR(a->b, "b", es);
+        KDA_REQ_PTR(a->o, "o", es);
+        if (!a->log_decay) KDA_REQ_PTR(a->z, "z (or log_decay)", es);
+        KDA_OPT_PTR(a->log_decay, "log_decay", 4);
+    }
+    KDA_OPT_PTR(a->initial_state, "initial_state", 4);
+    KDA_OPT_PTR(a->final_state, "final_state", 4);
+    const Buf ins[] = {
+        {a->S ? a->q : nullptr, nk * es, "q"}, {a->S ? a->k : nullptr, nk * es, "k"},
+        {a->S ? a->v : nullptr, nv * es, "v"}, {a->S ? a->a : nullptr, nk * es, "a"},
+        {a->S ? a->b : nullptr, nk * es, "b"}, {a->S && !a->log_decay ? a->z : nullptr, nk * es, "z"},
+        {a->S ? a->log_decay : nullptr, nk * 4, "log_decay"}, {a->initial_state, ns, "initial_state"},
+    };
+    const int nin = (int)(sizeof(ins) / sizeof(ins[0]));
+    if (a->S > 0) KDA_TRY(check_no_overlap(Buf{a->o, nv * es, "o"}, ins, nin));
+    if (a->final_state) {
+        KDA_TRY(check_no_overlap(Buf{a->final_state, ns, "final_state"}, ins, nin));
+        if (a->S > 0 && overlap(a->final_state, ns, a->o, nv * es)) return fail(KDA_ERR_INVALID_ARG, "final_state overlaps o");
+    }
+    if (a->S == 0) {
+        if (a->final_state) {
+            cudaError_t e = a->initial_state ? cudaMemcpyAsync(a->final_state, a->initial_state, ns,
+                                                               cudaMemcpyDeviceToDevice, (cudaStream_t)a->stream)
+                                             : cudaMemsetAsync(a->final_state, 0, ns, (cudaStream_t)a->stream);
+            if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "empty sequence: %s", cudaGetErrorString(e));
+        }
+        return KDA_OK;
+    }
+    return launch_dplr(*a, (cudaStream_t)a->stream);
+}
+
 kda_status_t kda_decode_step(const kda_decode_args *a) {
     g_err[0] = 0;
     if (!a) return fail(KDA_ERR_INVALID_ARG, "args is NULL");

@@ -21,14 +21,15 @@
 // recomputes the chunk's states from its checkpoint into a per-CTA stash, and
 // applies the reverse steps token by token.  The sums over key rows (p, dr)
 // are warp shuffles plus one shared-memory pass.
-#include "kda_internal.cuh"
+#include "rec_common.cuh"
 
 namespace kda {
 
 namespace {
 
-constexpr int RB_THREADS = 256;  // thread t: key row c = t >> 1, columns 8 (t & 1) .. 8 (t & 1) + 7 of the slice
-constexpr int RB_VS = 16;        // value columns per CTA
+using rec::rowsum16;
+constexpr int RB_THREADS = rec::THREADS;
+constexpr int RB_VS = rec::VS;
 constexpr int RB_C = 64;         // tokens per checkpoint interval
 
 struct RbArgs {
@@ -42,28 +43,6 @@ struct RbArgs {
     float *ckpt;   // [B*H][nslice][Nc][Dk][16]
     float *stash;  // [B*H][nslice][64][Dk][16]
 };
-
-// Sum over the key rows (threads) of x[8] for this thread's 8 columns; thread j < 16 gets column j's
-// total back (the return value; 0 elsewhere).  Two block barriers.
-__device__ __forceinline__ float rowsum16(const float (&x)[8], float *red, int tid) {
-    float y[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) y[e] = x[e];
-#pragma unroll
-    for (int off = 2; off < 32; off <<= 1)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) y[e] += __shfl_xor_sync(0xffffffffu, y[e], off);
-    const int lane = tid & 31, warp = tid >> 5;
-    if (lane < 2)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) red[warp * 16 + 8 * lane + e] = y[e];
-    __syncthreads();
-    float s = 0.f;
-    if (tid < 16)
-#pragma unroll
-        for (int w = 0; w < RB_THREADS / 32; ++w) s += red[w * 16 + tid];
-    return s;
-}
 
 template <typename T>
 struct Step {  // per-thread view of one token's inputs

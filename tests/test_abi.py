@@ -9,7 +9,7 @@ import subprocess
 import pytest
 
 from kimi_delta_attention_21_b200 import _lib
-from kimi_delta_attention_21_b200._lib import ChunkArgs, DecodeArgs, RecBwdArgs
+from kimi_delta_attention_21_b200._lib import ChunkArgs, DecodeArgs, DplrArgs, RecBwdArgs
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "kda.h")
@@ -35,7 +35,7 @@ def test_library_exports_every_declared_symbol():
 
 def test_struct_layout_matches_header(tmp_path):
     structs = {"c": ("kda_chunk_args", ChunkArgs), "d": ("kda_decode_args", DecodeArgs),
-               "r": ("kda_recurrent_bwd_args", RecBwdArgs)}
+               "r": ("kda_recurrent_bwd_args", RecBwdArgs), "p": ("kda_dplr_args", DplrArgs)}
     prog = tmp_path / "layout.c"
     lines = ['#include <stdio.h>', '#include <stddef.h>', f'#include "{HEADER}"', "int main(void){"]
     for tag, (cname, S) in structs.items():

@@ -379,3 +379,34 @@ def test_log_decay_gate_limits():
     np.testing.assert_allclose(g[:3], [-2.5, -5.0, 0.0], atol=1e-20)
     # sigmoid(1) = e/(1+e)
     np.testing.assert_allclose(g[3], -5.0 * np.e / (1 + np.e), rtol=1e-15)
+
+
+# ---------------------------------------------------------------- general DPLR (comparator)
+
+def test_dplr_with_kda_binding_is_kda():
+    # a = beta k, b = k * alpha and the write key beta k turn the general DPLR transition into Eq. 1
+    from oracle.dplr import dplr_recurrence
+    q, k, v, z, beta, S0 = _problem(2, 9, 2, 5, 3, 31)
+    alpha = _alpha(z, -4.0)
+    a = beta[..., None].astype(np.float64) * k.astype(np.float64)
+    b = k.astype(np.float64) * alpha
+    o, sf = dplr_recurrence(q, a, v, a, b, z=z, g_min=-4.0, initial_state=S0)
+    o2, sf2 = oracle.recurrence(q, k, v, beta, z=z, g_min=-4.0, initial_state=S0)
+    np.testing.assert_allclose(o, o2, rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(sf, sf2, rtol=1e-10, atol=1e-12)
+
+
+def test_dplr_without_erase_is_decayed_linear_attention():
+    # a = 0: S_T = Gamma_T S_0 + sum_i Gamma_{i->T} k_i v_i^T with Gamma the channel-wise decay products
+    from oracle.dplr import dplr_recurrence
+    q, k, v, z, beta, S0 = _problem(1, 7, 1, 4, 3, 32)
+    rng = np.random.default_rng(1)
+    b = rng.standard_normal(k.shape)
+    o, sf = dplr_recurrence(q, k, v, np.zeros_like(k), b, z=z, g_min=-2.0, initial_state=S0)
+    g = -2.0 / (1.0 + np.exp(-z[0, :, 0].astype(np.float64)))          # (S, Dk)
+    want = np.exp(g.sum(0))[:, None] * S0[0, 0].astype(np.float64)
+    for i in range(7):
+        want = want + np.exp(g[i + 1:].sum(0))[:, None] * np.outer(k[0, i, 0].astype(np.float64),
+                                                                   v[0, i, 0].astype(np.float64))
+    np.testing.assert_allclose(sf[0, 0], want, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(o[0, -1, 0], want.T @ q[0, -1, 0].astype(np.float64), rtol=1e-12, atol=1e-13)
