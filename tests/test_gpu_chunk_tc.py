@@ -76,19 +76,34 @@ def _close(got, want, what, tol=2e-2):
     assert err <= tol * scale, f"{what}: max-abs {err:.3e} (scale {scale:.3e})"
 
 
-def test_workspace_intermediates_match_chunk_mirror(K):
-    w = small("wsi", 1, 100, 2, 128, 128, 16, "bf16", seed=41)
+def _rel(got, want, what, tol):
+    """Max-abs error relative to the tensor's own largest entry (the images are bf16: 2^-9 rounding)."""
+    scale = max(float(np.max(np.abs(want))), 1e-30)
+    err = float(np.max(np.abs(got - want)))
+    assert err <= tol * scale, f"{what}: max-abs {err:.3e} against largest |entry| {scale:.3e}"
+
+
+@pytest.mark.parametrize("s0_std", [0.0, 0.05])
+def test_workspace_intermediates_match_chunk_mirror(K, s0_std):
+    """The records the prep writes (W, Q e^G, K e^{G_C - G}, M, U, e^{G_C}) against the fp64 mirror of
+    the chunk algebra, each to a few bf16 roundings of its own scale; then, from a nonzero initial
+    state, the state-corrected values V' = U - W S_0 formed from the record and the known S_0, and the
+    outputs and final state of the whole two-chunk sequence, against the mirror chained chunk by chunk."""
+    w = small("wsi", 1, 100, 2, 128, 128, 16, "bf16", seed=41, s0_std=s0_std)
     inp = ki.make_inputs(w)
     d = upload(inp, w)
     nb = K.chunk_workspace_bytes(1, 100, 2, 128, 128)
     assert nb == 1 * 2 * 2 * (REC + SIG)
     ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
-    K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=d["z"], engine="tc", workspace=ws)
+    o, sf = K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=d["z"], initial_state=d["S0"], engine="tc",
+                        workspace=ws)
     torch.cuda.synchronize()
     assert _timeouts(K) == 0
     wsh = ws.cpu().numpy()
     la = oracle.log_decay(inp["z"], w.g_min)
+    o_np, sf_np = to_np(o), to_np(sf)
     for h in range(2):
+        S = np.zeros((128, 128)) if inp["S0"] is None else inp["S0"][0, h].astype(np.float64)
         for n in range(2):
             t0, t1 = 64 * n, min(100, 64 * n + 64)
             L = t1 - t0
@@ -96,17 +111,25 @@ def test_workspace_intermediates_match_chunk_mirror(K):
             q = pad(inp["q"][0, t0:t1, h].astype(np.float64)); k = pad(inp["k"][0, t0:t1, h].astype(np.float64))
             v = pad(inp["v"][0, t0:t1, h].astype(np.float64)); beta = pad(inp["beta"][0, t0:t1, h].astype(np.float64))
             g = pad(la[0, t0:t1, h])
-            mir = chunk_mirror.matrix_chunk(q, k, v, beta, g, np.zeros((128, 128)))
+            mir = chunk_mirror.matrix_chunk(q, k, v, beta, g, S)
             G = mir["G"]
             rec = wsh[(h * 2 + n) * REC:(h * 2 + n + 1) * REC]
             wq = _kmajor_image(rec[0:32768], rows=128)  # stacked [-W; Q e^G]
-            _close(wq[64:], q * np.exp(G), f"Qg h{h} n{n}")
-            _close(-wq[:64], mir["W"], f"W h{h} n{n}")
-            _close(_kmajor_image(rec[32768:49152]), k * np.exp(G[-1] - G), f"Kt h{h} n{n}")
-            _close(_mt_image(rec[49152:57344]), mir["M"].T, f"M h{h} n{n}")
-            _close(_atom_image(rec[57344:73728], 128).T, mir["U"], f"U h{h} n{n}")  # stored as U^T
+            W_rec, U_rec = -wq[:64], _atom_image(rec[57344:73728], 128).T  # U stored as U^T
+            tag = f"h{h} n{n} S0 std {s0_std}"
+            _rel(wq[64:], q * np.exp(G), f"Q e^G {tag}", 8e-3)
+            _rel(W_rec, mir["W"], f"W {tag}", 8e-3)
+            _rel(_kmajor_image(rec[32768:49152]), k * np.exp(G[-1] - G), f"K~ {tag}", 8e-3)
+            _rel(_mt_image(rec[49152:57344]), mir["M"].T, f"M {tag}", 8e-3)
+            _rel(U_rec, mir["U"], f"U {tag}", 8e-3)
             gam = np.frombuffer(rec[73728:74240].tobytes(), dtype=np.float32)
             np.testing.assert_allclose(gam, np.exp(G[-1]), rtol=1e-4, atol=1e-30)
+            # V' from the record and the exact entering state, against the mirror's
+            _rel(U_rec - W_rec @ S, mir["Vp"], f"V' {tag}", 1.6e-2)
+            # the engine's outputs of this chunk against the mirror's O (o~ of the chunk's tokens)
+            _rel(o_np[0, t0:t1, h], mir["O"][:L], f"O {tag}", 1.6e-2)
+            S = mir["S_next"]
+        _rel(sf_np[0, h], S, f"final state h{h} S0 std {s0_std}", 1e-2)
 
 
 @pytest.mark.parametrize("B,S,H", [(1, 1, 1), (1, 64, 1), (1, 65, 2), (2, 130, 3), (1, 200, 2), (3, 257, 27),
