@@ -18,14 +18,17 @@
 //    batch) units; all chunks are independent): TMA loads of q, k, v; the
 //    cumulative log-decay (from z or the log-decay input, read directly);
 //    decay-scaled operands; A^T and M^T on tcgen05; the inverse T in fp32 SIMT;
-//    [W | U^T] = T [beta K e^G | beta V] on tcgen05; the sigmoid of the output
-//    gate.  It writes one workspace record per chunk holding [-W; Q*e^G],
-//    K*e^{G_C-G}, M^T and U^T as ready-made 128-byte-swizzled shared-memory
-//    images, and e^{G_C}.
-//  * chunk_state_kernel, one CTA per (head, batch, segment of the sequence),
-//    walks the chunks in order with the state resident in TMEM, streaming the
-//    records with bulk copies, and writes the gated, normalised output and
-//    the final state; chunk_combine_kernel chains the segments (below).
+//    [W | U^T] = T [beta K e^G | beta V] on tcgen05.  It writes one workspace
+//    record per chunk holding [-W; Q*e^G], K*e^{G_C-G}, M^T and U^T as
+//    ready-made 128-byte-swizzled shared-memory images, and e^{G_C}.
+//  * the state pass.  A long sequence is cut into G segments:
+//    chunk_map_pair_kernel gives every segment but the last its affine map
+//    S_end = A_g S_start + Y_g (both chains in one CTA), chunk_combine_kernel
+//    chains the maps into each segment's entering state, and
+//    chunk_state_kernel, one CTA per (head, batch, segment), walks the
+//    segment's chunks in order with the state resident in TMEM, streaming the
+//    records with bulk copies, and writes the gated, normalised output and the
+//    final state.
 //
 // Decay factors as GEMM operands.  exp(G_r - G_i) is split into a row factor
 // and a column factor around a reference point.  G spans up to |g_min| * 64
@@ -647,7 +650,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
 //   warps 0-7   the chain's register work (lane quarter = warp % 4, column
 //               half = warp / 4);
 //   warp 8      issues the chain's MMAs and the record copies (one thread);
-//   warps 9-12  the output stage (chains only; the maps have no output); its
+//   warps 9-12  the output stage; its
 //               first thread issues the output's transposition MMA itself, so
 //               the output never waits on the chain's MMA issue order.
 // Per chunk n:
@@ -662,7 +665,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
 // sigmoid of the output-gate logits (a bf16 tile loaded by TMA one chunk
 // ahead) and store the tile with a TMA tensor store.  PO is double-buffered;
 // a buffer is reused for chunk n + 2 once the output warps have read chunk n.
-// Records stream in by bulk copies, two stages deep (three for the maps).
+// Records stream in by bulk copies, two stages deep.
 struct StateArgs {
     int S, H, Nc;
     int L, G;              // chunks per segment, segments per sequence
@@ -682,7 +685,7 @@ constexpr int ST_THREADS_MAP = 288;            // warps 0-7 chain register work,
 constexpr int ST_THREADS_CHAIN = 416;          // ... and warps 9-12 the output stage
 constexpr int ST_OUT_WARP0 = 9;
 constexpr uint32_t ST_STAGE = REC_GAM;         // the image part of a record (73728 B)
-constexpr uint32_t ST_GAM = 2 * ST_STAGE;      // e^{G_C} [2 stages][128] fp32 (the maps: 3 stages, into OIMG)
+constexpr uint32_t ST_GAM = 2 * ST_STAGE;      // e^{G_C} [2 stages][128] fp32 (the map pass: 3, into OIMG)
 constexpr uint32_t ST_OIMG = ST_GAM + 1024;    // output tile [2 atoms (j / 64)][64 rows r][128 B]
 constexpr uint32_t ST_SIGT = ST_OIMG + 16384;  // output-gate logits tile (TMA), same layout, bf16
 constexpr uint32_t ST_OT = ST_SIGT + 16384;    // O^T image, K-major B [128 rows j][128 B: 64 r]
@@ -706,12 +709,8 @@ __device__ __forceinline__ float sigmoid_fast(float x) {
     return fmaf(0.5f, t, 0.5f);
 }
 
-// kMap = false: the chain over segment blockIdx.z from its entering state, with outputs.
-// kMap = true:  no outputs; z = 0 runs segment 0 from the initial state (its end state is S_1, the
-//               entering state of segment 1); for g >= 1 the map S_end = A_g S_start + Y_g of segment
-//               g = (z + 1) / 2: odd z from S = I without U (-> A_g), even z from S = 0 with U (-> Y_g).
-template <bool kMap>
-__global__ void __launch_bounds__(kMap ? ST_THREADS_MAP : ST_THREADS_CHAIN, 1)
+// The chain over segment blockIdx.z from its entering state, with outputs.
+__global__ void __launch_bounds__(ST_THREADS_CHAIN, 1)
 chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constant__ CUtensorMap tgl, StateArgs p) {
     pdl_trigger();
     pdl_wait();
@@ -721,17 +720,15 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
     const int q4 = warp & 3, hf = (warp >> 2) & 1;  // TMEM lane quarter, column half (warps 0-7)
     const int h = blockIdx.x, b = blockIdx.y;
     const int bh = b * p.H + h;
-    const int g = kMap ? (int)((blockIdx.z + 1) >> 1) : (int)blockIdx.z;
-    const bool ident = kMap && (blockIdx.z & 1) == 1;  // map from the identity (no U)
+    const int g = (int)blockIdx.z;
     const int n0 = g * p.L;
     const int nc = max(0, min(p.L, p.Nc - n0));  // chunks of this segment
-    // Record stages: the chains use whole records, two deep; the maps only -W, K~ and U^T (48 KB),
-    // three deep.  The e^{G_C} of each stage sits after the stages.
-    constexpr int STG = kMap ? 3 : 2;
-    constexpr uint32_t STB = kMap ? 49152u : ST_STAGE;
-    constexpr uint32_t O_W_ATOM = kMap ? 8192u : 16384u;  // atom stride of the [-W; Q e^G] (or -W) B operand
-    constexpr uint32_t O_KT = kMap ? 16384u : REC_KT;
-    constexpr uint32_t O_U = kMap ? 32768u : REC_U;
+    // Record stages: whole records, two deep; the e^{G_C} of each stage sits after the stages.
+    constexpr int STG = 2;
+    constexpr uint32_t STB = ST_STAGE;
+    constexpr uint32_t O_W_ATOM = 16384u;  // atom stride of the [-W; Q e^G] B operand
+    constexpr uint32_t O_KT = REC_KT;
+    constexpr uint32_t O_U = REC_U;
     static_assert(STG * STB == ST_GAM, "record stages end where e^{G_C} starts");
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ST_BAR);
     uint64_t *full = bars;           // [STG] record stage landed
@@ -798,14 +795,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
                 uint8_t *dst = sm + stg * STB;
                 const uint8_t *src = rec0 + (size_t)n * REC_BYTES;
                 mbar_arrive_expect_tx(&full[stg], STB + 512);
-                if (kMap) {  // -W rows of both atoms, K~, U^T
-                    bulk_load(dst, src + REC_WQ, 8192, &full[stg]);
-                    bulk_load(dst + 8192, src + REC_WQ + 16384, 8192, &full[stg]);
-                    bulk_load(dst + O_KT, src + REC_KT, 16384, &full[stg]);
-                    bulk_load(dst + O_U, src + REC_U, 16384, &full[stg]);
-                } else {
-                    bulk_load(dst, src, ST_STAGE, &full[stg]);
-                }
+                bulk_load(dst, src, ST_STAGE, &full[stg]);
                 bulk_load(sgam + stg * 128, src + REC_GAM, 512, &full[stg]);
                 ++issued;
             };
@@ -817,15 +807,14 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
                 const uint32_t po = tmem + T_PO + (uint32_t)(n & 1) * 128;
                 if (!mbar_wait(&full[n % STG], (n / STG) & 1)) { ok = false; break; }
                 landed = n + 1;
-                // PO = S_n^T [-W; Q e^G]^T (the maps: S_n^T (-W)^T), once the output warps have read chunk n - 2
+                // PO = S_n^T [-W; Q e^G]^T, once the output warps have read chunk n - 2
                 if (!mbar_wait(bar_simg, n & 1)) { ok = false; break; }
-                if (!kMap && n >= 2 && !mbar_wait(&pofree[n & 1], ((n - 2) >> 1) & 1)) { ok = false; break; }
+                if (n >= 2 && !mbar_wait(&pofree[n & 1], ((n - 2) >> 1) & 1)) { ok = false; break; }
                 tc_fence_after();
-                constexpr uint32_t id_po = kMap ? idesc_f16(128, 64, 0, 0) : id_kk;
 #pragma unroll
                 for (int s8 = 0; s8 < 8; ++s8) {
                     const uint32_t ko = s8 >> 2, kb = (s8 & 3) * 32;
-                    mma_f16_ts(po, tmem + T_S16 + 8 * s8, dadd(d_k, sgo + ko * O_W_ATOM + kb), id_po, s8 > 0);
+                    mma_f16_ts(po, tmem + T_S16 + 8 * s8, dadd(d_k, sgo + ko * O_W_ATOM + kb), id_kk, s8 > 0);
                 }
                 mma_commit(bar_p);
                 // the stage of record n - 1 is free once its last group is done: refill it, STG - 1 ahead
@@ -840,11 +829,9 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
                 for (int s4 = 0; s4 < 4; ++s4)
                     mma_f16_ts(tmem + T_S32, tmem + T_V16 + 8 * s4, dadd(d_mn, sgo + O_KT + s4 * 2048), id_s, 1);
                 mma_commit(bar_s);
-                if (!kMap) {
 #pragma unroll
-                    for (int s4 = 0; s4 < 4; ++s4)
-                        mma_f16_ts(po + 64, tmem + T_V16 + 8 * s4, dadd(d_mn, sgo + REC_MT + s4 * 2048), id_o, 1);
-                }
+                for (int s4 = 0; s4 < 4; ++s4)
+                    mma_f16_ts(po + 64, tmem + T_V16 + 8 * s4, dadd(d_mn, sgo + REC_MT + s4 * 2048), id_o, 1);
                 mma_commit(bar_of(n));
             }
             if (!ok) s_fail = 1;
@@ -959,16 +946,12 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
         const int j = 32 * q4 + lane;  // value column (TMEM lane) of this thread
         {   // entering state -> TMEM (S^T[j, c] = S[c, j]: a warp reads 128 contiguous bytes per c)
             const float *s_in = (g == 0) ? (p.S0 ? p.S0 + (size_t)bh * DD * DD : nullptr)
-                              : kMap     ? nullptr
                               : (g == 1) ? p.yt + (size_t)bh * (p.G - 1) * DD * DD  // S_1: segment 0's end state
                                          : p.seg_init + ((size_t)bh * p.G + g) * DD * DD;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t su[32];
-                if (ident) {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) su[e] = (64 * hf + 32 * hh + e == j) ? 0x3F800000u : 0u;
-                } else if (s_in) {
+                if (s_in) {
                     const float *src = s_in + (size_t)(64 * hf + 32 * hh) * DD + j;
 #pragma unroll
                     for (int e = 0; e < 32; ++e) su[e] = __float_as_uint(src[(size_t)e * DD]);
@@ -1035,10 +1018,8 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
                     unpack8(uu[k], u);
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
-                        pk[4 * k + e] = ident ? pack_bf16x2(__uint_as_float(pv[8 * k + 2 * e]),
-                                                            __uint_as_float(pv[8 * k + 2 * e + 1]))
-                                              : pack_bf16x2(u[2 * e] + __uint_as_float(pv[8 * k + 2 * e]),
-                                                            u[2 * e + 1] + __uint_as_float(pv[8 * k + 2 * e + 1]));
+                        pk[4 * k + e] = pack_bf16x2(u[2 * e] + __uint_as_float(pv[8 * k + 2 * e]),
+                                                    u[2 * e + 1] + __uint_as_float(pv[8 * k + 2 * e + 1]));
                 }
                 tmem_st_32x32b_x16(tmem + lrow + T_V16 + 16 * hf, pk);
                 tmem_wait_st();
@@ -1051,33 +1032,7 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
             if (!mbar_wait(bar_s, (nc - 1) & 1) || !mbar_wait(bar_of(nc - 1), par_of(nc - 1))) ok = false;
             tc_fence_after();
         }
-        if (ok && kMap && !ident) {  // Y_g (S_1 for segment 0), laid out like a state
-            float *dst0 = p.yt + ((size_t)bh * (p.G - 1) + g) * DD * DD;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                uint32_t sv[32];
-                tmem_ld_32x32b_x32(tmem + lrow + T_S32 + 64 * hf + 32 * hh, sv);
-                tmem_wait_ld();
-                float *dst = dst0 + (size_t)(64 * hf + 32 * hh) * DD + j;
-#pragma unroll
-                for (int e = 0; e < 32; ++e) dst[(size_t)e * DD] = __uint_as_float(sv[e]);
-            }
-        } else if (ok && ident) {  // A_g^T as the combine pass's MN-major B operand: image row j = lane j
-            uint8_t *img = p.xt + ((size_t)bh * (p.G - 1) + g) * 32768;
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                uint32_t sv[32];
-                tmem_ld_32x32b_x32(tmem + lrow + T_S32 + 64 * hf + 32 * hh, sv);
-                tmem_wait_ld();
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    float f[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(sv[8 * k + e]);
-                    *reinterpret_cast<uint4 *>(img + hf * 16384 + sw128(j, 4 * hh + k)) = pack8(f);
-                }
-            }
-        } else if (ok && p.Sf && g == p.G - 1) {  // (with no chunks TMEM still holds the entering state)
+        if (ok && p.Sf && g == p.G - 1) {  // (with no chunks TMEM still holds the entering state)
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t sv[32];
@@ -1096,8 +1051,266 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
         // let the bulk copies already issued land before the CTA exits
         for (int m = landed; m < issued; ++m) mbar_wait(&full[m % STG], (m / STG) & 1, 100000000ull);
     }
-    if (!kMap && tid == ST_OUT_WARP0 * 32 && s_fail && p.gated)
+    if (tid == ST_OUT_WARP0 * 32 && s_fail && p.gated)
         mbar_wait(bar_sig, 0, 100000000ull), mbar_wait(bar_sig, 1, 100000000ull);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, ST_TCOLS);
+}
+
+// ================================================================ K2b': chunk_map_pair_kernel
+// The map pass, two chains per CTA (H, B, G - 1 CTAs; blockIdx.z = segment g <= G - 2).  Chain Y runs
+// segment g with U from its entering state: the initial state for g = 0 (its end state is S_1, the
+// entering state of segment 1), zero for g >= 1 (its end state is Y_g).  Chain X runs segment g from the
+// identity without U (its end state is A_g; segment 0 needs none, and its slot stays unused).  Both read
+// one stream of records (-W, K~, U^T, e^{G_C}), three stages deep.  The chain warps alternate between
+// the two chains, so that each chain's register work fills the other's MMA round trips.  Per chain the
+// TMEM columns are S^T fp32 (+0), the bf16 copy of S^T (+128) and PO = S^T (-W)^T (+192); the bf16 V'^T
+// reuses the copy's first 32 columns (the copy is dead once PO is done, V'^T once the update is done).
+__device__ __forceinline__ constexpr uint32_t mp_base(int c) { return c ? 256u : 0u; }  // chain X, chain Y
+constexpr uint32_t MP_S16 = 128, MP_PO = 192;
+
+__global__ void __launch_bounds__(ST_THREADS_MAP, 1) chunk_map_pair_kernel(StateArgs p) {
+    pdl_trigger();
+    pdl_wait();
+    extern __shared__ uint8_t smraw[];
+    uint8_t *sm = align1024(smraw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q4 = warp & 3, hf = (warp >> 2) & 1;  // TMEM lane quarter, column half (warps 0-7)
+    const int h = blockIdx.x, b = blockIdx.y, g = (int)blockIdx.z;
+    const int bh = b * p.H + h;
+    const int n0 = g * p.L;
+    const int nc = max(0, min(p.L, p.Nc - n0));
+    constexpr int STG = 3;
+    constexpr uint32_t STB = 49152u;  // -W rows of both atoms (16 KB), K~ (16 KB), U^T (16 KB)
+    constexpr uint32_t O_KT = 16384u, O_U = 32768u;
+    static_assert(STG * STB == ST_GAM, "record stages end where e^{G_C} starts");
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + ST_BAR);
+    uint64_t *full = bars;       // [3] record stage landed
+    uint64_t *bar_p = bars + 3;  // [2] PO of chain c done
+    uint64_t *bar_s = bars + 5;  // [2] S^T += V'^T K~ of chain c done
+    uint64_t *simg = bars + 7;   // [2] bf16 copy of chain c's S^T written (8 chain warps)
+    uint64_t *vimg = bars + 9;   // [2] bf16 copy of chain c's V'^T written (8 chain warps)
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 11);
+    float *sgam = reinterpret_cast<float *>(sm + ST_GAM);
+    const uint8_t *rec0 = p.ws + ((size_t)bh * p.Nc + n0) * REC_BYTES;
+    __shared__ volatile int s_fail;
+
+    if (tid == 0) {
+        s_fail = 0;
+        for (int i = 0; i < 7; ++i) mbar_init(&bars[i], 1);
+        for (int i = 7; i < 11; ++i) mbar_init(&bars[i], 8);
+        fence_barrier_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, ST_TCOLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = true;
+    int issued = 0, landed = 0;  // records requested / seen complete (MMA warp)
+
+    if (warp == 8) {
+        // ======================================== MMA and copy issue (one thread)
+        if (lane == 0) {
+            constexpr uint32_t id_po = idesc_f16(128, 64, 0, 0);  // A (TMEM) and B K-major
+            constexpr uint32_t id_s = idesc_f16(128, 128, 0, 1);  // B MN-major
+            const uint64_t d_k = smem_desc(smem_u32(sm), 16, 1024, LAYOUT_SW128);
+            const uint64_t d_mn = smem_desc(smem_u32(sm), 8192, 1024, LAYOUT_SW128);
+            auto issue_record = [&](int n) {
+                const int stg = n % STG;
+                uint8_t *dst = sm + stg * STB;
+                const uint8_t *src = rec0 + (size_t)n * REC_BYTES;
+                mbar_arrive_expect_tx(&full[stg], STB + 512);
+                bulk_load(dst, src + REC_WQ, 8192, &full[stg]);
+                bulk_load(dst + 8192, src + REC_WQ + 16384, 8192, &full[stg]);
+                bulk_load(dst + O_KT, src + REC_KT, 16384, &full[stg]);
+                bulk_load(dst + O_U, src + REC_U, 16384, &full[stg]);
+                bulk_load(sgam + stg * 128, src + REC_GAM, 512, &full[stg]);
+                ++issued;
+            };
+            for (int n = 0; n < STG && n < nc; ++n) issue_record(n);
+            for (int n = 0; n < nc; ++n) {
+                if (s_fail) { ok = false; break; }
+                const uint32_t sgo = (n % STG) * STB;
+                if (!mbar_wait(&full[n % STG], (n / STG) & 1)) { ok = false; break; }
+                landed = n + 1;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {  // PO_c = S_c^T (-W)^T
+                    if (!mbar_wait(&simg[c], n & 1)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t base = tmem + mp_base(c);
+#pragma unroll
+                    for (int s8 = 0; s8 < 8; ++s8) {
+                        const uint32_t ko = s8 >> 2, kb = (s8 & 3) * 32;
+                        mma_f16_ts(base + MP_PO, base + MP_S16 + 8 * s8, dadd(d_k, sgo + ko * 8192 + kb), id_po, s8 > 0);
+                    }
+                    mma_commit(&bar_p[c]);
+                }
+                if (!ok) break;
+                // the stage of record n - 1 is free once chain Y's update of chunk n - 1 is done (the
+                // chain warps read its U^T and e^{G_C} before they signal that update's V')
+                if (n >= 1 && n + STG - 1 < nc) {
+                    if (!mbar_wait(&bar_s[1], (n - 1) & 1)) { ok = false; break; }
+                    issue_record(n + STG - 1);
+                }
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {  // S_c^T += V'_c^T K~
+                    if (!mbar_wait(&vimg[c], n & 1)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t base = tmem + mp_base(c);
+#pragma unroll
+                    for (int s4 = 0; s4 < 4; ++s4)
+                        mma_f16_ts(base, base + MP_S16 + 8 * s4, dadd(d_mn, sgo + O_KT + s4 * 2048), id_s, 1);
+                    mma_commit(&bar_s[c]);
+                }
+                if (!ok) break;
+            }
+            if (!ok) s_fail = 1;
+        }
+    } else {
+        // ======================================== chain register work (warps 0-7), both chains
+        const uint32_t lrow = (uint32_t)(32 * q4) << 16;
+        const int j = 32 * q4 + lane;  // value column (TMEM lane) of this thread
+        {   // entering states -> TMEM: X = identity, Y = S_0 (g = 0) or zero
+            const float *s_in = (g == 0 && p.S0) ? p.S0 + (size_t)bh * DD * DD : nullptr;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t su[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) su[e] = (64 * hf + 32 * hh + e == j) ? 0x3F800000u : 0u;
+                tmem_st_32x32b_x32(tmem + lrow + mp_base(0) + 64 * hf + 32 * hh, su);
+                if (s_in) {
+                    const float *src = s_in + (size_t)(64 * hf + 32 * hh) * DD + j;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) su[e] = __float_as_uint(src[(size_t)e * DD]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) su[e] = 0u;
+                }
+                tmem_st_32x32b_x32(tmem + lrow + mp_base(1) + 64 * hf + 32 * hh, su);
+            }
+            tmem_wait_st();
+        }
+
+        for (int n = 0; n < nc && ok; ++n) {
+            if (s_fail) { ok = false; break; }
+            const int stg = n % STG;
+            if (!mbar_wait(&full[stg], (n / STG) & 1)) { ok = false; break; }
+            const float4 *g4 = reinterpret_cast<const float4 *>(sgam + stg * 128 + 64 * hf);
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {  // S_n^T -> bf16 copy; S^T <- S^T Diag(e^{G_C})
+                const uint32_t base = tmem + lrow + mp_base(c);
+                if (n >= 1 && !mbar_wait(&bar_s[c], (n - 1) & 1)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t sv[64];
+                tmem_ld_32x32b_x32(base + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                tmem_ld_32x32b_x32(base + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+                tmem_wait_ld();
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int e = 0; e < 16; ++e)
+                        pk[e] = pack_bf16x2(__uint_as_float(sv[32 * hh + 2 * e]), __uint_as_float(sv[32 * hh + 2 * e + 1]));
+                    tmem_st_32x32b_x16(base + MP_S16 + 32 * hf + 16 * hh, pk);
+                }
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&simg[c]);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float4 gg = g4[e];
+                    sv[4 * e] = __float_as_uint(__uint_as_float(sv[4 * e]) * gg.x);
+                    sv[4 * e + 1] = __float_as_uint(__uint_as_float(sv[4 * e + 1]) * gg.y);
+                    sv[4 * e + 2] = __float_as_uint(__uint_as_float(sv[4 * e + 2]) * gg.z);
+                    sv[4 * e + 3] = __float_as_uint(__uint_as_float(sv[4 * e + 3]) * gg.w);
+                }
+                tmem_st_32x32b_x32(base + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+                tmem_st_32x32b_x32(base + 64 * hf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+                tmem_wait_st();
+            }
+            if (!ok) break;
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {  // V'^T = [U^T] - (W S_n)^T -> bf16, over the dead S copy
+                const uint32_t base = tmem + lrow + mp_base(c);
+                uint4 uu[4];
+                if (c == 1) {
+                    const uint8_t *ut = sm + stg * STB + O_U;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) uu[k] = *reinterpret_cast<const uint4 *>(ut + sw128(j, 4 * hf + k));
+                }
+                if (!mbar_wait(&bar_p[c], n & 1)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t pv[32], pk[16];
+                tmem_ld_32x32b_x32(base + MP_PO + 32 * hf, pv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    float u[8];
+                    if (c == 1) {
+                        unpack8(uu[k], u);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) u[e] = 0.f;
+                    }
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        pk[4 * k + e] = pack_bf16x2(u[2 * e] + __uint_as_float(pv[8 * k + 2 * e]),
+                                                    u[2 * e + 1] + __uint_as_float(pv[8 * k + 2 * e + 1]));
+                }
+                tmem_st_32x32b_x16(base + MP_S16 + 16 * hf, pk);
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&vimg[c]);
+            }
+        }
+        if (ok && nc > 0) {
+            if (!mbar_wait(&bar_s[0], (nc - 1) & 1) || !mbar_wait(&bar_s[1], (nc - 1) & 1)) ok = false;
+            tc_fence_after();
+        }
+        if (ok) {
+            // Y_g (S_1 for segment 0), laid out like a state
+            float *dst0 = p.yt + ((size_t)bh * (p.G - 1) + g) * DD * DD;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t sv[32];
+                tmem_ld_32x32b_x32(tmem + lrow + mp_base(1) + 64 * hf + 32 * hh, sv);
+                tmem_wait_ld();
+                float *dst = dst0 + (size_t)(64 * hf + 32 * hh) * DD + j;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) dst[(size_t)e * DD] = __uint_as_float(sv[e]);
+            }
+            if (g >= 1) {  // A_g^T as the combine pass's MN-major B operand: image row j = lane j
+                uint8_t *img = p.xt + ((size_t)bh * (p.G - 1) + g) * 32768;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    uint32_t sv[32];
+                    tmem_ld_32x32b_x32(tmem + lrow + mp_base(0) + 64 * hf + 32 * hh, sv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        float f[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(sv[8 * k + e]);
+                        *reinterpret_cast<uint4 *>(img + hf * 16384 + sw128(j, 4 * hh + k)) = pack8(f);
+                    }
+                }
+            }
+        }
+        if (!ok) s_fail = 1;
+    }
+    __syncthreads();
+    if (warp == 8 && lane == 0 && s_fail) {
+        report_timeout(p.timeouts, p.dev_status);
+        // let the bulk copies already issued land before the CTA exits
+        for (int m = landed; m < issued; ++m) mbar_wait(&full[m % STG], (m / STG) & 1, 100000000ull);
+    }
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, ST_TCOLS);
@@ -1232,12 +1445,10 @@ __global__ void __launch_bounds__(128, 1) chunk_combine_kernel(CombineArgs p) {
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-// Segments per sequence: as many as let the map pass (one CTA for segment 0, two for every later
-// segment but the last: BH (2G - 3) CTAs) and the chain pass (BH G CTAs) each run in one wave, with at
-// least 4 chunks per segment; 1 when (batch x heads) alone fills the GPU.
+// Segments per sequence: as many as let the chain pass (BH G CTAs), and so the map pass (BH (G - 1)
+// CTAs), run in one wave, with at least 4 chunks per segment; 1 when (batch x heads) alone fills the GPU.
 int pick_segments(int64_t BH, int64_t Nc, int sms) {
-    int64_t G = (sms / BH + 3) / 2;
-    if (G > sms / BH) G = sms / BH;
+    int64_t G = sms / BH;
     if (G > Nc / 4) G = Nc / 4;
     return (int)(G < 1 ? 1 : G);
 }
@@ -1252,11 +1463,11 @@ int device_sms() {
 kda_status_t launch_state(const CUtensorMap &tmo, const CUtensorMap &tgl, const StateArgs &sa, int B, int H,
                           cudaStream_t st) {
     if (sa.G > 1) {
-        cudaFuncSetAttribute(chunk_state_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
-        cudaError_t e = launch_pdl(chunk_state_kernel<true>, dim3(H, B, 2 * sa.G - 3), dim3(ST_THREADS_MAP),
-                                   STATE_SMEM, st, tmo, tgl, sa);
-        if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "chunk_state_kernel (segment maps): %s", cudaGetErrorString(e));
-        kda_status_t s = check_launch("chunk_state_kernel (segment maps)");
+        cudaFuncSetAttribute(chunk_map_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
+        cudaError_t e = launch_pdl(chunk_map_pair_kernel, dim3(H, B, sa.G - 1), dim3(ST_THREADS_MAP), STATE_SMEM, st,
+                                   sa);
+        if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "chunk_map_pair_kernel: %s", cudaGetErrorString(e));
+        kda_status_t s = check_launch("chunk_map_pair_kernel");
         if (s != KDA_OK) return s;
     }
     if (sa.G > 2) {  // (with two segments, segment 1 starts from S_1 itself)
@@ -1274,8 +1485,8 @@ kda_status_t launch_state(const CUtensorMap &tmo, const CUtensorMap &tgl, const 
         kda_status_t s = check_launch("chunk_combine_kernel");
         if (s != KDA_OK) return s;
     }
-    cudaFuncSetAttribute(chunk_state_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
-    cudaError_t e = launch_pdl(chunk_state_kernel<false>, dim3(H, B, sa.G), dim3(ST_THREADS_CHAIN), STATE_SMEM, st, tmo, tgl,
+    cudaFuncSetAttribute(chunk_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
+    cudaError_t e = launch_pdl(chunk_state_kernel, dim3(H, B, sa.G), dim3(ST_THREADS_CHAIN), STATE_SMEM, st, tmo, tgl,
                                sa);
     if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "chunk_state_kernel: %s", cudaGetErrorString(e));
     return check_launch("chunk_state_kernel");

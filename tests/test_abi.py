@@ -159,12 +159,12 @@ def test_workspace_query_needs_no_device():
 def _expected_tc_workspace(B, S, H, sms=148):
     """Workspace of the tensor-core chunk engine, from the rule it follows: per-chunk records, and,
     with G segments, BH (G - 1) map slots (A image + Y) and BH G entering states, G the
-    largest count for which the map pass (BH (2G - 3) CTAs) and the chain pass (BH G CTAs) each fit
+    largest count for which the chain pass (BH G CTAs, so also the map pass, BH (G - 1) CTAs) fits
     in one wave, at least 4 chunks per segment, and no empty segment."""
     rec = 74240
     bh, nc = B * H, (S + 63) // 64
     per_sm = sms // bh
-    g = min((per_sm + 3) // 2, per_sm, nc // 4)
+    g = min(per_sm, nc // 4)
     g = max(g, 1)
     L = (nc + g - 1) // g
     g = (nc + L - 1) // L
@@ -174,7 +174,7 @@ def _expected_tc_workspace(B, S, H, sms=148):
     return ws, g
 
 
-@pytest.mark.parametrize("B,S,H,G", [(1, 4096, 16, 6),      # prefill_4k: 6 segments of 11 chunks
+@pytest.mark.parametrize("B,S,H,G", [(1, 4096, 16, 8),      # prefill_4k: 8 segments of 8 chunks
                                      (8, 8192, 32, 1),      # batch_8x8k: one segment
                                      (1, 600, 1, 2), (1, 768, 2, 3), (1, 2560, 2, 10)])
 def test_tc_workspace_and_segment_count(B, S, H, G):
