@@ -41,7 +41,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     using Cfg = ProjCfg<BN>;
     constexpr int ST = Cfg::STAGES;
     extern __shared__ uint8_t smraw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smraw) + 1023) & ~uintptr_t(1023));
+    // first 1024-byte boundary, by pointer arithmetic on the shared base (keeps accesses ld/st.shared)
+    uint8_t *sm = smraw + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(smraw)) & 1023u)) & 1023u);
     uint8_t *sA = sm;
     uint8_t *sB = sm + ST * Cfg::A_BYTES;
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + ST * Cfg::STAGE_BYTES);

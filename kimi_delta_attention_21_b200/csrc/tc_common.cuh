@@ -79,8 +79,12 @@ __device__ __forceinline__ float log_alpha_fast(float z, float g_min) {
 // bits, which cannot carry for shared-memory addresses below 256 KB.
 __device__ __forceinline__ uint64_t dadd(uint64_t d, uint32_t off_bytes) { return d + (off_bytes >> 4); }
 
+// The first 1024-byte boundary at or after the dynamic shared-memory base p.  Pointer arithmetic on p
+// itself (not an integer round trip), so that the compiler still knows every access through the
+// result is a shared-memory access (ld.shared / st.shared, 32-bit addresses).
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
-    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+    const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(p));
+    return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
 __device__ __forceinline__ void named_sync(int id, int nthreads) {
