@@ -200,12 +200,15 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             const int c = t & 127, hv = t >> 7;
             float *qsum = reinterpret_cast<float *>(sm + P_XS);
             const int64_t i0 = (((int64_t)b * p.S + t0) * p.H + h) * DD + c, rstr = (int64_t)p.H * DD;
+            // Rows past the end are computed (from a row inside, or the zero-filled tile rows) and then
+            // multiplied by zero: no branch per element, so the 32 exponential chains overlap.
             float g[32];
             if (p.log_decay) {
 #pragma unroll
                 for (int rr = 0; rr < 32; ++rr) {
                     const int r = hv * 32 + rr;
-                    g[rr] = (r < len) ? clamp_log_decay(p.log_decay[i0 + r * rstr], p.g_min) : 0.f;
+                    const float lv = p.log_decay[i0 + (int64_t)min(r, len - 1) * rstr];
+                    g[rr] = clamp_log_decay(lv, p.g_min) * (r < len ? 1.f : 0.f);
                 }
             } else {
                 if (!mbar_wait(bar_z, zpar)) landed = false;
@@ -215,7 +218,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                 for (int rr = 0; rr < 32; ++rr) {
                     const int r = hv * 32 + rr;
                     const float zv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(zc + sw128(r, ch)));
-                    g[rr] = (r < len) ? log_alpha_fast(zv, p.g_min) : 0.f;
+                    g[rr] = log_alpha_fast(zv, p.g_min) * (r < len ? 1.f : 0.f);
                 }
             }
             float acc = 0.f;

@@ -223,12 +223,15 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             tmem_ld_32x32b_x32(base, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
             tmem_ld_32x32b_x32(base + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
             tmem_wait_ld();
+            // Every entry is computed and the masked ones multiplied by zero (no branch per entry, so the
+            // exponential chains overlap); the exponent is capped at 0, which only the masked entries
+            // reach (G never increases along the chunk), so that they stay finite.
             if (warp < 2) {  // A[r, i] = beta_r e^{G_r - G_i} k_r . k_i for i < r
                 float *sA = reinterpret_cast<float *>(sm + G_SA) + row * SA_LD;
                 const float br = sbeta[row];
 #pragma unroll
                 for (int i = 0; i < 64; ++i)
-                    sA[i] = (i < row) ? br * fexp(Gr - sG[i]) * __uint_as_float(v[i]) : 0.f;
+                    sA[i] = br * (fexp(fminf(Gr - sG[i], 0.f)) * (i < row ? 1.f : 0.f)) * __uint_as_float(v[i]);
             } else {         // M^T[i, r] = e^{G_r - G_i} q_r . k_i for i <= r (row = i)
 #pragma unroll
                 for (int k8 = 0; k8 < 8; ++k8) {
@@ -236,7 +239,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int r = 8 * k8 + e;
-                        t[e] = (row <= r) ? fexp(sG[r] - Gr) * __uint_as_float(v[r]) : 0.f;
+                        t[e] = (fexp(fminf(sG[r] - Gr, 0.f)) * (row <= r ? 1.f : 0.f)) * __uint_as_float(v[r]);
                     }
                     *reinterpret_cast<uint4 *>(sm + G_MT + sw128(row, k8)) = pack8(t);
                 }
