@@ -178,10 +178,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     // P1 and the per-channel tables of unit u: beta, G = in-chunk cumulative log-decay (rows past the
     // sequence end: no decay, beta 0), the block constants and e^{G_C}.  The decay input is z (the tile
     // at P_ZT, loaded one unit ahead, landed on bar_z with parity zpar) or the log-decay (read from
-    // global memory, prefetched into L2 one unit ahead); beta_row is row t's beta (t < 64), loaded one
-    // unit ahead.  Run by the decay group, warps 4-11 (t = tid - 128, named barrier 3): for the first
-    // unit before the loop, for every later one beside the previous unit's inverse.  Returns false if
-    // the z tile never landed.
+    // global memory, prefetched into L2 one unit ahead).  Beta is read from global memory here, its
+    // load issued first and its value stored last (a load still in flight holds up the next barrier).
+    // Run by the decay group, warps 4-11 (t = tid - 128, named barrier 3): for the first unit before
+    // the loop, for every later one beside the previous unit's inverse.  Returns false if the z tile
+    // never landed.
     constexpr int DT0 = 128, DTN = 256;
     auto load_beta = [&](int64_t u, int row) -> float {  // beta of row `row` of unit u; 0 past the end
         int n, h, b;
@@ -189,13 +190,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         const int t0 = n * CH;
         return (t0 + row < p.S) ? __bfloat162float(p.beta[((int64_t)b * p.S + t0 + row) * p.H + h]) : 0.f;
     };
-    auto decay_tables = [&](int64_t u, uint32_t zpar, float beta_row) -> bool {
+    auto decay_tables = [&](int64_t u, uint32_t zpar) -> bool {
         int n, h, b;
         unit_coords(u, n, h, b);
         const int t = tid - DT0;
         const int t0 = n * CH, len = min(CH, p.S - t0);
         bool landed = true;
-        if (t < CH) sbeta[t] = beta_row;
+        const float beta_row = t < CH ? load_beta(u, t) : 0.f;
         {   // one thread per channel c and 32 rows (half hv); the half sums through a scratch
             const int c = t & 127, hv = t >> 7;
             float *qsum = reinterpret_cast<float *>(sm + P_XS);
@@ -268,6 +269,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             }
             }
         }
+        if (t < CH) sbeta[t] = beta_row;
         return landed;
     };
 
@@ -294,8 +296,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
     if (warp >= 4 && warp < 12 && (int64_t)blockIdx.x < p.units) {  // the first unit's decay and tables
-        const int t = tid - DT0;
-        ok = decay_tables(blockIdx.x, 0u, t < CH ? load_beta(blockIdx.x, t) : 0.f);
+        ok = decay_tables(blockIdx.x, 0u);
     }
 
     int it = 0;
@@ -304,8 +305,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         unit_coords(u, n, h, b);
         const int64_t u_next = u + gridDim.x;
         const uint32_t par = it & 1;
-        // the next unit's beta, consumed by its decay during this unit's inverse
-        const float beta_next = (warp >= 4 && warp < 6 && u_next < p.units) ? load_beta(u_next, tid - DT0) : 0.f;
         if (u_next < p.units && tid < 256 && p.log_decay) {  // the next unit's log-decay input -> L2
             int n2, h2, b2;
             unit_coords(u_next, n2, h2, b2);
@@ -562,7 +561,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             invert_unit_lower64(reinterpret_cast<const float *>(sm + P_SA), reinterpret_cast<float *>(sm + P_ST),
                                 reinterpret_cast<float *>(sm + P_IX), sm + P_TI, tid);
         } else if (warp < 12 && u_next < p.units) {
-            ok = decay_tables(u_next, (uint32_t)(it + 1) & 1u, beta_next) && ok;
+            ok = decay_tables(u_next, (uint32_t)(it + 1) & 1u) && ok;
         }
         tc_fence_before();
         ok = __syncthreads_and(ok);

@@ -49,8 +49,9 @@ constexpr uint32_t G_U = 147456;      // U^T image [128 rows j][128 B: r]
 constexpr uint32_t G_SA = 163840;     // A [64][SA_LD] fp32
 constexpr uint32_t G_ST = G_SA + 64 * SA_LD * 4;   // T [64][ST_LD] fp32
 constexpr uint32_t G_IX = G_ST + 64 * ST_LD * 4;   // inverse scratch, 1536 fp32
-constexpr uint32_t G_GV = G_IX + 1536 * 4;         // G [64], e^G [64], beta [64], e^{G_C} [128], warp sums [2]
-constexpr uint32_t G_BAR = G_GV + 1536;            // mbarriers: inputs [2], A/M MMA, W/U MMA; TMEM slot
+constexpr uint32_t G_GV = G_IX + 1536 * 4;         // G [64], e^G [64], beta [64], e^{G_C} [128], warp sums [2],
+                                                   // the next unit's log-decay [64] and beta [64] (from 384)
+constexpr uint32_t G_BAR = G_GV + 2048;            // mbarriers: inputs [2], A/M MMA, W/U MMA; TMEM slot
 constexpr uint32_t G_END = G_BAR + 64;
 constexpr size_t GDN_SMEM = G_END + 1024;
 static_assert(GDN_SMEM <= 232448, "gdn prep shared memory");
@@ -84,6 +85,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     float *sbeta = sG + 128;
     float *sgam = sG + 192;
     float *wsum = sG + 320;
+    float *sgn = sG + 384, *sbn = sG + 448;  // the next unit's log-decay and beta, loaded during the inverse
 
     auto unit_coords = [&](int64_t u, int &n, int &h, int &b) {  // 32-bit: units < 2^31 (host check)
         const uint32_t uu = (uint32_t)u, nc = (uint32_t)p.Nc, hh = (uint32_t)p.H;
@@ -154,8 +156,10 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             bulk_wait_read_all();
             load_inputs(u_next, buf ^ 1);
         }
-        float g_next = 0.f, b_next = 0.f;
-        if (tid < CH && u_next < p.units) load_decay(u_next, tid, g_next, b_next);
+        if (it > 0 && tid < CH) {  // this unit's log-decay and beta (loaded during the previous inverse)
+            g_cur = sgn[tid];
+            b_cur = sbn[tid];
+        }
         // ---- cumulative log-decay over the chunk (warps 0-1: one token per thread), e^G, beta
         if (tid < CH) {
             float x = g_cur;
@@ -171,8 +175,6 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             sG[tid] = x;
             seG[tid] = fexp(x);
         }
-        g_cur = g_next;
-        b_cur = b_next;
         ok = mbar_wait(&bar_in[buf], ipar) && ok;
         ok = __syncthreads_and(ok);
         if (!ok) break;
@@ -267,10 +269,17 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             bulk_store(rec + REC_GAM, sgam, 512);
             bulk_commit();
         }
-        // ---- T = (I + A)^{-1} (warps 0-3)
-        if (warp < 4)
+        // ---- T = (I + A)^{-1} (warps 0-3); meanwhile warps 4-5 read the next unit's log-decay and beta
+        //      (global loads still in flight would hold up a barrier: these have the inverse to land)
+        if (warp < 4) {
             invert_unit_lower64(reinterpret_cast<const float *>(sm + G_SA), reinterpret_cast<float *>(sm + G_ST),
                                 reinterpret_cast<float *>(sm + G_IX), sm + G_TI, tid);
+        } else if (warp < 6 && u_next < p.units) {
+            float g, bt;
+            load_decay(u_next, tid - 128, g, bt);
+            sgn[tid - 128] = g;
+            sbn[tid - 128] = bt;
+        }
         tc_fence_before();
         __syncthreads();
         // ---- W = T (beta K e^G) (M = 64, N = 128, K = 64) and U^T = (beta V)^T T^T (M = 128, N = 64, K = 64)
