@@ -58,11 +58,20 @@ CHUNK = 64
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one chunk-engine
 # call or one decode step, from an ncu capture of the named kernels on the
 # named workload, valid only while the kernel source is unchanged (sha256
-# prefix of the listed files).  "scale" marks a figure taken on a smaller
-# workload and scaled by the number of (batch, head, chunk) units.
+# prefix of the listed files).  "units" marks a figure taken on a smaller
+# workload, scaled by the number of (batch, head, chunk) units of the one timed.
+_CHUNK_SRC = {"kimi_delta_attention_21_b200/csrc/chunk_tc.cu": "1af918c89471cb76",
+              "kimi_delta_attention_21_b200/csrc/tc_common.cuh": "2c040ed7e721efb8",
+              "kimi_delta_attention_21_b200/csrc/sm100_ptx.cuh": "b75f6e1e7fa94863"}
 NCU_TRAFFIC = {
-    "decode@decode_256": {"bytes": 1027173120, "src_sha": {"kimi_delta_attention_21_b200/csrc/decode.cu":
-                                                              "079db3bd726bd665"}},
+    # chunk engine (prep, map pass, combine, chain pass) on prefill_4k, 1,024 units; long_1m scaled by
+    # units (the records dominate; its map pass covers 8 of 9 segments against 7 of 8); none for
+    # batch_8x8k, which runs no map pass
+    "chunk_engine@prefill_4k": {"bytes": 247777194, "units": 1024, "src_sha": _CHUNK_SRC},
+    "chunk_engine@long_1m": {"bytes": 247777194, "units": 1024, "src_sha": _CHUNK_SRC},
+    "decode@decode_256": {"bytes": 1024244608,
+                          "src_sha": {"kimi_delta_attention_21_b200/csrc/decode.cu": "88b9a3ab7b5af3e2",
+                                      "kimi_delta_attention_21_b200/csrc/sm100_ptx.cuh": "b75f6e1e7fa94863"}},
 }
 
 
