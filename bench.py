@@ -60,7 +60,7 @@ CHUNK = 64
 # named workload, valid only while the kernel source is unchanged (sha256
 # prefix of the listed files).  "units" marks a figure taken on a smaller
 # workload, scaled by the number of (batch, head, chunk) units of the one timed.
-_CHUNK_SRC = {"kimi_delta_attention_21_b200/csrc/chunk_tc.cu": "1af918c89471cb76",
+_CHUNK_SRC = {"kimi_delta_attention_21_b200/csrc/chunk_tc.cu": "6a80f033b594d956",
               "kimi_delta_attention_21_b200/csrc/tc_common.cuh": "2c040ed7e721efb8",
               "kimi_delta_attention_21_b200/csrc/sm100_ptx.cuh": "b75f6e1e7fa94863"}
 NCU_TRAFFIC = {
@@ -310,23 +310,27 @@ class Timer:
         return a, b
 
 
-def time_prefill(K, torch, w, d, steps, warmup, world, dev, flush, lib, sampler=None, gdn=False):
+def time_prefill(K, torch, w, d, steps, warmup, world, dev, flush, lib, sampler=None, gdn=False, engine="auto"):
     """Times `steps` layer forwards of workload `w` (device inputs `d`).  Returns
     per-step seconds (chunk engine, projection; max over ranks) and launches.
     gdn: the scalar-decay (Gated DeltaNet) engine, one decay logit per token and
-    head (the first channel's logit of the same inputs)."""
+    head (the first channel's logit of the same inputs).  engine: "auto" (the
+    tensor-core engine inside its envelope) or "simt" (the exact engine the
+    library falls back to outside it)."""
     B, S, H = w.B, w.S, w.H
     N = B * S
     x = torch.empty((B, S, H, w.Dv), dtype=d["v"].dtype, device=dev)
     y = torch.empty((N, w.D_model), dtype=d["v"].dtype, device=dev)
     sf = torch.empty((B, H, w.Dk, w.Dv), dtype=torch.float32, device=dev)
-    ws = torch.empty(K.chunk_workspace_bytes(B, S, H, w.Dk, w.Dv, scalar_decay=gdn), dtype=torch.uint8, device=dev)
+    ws = torch.empty(K.chunk_workspace_bytes(B, S, H, w.Dk, w.Dv, scalar_decay=gdn, engine=engine), dtype=torch.uint8,
+                     device=dev)
     stream = torch.cuda.current_stream(dev)
     z = d["z"][..., 0].contiguous() if gdn else d["z"]
 
     def chunk():
         K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=z, g_min=w.g_min, initial_state=d["S0"],
-                    gate_logits=d["gate"], eps=w.eps, out=x, final_state=sf, workspace=ws, scalar_decay=gdn)
+                    gate_logits=d["gate"], eps=w.eps, out=x, final_state=sf, workspace=ws, scalar_decay=gdn,
+                    engine=engine)
 
     def proj():
         K.out_proj(x.view(N, H * w.Dv), d["W_o"], out=y)
@@ -627,6 +631,17 @@ def run_ours(args, rank, world, local):
             "chunk_engine_tokens_per_s": round(w.B * w.S * world / tg["t_chunk"], 1),
             "roofline": {k: gr[k] for k in ("bound", "achieved", "peak", "unit", "frac")},
             "kda_over_gdn_chunk_time": round(tm["t_chunk"] / tg["t_chunk"], 3)}
+        if name == "prefill_4k":
+            # the exact SIMT engine, which the library uses outside the tensor-core engine's envelope
+            ts = time_prefill(K, torch, w, d, max(3, args.steps // 4), args.warmup, world, dev, flush, lib,
+                              engine="simt")
+            records[name]["simt_engine"] = {
+                "engine": "kda_chunk_fwd with engine = SIMT (exact; fp64 G and accumulation for fp32 inputs)",
+                "used_when": "auto: inputs not bf16, D_k or D_v not 128, chunk not 64, g_min < -5.5, or a pointer "
+                             "not 16-byte aligned",
+                "chunk_engine_ms": round(ts["t_chunk"] * 1e3, 4),
+                "chunk_engine_tokens_per_s": round(w.B * w.S * world / ts["t_chunk"], 1),
+                "simt_over_tc_chunk_time": round(ts["t_chunk"] / tm["t_chunk"], 2)}
         if name == HEADLINE:
             head_tm = tm
         if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -80,8 +80,8 @@ constexpr uint32_t P_A = 65536;      // A operand of the A/M MMAs [2 atoms][224 
                                      // one (rows 160-223); later -W, U^T and the M^T image
 constexpr uint32_t P_B = 122880;     // B operand [2 atoms][192 rows][128 B]: row operands from k, q and the low
                                      // part of the q one; later the T image and the diagonal residues
-constexpr uint32_t P_SG = 172032;    // G fp32 [64][132]; later A [64][65] and T [64][68] fp32
-constexpr uint32_t P_TAB = 206080;   // per-channel block constants [26][128] fp32; then inverse scratch
+constexpr uint32_t P_SG = 172032;    // G fp32 [64][132] (the next unit's, written beside this unit's inverse)
+constexpr uint32_t P_TAB = 206080;   // per-channel block constants [26][128] fp32 (likewise)
 constexpr uint32_t P_XS = 219392;    // quarter sums of the cumulative log-decay [4][128] fp32
 constexpr uint32_t P_BETA = 222464;  // beta [64] fp32
 constexpr uint32_t P_GAM = 222720;   // e^{G_C} [128] fp32
