@@ -9,7 +9,7 @@
 // b = k * alpha) the chunkwise UT/WY form does not apply as is, and this is the
 // form every such transition has.  Exact fp32; a block owns one (b, h) and 16
 // value columns with the state slice in registers (two sums over the key rows
-// per token).
+// per token, one block barrier each).
 #include "rec_common.cuh"
 
 namespace kda {
@@ -27,10 +27,19 @@ struct DplrParams {
     float *Sf;
 };
 
+// A chunk of 64 tokens is staged in shared memory by coalesced loads (k, q, a, b and log alpha [64][D_k],
+// the block's 16 columns of v [64][16]) and its outputs leave together (o [64][16]), so that no token
+// step waits on global memory; the two sums per token take one block barrier each.
+constexpr int DP_C = 64;
+
+size_t dplr_smem_bytes(int Dk) { return (size_t)(5 * DP_C * Dk + 2 * DP_C * rec::VS) * 4; }
+
 template <typename T>
 __global__ void __launch_bounds__(rec::THREADS) dplr_recurrent_kernel(DplrParams p) {
-    __shared__ float red[rec::THREADS / 32 * 16];
-    __shared__ float sw[16], sv[16];
+    extern __shared__ __align__(16) float smf[];
+    __shared__ __align__(16) float red[2][rec::THREADS / 32 * 16];
+    float *sk = smf, *sq = sk + DP_C * p.Dk, *sa = sq + DP_C * p.Dk, *sbv = sa + DP_C * p.Dk;
+    float *sg = sbv + DP_C * p.Dk, *sv = sg + DP_C * p.Dk, *so = sv + DP_C * rec::VS;
     const int tid = threadIdx.x, c = tid >> 1, half = tid & 1;
     const int bh = blockIdx.x, b = bh / p.H, h = bh % p.H, j0 = blockIdx.y * rec::VS, jc = j0 + 8 * half;
     const bool row_ok = c < p.Dk;
@@ -38,36 +47,51 @@ __global__ void __launch_bounds__(rec::THREADS) dplr_recurrent_kernel(DplrParams
 #pragma unroll
     for (int e = 0; e < 8; ++e)
         S[e] = (p.S0 && row_ok && jc + e < p.Dv) ? p.S0[((int64_t)bh * p.Dk + c) * p.Dv + jc + e] : 0.f;
-    for (int64_t t = 0; t < p.S; ++t) {
-        const int64_t row = ((int64_t)b * p.S + t) * p.H + h;
-        float al = 1.f, ac = 0.f, bc = 0.f, kc = 0.f, qc = 0.f;
-        if (row_ok) {
-            const int64_t i = row * p.Dk + c;
-            const float g = p.log_decay ? clamp_log_decay(p.log_decay[i], p.g_min)
-                                        : log_alpha_of(load_elem((const T *)p.z, i), p.g_min);
-            al = expf(g);
-            ac = load_elem((const T *)p.a, i);
-            bc = load_elem((const T *)p.b, i);
-            kc = load_elem((const T *)p.k, i);
-            qc = load_elem((const T *)p.q, i);
+    int par = 0;  // which of the two partial-sum buffers the next sum uses
+    for (int64_t t0 = 0; t0 < p.S; t0 += DP_C) {
+        const int len = (int)min((int64_t)DP_C, p.S - t0);
+        const int64_t row0 = (int64_t)b * p.S + t0;
+        __syncthreads();  // the previous chunk's steps and output flush are done with the staged arrays
+        for (int idx = tid; idx < len * p.Dk; idx += rec::THREADS) {
+            const int r = idx / p.Dk, cc = idx - r * p.Dk;
+            const int64_t i = ((row0 + r) * p.H + h) * p.Dk + cc;
+            sk[idx] = load_elem((const T *)p.k, i);
+            sq[idx] = load_elem((const T *)p.q, i);
+            sa[idx] = load_elem((const T *)p.a, i);
+            sbv[idx] = load_elem((const T *)p.b, i);
+            sg[idx] = p.log_decay ? clamp_log_decay(p.log_decay[i], p.g_min)
+                                  : log_alpha_of(load_elem((const T *)p.z, i), p.g_min);
         }
-        float x[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = bc * S[e];
-        const float wj = rec::rowsum16(x, red, tid);  // w = b^T S_{t-1}
-        if (tid < 16) {
-            sw[tid] = wj;
-            sv[tid] = (j0 + tid < p.Dv) ? load_elem((const T *)p.v, row * p.Dv + j0 + tid) : 0.f;
+        for (int idx = tid; idx < len * rec::VS; idx += rec::THREADS) {
+            const int r = idx / rec::VS, j = idx - r * rec::VS;
+            sv[idx] = (j0 + j < p.Dv) ? load_elem((const T *)p.v, ((row0 + r) * p.H + h) * p.Dv + j0 + j) : 0.f;
         }
         __syncthreads();
+        for (int r = 0; r < len; ++r) {
+            const int ri = r * p.Dk + c;
+            const float al = row_ok ? expf(sg[ri]) : 1.f, ac = row_ok ? sa[ri] : 0.f, bc = row_ok ? sbv[ri] : 0.f;
+            const float kc = row_ok ? sk[ri] : 0.f, qc = row_ok ? sq[ri] : 0.f;
+            float x[8], w[8], o[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            S[e] = fmaf(al, S[e], fmaf(-ac, sw[8 * half + e], kc * sv[8 * half + e]));
-            x[e] = qc * S[e];
+            for (int e = 0; e < 8; ++e) x[e] = bc * S[e];
+            rec::rowsum16_all(x, red[par], tid, w);  // w = b^T S_{t-1}
+            par ^= 1;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                S[e] = fmaf(al, S[e], fmaf(-ac, w[e], kc * sv[r * rec::VS + 8 * half + e]));
+                x[e] = qc * S[e];
+            }
+            rec::rowsum16_all(x, red[par], tid, o);  // o = S_t^T q
+            par ^= 1;
+            if (tid < 2)
+#pragma unroll
+                for (int e = 0; e < 8; ++e) so[r * rec::VS + 8 * half + e] = o[e];
         }
-        const float oj = rec::rowsum16(x, red, tid);  // o = S_t^T q
-        if (tid < 16 && j0 + tid < p.Dv) store_elem((T *)p.o, row * p.Dv + j0 + tid, oj);
-        __syncthreads();  // the next token's first sum reuses `red`
+        __syncthreads();
+        for (int idx = tid; idx < len * rec::VS; idx += rec::THREADS) {
+            const int r = idx / rec::VS, j = idx - r * rec::VS;
+            if (j0 + j < p.Dv) store_elem((T *)p.o, ((row0 + r) * p.H + h) * p.Dv + j0 + j, so[idx]);
+        }
     }
     if (p.Sf && row_ok)
 #pragma unroll
@@ -90,8 +114,15 @@ kda_status_t launch_dplr(const kda_dplr_args &a, cudaStream_t st) {
     p.o = a.o;
     p.Sf = a.final_state;
     const dim3 grid((unsigned)(a.B * a.H), (unsigned)((a.D_v + rec::VS - 1) / rec::VS));
-    if (a.dtype == KDA_F32) dplr_recurrent_kernel<float><<<grid, rec::THREADS, 0, st>>>(p);
-    else dplr_recurrent_kernel<__nv_bfloat16><<<grid, rec::THREADS, 0, st>>>(p);
+    const size_t smem = dplr_smem_bytes(a.D_k);
+    if (a.dtype == KDA_F32) {
+        cudaFuncSetAttribute(dplr_recurrent_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        dplr_recurrent_kernel<float><<<grid, rec::THREADS, smem, st>>>(p);
+    } else {
+        cudaFuncSetAttribute(dplr_recurrent_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
+        dplr_recurrent_kernel<__nv_bfloat16><<<grid, rec::THREADS, smem, st>>>(p);
+    }
     return check_launch("dplr_recurrent_kernel");
 }
 
