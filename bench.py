@@ -60,7 +60,7 @@ CHUNK = 64
 # named workload, valid only while the kernel source is unchanged (sha256
 # prefix of the listed files).  "units" marks a figure taken on a smaller
 # workload, scaled by the number of (batch, head, chunk) units of the one timed.
-_CHUNK_SRC = {"kimi_delta_attention_21_b200/csrc/chunk_tc.cu": "6a80f033b594d956",
+_CHUNK_SRC = {"kimi_delta_attention_21_b200/csrc/chunk_tc.cu": "6b4e19675db3b528",
               "kimi_delta_attention_21_b200/csrc/tc_common.cuh": "2c040ed7e721efb8",
               "kimi_delta_attention_21_b200/csrc/sm100_ptx.cuh": "b75f6e1e7fa94863"}
 NCU_TRAFFIC = {

@@ -76,6 +76,15 @@ uint64_t kda_launch_count(void);
  * the last reset (0 in a healthy run); reset != 0 clears it.  Synchronous. */
 kda_status_t kda_device_timeouts(uint32_t *count, int reset);
 
+/* Writes that a checked build (compiled with -DKDA_CHECKED: libkda_checked.so)
+ * found outside their buffer and skipped, on the current device, since the
+ * last reset; reset != 0 clears it.  *checked_build (if not NULL) is set to 1
+ * in a checked build, 0 otherwise (where the count stays 0).  The checks cover
+ * every global write through an offset the library computes: workspace
+ * records, segment maps and entering states, checkpoints and stashes, final
+ * states and staged outputs.  Synchronous. */
+kda_status_t kda_device_bounds_errors(uint32_t *count, int reset, int *checked_build);
+
 /* Self-test of the bounded-wait path the tensor-core kernels use: launches a
  * one-CTA kernel that waits on a barrier nothing completes, gives up after
  * limit_us microseconds (1 .. 1e6), writes KDA_ERR_TIMEOUT to *dev_status (a

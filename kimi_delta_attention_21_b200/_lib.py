@@ -8,7 +8,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libkda.so")
+# KDA_LIBRARY picks another in-tree build of the same ABI by file name (libkda_checked.so: the
+# bounds-checked build); absent, the library is libkda.so
+LIB_PATH = os.path.join(_HERE, os.path.basename(os.environ.get("KDA_LIBRARY", "libkda.so")))
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(6)
 KDA_F32, KDA_BF16 = 0, 1
@@ -81,6 +83,7 @@ SIGNATURES = {
     "kda_version": (ctypes.c_int, []),
     "kda_launch_count": (ctypes.c_uint64, []),
     "kda_device_timeouts": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]),
+    "kda_device_bounds_errors": (ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, _p]),
     "kda_selftest_wait_timeout": (ctypes.c_int, [_p, ctypes.c_uint32, _p]),
     "kda_gate": (ctypes.c_int, [_p, ctypes.c_int, _i64, _f32, _p, _p]),
     "kda_chunk_workspace_size": (ctypes.c_int, [ctypes.POINTER(ChunkArgs), ctypes.POINTER(ctypes.c_size_t)]),

@@ -120,6 +120,8 @@ struct PrepArgs {
     const __nv_bfloat16 *beta;
     const float *log_decay;
     uint8_t *ws;
+    size_t rec_bytes;        // the records' part of ws (checked builds test the record stores against it)
+    unsigned int *bounds;
     unsigned int *timeouts;
     int *dev_status;
 };
@@ -429,7 +431,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         // ---------------- tcgen05: A^T (cols 0-63), M^T (64-127), residues of M's diagonal blocks (128-191);
         // meanwhile Q e^G, K e^{G_C - G} and e^{G_C} leave (thread 96; once the stores have read them,
         // during P3, the next unit's q and k tiles take their place: they are not operands of these MMAs)
-        if (tid == 96) {
+        if (tid == 96 && in_bounds(rec, REC_BYTES, p.ws, p.rec_bytes, p.bounds)) {
             // Q e^G fills rows 64-127 of each atom of the stacked [W; Q e^G] image
             bulk_store(rec + REC_WQ + 8192, sm + P_QI, 8192);
             bulk_store(rec + REC_WQ + 16384 + 8192, sm + P_QI + 8192, 8192);
@@ -628,7 +630,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (tid == 0) {
+        if (tid == 0 && in_bounds(rec, REC_BYTES, p.ws, p.rec_bytes, p.bounds)) {
             bulk_store(rec + REC_WQ, sm + P_WI, 8192);
             bulk_store(rec + REC_WQ + 16384, sm + P_WI + 8192, 8192);
             bulk_store(rec + REC_MT, sm + P_MT, 8192);
@@ -678,6 +680,8 @@ struct StateArgs {
     const float *seg_init; // state entering segment g >= 1, [B*H][G][128][128] (after the combine pass)
     uint8_t *xt;           // map pass: A_g^T as bf16 operand images [B*H][G-1][32 KB]
     float *yt;             // map pass: Y_g [B*H][G-1][128][128]
+    size_t sf_bytes, xt_bytes, yt_bytes;  // sizes of Sf, xt, yt (checked builds test the writes against them)
+    unsigned int *bounds;
     float eps;
     unsigned int *timeouts;
     int *dev_status;
@@ -1034,7 +1038,8 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
             if (!mbar_wait(bar_s, (nc - 1) & 1) || !mbar_wait(bar_of(nc - 1), par_of(nc - 1))) ok = false;
             tc_fence_after();
         }
-        if (ok && p.Sf && g == p.G - 1) {  // (with no chunks TMEM still holds the entering state)
+        if (ok && p.Sf && g == p.G - 1 &&  // (with no chunks TMEM still holds the entering state)
+            in_bounds(p.Sf + (size_t)bh * DD * DD, DD * DD * 4, p.Sf, p.sf_bytes, p.bounds)) {
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t sv[32];
@@ -1276,7 +1281,7 @@ __global__ void __launch_bounds__(ST_THREADS_MAP, 1) chunk_map_pair_kernel(State
             if (!mbar_wait(&bar_s[0], (nc - 1) & 1) || !mbar_wait(&bar_s[1], (nc - 1) & 1)) ok = false;
             tc_fence_after();
         }
-        if (ok) {
+        if (ok && in_bounds(p.yt + ((size_t)bh * (p.G - 1) + g) * DD * DD, DD * DD * 4, p.yt, p.yt_bytes, p.bounds)) {
             // Y_g (S_1 for segment 0), laid out like a state
             float *dst0 = p.yt + ((size_t)bh * (p.G - 1) + g) * DD * DD;
 #pragma unroll
@@ -1288,7 +1293,8 @@ __global__ void __launch_bounds__(ST_THREADS_MAP, 1) chunk_map_pair_kernel(State
 #pragma unroll
                 for (int e = 0; e < 32; ++e) dst[(size_t)e * DD] = __uint_as_float(sv[e]);
             }
-            if (g >= 1) {  // A_g^T as the combine pass's MN-major B operand: image row j = lane j
+            if (g >= 1 && in_bounds(p.xt + ((size_t)bh * (p.G - 1) + g) * 32768, 32768, p.xt, p.xt_bytes, p.bounds)) {
+                // A_g^T as the combine pass's MN-major B operand: image row j = lane j
                 uint8_t *img = p.xt + ((size_t)bh * (p.G - 1) + g) * 32768;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
@@ -1330,6 +1336,8 @@ struct CombineArgs {
     const uint8_t *xt;
     const float *yt;
     float *seg_init;
+    size_t seg_bytes;  // size of seg_init (checked builds test the writes against it)
+    unsigned int *bounds;
     unsigned int *timeouts;
     int *dev_status;
 };
@@ -1407,7 +1415,8 @@ __global__ void __launch_bounds__(128, 1) chunk_combine_kernel(CombineArgs p) {
         }
         // while the MMA runs: S_g leaves for its segment chain (S_1 is read where the map pass left it)
         // and Y_g comes into registers
-        if (g > 1) {
+        if (g > 1 && in_bounds(p.seg_init + ((size_t)bh * p.G + g) * DD * DD, DD * DD * 4, p.seg_init, p.seg_bytes,
+                               p.bounds)) {
             float *dst = p.seg_init + ((size_t)bh * p.G + g) * DD * DD + j;
 #pragma unroll
             for (int c = 0; c < 128; ++c) dst[(size_t)c * DD] = sv[c];
@@ -1479,6 +1488,8 @@ kda_status_t launch_state(const CUtensorMap &tmo, const CUtensorMap &tgl, const 
         ca.xt = sa.xt;
         ca.yt = sa.yt;
         ca.seg_init = const_cast<float *>(sa.seg_init);
+        ca.seg_bytes = (size_t)B * H * sa.G * DD * DD * 4;
+        ca.bounds = sa.bounds;
         ca.timeouts = sa.timeouts;
         ca.dev_status = sa.dev_status;
         cudaFuncSetAttribute(chunk_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)COMB_SMEM);
@@ -1574,6 +1585,13 @@ kda_status_t tc::launch_chunk_state_pass(const kda_chunk_args &a, cudaStream_t s
     sa.xt = ws + lay.xt;
     sa.yt = reinterpret_cast<float *>(ws + lay.yt);
     sa.seg_init = reinterpret_cast<const float *>(ws + lay.seg);
+    {
+        const size_t BH = (size_t)a.B * a.H, nmap = sa.G > 1 ? BH * (sa.G - 1) : 0;
+        sa.sf_bytes = BH * DD * DD * 4;
+        sa.xt_bytes = nmap * 32768;
+        sa.yt_bytes = nmap * DD * DD * 4;
+        sa.bounds = device_bounds_counter();
+    }
     sa.eps = a.eps;
     sa.timeouts = device_timeout_counter();
     sa.dev_status = a.dev_status;
@@ -1608,6 +1626,8 @@ kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
         pa.beta = (const __nv_bfloat16 *)a.beta;
         pa.log_decay = a.log_decay;
         pa.ws = (uint8_t *)a.workspace;
+        pa.rec_bytes = (size_t)pa.units * REC_BYTES;
+        pa.bounds = device_bounds_counter();
         pa.timeouts = timeouts;
         pa.dev_status = a.dev_status;
         const int sms = device_sms();

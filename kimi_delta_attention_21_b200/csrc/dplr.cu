@@ -25,6 +25,8 @@ struct DplrParams {
     const float *S0;
     void *o;
     float *Sf;
+    size_t o_bytes, sf_bytes;  // (checked builds test the writes against them)
+    unsigned int *bounds;
 };
 
 // A chunk of 64 tokens is staged in shared memory by coalesced loads (k, q, a, b and log alpha [64][D_k],
@@ -88,12 +90,14 @@ __global__ void __launch_bounds__(rec::THREADS) dplr_recurrent_kernel(DplrParams
                 for (int e = 0; e < 8; ++e) so[r * rec::VS + 8 * half + e] = o[e];
         }
         __syncthreads();
-        for (int idx = tid; idx < len * rec::VS; idx += rec::THREADS) {
+        const int64_t o_lo = (row0 * p.H + h) * p.Dv, o_n = ((int64_t)(len - 1) * p.H) * p.Dv + p.Dv;
+        const bool o_ok = in_bounds((const T *)p.o + o_lo, (size_t)o_n * sizeof(T), p.o, p.o_bytes, p.bounds);
+        for (int idx = tid; o_ok && idx < len * rec::VS; idx += rec::THREADS) {
             const int r = idx / rec::VS, j = idx - r * rec::VS;
             if (j0 + j < p.Dv) store_elem((T *)p.o, ((row0 + r) * p.H + h) * p.Dv + j0 + j, so[idx]);
         }
     }
-    if (p.Sf && row_ok)
+    if (p.Sf && row_ok && in_bounds(p.Sf + (int64_t)bh * p.Dk * p.Dv, (size_t)p.Dk * p.Dv * 4, p.Sf, p.sf_bytes, p.bounds))
 #pragma unroll
         for (int e = 0; e < 8; ++e)
             if (jc + e < p.Dv) p.Sf[((int64_t)bh * p.Dk + c) * p.Dv + jc + e] = S[e];
@@ -113,6 +117,9 @@ kda_status_t launch_dplr(const kda_dplr_args &a, cudaStream_t st) {
     p.S0 = a.initial_state;
     p.o = a.o;
     p.Sf = a.final_state;
+    p.o_bytes = (size_t)a.B * a.S * a.H * a.D_v * (a.dtype == KDA_F32 ? 4 : 2);
+    p.sf_bytes = (size_t)a.B * a.H * a.D_k * a.D_v * 4;
+    p.bounds = device_bounds_counter();
     const dim3 grid((unsigned)(a.B * a.H), (unsigned)((a.D_v + rec::VS - 1) / rec::VS));
     const size_t smem = dplr_smem_bytes(a.D_k);
     if (a.dtype == KDA_F32) {

@@ -64,6 +64,8 @@ struct GdnArgs {
     const __nv_bfloat16 *z;        // (B, S, H) decay logits, or null
     const float *log_decay;        // (B, S, H) log alpha, or null (wins over z)
     uint8_t *ws;
+    size_t rec_bytes;              // the records' part of ws (checked builds test the record stores against it)
+    unsigned int *bounds;
     unsigned int *timeouts;
     int *dev_status;
 };
@@ -263,7 +265,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
         tc_fence_before();
         ok = __syncthreads_and(ok);
         if (!ok) break;
-        if (tid == 32) {
+        if (tid == 32 && in_bounds(rec, REC_BYTES, p.ws, p.rec_bytes, p.bounds)) {
             bulk_store(rec + REC_KT, sm + G_KT, 16384);
             bulk_store(rec + REC_MT, sm + G_MT, 8192);
             bulk_store(rec + REC_GAM, sgam, 512);
@@ -340,7 +342,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (tid == 0) {
+        if (tid == 0 && in_bounds(rec, REC_BYTES, p.ws, p.rec_bytes, p.bounds)) {
             bulk_store(rec + REC_WQ, kq, 32768);
             bulk_store(rec + REC_U, sm + G_U, 16384);
             bulk_commit();
@@ -388,6 +390,8 @@ kda_status_t launch_gdn_tc(const kda_chunk_args &a, cudaStream_t st) {
         ga.z = (const __nv_bfloat16 *)a.z;
         ga.log_decay = a.log_decay;
         ga.ws = (uint8_t *)a.workspace;
+        ga.rec_bytes = (size_t)ga.units * REC_BYTES;
+        ga.bounds = device_bounds_counter();
         ga.timeouts = device_timeout_counter();
         ga.dev_status = a.dev_status;
         int dev = 0, sms = 148;

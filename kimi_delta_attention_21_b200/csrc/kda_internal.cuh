@@ -46,6 +46,27 @@ __device__ __forceinline__ float log_alpha_of(float z, float g_min) {
     return g_min * sigmoid_precise(z);
 }
 
+// ----------------------------------------------------------------- checked builds
+// A build with -DKDA_CHECKED tests every global write through an offset the library computes itself
+// (workspace records, segment maps and entering states, checkpoints and stashes, final states, staged
+// outputs) against the buffer it has to land in: a write that would leave its buffer is skipped and
+// counted in a device counter (kda_device_bounds_errors), never trapped.  Other builds compile the
+// test away.
+#ifdef KDA_CHECKED
+__device__ __forceinline__ bool in_bounds(const void *p, size_t n, const void *base, size_t size,
+                                          unsigned int *errors) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p), b = reinterpret_cast<uintptr_t>(base);
+    const bool ok = base != nullptr && a >= b && n <= size && a - b <= size - n;
+    if (!ok && errors) atomicAdd(errors, 1u);
+    return ok;
+}
+#else
+__device__ __forceinline__ constexpr bool in_bounds(const void *, size_t, const void *, size_t, unsigned int *) {
+    return true;
+}
+#endif
+unsigned int *device_bounds_counter();  // device address of the counter (host)
+
 // ----------------------------------------------------------------- launchers (one per .cu)
 kda_status_t launch_gate(const void *z, kda_dtype_t dt, int64_t n, float g_min, float *out,
                          cudaStream_t st);

@@ -44,6 +44,9 @@ struct RbArgs {
     float *dq, *dk, *dv, *dbeta, *dz, *dS0;
     float *ckpt;   // [B*H][nslice][Nc][Dk][16]
     float *stash;  // [B*H][nslice][64][Dk][16]
+    // buffer sizes in bytes (checked builds test the workspace accesses and the writes against them)
+    size_t ckpt_bytes, stash_bytes, nk_bytes, nv_bytes, nb_bytes, ns_bytes;
+    unsigned int *bounds;
 };
 
 // The inputs of one 64-token chunk, staged in shared memory by coalesced loads once per chunk (the
@@ -132,7 +135,7 @@ __global__ void __launch_bounds__(RB_THREADS) rec_ckpt_kernel(RbArgs p) {
         S[e] = (p.S0 && c < p.Dk && jc + e < p.Dv) ? p.S0[((int64_t)bh * p.Dk + c) * p.Dv + jc + e] : 0.f;
     float *ck = p.ckpt + ((int64_t)bh * p.nslice + slice) * p.Nc * p.Dk * RB_VS;
     for (int n = 0; n < p.Nc; ++n) {
-        if (c < p.Dk)
+        if (c < p.Dk && in_bounds(ck + (int64_t)n * p.Dk * RB_VS, (size_t)p.Dk * RB_VS * 4, p.ckpt, p.ckpt_bytes, p.bounds))
 #pragma unroll
             for (int e = 0; e < 8; ++e) ck[((int64_t)n * p.Dk + c) * RB_VS + 8 * half + e] = S[e];
         const int64_t t0 = (int64_t)n * RB_C;
@@ -164,6 +167,7 @@ __global__ void __launch_bounds__(RB_THREADS) rec_bwd_kernel(RbArgs p) {
     const float *ck = p.ckpt + cta * p.Nc * p.Dk * RB_VS;
     float *stash = p.stash + cta * RB_C * p.Dk * RB_VS;
     const int soff = c * RB_VS + 8 * half;  // this thread's 8 floats within a token's [D_k][16] slice
+    const bool stash_ok = in_bounds(stash, (size_t)RB_C * p.Dk * RB_VS * 4, p.stash, p.stash_bytes, p.bounds);
     for (int n = p.Nc - 1; n >= 0; --n) {
         const int64_t t0 = (int64_t)n * RB_C;
         const int len = (int)min((int64_t)RB_C, p.S - t0);
@@ -171,10 +175,13 @@ __global__ void __launch_bounds__(RB_THREADS) rec_bwd_kernel(RbArgs p) {
         stage_chunk<T>(p, st, b, h, t0, len, j0, true, true, tid);
         __syncthreads();
         // recompute the chunk forward from its checkpoint, keeping S_{t-1} (stash) and u_t of every token
+        const bool ck_ok =
+            in_bounds(ck + (int64_t)n * p.Dk * RB_VS, (size_t)p.Dk * RB_VS * 4, p.ckpt, p.ckpt_bytes, p.bounds);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) S[e] = row_ok ? ck[((int64_t)n * p.Dk + c) * RB_VS + 8 * half + e] : 0.f;
+        for (int e = 0; e < 8; ++e)
+            S[e] = (row_ok && ck_ok) ? ck[((int64_t)n * p.Dk + c) * RB_VS + 8 * half + e] : 0.f;
         for (int r = 0; r < len; ++r) {
-            if (row_ok)
+            if (row_ok && stash_ok)
 #pragma unroll
                 for (int e = 0; e < 8; ++e) stash[(size_t)r * p.Dk * RB_VS + soff + e] = S[e];
             fwd_step(p, st, r, c, half, S, red, su, tid);
@@ -184,7 +191,7 @@ __global__ void __launch_bounds__(RB_THREADS) rec_bwd_kernel(RbArgs p) {
         __syncthreads();  // u_t of the last token is read by every thread below
         // the stash of the last RB_NR tokens into the ring (slot r % RB_NR for token r of the chunk)
         auto prefetch = [&](int r) {
-            if (r >= 0 && row_ok) {
+            if (r >= 0 && row_ok && stash_ok) {
                 float *dst = st.ring + (r % RB_NR) * p.Dk * RB_VS + soff;
                 const float *src = stash + (size_t)r * p.Dk * RB_VS + soff;
                 cp_async16(dst, src);
@@ -260,20 +267,29 @@ __global__ void __launch_bounds__(RB_THREADS) rec_bwd_kernel(RbArgs p) {
         // with fp32 atomics, dq, dk, dz and dbeta (no global access in the token steps above)
         __syncthreads();
         const int64_t row0 = (int64_t)b * p.S + t0;
-        for (int idx = tid; idx < len * p.Dk; idx += RB_THREADS) {
+        // the chunk's rows of each output span [(row0 H + h) D, ((row0 + len - 1) H + h) D + D)
+        const int64_t k_lo = (row0 * p.H + h) * p.Dk, k_n = ((int64_t)(len - 1) * p.H) * p.Dk + p.Dk;
+        const int64_t v_lo = (row0 * p.H + h) * p.Dv, v_n = ((int64_t)(len - 1) * p.H) * p.Dv + p.Dv;
+        const int64_t b_lo = row0 * p.H + h, b_n = (int64_t)(len - 1) * p.H + 1;
+        const bool k_ok = in_bounds(p.dq + k_lo, k_n * 4, p.dq, p.nk_bytes, p.bounds) &&
+                          in_bounds(p.dk + k_lo, k_n * 4, p.dk, p.nk_bytes, p.bounds) &&
+                          in_bounds(p.dz + k_lo, k_n * 4, p.dz, p.nk_bytes, p.bounds);
+        const bool v_ok = in_bounds(p.dv + v_lo, v_n * 4, p.dv, p.nv_bytes, p.bounds);
+        const bool b_ok = in_bounds(p.dbeta + b_lo, b_n * 4, p.dbeta, p.nb_bytes, p.bounds);
+        for (int idx = tid; k_ok && idx < len * p.Dk; idx += RB_THREADS) {
             const int r = idx / p.Dk, cc = idx - r * p.Dk;
             const int64_t i = ((row0 + r) * p.H + h) * p.Dk + cc;
             atomicAdd(p.dq + i, st.q[idx]);
             atomicAdd(p.dk + i, st.k[idx]);
             atomicAdd(p.dz + i, st.g[idx]);
         }
-        for (int idx = tid; idx < len * RB_VS; idx += RB_THREADS) {
+        for (int idx = tid; v_ok && idx < len * RB_VS; idx += RB_THREADS) {
             const int r = idx / RB_VS, j = idx - r * RB_VS;
             if (j0 + j < p.Dv) p.dv[((row0 + r) * p.H + h) * p.Dv + j0 + j] = st.v[idx];
         }
-        for (int r = tid; r < len; r += RB_THREADS) atomicAdd(p.dbeta + (row0 + r) * p.H + h, st.b[r]);
+        for (int r = tid; b_ok && r < len; r += RB_THREADS) atomicAdd(p.dbeta + (row0 + r) * p.H + h, st.b[r]);
     }
-    if (p.dS0 && row_ok)
+    if (p.dS0 && row_ok && in_bounds(p.dS0 + (int64_t)bh * p.Dk * p.Dv, (size_t)p.Dk * p.Dv * 4, p.dS0, p.ns_bytes, p.bounds))
 #pragma unroll
         for (int e = 0; e < 8; ++e)
             if (jc + e < p.Dv) p.dS0[((int64_t)bh * p.Dk + c) * p.Dv + jc + e] = dS[e];
@@ -320,6 +336,13 @@ kda_status_t launch_rec_bwd(const kda_recurrent_bwd_args &a, cudaStream_t st) {
     uint8_t *ws = (uint8_t *)a.workspace;
     p.ckpt = reinterpret_cast<float *>(ws);
     p.stash = reinterpret_cast<float *>(ws + (size_t)nbh * p.nslice * p.Nc * a.D_k * RB_VS * sizeof(float));
+    p.ckpt_bytes = (size_t)nbh * p.nslice * p.Nc * a.D_k * RB_VS * sizeof(float);
+    p.stash_bytes = (size_t)nbh * p.nslice * RB_C * a.D_k * RB_VS * sizeof(float);
+    p.nk_bytes = nk;
+    p.nv_bytes = (size_t)nbh * a.S * a.D_v * sizeof(float);
+    p.nb_bytes = nb;
+    p.ns_bytes = (size_t)nbh * a.D_k * a.D_v * sizeof(float);
+    p.bounds = device_bounds_counter();
     const dim3 grid((unsigned)nbh, (unsigned)p.nslice);
     const size_t smem = rec_smem_bytes(a.D_k);
     if (a.dtype == KDA_F32) {

@@ -11,6 +11,7 @@ namespace kda {
 
 // Counts bounded device-side waits that ran out (all kernels of this library).
 __device__ unsigned int g_kda_wait_timeouts;
+__device__ unsigned int g_kda_bounds_errors;  // writes a checked build skipped (always 0 otherwise)
 
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static std::once_flag once;
@@ -90,7 +91,41 @@ unsigned int *device_timeout_counter() {
     return p;
 }
 
+unsigned int *device_bounds_counter() {
+    static std::atomic<unsigned int *> ptrs[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    unsigned int *p = ptrs[dev].load();
+    if (!p) {
+        void *q = nullptr;
+        if (cudaGetSymbolAddress(&q, g_kda_bounds_errors) != cudaSuccess) return nullptr;
+        p = static_cast<unsigned int *>(q);
+        ptrs[dev].store(p);
+    }
+    return p;
+}
+
 }  // namespace kda
+
+extern "C" kda_status_t kda_device_bounds_errors(uint32_t *count, int reset, int *checked_build) {
+    using namespace kda;
+    if (!count) return fail(KDA_ERR_INVALID_ARG, "count is NULL");
+#ifdef KDA_CHECKED
+    if (checked_build) *checked_build = 1;
+#else
+    if (checked_build) *checked_build = 0;
+#endif
+    unsigned int v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_kda_bounds_errors, sizeof(v));
+    if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "reading the bounds counter: %s", cudaGetErrorString(e));
+    *count = v;
+    if (reset) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_kda_bounds_errors, &zero, sizeof(zero));
+        if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "resetting the bounds counter: %s", cudaGetErrorString(e));
+    }
+    return KDA_OK;
+}
 
 extern "C" kda_status_t kda_device_timeouts(uint32_t *count, int reset) {
     using namespace kda;
