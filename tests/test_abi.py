@@ -199,3 +199,22 @@ def test_noalloc_size_check_cannot_be_wrapped():
     assert st == _lib.KDA_ERR_UNSUPPORTED
     assert "scratch" in lib.kda_last_error().decode()
     assert lib.kda_launch_count() == n0
+
+
+def test_checked_build_reports_itself():
+    """build() makes a bounds-checked variant beside the library; each reports which one it is before
+    any CUDA call (here, without a GPU, the counter read itself then fails with KDA_ERR_CUDA)."""
+    import os
+    pkg = os.path.dirname(_lib.LIB_PATH)
+    for name, want in (("libkda.so", 0), ("libkda_checked.so", 1)):
+        path = os.path.join(pkg, name)
+        assert os.path.exists(path), f"{name} missing: run the build"
+        lib = ctypes.CDLL(path)
+        f = lib.kda_device_bounds_errors
+        f.restype = ctypes.c_int
+        f.argtypes = [ctypes.POINTER(ctypes.c_uint32), ctypes.c_int, ctypes.c_void_p]
+        n, chk = ctypes.c_uint32(7), ctypes.c_int(-1)
+        st = f(ctypes.byref(n), 0, ctypes.cast(ctypes.pointer(chk), ctypes.c_void_p))
+        assert chk.value == want
+        assert st in (_lib.KDA_OK, _lib.KDA_ERR_CUDA)
+        assert f(None, 0, None) == _lib.KDA_ERR_INVALID_ARG
