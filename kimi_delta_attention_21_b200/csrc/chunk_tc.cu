@@ -122,6 +122,7 @@ struct PrepArgs {
     uint8_t *ws;
     size_t rec_bytes;        // the records' part of ws (checked builds test the record stores against it)
     unsigned int *bounds;
+    float *lbound;           // per-chunk log-bounds of the transition norm [B*H][Nc] (null: one segment)
     unsigned int *timeouts;
     int *dev_status;
 };
@@ -147,6 +148,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     float *sbeta = reinterpret_cast<float *>(sm + P_BETA);
     float *sgam = reinterpret_cast<float *>(sm + P_GAM);
     const uint32_t in_bytes = 4u * 8192u;  // q, k
+    // the chunk's log-bound of the transition norm: the largest log(alpha) of its tokens (from the decay
+    // group, per warp then per unit) and beta |k|^2 of each token (from the readout)
+    __shared__ float s_gmax_w[8], s_unit_gmax, s_bk[CH];
 
     auto unit_coords = [&](int64_t u, int &n, int &h, int &b) {  // 32-bit: units < 2^31 (host check)
         const uint32_t uu = (uint32_t)u, nc = (uint32_t)p.Nc, hh = (uint32_t)p.H;
@@ -224,6 +228,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                     g[rr] = log_alpha_fast(zv, p.g_min) * (r < len ? 1.f : 0.f);
                 }
             }
+            // the largest log(alpha) among this thread's rows (rows past the end, 0, only occur in the
+            // sequence's last chunk, in the last segment, whose bound no map reads)
+            float gm = g[0];
+#pragma unroll
+            for (int rr = 1; rr < 32; ++rr) gm = fmaxf(gm, g[rr]);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) gm = fmaxf(gm, __shfl_xor_sync(0xffffffffu, gm, off));
+            if ((t & 31) == 0) s_gmax_w[t >> 5] = gm;
             float acc = 0.f;
 #pragma unroll
             for (int rr = 0; rr < 32; ++rr) {
@@ -232,6 +244,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
             }
             qsum[hv * 128 + c] = acc;
             named_sync(3, DTN);
+            if (t == 0) {
+                float m = s_gmax_w[0];
+#pragma unroll
+                for (int w = 1; w < 8; ++w) m = fmaxf(m, s_gmax_w[w]);
+                s_unit_gmax = m;  // read by this unit's readout, one iteration later
+            }
             const float base = hv ? qsum[c] : 0.f;
 #pragma unroll
             for (int rr = 0; rr < 32; ++rr) sG[(hv * 32 + rr) * SG_LD + c] = g[rr] + base;
@@ -509,11 +527,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                     }
                 }
                 float *sA = reinterpret_cast<float *>(sm + P_SA);
+                float kk = 0.f;  // |k_i|^2: the diagonal entry (r = i), whose row and column factors cancel
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const int r = 16 * V + e;
                     sA[r * SA_LD + i] = (i < r) ? sbeta[r] * __uint_as_float(a_[e]) : 0.f;
+                    if (r == i) kk = __uint_as_float(a_[e]);
                 }
+                if (diag) s_bk[i] = sbeta[i] * kk;  // beta_i |k_i|^2, for the chunk's log-bound
             }
             if (warp == 6 || warp == 7) {  // low part of the diagonal column operand x q: row i, block R = i / 16
                 const int il = 32 * (warp - 6) + lane, R = il >> 4;
@@ -551,8 +572,21 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
                         *reinterpret_cast<uint4 *>(sm + P_MT + sw128(i, cc)) = make_uint4(0u, 0u, 0u, 0u);
             }
         }
+        const float gmax_u = s_unit_gmax;  // (this unit's: the next unit's decay rewrites it only below)
         tc_fence_before();
         __syncthreads();
+        if (warp == 12 && p.lbound) {  // (idle in P4) the chunk's log-bound: len tokens of at most gmax_u, and
+                                       // each token's log max(1, |1 - beta |k|^2|), |k|^2 widened by 2^-7 (bf16)
+            float lf = 0.f;
+#pragma unroll
+            for (int k2 = 0; k2 < 2; ++k2) {
+                const float bk = s_bk[lane + 32 * k2];
+                lf += __logf(fmaxf(1.f, fmaxf(fabsf(1.f - bk * (1.f - 0.0078125f)), fabsf(1.f - bk * (1.f + 0.0078125f)))));
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) lf += __shfl_xor_sync(0xffffffffu, lf, off);
+            if (lane == 0) p.lbound[((size_t)b * p.H + h) * p.Nc + n] = (float)min(CH, p.S - n * CH) * gmax_u + lf;
+        }
 
         // ---------------- P4: T = (I + A)^{-1} (fp32) by block doubling: the four diagonal 16x16 blocks by
         // forward substitution, then T_{R,R-1} = -T_RR A_{R,R-1} T_{R-1,R-1} for R = 1, 3, then the lower-left
@@ -681,6 +715,7 @@ struct StateArgs {
     uint8_t *xt;           // map pass: A_g^T as bf16 operand images [B*H][G-1][32 KB]
     float *yt;             // map pass: Y_g [B*H][G-1][128][128]
     size_t sf_bytes, xt_bytes, yt_bytes;  // sizes of Sf, xt, yt (checked builds test the writes against them)
+    const float *lbound;   // map pass: per-chunk log-bounds of the transition norm [B*H][Nc], or null
     unsigned int *bounds;
     float eps;
     unsigned int *timeouts;
@@ -1074,6 +1109,15 @@ chunk_state_kernel(const __grid_constant__ CUtensorMap tmo, const __grid_constan
 // the two chains, so that each chain's register work fills the other's MMA round trips.  Per chain the
 // TMEM columns are S^T fp32 (+0), the bf16 copy of S^T (+128) and PO = S^T (-W)^T (+192); the bf16 V'^T
 // reuses the copy's first 32 columns (the copy is dead once PO is done, V'^T once the update is done).
+//
+// Windows.  Each token's transition S -> (I - beta k k^T) Diag(alpha) S has spectral norm at most
+// max_c alpha_c max(1, |1 - beta |k|^2|), so the segment's linear part A_g and everything before a chunk
+// reach the end state scaled by at most the product of those bounds over the chunks that follow.  The
+// prep leaves each chunk's log-bound in p.lbound.  When the bounds of the segment's last chunks [nb, nc)
+// add up below -WINDOW_LOG (e^-200: below the smallest fp32 number even for states of 1e38), A_g is zero
+// to fp32 and Y_g is the chain over [nb, nc) alone, from zero: chain X is skipped (A_g's image written as
+// zeros) and chain Y runs from chunk nb.  Otherwise (slow decay) both chains run the whole segment.
+constexpr float WINDOW_LOG = 200.f;
 __device__ __forceinline__ constexpr uint32_t mp_base(int c) { return c ? 256u : 0u; }  // chain X, chain Y
 constexpr uint32_t MP_S16 = 128, MP_PO = 192;
 
@@ -1102,6 +1146,7 @@ __global__ void __launch_bounds__(ST_THREADS_MAP, 1) chunk_map_pair_kernel(State
     float *sgam = reinterpret_cast<float *>(sm + ST_GAM);
     const uint8_t *rec0 = p.ws + ((size_t)bh * p.Nc + n0) * REC_BYTES;
     __shared__ volatile int s_fail;
+    __shared__ int s_nb, s_win;  // first chunk the chains run (within the segment); whether it is a window
 
     if (tid == 0) {
         s_fail = 0;
@@ -1112,11 +1157,37 @@ __global__ void __launch_bounds__(ST_THREADS_MAP, 1) chunk_map_pair_kernel(State
     if (warp == 0) {
         tmem_alloc(tmem_slot, ST_TCOLS);
         tmem_relinquish();
+        // the shortest suffix [nb, nc) whose log-bounds add up below -WINDOW_LOG: lane l of a pass takes
+        // chunk top - 1 - l, so a prefix over lanes plus the later passes' sum is a suffix sum
+        int nb = -1;
+        if (p.lbound) {
+            const float *lb = p.lbound + (size_t)bh * p.Nc + n0;
+            float carry = 0.f;
+            for (int top = nc; top > 0 && nb < 0; top -= 32) {
+                const int idx = top - 1 - lane;
+                float v = idx >= 0 ? lb[idx] : 0.f;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, v, off);
+                    if (lane >= off) v += y;
+                }
+                const unsigned hit = __ballot_sync(0xffffffffu, idx >= 0 && carry + v < -WINDOW_LOG);
+                if (hit) nb = top - 1 - (__ffs(hit) - 1);
+                carry += __shfl_sync(0xffffffffu, v, 31);
+            }
+        }
+        if (lane == 0) {
+            s_win = nb >= 0;
+            s_nb = nb >= 0 ? nb : 0;
+        }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    const bool windowed = s_win != 0;
+    const int nb = s_nb, nrun = nc - nb;  // chunks the chains run: nb .. nc - 1
+    const int c0 = windowed ? 1 : 0;      // first chain that runs (chain X only without a window)
     bool ok = true;
     int issued = 0, landed = 0;  // records requested / seen complete (MMA warp)
 
@@ -1127,10 +1198,11 @@ __global__ void __launch_bounds__(ST_THREADS_MAP, 1) chunk_map_pair_kernel(State
             constexpr uint32_t id_s = idesc_f16(128, 128, 0, 1);  // B MN-major
             const uint64_t d_k = smem_desc(smem_u32(sm), 16, 1024, LAYOUT_SW128);
             const uint64_t d_mn = smem_desc(smem_u32(sm), 8192, 1024, LAYOUT_SW128);
-            auto issue_record = [&](int n) {
-                const int stg = n % STG;
+            // (m counts the chunks run, from chunk nb: stages and barrier phases follow m)
+            auto issue_record = [&](int m) {
+                const int stg = m % STG;
                 uint8_t *dst = sm + stg * STB;
-                const uint8_t *src = rec0 + (size_t)n * REC_BYTES;
+                const uint8_t *src = rec0 + (size_t)(nb + m) * REC_BYTES;
                 mbar_arrive_expect_tx(&full[stg], STB + 512);
                 bulk_load(dst, src + REC_WQ, 8192, &full[stg]);
                 bulk_load(dst + 8192, src + REC_WQ + 16384, 8192, &full[stg]);
@@ -1139,15 +1211,15 @@ __global__ void __launch_bounds__(ST_THREADS_MAP, 1) chunk_map_pair_kernel(State
                 bulk_load(sgam + stg * 128, src + REC_GAM, 512, &full[stg]);
                 ++issued;
             };
-            for (int n = 0; n < STG && n < nc; ++n) issue_record(n);
-            for (int n = 0; n < nc; ++n) {
+            for (int m = 0; m < STG && m < nrun; ++m) issue_record(m);
+            for (int m = 0; m < nrun; ++m) {
                 if (s_fail) { ok = false; break; }
-                const uint32_t sgo = (n % STG) * STB;
-                if (!mbar_wait(&full[n % STG], (n / STG) & 1)) { ok = false; break; }
-                landed = n + 1;
+                const uint32_t sgo = (m % STG) * STB;
+                if (!mbar_wait(&full[m % STG], (m / STG) & 1)) { ok = false; break; }
+                landed = m + 1;
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {  // PO_c = S_c^T (-W)^T
-                    if (!mbar_wait(&simg[c], n & 1)) { ok = false; break; }
+                for (int c = c0; c < 2; ++c) {  // PO_c = S_c^T (-W)^T
+                    if (!mbar_wait(&simg[c], m & 1)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t base = tmem + mp_base(c);
 #pragma unroll
@@ -1158,15 +1230,15 @@ __global__ void __launch_bounds__(ST_THREADS_MAP, 1) chunk_map_pair_kernel(State
                     mma_commit(&bar_p[c]);
                 }
                 if (!ok) break;
-                // the stage of record n - 1 is free once chain Y's update of chunk n - 1 is done (the
-                // chain warps read its U^T and e^{G_C} before they signal that update's V')
-                if (n >= 1 && n + STG - 1 < nc) {
-                    if (!mbar_wait(&bar_s[1], (n - 1) & 1)) { ok = false; break; }
-                    issue_record(n + STG - 1);
+                // the stage of record m - 1 is free once chain Y's update of it is done (the chain warps
+                // read its U^T and e^{G_C} before they signal that update's V')
+                if (m >= 1 && m + STG - 1 < nrun) {
+                    if (!mbar_wait(&bar_s[1], (m - 1) & 1)) { ok = false; break; }
+                    issue_record(m + STG - 1);
                 }
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {  // S_c^T += V'_c^T K~
-                    if (!mbar_wait(&vimg[c], n & 1)) { ok = false; break; }
+                for (int c = c0; c < 2; ++c) {  // S_c^T += V'_c^T K~
+                    if (!mbar_wait(&vimg[c], m & 1)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t base = tmem + mp_base(c);
 #pragma unroll
@@ -1182,8 +1254,8 @@ __global__ void __launch_bounds__(ST_THREADS_MAP, 1) chunk_map_pair_kernel(State
         // ======================================== chain register work (warps 0-7), both chains
         const uint32_t lrow = (uint32_t)(32 * q4) << 16;
         const int j = 32 * q4 + lane;  // value column (TMEM lane) of this thread
-        {   // entering states -> TMEM: X = identity, Y = S_0 (g = 0) or zero
-            const float *s_in = (g == 0 && p.S0) ? p.S0 + (size_t)bh * DD * DD : nullptr;
+        {   // entering states -> TMEM: X = identity, Y = S_0 (segment 0 without a window) or zero
+            const float *s_in = (g == 0 && p.S0 && !windowed) ? p.S0 + (size_t)bh * DD * DD : nullptr;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 uint32_t su[32];
@@ -1203,15 +1275,15 @@ __global__ void __launch_bounds__(ST_THREADS_MAP, 1) chunk_map_pair_kernel(State
             tmem_wait_st();
         }
 
-        for (int n = 0; n < nc && ok; ++n) {
+        for (int m = 0; m < nrun && ok; ++m) {  // chunk nb + m
             if (s_fail) { ok = false; break; }
-            const int stg = n % STG;
-            if (!mbar_wait(&full[stg], (n / STG) & 1)) { ok = false; break; }
+            const int stg = m % STG;
+            if (!mbar_wait(&full[stg], (m / STG) & 1)) { ok = false; break; }
             const float4 *g4 = reinterpret_cast<const float4 *>(sgam + stg * 128 + 64 * hf);
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {  // S_n^T -> bf16 copy; S^T <- S^T Diag(e^{G_C})
+            for (int c = c0; c < 2; ++c) {  // S^T -> bf16 copy; S^T <- S^T Diag(e^{G_C})
                 const uint32_t base = tmem + lrow + mp_base(c);
-                if (n >= 1 && !mbar_wait(&bar_s[c], (n - 1) & 1)) { ok = false; break; }
+                if (m >= 1 && !mbar_wait(&bar_s[c], (m - 1) & 1)) { ok = false; break; }
                 tc_fence_after();
                 uint32_t sv[64];
                 tmem_ld_32x32b_x32(base + 64 * hf, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
@@ -1243,7 +1315,7 @@ __global__ void __launch_bounds__(ST_THREADS_MAP, 1) chunk_map_pair_kernel(State
             }
             if (!ok) break;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {  // V'^T = [U^T] - (W S_n)^T -> bf16, over the dead S copy
+            for (int c = c0; c < 2; ++c) {  // V'^T = [U^T] - (W S)^T -> bf16, over the dead S copy
                 const uint32_t base = tmem + lrow + mp_base(c);
                 uint4 uu[4];
                 if (c == 1) {
@@ -1251,7 +1323,7 @@ __global__ void __launch_bounds__(ST_THREADS_MAP, 1) chunk_map_pair_kernel(State
 #pragma unroll
                     for (int k = 0; k < 4; ++k) uu[k] = *reinterpret_cast<const uint4 *>(ut + sw128(j, 4 * hf + k));
                 }
-                if (!mbar_wait(&bar_p[c], n & 1)) { ok = false; break; }
+                if (!mbar_wait(&bar_p[c], m & 1)) { ok = false; break; }
                 tc_fence_after();
                 uint32_t pv[32], pk[16];
                 tmem_ld_32x32b_x32(base + MP_PO + 32 * hf, pv);
@@ -1277,8 +1349,9 @@ __global__ void __launch_bounds__(ST_THREADS_MAP, 1) chunk_map_pair_kernel(State
                 if (lane == 0) mbar_arrive(&vimg[c]);
             }
         }
-        if (ok && nc > 0) {
-            if (!mbar_wait(&bar_s[0], (nc - 1) & 1) || !mbar_wait(&bar_s[1], (nc - 1) & 1)) ok = false;
+        if (ok && nrun > 0) {
+            if ((!windowed && !mbar_wait(&bar_s[0], (nrun - 1) & 1)) || !mbar_wait(&bar_s[1], (nrun - 1) & 1))
+                ok = false;
             tc_fence_after();
         }
         if (ok && in_bounds(p.yt + ((size_t)bh * (p.G - 1) + g) * DD * DD, DD * DD * 4, p.yt, p.yt_bytes, p.bounds)) {
@@ -1293,7 +1366,14 @@ __global__ void __launch_bounds__(ST_THREADS_MAP, 1) chunk_map_pair_kernel(State
 #pragma unroll
                 for (int e = 0; e < 32; ++e) dst[(size_t)e * DD] = __uint_as_float(sv[e]);
             }
-            if (g >= 1 && in_bounds(p.xt + ((size_t)bh * (p.G - 1) + g) * 32768, 32768, p.xt, p.xt_bytes, p.bounds)) {
+            if (g >= 1 && windowed &&
+                in_bounds(p.xt + ((size_t)bh * (p.G - 1) + g) * 32768, 32768, p.xt, p.xt_bytes, p.bounds)) {
+                // A_g = 0 to fp32 (the window's bound): its image is zeros, 128 bytes a thread
+                uint4 *img = reinterpret_cast<uint4 *>(p.xt + ((size_t)bh * (p.G - 1) + g) * 32768) + tid * 8;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) img[k] = make_uint4(0u, 0u, 0u, 0u);
+            } else if (g >= 1 &&
+                       in_bounds(p.xt + ((size_t)bh * (p.G - 1) + g) * 32768, 32768, p.xt, p.xt_bytes, p.bounds)) {
                 // A_g^T as the combine pass's MN-major B operand: image row j = lane j
                 uint8_t *img = p.xt + ((size_t)bh * (p.G - 1) + g) * 32768;
 #pragma unroll
@@ -1535,7 +1615,7 @@ namespace {
 // A_g^T (bf16 images) and Y_g, and the segments' entering states.
 struct TcLayout {
     int G, L;
-    size_t xt, yt, seg, total;
+    size_t xt, yt, seg, lb, total;
 };
 
 TcLayout tc_layout(const kda_chunk_args &a) {
@@ -1548,13 +1628,19 @@ TcLayout tc_layout(const kda_chunk_args &a) {
     const size_t nmap = t.G > 1 ? (size_t)BH * (t.G - 1) : 0;
     t.yt = t.xt + nmap * 32768;
     t.seg = t.yt + nmap * DD * DD * 4;
-    t.total = t.seg + (t.G > 1 ? (size_t)BH * t.G * DD * DD * 4 : 0);
+    t.lb = t.seg + (t.G > 1 ? (size_t)BH * t.G * DD * DD * 4 : 0);
+    t.total = t.lb + (t.G > 1 ? (size_t)BH * Nc * 4 : 0);  // per-chunk log-bounds, for the map pass's windows
     return t;
 }
 
 }  // namespace
 
 size_t chunk_tc_workspace(const kda_chunk_args &a) { return tc_layout(a).total; }
+
+float *tc::chunk_log_bounds(const kda_chunk_args &a) {
+    const TcLayout lay = tc_layout(a);
+    return lay.G > 1 ? reinterpret_cast<float *>((uint8_t *)a.workspace + lay.lb) : nullptr;
+}
 
 kda_status_t tc::launch_chunk_state_pass(const kda_chunk_args &a, cudaStream_t st) {
     const int64_t Nc = (a.S + CH - 1) / CH;
@@ -1592,6 +1678,7 @@ kda_status_t tc::launch_chunk_state_pass(const kda_chunk_args &a, cudaStream_t s
         sa.yt_bytes = nmap * DD * DD * 4;
         sa.bounds = device_bounds_counter();
     }
+    sa.lbound = (Nc > 0 && lay.G > 1) ? reinterpret_cast<const float *>(ws + lay.lb) : nullptr;
     sa.eps = a.eps;
     sa.timeouts = device_timeout_counter();
     sa.dev_status = a.dev_status;
@@ -1628,6 +1715,7 @@ kda_status_t launch_chunk_tc(const kda_chunk_args &a, cudaStream_t st) {
         pa.ws = (uint8_t *)a.workspace;
         pa.rec_bytes = (size_t)pa.units * REC_BYTES;
         pa.bounds = device_bounds_counter();
+        pa.lbound = tc::chunk_log_bounds(a);
         pa.timeouts = timeouts;
         pa.dev_status = a.dev_status;
         const int sms = device_sms();

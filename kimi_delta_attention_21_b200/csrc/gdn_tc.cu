@@ -66,6 +66,7 @@ struct GdnArgs {
     uint8_t *ws;
     size_t rec_bytes;              // the records' part of ws (checked builds test the record stores against it)
     unsigned int *bounds;
+    float *lbound;                 // per-chunk log-bounds of the transition norm [B*H][Nc] (null: one segment)
     unsigned int *timeouts;
     int *dev_status;
 };
@@ -88,6 +89,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
     float *sgam = sG + 192;
     float *wsum = sG + 320;
     float *sgn = sG + 384, *sbn = sG + 448;  // the next unit's log-decay and beta, loaded during the inverse
+    __shared__ float s_lf;  // sum over the chunk's tokens of log max(1, |1 - beta |k|^2|)
 
     auto unit_coords = [&](int64_t u, int &n, int &h, int &b) {  // 32-bit: units < 2^31 (host check)
         const uint32_t uu = (uint32_t)u, nc = (uint32_t)p.Nc, hh = (uint32_t)p.H;
@@ -162,6 +164,7 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             g_cur = sgn[tid];
             b_cur = sbn[tid];
         }
+        if (tid == 0) s_lf = 0.f;
         // ---- cumulative log-decay over the chunk (warps 0-1: one token per thread), e^G, beta
         if (tid < CH) {
             float x = g_cur;
@@ -233,9 +236,20 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
             if (warp < 2) {  // A[r, i] = beta_r e^{G_r - G_i} k_r . k_i for i < r
                 float *sA = reinterpret_cast<float *>(sm + G_SA) + row * SA_LD;
                 const float br = sbeta[row];
+                float kk = 0.f;  // |k_row|^2, the diagonal entry
 #pragma unroll
-                for (int i = 0; i < 64; ++i)
+                for (int i = 0; i < 64; ++i) {
                     sA[i] = br * (fexp(fminf(Gr - sG[i], 0.f)) * (i < row ? 1.f : 0.f)) * __uint_as_float(v[i]);
+                    if (i == row) kk = __uint_as_float(v[i]);
+                }
+                if (p.lbound) {  // this token's log max(1, |1 - beta |k|^2|), |k|^2 widened by 2^-7;
+                                 // summed over the warp, one shared add per warp
+                    const float lo = kk * (1.f - 0.0078125f), hi = kk * (1.f + 0.0078125f);
+                    float lf = __logf(fmaxf(1.f, fmaxf(fabsf(1.f - br * lo), fabsf(1.f - br * hi))));
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) lf += __shfl_xor_sync(0xffffffffu, lf, off);
+                    if (lane == 0 && lf != 0.f) atomicAdd(&s_lf, lf);
+                }
             } else {         // M^T[i, r] = e^{G_r - G_i} q_r . k_i for i <= r (row = i)
 #pragma unroll
                 for (int k8 = 0; k8 < 8; ++k8) {
@@ -265,6 +279,9 @@ gdn_prep_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ 
         tc_fence_before();
         ok = __syncthreads_and(ok);
         if (!ok) break;
+        if (tid == 256 && p.lbound)  // (warp 8, idle in the inverse) the chunk's log-bound: its exact log-decay
+                                     // sum (one alpha per token) and the |k| terms
+            p.lbound[((size_t)b * p.H + h) * p.Nc + n] = sG[CH - 1] + s_lf;
         if (tid == 32 && in_bounds(rec, REC_BYTES, p.ws, p.rec_bytes, p.bounds)) {
             bulk_store(rec + REC_KT, sm + G_KT, 16384);
             bulk_store(rec + REC_MT, sm + G_MT, 8192);
@@ -392,6 +409,7 @@ kda_status_t launch_gdn_tc(const kda_chunk_args &a, cudaStream_t st) {
         ga.ws = (uint8_t *)a.workspace;
         ga.rec_bytes = (size_t)ga.units * REC_BYTES;
         ga.bounds = device_bounds_counter();
+        ga.lbound = tc::chunk_log_bounds(a);
         ga.timeouts = device_timeout_counter();
         ga.dev_status = a.dev_status;
         int dev = 0, sms = 148;

@@ -240,5 +240,10 @@ kda_status_t make_tmap_tokens(CUtensorMap *m, const void *base, int H, int64_t S
 // the per-chunk records in a.workspace, which a prep kernel has written for every (b, h, chunk).
 kda_status_t launch_chunk_state_pass(const kda_chunk_args &a, cudaStream_t st);
 
+// Where a prep leaves each chunk's log-bound of the transition norm ([B*H][Nc] fp32 in a.workspace: the
+// sum over its tokens of log(max_c alpha_c) + log(max(1, |1 - beta |k|^2|)), or an upper bound of it),
+// or null when the sequence is one segment (the map pass, which reads them, does not run).
+float *chunk_log_bounds(const kda_chunk_args &a);
+
 }  // namespace tc
 }  // namespace kda

@@ -158,7 +158,8 @@ def test_workspace_query_needs_no_device():
 
 def _expected_tc_workspace(B, S, H, sms=148):
     """Workspace of the tensor-core chunk engine, from the rule it follows: per-chunk records, and,
-    with G segments, BH (G - 1) map slots (A image + Y) and BH G entering states, G the
+    with G segments, BH (G - 1) map slots (A image + Y), BH G entering states and a 4-byte log-bound
+    per chunk, G the
     largest count for which the chain pass (BH G CTAs, so also the map pass, BH (G - 1) CTAs) fits
     in one wave, at least 4 chunks per segment, and no empty segment."""
     rec = 74240
@@ -169,8 +170,8 @@ def _expected_tc_workspace(B, S, H, sms=148):
     L = (nc + g - 1) // g
     g = (nc + L - 1) // L
     ws = bh * nc * rec
-    if g > 1:
-        ws += bh * (g - 1) * (32768 + 65536) + bh * g * 128 * 128 * 4
+    if g > 1:  # segment maps (A image + Y), entering states, per-chunk log-bounds for the map windows
+        ws += bh * (g - 1) * (32768 + 65536) + bh * g * 128 * 128 * 4 + bh * nc * 4
     return ws, g
 
 

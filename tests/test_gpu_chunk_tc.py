@@ -301,3 +301,24 @@ def test_tc_random_shapes(K, seed):
     else:
         assert_bf16_outputs(to_np(o), o_ref, "o~, " + what)
     assert_bf16_state(to_np(sf), s_ref, "final_state, " + what)
+
+
+def test_tc_segment_windows(K):
+    """Strong decay (z shifted by +5): every chunk's log-bound of the transition norm is below -100 (checked
+    here from the same inputs: 64 tokens of at most the chunk's largest log(alpha); unit keys and beta < 1
+    add nothing), so each segment's map runs a window of its last two or three chunks and writes A_g = 0.
+    The segmented state pass (8 segments of 8 chunks) still matches the oracle."""
+    w = small("win", 1, 4096, 16, 128, 128, 16, "bf16", seed=77, s0_std=0.5)
+    inp = ki.make_inputs(w)
+    inp["z"] = ki.round_bf16(inp["z"].astype(np.float64) + 5.0).astype(inp["z"].dtype)
+    g = w.g_min / (1.0 + np.exp(-inp["z"].astype(np.float64)))            # (B, S, H, D_k)
+    per_chunk = 64 * g.reshape(1, 64, 64, 16, 128).max(axis=(2, 4))        # (B, chunks, H)
+    assert per_chunk.max() < -100.0
+    d = upload(inp, w)
+    o, sf = K.chunk_fwd(d["q"], d["k"], d["v"], d["beta"], z=d["z"], initial_state=d["S0"], engine="tc")
+    torch.cuda.synchronize()
+    assert _timeouts(K) == 0
+    o_ref, s_ref = oracle.recurrence(inp["q"], inp["k"], inp["v"], inp["beta"], z=inp["z"], g_min=w.g_min,
+                                     initial_state=inp["S0"])
+    assert_bf16_outputs(to_np(o), o_ref, "o~")
+    assert_bf16_state(to_np(sf), s_ref, "final_state")
