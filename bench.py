@@ -706,6 +706,8 @@ def run_ours(args, rank, world, local):
         "wall_s_timed_region": round(head_tm["wall"], 4),
         "workloads": records,
     }
+    if "gdn" in rec:
+        line["gdn"] = rec["gdn"]
     if "cpu_baseline" in rec:
         line["cpu_baseline"] = rec["cpu_baseline"]
     return line
