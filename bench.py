@@ -484,10 +484,17 @@ def run_e2e(K, torch, w, d, steps, world, dev):
             "api": "kimi_delta_attention_21_b200.kda_forward (pinned host tensors in and out)"}
 
 
-def time_backward(K, torch, w, d, warmup, world, dev, flush, lib, steps=3):
-    """The recurrent backward (kda_recurrent_bwd) on the workload: gradients of the
-    core recurrence w.r.t. q, k, v, beta, z and the initial state from a seeded
-    dL/do~ and dL/dS_T.  Exact fp32, token by token (not the chunkwise form)."""
+BACKWARD_ENTRY = {
+    "recurrent_bwd": "kda_recurrent_bwd (exact fp32, recurrent form with 64-token checkpoints)",
+    "chunk_bwd": "kda_chunk_bwd (exact fp32, chunk form: chunks in parallel, state and its gradient in order)",
+}
+
+
+def time_backward(K, torch, w, d, warmup, world, dev, flush, lib, steps=3, engine="recurrent_bwd"):
+    """A backward entry point on the workload: gradients of the core recurrence
+    w.r.t. q, k, v, beta, z and the initial state from a seeded dL/do~ and
+    dL/dS_T, by the recurrent form (kda_recurrent_bwd) or the chunk form
+    (kda_chunk_bwd)."""
     g = torch.Generator(device=dev)
     g.manual_seed(w.seed + 99)
     d_o = torch.randn((w.B, w.S, w.H, w.Dv), generator=g, device=dev).to(d["q"].dtype)
@@ -495,8 +502,8 @@ def time_backward(K, torch, w, d, warmup, world, dev, flush, lib, steps=3):
     ws = None  # (the binding allocates the outputs and the workspace per call)
 
     def one():
-        return K.recurrent_bwd(d["q"], d["k"], d["v"], d["beta"], d_o, z=d["z"], g_min=w.g_min,
-                               initial_state=d["S0"], d_final_state=d_st, workspace=ws)
+        return getattr(K, engine)(d["q"], d["k"], d["v"], d["beta"], d_o, z=d["z"], g_min=w.g_min,
+                                  initial_state=d["S0"], d_final_state=d_st, workspace=ws)
 
     for _ in range(max(1, warmup // 3)):
         one()
@@ -511,8 +518,7 @@ def time_backward(K, torch, w, d, warmup, world, dev, flush, lib, steps=3):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     (t,) = reduce_max([e0.elapsed_time(e1) / steps * 1e-3], world, dev)
-    return {"entry_point": "kda_recurrent_bwd (exact fp32, recurrent form with 64-token checkpoints)",
-            "ms": round(t * 1e3, 3), "tokens_per_s": round(w.B * w.S * world / t, 1),
+    return {"entry_point": BACKWARD_ENTRY[engine], "ms": round(t * 1e3, 3), "tokens_per_s": round(w.B * w.S * world / t, 1),
             "gpu_launches_per_call": int((lib.kda_launch_count() - n0) // steps)}
 
 
@@ -656,8 +662,10 @@ def run_ours(args, rank, world, local):
     if "prefill_4k" in only and not args.no_backward:
         w = rank_workload("prefill_4k", rank)
         d = ki.device_inputs(w, dev)
-        records.setdefault("prefill_4k", {})["backward"] = time_backward(K, torch, w, d, args.warmup, world, dev,
-                                                                         flush, lib)
+        rb = records.setdefault("prefill_4k", {})
+        rb["backward"] = time_backward(K, torch, w, d, args.warmup, world, dev, flush, lib)
+        rb["chunk_backward"] = time_backward(K, torch, w, d, args.warmup, world, dev, flush, lib, engine="chunk_bwd")
+        rb["chunk_backward"]["recurrent_over_chunk_time"] = round(rb["backward"]["ms"] / rb["chunk_backward"]["ms"], 2)
         del d
         torch.cuda.empty_cache()
 

@@ -239,6 +239,27 @@ kda_status_t kda_recurrent_bwd_workspace_size(const kda_recurrent_bwd_args *args
 kda_status_t kda_recurrent_bwd(const kda_recurrent_bwd_args *args);
 
 /*
+ * kda_chunk_bwd — the same gradients as kda_recurrent_bwd (same arguments,
+ * same outputs), computed in the chunk form of the recurrence (Kimi Linear
+ * report, section 3.1 and appendix B, Props. 1-2: the WY/UT representation the
+ * pages motivate by training).  Chunks of 64 tokens run in parallel for the
+ * per-chunk algebra (decayed K K^T and Q K^T, T = (I + A)^{-1} by forward
+ * substitution, W, U, and every per-chunk gradient); only the state and its
+ * gradient pass through the chunks in order (one 16-value-column slice of
+ * the state per CTA).  Exact fp32 arithmetic; every decay factor is the
+ * exponential of a difference <= 0, so any g_min works.  The reverse-mode
+ * lines it evaluates are listed in csrc/chunk_bwd.cu.
+ * Outputs are fully written (no zeroing needed).  The workspace holds one
+ * record per (b, h, chunk): 4 (C (4 D_k + 3 D_v + 3 C) + 2 D_k D_v
+ * + ceil(D_v / 16) D_k) bytes with C = 64, rounded up to 16 bytes (404 KB at
+ * D_k = D_v = 128); query it with kda_chunk_bwd_workspace_size.
+ * Errors: as kda_recurrent_bwd; UNSUPPORTED if B*H*chunks exceeds 2^31 - 1.
+ */
+kda_status_t kda_chunk_bwd_workspace_size(const kda_recurrent_bwd_args *args, size_t *bytes);
+
+kda_status_t kda_chunk_bwd(const kda_recurrent_bwd_args *args);
+
+/*
  * kda_dplr_recurrent_fwd — the general diagonal-plus-low-rank recurrence of the
  * "Diagonal-Plus-Low-Rank Matrices and Kimi Delta Attention" post (sections 1
  * and 3), the comparator of the KDA engines:

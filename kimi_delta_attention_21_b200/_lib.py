@@ -93,6 +93,8 @@ SIGNATURES = {
     "kda_decode_step": (ctypes.c_int, [ctypes.POINTER(DecodeArgs)]),
     "kda_recurrent_bwd_workspace_size": (ctypes.c_int, [ctypes.POINTER(RecBwdArgs), ctypes.POINTER(ctypes.c_size_t)]),
     "kda_recurrent_bwd": (ctypes.c_int, [ctypes.POINTER(RecBwdArgs)]),
+    "kda_chunk_bwd_workspace_size": (ctypes.c_int, [ctypes.POINTER(RecBwdArgs), ctypes.POINTER(ctypes.c_size_t)]),
+    "kda_chunk_bwd": (ctypes.c_int, [ctypes.POINTER(RecBwdArgs)]),
     "kda_dplr_recurrent_fwd": (ctypes.c_int, [ctypes.POINTER(DplrArgs)]),
     "kda_norm_gate": (ctypes.c_int, [_p, _p, _i64, _i32, _i32, _f32, _p, ctypes.c_int, _p]),
     "kda_out_proj": (ctypes.c_int, [_p, _p, _i64, _i32, _i32, _p, ctypes.c_int, _p]),

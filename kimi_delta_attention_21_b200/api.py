@@ -134,6 +134,20 @@ def recurrent_bwd(q, k, v, beta, d_o, *, z=None, log_decay=None, g_min=-5.0, ini
     (B,S,H,D_v) and d_final_state = dL/dS_T (B,H,D_k,D_v) or None, returns a dict
     of fp32 tensors dq, dk, dv, dbeta, dz (d/dz, or d/dlog_decay when log_decay is
     given) and d_initial_state (or None)."""
+    return _bwd("kda_recurrent_bwd", q, k, v, beta, d_o, z, log_decay, g_min, initial_state, d_final_state,
+                want_d_initial_state, workspace)
+
+
+def chunk_bwd(q, k, v, beta, d_o, *, z=None, log_decay=None, g_min=-5.0, initial_state=None,
+              d_final_state=None, want_d_initial_state=True, workspace=None):
+    """The same gradients as ``recurrent_bwd``, in the chunk form (kda_chunk_bwd:
+    chunks in parallel, only the state and its gradient carried in order)."""
+    return _bwd("kda_chunk_bwd", q, k, v, beta, d_o, z, log_decay, g_min, initial_state, d_final_state,
+                want_d_initial_state, workspace)
+
+
+def _bwd(entry, q, k, v, beta, d_o, z, log_decay, g_min, initial_state, d_final_state, want_d_initial_state,
+         workspace):
     _dev(q, "q")
     dt = q.dtype
     B, S, H, Dk = q.shape
@@ -161,7 +175,7 @@ def recurrent_bwd(q, k, v, beta, d_o, *, z=None, log_decay=None, g_min=-5.0, ini
                    workspace_bytes=0, stream=_stream(q.device))
     lib = _lib.load()
     n = ctypes.c_size_t(0)
-    check("kda_recurrent_bwd_workspace_size", lib.kda_recurrent_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)))
+    check(entry + "_workspace_size", getattr(lib, entry + "_workspace_size")(ctypes.byref(a), ctypes.byref(n)))
     ws = workspace
     if n.value:
         if ws is None:
@@ -169,7 +183,7 @@ def recurrent_bwd(q, k, v, beta, d_o, *, z=None, log_decay=None, g_min=-5.0, ini
         _dev(ws, "workspace", torch.uint8)
         a.workspace = _ptr(ws)
         a.workspace_bytes = ws.numel()
-    check("kda_recurrent_bwd", lib.kda_recurrent_bwd(ctypes.byref(a)))
+    check(entry, getattr(lib, entry)(ctypes.byref(a)))
     if log_decay is not None:
         out["dlog_decay"] = out.pop("dz")
     return out

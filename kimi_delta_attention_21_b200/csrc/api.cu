@@ -271,10 +271,16 @@ kda_status_t kda_recurrent_bwd_workspace_size(const kda_recurrent_bwd_args *a, s
     return KDA_OK;
 }
 
-kda_status_t kda_recurrent_bwd(const kda_recurrent_bwd_args *a) {
+kda_status_t kda_chunk_bwd_workspace_size(const kda_recurrent_bwd_args *a, size_t *bytes) {
     g_err[0] = 0;
+    if (!bytes) return fail(KDA_ERR_INVALID_ARG, "bytes is NULL");
     KDA_TRY(rec_bwd_validate(a));
-    if (a->B == 0) return KDA_OK;
+    *bytes = chunk_bwd_workspace(a->B, a->S, a->H, a->D_k, a->D_v);
+    return KDA_OK;
+}
+
+// The pointer, workspace and overlap checks both backward entry points share (need: the workspace bytes).
+static kda_status_t bwd_check_buffers(const kda_recurrent_bwd_args *a, size_t need) {
     const size_t es = esize(a->dtype);
     const size_t nk = (size_t)a->B * a->S * a->H * a->D_k, nv = (size_t)a->B * a->S * a->H * a->D_v;
     const size_t nb = (size_t)a->B * a->S * a->H, ns = (size_t)a->B * a->H * a->D_k * a->D_v * 4;
@@ -296,7 +302,6 @@ kda_status_t kda_recurrent_bwd(const kda_recurrent_bwd_args *a) {
     KDA_OPT_PTR(a->d_final_state, "d_final_state", 4);
     KDA_OPT_PTR(a->d_initial_state, "d_initial_state", 4);
     KDA_OPT_PTR(a->workspace, "workspace", 256);
-    const size_t need = rec_bwd_workspace(a->B, a->S, a->H, a->D_k, a->D_v);
     if (a->S > 0 && need > 0 && (!a->workspace || a->workspace_bytes < need))
         return fail(KDA_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", need,
                     a->workspace ? a->workspace_bytes : (size_t)0);
@@ -318,7 +323,23 @@ kda_status_t kda_recurrent_bwd(const kda_recurrent_bwd_args *a) {
             if (&o2 != &o && o2.p && overlap(o.p, o.n, o2.p, o2.n))
                 return fail(KDA_ERR_INVALID_ARG, "outputs %s and %s overlap", o.name, o2.name);
     }
+    return KDA_OK;
+}
+
+kda_status_t kda_recurrent_bwd(const kda_recurrent_bwd_args *a) {
+    g_err[0] = 0;
+    KDA_TRY(rec_bwd_validate(a));
+    if (a->B == 0) return KDA_OK;
+    KDA_TRY(bwd_check_buffers(a, rec_bwd_workspace(a->B, a->S, a->H, a->D_k, a->D_v)));
     return launch_rec_bwd(*a, (cudaStream_t)a->stream);
+}
+
+kda_status_t kda_chunk_bwd(const kda_recurrent_bwd_args *a) {
+    g_err[0] = 0;
+    KDA_TRY(rec_bwd_validate(a));
+    if (a->B == 0) return KDA_OK;
+    KDA_TRY(bwd_check_buffers(a, chunk_bwd_workspace(a->B, a->S, a->H, a->D_k, a->D_v)));
+    return launch_chunk_bwd(*a, (cudaStream_t)a->stream);
 }
 
 kda_status_t kda_dplr_recurrent_fwd(const kda_dplr_args *a) {

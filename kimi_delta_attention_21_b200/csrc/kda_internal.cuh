@@ -94,6 +94,10 @@ kda_status_t launch_gdn_tc(const kda_chunk_args &a, cudaStream_t st);
 size_t rec_bwd_workspace(int64_t B, int64_t S, int H, int Dk, int Dv);
 kda_status_t launch_rec_bwd(const kda_recurrent_bwd_args &a, cudaStream_t st);
 
+// Chunkwise backward (exact fp32): per-chunk records, forward and backward state chains.
+size_t chunk_bwd_workspace(int64_t B, int64_t S, int H, int Dk, int Dv);
+kda_status_t launch_chunk_bwd(const kda_recurrent_bwd_args &a, cudaStream_t st);
+
 // General DPLR recurrence, token by token (the comparator).
 kda_status_t launch_dplr(const kda_dplr_args &a, cudaStream_t st);
 

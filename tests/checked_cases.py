@@ -1,7 +1,7 @@
 """The calls the checked-build test runs, shared by the test and the child
 process that runs them on libkda_checked.so: the tensor-core chunk engine on
 segmented sequences (maps, combine, chains; z and log-decay inputs, gate), the
-GDN engine, the recurrent backward and the DPLR comparator.  As a script:
+GDN engine, the recurrent and chunkwise backward and the DPLR comparator.  As a script:
 `python tests/checked_cases.py OUT.npz` runs them on the library the binding
 loads (KDA_LIBRARY picks it) and saves the results with the device counters."""
 import ctypes
@@ -62,6 +62,12 @@ def run_cases():
     for n, t in grads.items():
         if t is not None:
             keep("bwd_" + n, t)
+    # chunkwise backward on the same inputs (three chunks, ragged)
+    grads = K.chunk_bwd(d["q"], d["k"], d["v"], d["beta"], d_o, z=d["z"], initial_state=d["S0"],
+                        d_final_state=d_st)
+    for n, t in grads.items():
+        if t is not None:
+            keep("bwd_chunk_" + n, t)
     # DPLR comparator (two chunks, ragged)
     w = small("chk5", 1, 100, 2, 128, 128, 16, "bf16", seed=49, s0_std=0.1)
     d = upload(ki.make_inputs(w), w)
