@@ -41,7 +41,8 @@ namespace kda {
 namespace {
 
 constexpr int CB_C = 64;    // tokens per chunk
-constexpr int CB_NT = 256;  // threads per CTA
+constexpr int CB_NT = 256;   // threads per CTA of the chain kernels
+constexpr int CB_NTC = 512;  // threads per CTA of the per-chunk kernels
 constexpr int CB_VS = 16;   // value columns per chain CTA
 
 __host__ __device__ inline int cb_pad8(int x) { return (x + 7) & ~7; }
@@ -125,6 +126,78 @@ __device__ __forceinline__ int64_t cb_idx(const CbArgs &p, const CbUnit &w, int 
     return (((int64_t)w.b * p.S + w.t0 + r) * p.H + w.h) * D + c;
 }
 
+// Staging into shared memory.  Record blocks (fp32) go by cp.async, every element of a tile in flight at
+// once; dst[r * ld + c] = src[r * D + c] for r < rows, c < D, and zero for r < rows_p, c < D_p outside
+// that (the padding the products read).  16-byte copies where D, D_p, ld and both addresses allow them.
+// (r, c) advance by a fixed step per pass: no division per element.
+__device__ __forceinline__ void cb_copy(float *dst, int ld, const float *src, int rows, int D, int rows_p,
+                                        int D_p) {
+    const int nt = blockDim.x;
+    const bool wide = ((D | D_p | ld) & 3) == 0 &&
+                      ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15) == 0;
+    const int e = wide ? 4 : 1, W = D_p / e, n = rows_p * W, sr = nt / W, sc = nt - sr * W;
+    int r = threadIdx.x / W, c = threadIdx.x - r * W;
+    for (int idx = threadIdx.x; idx < n; idx += nt) {
+        const bool in = r < rows && e * c < D;
+        const float *g = src + (in ? (int64_t)r * D + e * c : 0);
+        if (wide) cp_async16_fill(dst + r * ld + e * c, g, in);
+        else cp_async4(dst + r * ld + c, g, in);
+        c += sc;
+        r += sr;
+        if (c >= W) {
+            c -= W;
+            ++r;
+        }
+    }
+}
+// columns j0 .. j0 + 15 of a [rows][D] block into [rows][16] (zero past D)
+__device__ __forceinline__ void cb_copy_cols(float *dst, const float *src, int rows, int D, int j0) {
+    const int nt = blockDim.x;
+    const bool wide = ((D | j0) & 3) == 0 &&
+                      ((reinterpret_cast<uintptr_t>(src) | reinterpret_cast<uintptr_t>(dst)) & 15) == 0;
+    const int e = wide ? 4 : 1, W = CB_VS / e, n = rows * W;
+    for (int idx = threadIdx.x; idx < n; idx += nt) {
+        const int r = idx / W, c = idx - r * W;  // (W is 4 or 16: a shift)
+        const bool in = j0 + e * c < D;
+        const float *g = src + (in ? (int64_t)r * D + j0 + e * c : 0);
+        if (wide) cp_async16_fill(dst + r * CB_VS + e * c, g, in);
+        else cp_async4(dst + r * CB_VS + c, g, in);
+    }
+}
+// Token rows of an input tensor (rs elements from one row to the next), converted to fp32, times
+// e^{gsrc[r * D + c]} when gsrc is given (a record block): rows < valid, columns < D; zero elsewhere up
+// to rows x D_p.  Eight loads in flight per thread.
+template <typename T>
+__device__ __forceinline__ void cb_load_rows(float *dst, int ld, const T *src, int64_t rs, int rows, int valid,
+                                             int D, int D_p, const float *gsrc = nullptr) {
+    const int nt = blockDim.x, n = rows * D_p, sr = nt / D_p, sc = nt - sr * D_p;
+    int r0 = threadIdx.x / D_p, c0 = threadIdx.x - r0 * D_p;
+    for (int base = threadIdx.x; base < n; base += 8 * nt) {
+        float v[8], g[8];
+        int rr[8], cc[8];
+        int r = r0, c = c0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            rr[u] = r;
+            cc[u] = c;
+            const bool in = base + u * nt < n && r < valid && c < D;
+            v[u] = in ? load_elem(src, (int64_t)r * rs + c) : 0.f;
+            g[u] = (in && gsrc) ? gsrc[(int64_t)r * D + c] : 0.f;
+            c += sc;
+            r += sr;
+            if (c >= D_p) {
+                c -= D_p;
+                ++r;
+            }
+        }
+        r0 = r;
+        c0 = c;
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            if (base + u * nt < n) dst[rr[u] * ld + cc[u]] = gsrc ? v[u] * cb_exp(g[u]) : v[u];
+    }
+}
+
 // out(r, c) = sum_k X(r, k) Y(c, k) for r < R, c < N (R, N multiples of 4), each thread a 4 x 4 block
 // of strided elements (rows rt + a R/4, columns ct + b N/4, so that neighbouring threads read
 // neighbouring rows of Y).  X(r, k) = X[r * ldx + k], or X[k * ldx + r] with XT; likewise Y.
@@ -132,7 +205,7 @@ template <bool XT, bool YT, typename F>
 __device__ __forceinline__ void cb_mm(const float *X, int ldx, const float *Y, int ldy, int R, int N, int K,
                                       F &&emit) {
     const int R4 = R >> 2, N4 = N >> 2;
-    for (int tile = threadIdx.x; tile < R4 * N4; tile += CB_NT) {
+    for (int tile = threadIdx.x; tile < R4 * N4; tile += blockDim.x) {
         const int rt = tile / N4, ct = tile - rt * N4;
         float acc[4][4];
 #pragma unroll
@@ -166,7 +239,7 @@ __host__ __device__ inline size_t cb_prep_smem(int Dk, int Dv) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(CB_NT) cb_prep_kernel(CbArgs p) {
+__global__ void __launch_bounds__(CB_NTC) cb_prep_kernel(CbArgs p) {
     extern __shared__ __align__(16) float cb_sm[];
     const int tid = threadIdx.x;
     const CbUnit w = cb_unit(p, blockIdx.x);
@@ -178,36 +251,27 @@ __global__ void __launch_bounds__(CB_NT) cb_prep_kernel(CbArgs p) {
     float *rec = p.ws + w.u * R.size;
     const bool ok = in_bounds(rec, (size_t)R.size * 4, p.ws, p.ws_bytes, p.bounds);
 
-    // inputs; rows past the sequence end: zero, no decay
-    for (int idx = tid; idx < C * Dk; idx += CB_NT) {
-        const int r = idx / Dk, c = idx - r * Dk;
-        float kv = 0.f, qv = 0.f, g = 0.f;
-        if (r < len) {
-            const int64_t i = cb_idx(p, w, r, Dk, c);
-            kv = load_elem((const T *)p.k, i);
-            qv = load_elem((const T *)p.q, i);
-            g = p.log_decay ? clamp_log_decay(p.log_decay[i], p.g_min)
-                            : log_alpha_of(load_elem((const T *)p.z, i), p.g_min);
-        }
-        sK[r * LK + c] = kv;
-        sQ[r * LK + c] = qv;
-        sG[r * LK + c] = g;
-    }
-    for (int idx = tid; idx < C * Dv; idx += CB_NT) {
-        const int r = idx / Dv, j = idx - r * Dv;
-        sV[r * LV + j] = r < len ? load_elem((const T *)p.v, cb_idx(p, w, r, Dv, j)) : 0.f;
-    }
+    // inputs; rows past the sequence end: zero, no decay (the raw decay input first, log(alpha) below)
+    const int64_t rk = (int64_t)p.H * Dk, rv = (int64_t)p.H * Dv;
+    cb_load_rows(sK, LK, (const T *)p.k + cb_idx(p, w, 0, Dk, 0), rk, C, len, Dk, Dk);
+    cb_load_rows(sQ, LK, (const T *)p.q + cb_idx(p, w, 0, Dk, 0), rk, C, len, Dk, Dk);
+    if (p.log_decay)
+        cb_load_rows(sG, LK, p.log_decay + cb_idx(p, w, 0, Dk, 0), rk, C, len, Dk, Dk);
+    else
+        cb_load_rows(sG, LK, (const T *)p.z + cb_idx(p, w, 0, Dk, 0), rk, C, len, Dk, Dk);
+    cb_load_rows(sV, LV, (const T *)p.v + cb_idx(p, w, 0, Dv, 0), rv, C, len, Dv, Dv);
     if (tid < C) sb[tid] = tid < len ? load_elem((const T *)p.beta, cb_idx(p, w, tid, 1, 0)) : 0.f;
     __syncthreads();
-    for (int c = tid; c < Dk; c += CB_NT) {  // G: cumulative sum over the chunk's rows
+    for (int c = tid; c < Dk; c += CB_NTC) {  // G: cumulative sum of log(alpha) over the chunk's rows
         float acc = 0.f;
         for (int r = 0; r < C; ++r) {
-            acc += sG[r * LK + c];
+            const float x = sG[r * LK + c];
+            acc += r < len ? (p.log_decay ? clamp_log_decay(x, p.g_min) : log_alpha_of(x, p.g_min)) : 0.f;
             sG[r * LK + c] = acc;
         }
     }
     __syncthreads();
-    for (int idx = tid; ok && idx < C * Dk; idx += CB_NT) {
+    for (int idx = tid; ok && idx < C * Dk; idx += CB_NTC) {
         const int r = idx / Dk, c = idx - r * Dk;
         const float G = sG[r * LK + c];
         rec[R.G + idx] = G;
@@ -215,7 +279,7 @@ __global__ void __launch_bounds__(CB_NT) cb_prep_kernel(CbArgs p) {
         rec[R.Kd + idx] = sK[r * LK + c] * cb_exp(sG[(C - 1) * LK + c] - G);
     }
     // P (i < r) and M (i <= r) over the triangle of pairs; neighbouring threads take neighbouring i
-    for (int pi = tid; pi < C * (C + 1) / 2; pi += CB_NT) {
+    for (int pi = tid; pi < C * (C + 1) / 2; pi += CB_NTC) {
         int r = (int)((sqrtf(8.f * (float)pi + 1.f) - 1.f) * 0.5f);
         while (r > 0 && r * (r + 1) / 2 > pi) --r;
         while ((r + 1) * (r + 2) / 2 <= pi) ++r;
@@ -234,7 +298,7 @@ __global__ void __launch_bounds__(CB_NT) cb_prep_kernel(CbArgs p) {
             rec[R.M + r * C + i] = mq;
         }
     }
-    for (int idx = tid; idx < C * C; idx += CB_NT) {  // the upper triangles
+    for (int idx = tid; idx < C * C; idx += CB_NTC) {  // the upper triangles
         const int r = idx / C, i = idx - r * C;
         if (i > r) {
             sP[r * LC + i] = 0.f;
@@ -263,27 +327,31 @@ __global__ void __launch_bounds__(CB_NT) cb_prep_kernel(CbArgs p) {
         }
     }
     __syncthreads();
-    for (int idx = tid; ok && idx < C * C; idx += CB_NT) {
+    for (int idx = tid; ok && idx < C * C; idx += CB_NTC) {
         const int r = idx / C, m = idx - r * C;
         rec[R.T + idx] = sT[r * LC + m];
     }
     // beta K e^G and beta V in place: the right-hand sides of W and U
-    for (int idx = tid; idx < C * Dk; idx += CB_NT) {
+    for (int idx = tid; idx < C * Dk; idx += CB_NTC) {
         const int r = idx / Dk, c = idx - r * Dk;
         sK[r * LK + c] = sb[r] * sK[r * LK + c] * cb_exp(sG[r * LK + c]);
     }
-    for (int idx = tid; idx < C * Dv; idx += CB_NT) {
+    for (int idx = tid; idx < C * Dv; idx += CB_NTC) {
         const int r = idx / Dv, j = idx - r * Dv;
         sV[r * LV + j] *= sb[r];
     }
     __syncthreads();
-    // [W | U] = T [beta K e^G | beta V]: a thread per column, four rows at a time
-    for (int col = tid; ok && col < Dk + Dv; col += CB_NT) {
+    // [W | U] = T [beta K e^G | beta V]: a thread per column (D_k + D_v <= 256) and every other group of
+    // four rows (the two halves of the CTA take alternate groups, so that both get short and long ones)
+    static_assert(CB_NTC == 512, "two threads per column");
+    const int col = tid & 255, half = tid >> 8;
+    if (ok && col < Dk + Dv) {
         const bool isw = col < Dk;
         const float *Bc = isw ? sK + col : sV + (col - Dk);
         const int ldb = isw ? LK : LV, ldd = isw ? Dk : Dv;
         float *dst = isw ? rec + R.W + col : rec + R.U + (col - Dk);
-        for (int r0 = 0; r0 < C; r0 += 4) {
+        for (int g = 0; g < C / 8; ++g) {
+            const int r0 = 4 * (2 * g + half);
             float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
             for (int m = 0; m <= r0 + 3; ++m) {
                 const float x = Bc[m * ldb];
@@ -301,49 +369,62 @@ __global__ void __launch_bounds__(CB_NT) cb_prep_kernel(CbArgs p) {
 }
 
 // ---------------------------------------------------------------- the state chains, per 16 value columns
+// Row pitches of the chain kernels: multiples of 4 floats (16-byte copies) that are 4 mod 8, so that the
+// eight rows a warp reads at one column fall in different banks.
+__host__ __device__ inline int cb_lk(int Dk) { return cb_pad8(Dk) + 4; }
+constexpr int CB_LCC = CB_C + 4;
+// forward stages: {W, Kd [C][LK], U columns [C][16], last row of G [Dk]}, two of them
+__host__ __device__ inline int cb_fstage(int Dk) {
+    return (2 * CB_C * cb_lk(Dk) + CB_C * CB_VS + Dk + 3) & ~3;
+}
 __host__ __device__ inline size_t cb_chain_smem(int Dk) {
-    const int LK = cb_pad8(Dk) + 1, LC = CB_C + 1;
-    // forward: W, Kd [C][LK], U, V' [C][16], S [Dk][16], gamma;  backward: M [C][LC], Kd, Qg, W [C][LK],
-    // dO, dV' [C][16], S, dS [Dk][16], gamma
-    const size_t fwd = (size_t)2 * CB_C * LK + 2 * CB_C * CB_VS + (size_t)Dk * CB_VS + Dk;
-    const size_t bwd = (size_t)CB_C * LC + (size_t)3 * CB_C * LK + 2 * CB_C * CB_VS + (size_t)2 * Dk * CB_VS + Dk;
+    const int LK = cb_lk(Dk), LC = CB_LCC, Dk4 = (Dk + 3) & ~3;
+    // forward: two stages, V' [C][16], S [Dk][16];  backward: M [C][LC], Kd [C][LK], S [Dk][16] (one copy
+    // group), Q e^G, W [C][LK], last row of G (the other), dO, dV' [C][16], dS [Dk][16]
+    const size_t fwd = (size_t)2 * cb_fstage(Dk) + CB_C * CB_VS + (size_t)Dk * CB_VS;
+    const size_t bwd = (size_t)CB_C * LC + (size_t)3 * CB_C * LK + (size_t)2 * Dk * CB_VS + Dk4 + 2 * CB_C * CB_VS;
     return sizeof(float) * (fwd > bwd ? fwd : bwd);
 }
 
 // Forward over the chunks of one (b, h) for value columns j0 .. j0 + 15: the state entering every chunk
-// and V' go to the chunk's record.
+// and V' go to the chunk's record.  The next chunk's blocks are copied in while this one is computed.
 __global__ void __launch_bounds__(CB_NT) cb_fwd_chain_kernel(CbArgs p) {
     extern __shared__ __align__(16) float cb_sm[];
     const int tid = threadIdx.x;
     const int64_t bh = blockIdx.x;
     const int j0 = blockIdx.y * CB_VS;
-    const int C = CB_C, Dk = p.Dk, Dv = p.Dv, LK = cb_pad8(Dk) + 1;
-    float *sW = cb_sm, *sKd = sW + C * LK, *sU = sKd + C * LK, *sVp = sU + C * CB_VS, *sS = sVp + C * CB_VS;
-    float *sgam = sS + Dk * CB_VS;
+    const int C = CB_C, Dk = p.Dk, Dv = p.Dv, LK = cb_lk(Dk), FS = cb_fstage(Dk);
+    float *sVp = cb_sm + 2 * FS, *sS = sVp + C * CB_VS;
     const CbRec R = cb_rec(Dk, Dv, p.nslice);
+    auto stage = [&](int n) {  // chunk n's blocks into stage n & 1, one copy group
+        const float *rec = p.ws + (bh * p.Nc + n) * R.size;
+        float *st = cb_sm + (n & 1) * FS;
+        if (in_bounds(rec, (size_t)R.size * 4, p.ws, p.ws_bytes, p.bounds)) {
+            cb_copy(st, LK, rec + R.W, C, Dk, C, Dk);
+            cb_copy(st + C * LK, LK, rec + R.Kd, C, Dk, C, Dk);
+            cb_copy_cols(st + 2 * C * LK, rec + R.U, C, Dv, j0);
+            cb_copy(st + 2 * C * LK + C * CB_VS, Dk, rec + R.G + (int64_t)(C - 1) * Dk, 1, Dk, 1, Dk);
+        }
+        cp_async_commit_group();
+    };
     for (int idx = tid; idx < Dk * CB_VS; idx += CB_NT) {
         const int c = idx / CB_VS, j = idx - c * CB_VS;
         sS[idx] = (p.S0 && j0 + j < Dv) ? p.S0[(bh * Dk + c) * Dv + j0 + j] : 0.f;
     }
+    stage(0);
     for (int n = 0; n < p.Nc; ++n) {
+        if (n + 1 < p.Nc) stage(n + 1);
+        else cp_async_commit_group();
+        cp_async_wait<1>();  // chunk n's copies
+        __syncthreads();
+        const float *st = cb_sm + (n & 1) * FS;
+        const float *sW = st, *sKd = st + C * LK, *sU = st + 2 * C * LK, *sGl = sU + C * CB_VS;
         float *rec = p.ws + (bh * p.Nc + n) * R.size;
         const bool ok = in_bounds(rec, (size_t)R.size * 4, p.ws, p.ws_bytes, p.bounds);
-        __syncthreads();  // the previous chunk's reads of W, Kd and V' are done
-        for (int idx = tid; idx < C * Dk; idx += CB_NT) {
-            const int r = idx / Dk, c = idx - r * Dk;
-            sW[r * LK + c] = ok ? rec[R.W + idx] : 0.f;
-            sKd[r * LK + c] = ok ? rec[R.Kd + idx] : 0.f;
-        }
-        for (int idx = tid; idx < C * CB_VS; idx += CB_NT) {
-            const int r = idx / CB_VS, j = idx - r * CB_VS;
-            sU[idx] = (ok && j0 + j < Dv) ? rec[R.U + (int64_t)r * Dv + j0 + j] : 0.f;
-        }
-        for (int c = tid; c < Dk; c += CB_NT) sgam[c] = ok ? cb_exp(rec[R.G + (int64_t)(C - 1) * Dk + c]) : 0.f;
         for (int idx = tid; ok && idx < Dk * CB_VS; idx += CB_NT) {  // the state entering chunk n
             const int c = idx / CB_VS, j = idx - c * CB_VS;
             if (j0 + j < Dv) rec[R.S + (int64_t)c * Dv + j0 + j] = sS[idx];
         }
-        __syncthreads();
         {  // V' = U - W S: thread (row r, four columns)
             const int r = tid >> 2, jq = (tid & 3) * 4;
             float a[4];
@@ -366,9 +447,10 @@ __global__ void __launch_bounds__(CB_NT) cb_fwd_chain_kernel(CbArgs p) {
         __syncthreads();
         if (tid < 2 * Dk) {  // S <- Diag(gamma) S + Kd^T V': thread (key row c, eight columns)
             const int c = tid >> 1, jh = (tid & 1) * 8;
+            const float gam = cb_exp(sGl[c]);
             float a[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) a[e] = sgam[c] * sS[c * CB_VS + jh + e];
+            for (int e = 0; e < 8; ++e) a[e] = gam * sS[c * CB_VS + jh + e];
             for (int r = 0; r < C; ++r) {
                 const float kd = sKd[r * LK + c];
                 const float4 v0 = *reinterpret_cast<const float4 *>(sVp + r * CB_VS + jh);
@@ -385,55 +467,78 @@ __global__ void __launch_bounds__(CB_NT) cb_fwd_chain_kernel(CbArgs p) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) sS[c * CB_VS + jh + e] = a[e];
         }
+        __syncthreads();  // stage n & 1 takes chunk n + 2 next
     }
 }
 
 // Backward over the chunks of one (b, h) for value columns j0 .. j0 + 15: dS_next, dV' and the
-// partial dgamma of every chunk go to its record; dL/dS_0 to the output.
+// partial dgamma of every chunk go to its record; dL/dS_0 to the output.  The blocks the first half of
+// a step reads (M, Kd, S) and those of its second half (Q e^G, W, G) are two copy groups, each refilled
+// with the previous chunk's as soon as its half is done.
 template <typename T>
 __global__ void __launch_bounds__(CB_NT) cb_bwd_chain_kernel(CbArgs p) {
     extern __shared__ __align__(16) float cb_sm[];
     const int tid = threadIdx.x;
     const int64_t bh = blockIdx.x;
     const int sl = blockIdx.y, j0 = sl * CB_VS;
-    const int C = CB_C, Dk = p.Dk, Dv = p.Dv, LK = cb_pad8(Dk) + 1, LC = C + 1;
+    const int C = CB_C, Dk = p.Dk, Dv = p.Dv, LK = cb_lk(Dk), LC = CB_LCC, Dk4 = (Dk + 3) & ~3;
     const int b = (int)(bh / p.H), h = (int)(bh - (int64_t)b * p.H);
-    float *sM = cb_sm, *sKd = sM + C * LC, *sQg = sKd + C * LK, *sW = sQg + C * LK, *sdO = sW + C * LK;
-    float *sdV = sdO + C * CB_VS, *sSn = sdV + C * CB_VS, *sdS = sSn + Dk * CB_VS, *sgam = sdS + Dk * CB_VS;
+    float *sM = cb_sm, *sKd = sM + C * LC, *sSn = sKd + C * LK;
+    float *sQg = sSn + Dk * CB_VS, *sW = sQg + C * LK, *sGl = sW + C * LK;
+    float *sdO = sGl + Dk4, *sdV = sdO + C * CB_VS, *sdS = sdV + C * CB_VS;
     const CbRec R = cb_rec(Dk, Dv, p.nslice);
+    auto rec_of = [&](int n) { return p.ws + (bh * p.Nc + n) * R.size; };
+    auto stage_a = [&](int n) {
+        const float *rec = rec_of(n);
+        if (in_bounds(rec, (size_t)R.size * 4, p.ws, p.ws_bytes, p.bounds)) {
+            cb_copy(sM, LC, rec + R.M, C, C, C, C);
+            cb_copy(sKd, LK, rec + R.Kd, C, Dk, C, Dk);
+            cb_copy_cols(sSn, rec + R.S, Dk, Dv, j0);
+        }
+        cp_async_commit_group();
+    };
+    auto stage_b = [&](int n) {
+        const float *rec = rec_of(n);
+        if (in_bounds(rec, (size_t)R.size * 4, p.ws, p.ws_bytes, p.bounds)) {
+            cb_copy(sQg, LK, rec + R.Qg, C, Dk, C, Dk);
+            cb_copy(sW, LK, rec + R.W, C, Dk, C, Dk);
+            cb_copy(sGl, Dk, rec + R.G + (int64_t)(C - 1) * Dk, 1, Dk, 1, Dk);
+        }
+        cp_async_commit_group();
+    };
+    float pre[C * CB_VS / CB_NT];  // this thread's dO elements of a chunk: element tid + CB_NT u of [C][16]
+    auto load_do = [&](int n) {
+        const int64_t t0 = (int64_t)n * C;
+        const int len = (int)min((int64_t)C, p.S - t0);
+#pragma unroll
+        for (int u = 0; u < C * CB_VS / CB_NT; ++u) {
+            const int idx = tid + u * CB_NT, r = idx / CB_VS, j = idx - r * CB_VS;
+            pre[u] = (r < len && j0 + j < Dv)
+                         ? load_elem((const T *)p.dO, (((int64_t)b * p.S + t0 + r) * p.H + h) * Dv + j0 + j)
+                         : 0.f;
+        }
+    };
+    auto store_do = [&]() {
+#pragma unroll
+        for (int u = 0; u < C * CB_VS / CB_NT; ++u) sdO[tid + u * CB_NT] = pre[u];
+    };
     for (int idx = tid; idx < Dk * CB_VS; idx += CB_NT) {
         const int c = idx / CB_VS, j = idx - c * CB_VS;
         sdS[idx] = (p.dST && j0 + j < Dv) ? p.dST[(bh * Dk + c) * Dv + j0 + j] : 0.f;
     }
+    stage_a(p.Nc - 1);
+    stage_b(p.Nc - 1);
+    load_do(p.Nc - 1);
+    store_do();
     for (int n = p.Nc - 1; n >= 0; --n) {
-        float *rec = p.ws + (bh * p.Nc + n) * R.size;
+        float *rec = rec_of(n);
         const bool ok = in_bounds(rec, (size_t)R.size * 4, p.ws, p.ws_bytes, p.bounds);
-        const int64_t t0 = (int64_t)n * C;
-        const int len = (int)min((int64_t)C, p.S - t0);
-        __syncthreads();  // the previous chunk's reads are done
-        for (int idx = tid; idx < C * C; idx += CB_NT) {
-            const int r = idx / C, i = idx - r * C;
-            sM[r * LC + i] = ok ? rec[R.M + idx] : 0.f;
-        }
-        for (int idx = tid; idx < C * Dk; idx += CB_NT) {
-            const int r = idx / Dk, c = idx - r * Dk;
-            sKd[r * LK + c] = ok ? rec[R.Kd + idx] : 0.f;
-            sQg[r * LK + c] = ok ? rec[R.Qg + idx] : 0.f;
-            sW[r * LK + c] = ok ? rec[R.W + idx] : 0.f;
-        }
-        for (int idx = tid; idx < C * CB_VS; idx += CB_NT) {
-            const int r = idx / CB_VS, j = idx - r * CB_VS;
-            sdO[idx] = (r < len && j0 + j < Dv)
-                           ? load_elem((const T *)p.dO, (((int64_t)b * p.S + t0 + r) * p.H + h) * Dv + j0 + j)
-                           : 0.f;
-        }
-        for (int idx = tid; idx < Dk * CB_VS; idx += CB_NT) {
-            const int c = idx / CB_VS, j = idx - c * CB_VS;
-            sSn[idx] = (ok && j0 + j < Dv) ? rec[R.S + (int64_t)c * Dv + j0 + j] : 0.f;
-            if (ok && j0 + j < Dv) rec[R.dS + (int64_t)c * Dv + j0 + j] = sdS[idx];
-        }
-        for (int c = tid; c < Dk; c += CB_NT) sgam[c] = ok ? cb_exp(rec[R.G + (int64_t)(C - 1) * Dk + c]) : 0.f;
+        cp_async_wait<1>();  // M, Kd and S of chunk n
         __syncthreads();
+        for (int idx = tid; ok && idx < Dk * CB_VS; idx += CB_NT) {  // dS_next of chunk n
+            const int c = idx / CB_VS, j = idx - c * CB_VS;
+            if (j0 + j < Dv) rec[R.dS + (int64_t)c * Dv + j0 + j] = sdS[idx];
+        }
         for (int c = tid; ok && c < Dk; c += CB_NT) {  // this slice's part of dgamma = rowsum(dS_next * S)
             float s = 0.f;
 #pragma unroll
@@ -465,12 +570,21 @@ __global__ void __launch_bounds__(CB_NT) cb_bwd_chain_kernel(CbArgs p) {
                 if (ok && j0 + jq + e < Dv) rec[R.dVp + (int64_t)r * Dv + j0 + jq + e] = a[e];
             }
         }
+        __syncthreads();  // M, Kd and S of chunk n are read: the previous chunk's come in
+        if (n > 0) {
+            stage_a(n - 1);
+            load_do(n - 1);
+        } else {
+            cp_async_commit_group();
+        }
+        cp_async_wait<1>();  // Q e^G, W and G of chunk n
         __syncthreads();
         if (tid < 2 * Dk) {  // dS <- Diag(gamma) dS_next + (Q e^G)^T dO - W^T dV'
             const int c = tid >> 1, jh = (tid & 1) * 8;
+            const float gam = cb_exp(sGl[c]);
             float a[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) a[e] = sgam[c] * sdS[c * CB_VS + jh + e];
+            for (int e = 0; e < 8; ++e) a[e] = gam * sdS[c * CB_VS + jh + e];
             for (int r = 0; r < C; ++r) {
                 const float qg = sQg[r * LK + c], wv = sW[r * LK + c];
 #pragma unroll
@@ -479,6 +593,13 @@ __global__ void __launch_bounds__(CB_NT) cb_bwd_chain_kernel(CbArgs p) {
             }
 #pragma unroll
             for (int e = 0; e < 8; ++e) sdS[c * CB_VS + jh + e] = a[e];
+        }
+        __syncthreads();  // Q e^G, W, G and dO of chunk n are read
+        if (n > 0) {
+            stage_b(n - 1);
+            store_do();
+        } else {
+            cp_async_commit_group();
         }
     }
     __syncthreads();
@@ -494,7 +615,8 @@ __global__ void __launch_bounds__(CB_NT) cb_bwd_chain_kernel(CbArgs p) {
 __host__ __device__ inline size_t cb_mat_smem(int Dk, int Dv) {
     const int Dkp = cb_pad8(Dk), LK = Dkp + 1, LV = cb_pad8(Dv) + 1, LC = CB_C + 1;
     const int LVC = cb_max(LV, LC);
-    const size_t big = cb_max(Dkp * LV, CB_C * (LV + LK));  // S or dS_next [Dk][Dv]; later V and K e^G
+    // S or dS_next [Dk][Dv]; later V and K e^G [C][LV + LK]; later P [C][LC]
+    const size_t big = cb_max(cb_max(Dkp * LV, CB_C * (LV + LK)), CB_C * LC);
     return sizeof(float) * (big + (size_t)CB_C * LVC      // dO, later T
                             + (size_t)CB_C * LV            // dV'
                             + (size_t)CB_C * LVC           // V', later dT
@@ -504,7 +626,7 @@ __host__ __device__ inline size_t cb_mat_smem(int Dk, int Dv) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(CB_NT) cb_grad_mat_kernel(CbArgs p) {
+__global__ void __launch_bounds__(CB_NTC) cb_grad_mat_kernel(CbArgs p) {
     extern __shared__ __align__(16) float cb_sm[];
     const int tid = threadIdx.x;
     const CbUnit w = cb_unit(p, blockIdx.x);
@@ -512,7 +634,7 @@ __global__ void __launch_bounds__(CB_NT) cb_grad_mat_kernel(CbArgs p) {
     const int Dkp = cb_pad8(Dk), Dvp = cb_pad8(Dv), LK = Dkp + 1, LV = Dvp + 1, LC = C + 1;
     const int LVC = cb_max(LV, LC);
     float *sX = cb_sm;
-    float *sdO = sX + cb_max(Dkp * LV, C * (LV + LK));
+    float *sdO = sX + cb_max(cb_max(Dkp * LV, C * (LV + LK)), C * LC);
     float *sdV = sdO + C * LVC, *sV = sdV + C * LV, *sdW = sV + C * LVC, *sdM = sdW + C * LK;
     float *sb = sdM + C * LC, *sdb = sb + C;
     const CbRec R = cb_rec(Dk, Dv, p.nslice);
@@ -520,21 +642,17 @@ __global__ void __launch_bounds__(CB_NT) cb_grad_mat_kernel(CbArgs p) {
     const bool ok = in_bounds(rec, (size_t)R.size * 4, p.ws, p.ws_bytes, p.bounds);
     if (!ok) return;
 
-    // S [c][j], dO [r][j], dV' [r][j] (zero padding to multiples of 8)
-    for (int idx = tid; idx < Dkp * Dvp; idx += CB_NT) {
-        const int c = idx / Dvp, j = idx - c * Dvp;
-        sX[c * LV + j] = (c < Dk && j < Dv) ? rec[R.S + (int64_t)c * Dv + j] : 0.f;
-    }
-    for (int idx = tid; idx < C * Dvp; idx += CB_NT) {
-        const int r = idx / Dvp, j = idx - r * Dvp;
-        const bool in = r < len && j < Dv;
-        sdO[r * LV + j] = in ? load_elem((const T *)p.dO, cb_idx(p, w, r, Dv, j)) : 0.f;
-        sdV[r * LV + j] = j < Dv ? rec[R.dVp + (int64_t)r * Dv + j] : 0.f;
-    }
+    // S [c][j], dV' [r][j], V' [r][j] (copies), dO [r][j] (zero padding to multiples of 8)
+    cb_copy(sX, LV, rec + R.S, Dk, Dv, Dkp, Dvp);
+    cb_copy(sdV, LV, rec + R.dVp, C, Dv, C, Dvp);
+    cb_copy(sV, LV, rec + R.Vp, C, Dv, C, Dvp);
+    cp_async_commit_group();
+    cb_load_rows(sdO, LV, (const T *)p.dO + cb_idx(p, w, 0, Dv, 0), (int64_t)p.H * Dv, C, len, Dv, Dvp);
     if (tid < C) {
         sb[tid] = tid < len ? load_elem((const T *)p.beta, cb_idx(p, w, tid, 1, 0)) : 0.f;
         sdb[tid] = 0.f;
     }
+    cp_async_wait<0>();
     __syncthreads();
     // dQg = dO S^T -> record (Q e^G's place);  dW = -dV' S^T -> shared
     cb_mm<false, false>(sdO, LV, sX, LV, C, Dkp, Dvp, [&](int r, int c, float v) {
@@ -542,15 +660,10 @@ __global__ void __launch_bounds__(CB_NT) cb_grad_mat_kernel(CbArgs p) {
     });
     cb_mm<false, false>(sdV, LV, sX, LV, C, Dkp, Dvp, [&](int r, int c, float v) { sdW[r * LK + c] = -v; });
     __syncthreads();
-    // dS_next [c][j] over S; V' [r][j]
-    for (int idx = tid; idx < Dkp * Dvp; idx += CB_NT) {
-        const int c = idx / Dvp, j = idx - c * Dvp;
-        sX[c * LV + j] = (c < Dk && j < Dv) ? rec[R.dS + (int64_t)c * Dv + j] : 0.f;
-    }
-    for (int idx = tid; idx < C * Dvp; idx += CB_NT) {
-        const int r = idx / Dvp, j = idx - r * Dvp;
-        sV[r * LV + j] = j < Dv ? rec[R.Vp + (int64_t)r * Dv + j] : 0.f;
-    }
+    // dS_next [c][j] over S
+    cb_copy(sX, LV, rec + R.dS, Dk, Dv, Dkp, Dvp);
+    cp_async_commit_group();
+    cp_async_wait<0>();
     __syncthreads();
     // dKd = V' dS_next^T -> record (Kd's place);  dM = dO V'^T (i <= r) -> shared and record (M's place)
     cb_mm<false, false>(sV, LV, sX, LV, C, Dkp, Dvp, [&](int r, int c, float v) {
@@ -564,20 +677,11 @@ __global__ void __launch_bounds__(CB_NT) cb_grad_mat_kernel(CbArgs p) {
     __syncthreads();
     // V [m][j] and K e^G [m][c] over S's space; T [r][m] over dO's
     float *sVin = sX, *sKg = sX + C * LV, *sT = sdO, *sdT = sV;
-    for (int idx = tid; idx < C * Dvp; idx += CB_NT) {
-        const int r = idx / Dvp, j = idx - r * Dvp;
-        sVin[r * LV + j] = (r < len && j < Dv) ? load_elem((const T *)p.v, cb_idx(p, w, r, Dv, j)) : 0.f;
-    }
-    for (int idx = tid; idx < C * Dkp; idx += CB_NT) {
-        const int r = idx / Dkp, c = idx - r * Dkp;
-        sKg[r * LK + c] = (r < len && c < Dk)
-                              ? load_elem((const T *)p.k, cb_idx(p, w, r, Dk, c)) * cb_exp(rec[R.G + (int64_t)r * Dk + c])
-                              : 0.f;
-    }
-    for (int idx = tid; idx < C * C; idx += CB_NT) {
-        const int r = idx / C, m = idx - r * C;
-        sT[r * LC + m] = rec[R.T + idx];
-    }
+    cb_copy(sT, LC, rec + R.T, C, C, C, C);
+    cp_async_commit_group();
+    cb_load_rows(sVin, LV, (const T *)p.v + cb_idx(p, w, 0, Dv, 0), (int64_t)p.H * Dv, C, len, Dv, Dvp);
+    cb_load_rows(sKg, LK, (const T *)p.k + cb_idx(p, w, 0, Dk, 0), (int64_t)p.H * Dk, C, len, Dk, Dkp, rec + R.G);
+    cp_async_wait<0>();
     __syncthreads();
     // dT = (dV' V^T + dW (K e^G)^T) Diag(beta), in two passes over the same threads' elements
     cb_mm<false, false>(sdV, LV, sVin, LV, C, C, Dvp, [&](int r, int m, float v) { sdT[r * LC + m] = v; });
@@ -599,15 +703,19 @@ __global__ void __launch_bounds__(CB_NT) cb_grad_mat_kernel(CbArgs p) {
             atomicAdd(sdb + m, v * sKg[m * LK + c]);
         }
     });
-    // X = dT T^T over dM's space
-    float *sX1 = sdM;
+    __syncthreads();
+    // P over S's space (V and K e^G are read) while X = dT T^T goes to dM's
+    float *sP = sX, *sX1 = sdM;
+    cb_copy(sP, LC, rec + R.P, C, C, C, C);
+    cp_async_commit_group();
     cb_mm<false, false>(sdT, LC, sT, LC, C, C, C, [&](int r, int m, float v) { sX1[r * LC + m] = v; });
+    cp_async_wait<0>();
     __syncthreads();
     // dA^T = -X^T T (dA[r][i], i < r) -> record (T's place); dbeta += rowsum(dA * P)
     cb_mm<true, true>(sX1, LC, sT, LC, C, C, C, [&](int i, int r, float v) {
         const float a = i < r ? -v : 0.f;
         rec[R.T + r * C + i] = a;
-        atomicAdd(sdb + r, a * rec[R.P + r * C + i]);
+        atomicAdd(sdb + r, a * sP[r * LC + i]);
     });
     __syncthreads();
     if (tid < len) p.dbeta[cb_idx(p, w, tid, 1, 0)] = sdb[tid];
@@ -620,7 +728,7 @@ __host__ __device__ inline size_t cb_pair_smem(int Dk) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(CB_NT) cb_grad_pair_kernel(CbArgs p) {
+__global__ void __launch_bounds__(CB_NTC) cb_grad_pair_kernel(CbArgs p) {
     extern __shared__ __align__(16) float cb_sm[];
     const int tid = threadIdx.x;
     const CbUnit w = cb_unit(p, blockIdx.x);
@@ -632,24 +740,20 @@ __global__ void __launch_bounds__(CB_NT) cb_grad_pair_kernel(CbArgs p) {
     const float *rec = p.ws + w.u * R.size;
     if (!in_bounds(rec, (size_t)R.size * 4, p.ws, p.ws_bytes, p.bounds)) return;
 
-    for (int idx = tid; idx < C * Dk; idx += CB_NT) {
-        const int r = idx / Dk, c = idx - r * Dk;
-        const bool in = r < len;
-        const int64_t i = in ? cb_idx(p, w, r, Dk, c) : 0;
-        sG[r * LK + c] = rec[R.G + idx];
-        sK[r * LK + c] = in ? load_elem((const T *)p.k, i) : 0.f;
-        sQ[r * LK + c] = in ? load_elem((const T *)p.q, i) : 0.f;
-    }
-    for (int idx = tid; idx < C * C; idx += CB_NT) {
-        const int r = idx / C, i = idx - r * C;
-        sdA[r * LC + i] = rec[R.T + idx];
-        sdM[r * LC + i] = rec[R.M + idx];
-    }
+    const int64_t rk = (int64_t)p.H * Dk, row0 = cb_idx(p, w, 0, Dk, 0);
+    cb_copy(sG, LK, rec + R.G, C, Dk, C, Dk);
+    cb_copy(sdA, LC, rec + R.T, C, C, C, C);
+    cb_copy(sdM, LC, rec + R.M, C, C, C, C);
+    cp_async_commit_group();
+    cb_load_rows(sK, LK, (const T *)p.k + row0, rk, C, len, Dk, Dk);
+    cb_load_rows(sQ, LK, (const T *)p.q + row0, rk, C, len, Dk, Dk);
     if (tid < C) sb[tid] = tid < len ? load_elem((const T *)p.beta, cb_idx(p, w, tid, 1, 0)) : 0.f;
+    cp_async_wait<0>();
     __syncthreads();
     // row roles: token r against the earlier tokens i <= r; dq is final here
-    for (int idx = tid; idx < C * Dk; idx += CB_NT) {
+    for (int idx = tid; idx < C * Dk; idx += CB_NTC) {
         const int r = idx / Dk, c = idx - r * Dk;
+        const float dQg = rec[R.Qg + idx], dKg = rec[R.W + idx], dKd = rec[R.Kd + idx];  // (in flight meanwhile)
         const float Gr = sG[r * LK + c];
         float xa = 0.f, y = 0.f;
         for (int i = 0; i <= r; ++i) {
@@ -658,7 +762,6 @@ __global__ void __launch_bounds__(CB_NT) cb_grad_pair_kernel(CbArgs p) {
             y = fmaf(sdM[r * LC + i], e, y);
         }
         const float eG = cb_exp(Gr), eD = cb_exp(sG[(C - 1) * LK + c] - Gr);
-        const float dQg = rec[R.Qg + idx], dKg = rec[R.W + idx], dKd = rec[R.Kd + idx];
         const float kv = sK[r * LK + c], qv = sQ[r * LK + c], bxa = sb[r] * xa;
         if (r < len) p.dq[cb_idx(p, w, r, Dk, c)] = fmaf(dQg, eG, y);
         sdk[r * LK + c] = dKg * eG + dKd * eD + bxa;
@@ -666,7 +769,7 @@ __global__ void __launch_bounds__(CB_NT) cb_grad_pair_kernel(CbArgs p) {
     }
     __syncthreads();
     // column roles: token i against the later tokens r >= i
-    for (int idx = tid; idx < C * Dk; idx += CB_NT) {
+    for (int idx = tid; idx < C * Dk; idx += CB_NTC) {
         const int i = idx / Dk, c = idx - i * Dk;
         const float Gi = sG[i * LK + c];
         float x = 0.f;
@@ -678,11 +781,21 @@ __global__ void __launch_bounds__(CB_NT) cb_grad_pair_kernel(CbArgs p) {
         sdG[i * LK + c] -= sK[i * LK + c] * x;
     }
     __syncthreads();
+    // dKd over dA's and dM's space, the raw decay input over Q's
+    float *sdKd = sdA, *sZ = sQ;
+    cb_copy(sdKd, LK, rec + R.Kd, C, Dk, C, Dk);
+    cp_async_commit_group();
+    if (p.log_decay)
+        cb_load_rows(sZ, LK, p.log_decay + row0, rk, C, len, Dk, Dk);
+    else
+        cb_load_rows(sZ, LK, (const T *)p.z + row0, rk, C, len, Dk, Dk);
+    cp_async_wait<0>();
+    __syncthreads();
     // per channel: the last row's gamma and Kd terms, the reverse cumulative sum, dz and dk
-    for (int c = tid; c < Dk; c += CB_NT) {
+    for (int c = tid; c < Dk; c += CB_NTC) {
         const float Gl = sG[(C - 1) * LK + c];
         float s = 0.f;
-        for (int r = 0; r < C; ++r) s = fmaf(rec[R.Kd + (int64_t)r * Dk + c] * sK[r * LK + c], cb_exp(Gl - sG[r * LK + c]), s);
+        for (int r = 0; r < C; ++r) s = fmaf(sdKd[r * LK + c] * sK[r * LK + c], cb_exp(Gl - sG[r * LK + c]), s);
         float dgam = 0.f;
         for (int sl = 0; sl < p.nslice; ++sl) dgam += rec[R.dgam + (int64_t)sl * Dk + c];
         float acc = s + dgam * cb_exp(Gl);
@@ -690,12 +803,12 @@ __global__ void __launch_bounds__(CB_NT) cb_grad_pair_kernel(CbArgs p) {
             acc += sdG[r * LK + c];
             if (r < len) {
                 const int64_t i = cb_idx(p, w, r, Dk, c);
+                const float raw = sZ[r * LK + c];
                 float dz;
                 if (p.log_decay) {
-                    const float raw = p.log_decay[i];
                     dz = (raw >= p.g_min && raw <= 0.f) ? acc : 0.f;  // a clamped input has no gradient
                 } else {  // g = g_min sigmoid(z): dg/dz = g (1 - g / g_min)
-                    const float g = log_alpha_of(load_elem((const T *)p.z, i), p.g_min);
+                    const float g = log_alpha_of(raw, p.g_min);
                     dz = acc * g * (1.0f - g / p.g_min);
                 }
                 p.dz[i] = dz;
@@ -758,15 +871,15 @@ kda_status_t launch_chunk_bwd(const kda_recurrent_bwd_args &a, cudaStream_t st) 
         cudaFuncSetAttribute(mat, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s4);
         cudaFuncSetAttribute(pair, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s5);
         kda_status_t s;
-        prep<<<gu, CB_NT, s1, st>>>(p);
+        prep<<<gu, CB_NTC, s1, st>>>(p);
         if ((s = check_launch("cb_prep_kernel")) != KDA_OK) return s;
         cb_fwd_chain_kernel<<<gc, CB_NT, s2, st>>>(p);
         if ((s = check_launch("cb_fwd_chain_kernel")) != KDA_OK) return s;
         bchain<<<gc, CB_NT, s2, st>>>(p);
         if ((s = check_launch("cb_bwd_chain_kernel")) != KDA_OK) return s;
-        mat<<<gu, CB_NT, s4, st>>>(p);
+        mat<<<gu, CB_NTC, s4, st>>>(p);
         if ((s = check_launch("cb_grad_mat_kernel")) != KDA_OK) return s;
-        pair<<<gu, CB_NT, s5, st>>>(p);
+        pair<<<gu, CB_NTC, s5, st>>>(p);
         return check_launch("cb_grad_pair_kernel");
     };
     if (a.dtype == KDA_F32)

@@ -67,6 +67,25 @@ __device__ __forceinline__ constexpr bool in_bounds(const void *, size_t, const 
 #endif
 unsigned int *device_bounds_counter();  // device address of the counter (host)
 
+// ----------------------------------------------------------------- asynchronous global -> shared copies
+// One fp32 element by cp.async (4-byte aligned addresses); with fill == false the destination gets
+// zero and nothing is read.  A thread's copies have landed after cp_async_wait<n>() leaves at most n of
+// its committed groups pending; other threads see them after a block barrier that follows.
+__device__ __forceinline__ void cp_async4(float *smem_dst, const float *gsrc, bool fill = true) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
+                 "l"(gsrc), "r"(fill ? 4 : 0)
+                 : "memory");
+}
+// Four fp32 elements (16-byte aligned addresses); zero and no read with fill == false.
+__device__ __forceinline__ void cp_async16_fill(float *smem_dst, const float *gsrc, bool fill = true) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"((uint32_t)__cvta_generic_to_shared(smem_dst)),
+                 "l"(gsrc), "r"(fill ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit_group() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // ----------------------------------------------------------------- launchers (one per .cu)
 kda_status_t launch_gate(const void *z, kda_dtype_t dt, int64_t n, float g_min, float *out,
                          cudaStream_t st);

@@ -69,9 +69,10 @@ def test_backward_matches_oracle(K, engine, B, S, H, D, dtype):
 
 
 @pytest.mark.parametrize("B,S,H,Dk,Dv,dtype", [(1, 200, 2, 32, 128, "bf16"), (2, 70, 1, 128, 20, "f32"),
-                                               (1, 640, 2, 128, 128, "bf16")])
+                                               (1, 100, 2, 18, 13, "f32"), (1, 640, 2, 128, 128, "bf16")])
 def test_chunk_backward_unequal_heads_and_long(K, B, S, H, Dk, Dv, dtype):
-    """D_k != D_v (value slices of 16 with a ragged last one), and ten chunks of 64 at D = 128."""
+    """D_k != D_v (value slices of 16 with a ragged last one; sizes that are not multiples of 4, which
+    take the element-wise copies), and ten chunks of 64 at D = 128."""
     w = small("bwdc", B, S, H, Dk, Dv, 16, dtype, seed=S + Dk, s0_std=0.05)
     got, want = _run(K, w, seed=S + 1, with_s0=True, with_dst=True, use_log=False, engine="chunk_bwd")
     for n in NAMES:
