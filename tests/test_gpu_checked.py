@@ -1,8 +1,9 @@
 """The bounds-checked build (libkda_checked.so, compiled with -DKDA_CHECKED):
 in a child process that loads it, the segmented tensor-core forward, the GDN
-engine, the recurrent backward and the DPLR comparator find no write outside
-its buffer, and give the results the normal library gives on the same inputs
-(bit for bit where no floating-point atomics are involved)."""
+engine, the recurrent and chunkwise backward passes and the DPLR comparator
+find no write outside its buffer, and give the results the normal library
+gives on the same inputs (bit for bit where no floating-point atomics are
+involved)."""
 import os
 import subprocess
 import sys
@@ -36,7 +37,7 @@ def test_checked_build_runs_clean_and_matches(tmp_path):
     assert set(want) == {k for k in got.files if not k.startswith("_")}
     for k, v in want.items():
         g = got[k]
-        if k.startswith("bwd_"):  # fp32 atomics add the value-column slices in any order
+        if k.startswith("bwd_"):  # fp32 atomics add in any order (value-column slices, dbeta terms)
             scale = max(1e-30, float(np.abs(v).max()))
             np.testing.assert_allclose(g, v, rtol=1e-5, atol=1e-6 * scale, err_msg=k)
         else:
