@@ -524,9 +524,10 @@ def time_backward(K, torch, w, d, warmup, world, dev, flush, lib, steps=3, engin
 
 def time_dplr(K, torch, w, d, warmup, world, dev, rec, steps=3):
     """The general DPLR transition (free erase directions; here random unit
-    directions drawn on the device) evaluated token by token on the workload,
-    against the KDA chunk engine's time on the same workload: what KDA's
-    binding, which makes the chunkwise form possible, is worth on this GPU."""
+    directions drawn on the device) on the workload, token by token and in
+    chunk form, against the KDA chunk engine's time on the same workload: what
+    KDA's binding (two decayed products per chunk instead of four, a state-only
+    chain, tensor-core operands) is worth on this GPU."""
     g = torch.Generator(device=dev)
     g.manual_seed(w.seed + 7)
     shp = (w.B, w.S, w.H, w.Dk)
@@ -535,26 +536,40 @@ def time_dplr(K, torch, w, d, warmup, world, dev, rec, steps=3):
     o = torch.empty((w.B, w.S, w.H, w.Dv), dtype=d["q"].dtype, device=dev)
     sf = torch.empty((w.B, w.H, w.Dk, w.Dv), dtype=torch.float32, device=dev)
 
-    def one():
+    ws = torch.empty(K.api.dplr_chunk_workspace_bytes(w.B, w.S, w.H, w.Dk, w.Dv), dtype=torch.uint8, device=dev)
+
+    def recurrent():
         K.dplr_recurrent_fwd(d["q"], d["k"], d["v"], a, b, z=d["z"], g_min=w.g_min, initial_state=d["S0"], out=o,
                              final_state=sf)
 
-    for _ in range(max(1, warmup // 3)):
-        one()
-    torch.cuda.synchronize(dev)
-    stream = torch.cuda.current_stream(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    e0.record(stream)
-    for _ in range(steps):
-        one()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    (t,) = reduce_max([e0.elapsed_time(e1) / steps * 1e-3], world, dev)
+    def chunked():
+        K.dplr_chunk_fwd(d["q"], d["k"], d["v"], a, b, z=d["z"], g_min=w.g_min, initial_state=d["S0"], out=o,
+                         final_state=sf, workspace=ws)
+
+    def timed(one):
+        for _ in range(max(1, warmup // 3)):
+            one()
+        torch.cuda.synchronize(dev)
+        stream = torch.cuda.current_stream(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        e0.record(stream)
+        for _ in range(steps):
+            one()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        (t,) = reduce_max([e0.elapsed_time(e1) / steps * 1e-3], world, dev)
+        return t
+
+    t, tc = timed(recurrent), timed(chunked)
     out = {"entry_point": "kda_dplr_recurrent_fwd (general DPLR, token by token, exact fp32)",
-           "ms": round(t * 1e3, 3), "tokens_per_s": round(w.B * w.S * world / t, 1)}
+           "ms": round(t * 1e3, 3), "tokens_per_s": round(w.B * w.S * world / t, 1),
+           "chunk": {"entry_point": "kda_dplr_chunk_fwd (general DPLR in chunk form, exact fp32 SIMT)",
+                     "ms": round(tc * 1e3, 3), "tokens_per_s": round(w.B * w.S * world / tc, 1),
+                     "recurrent_over_chunk_time": round(t / tc, 2)}}
     if rec and "kernels_ms" in rec:
         out["dplr_over_kda_chunk_engine_time"] = round(t * 1e3 / rec["kernels_ms"]["chunk_engine"], 2)
+        out["chunk"]["dplr_chunk_over_kda_chunk_engine_time"] = round(tc * 1e3 / rec["kernels_ms"]["chunk_engine"], 2)
     return out
 
 

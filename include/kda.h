@@ -295,6 +295,29 @@ typedef struct kda_dplr_args {
 kda_status_t kda_dplr_recurrent_fwd(const kda_dplr_args *args);
 
 /*
+ * kda_dplr_chunk_fwd — the same recurrence and outputs as kda_dplr_recurrent_fwd,
+ * in chunk form: with y_t = b_t^T S_{t-1}, the chunk's erased rows Y solve a
+ * unit-lower-triangular system (I + Ba) Y = (b * e^{G_{t-1}}) S + Bk V built
+ * from decayed products of b with a and k, and the outputs and the next state
+ * follow from S, V and Y (derivation in csrc/dplr_chunk.cu; the post's
+ * sections 1 and 3 give the recurrence, the Kimi Linear report's appendix B
+ * the same construction for KDA's binding).  Chunks of 64 tokens in parallel
+ * for the per-chunk algebra; the state passes through the chunks in order (one
+ * 16-value-column slice per CTA).  Exact fp32 arithmetic; any g_min.
+ *   args            : as kda_dplr_recurrent_fwd
+ *   workspace       : device memory, 256-byte aligned, at least the size
+ *                     kda_dplr_chunk_workspace_size returns: one record per
+ *                     (b, h, chunk) of 4 (D_k rounded up to 4 + C (3 D_k +
+ *                     C + 2 D_v) + D_k D_v) bytes with C = 64, rounded up to
+ *                     16 bytes (240.5 KB at D_k = D_v = 128)
+ * Errors: as kda_dplr_recurrent_fwd; WORKSPACE; UNSUPPORTED if B*H*chunks
+ * exceeds 2^31 - 1.
+ */
+kda_status_t kda_dplr_chunk_workspace_size(const kda_dplr_args *args, size_t *bytes);
+
+kda_status_t kda_dplr_chunk_fwd(const kda_dplr_args *args, void *workspace, size_t workspace_bytes);
+
+/*
  * kda_decode_step — one token of the Eq. 1 recurrence for B independent
  * sequences, fused in one pass over the fp32 state (the fused recurrent
  * form: decay the state, predict k^T S, form the residual beta (v - pred),

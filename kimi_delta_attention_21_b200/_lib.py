@@ -96,6 +96,8 @@ SIGNATURES = {
     "kda_chunk_bwd_workspace_size": (ctypes.c_int, [ctypes.POINTER(RecBwdArgs), ctypes.POINTER(ctypes.c_size_t)]),
     "kda_chunk_bwd": (ctypes.c_int, [ctypes.POINTER(RecBwdArgs)]),
     "kda_dplr_recurrent_fwd": (ctypes.c_int, [ctypes.POINTER(DplrArgs)]),
+    "kda_dplr_chunk_workspace_size": (ctypes.c_int, [ctypes.POINTER(DplrArgs), ctypes.POINTER(ctypes.c_size_t)]),
+    "kda_dplr_chunk_fwd": (ctypes.c_int, [ctypes.POINTER(DplrArgs), ctypes.c_void_p, ctypes.c_size_t]),
     "kda_norm_gate": (ctypes.c_int, [_p, _p, _i64, _i32, _i32, _f32, _p, ctypes.c_int, _p]),
     "kda_out_proj": (ctypes.c_int, [_p, _p, _i64, _i32, _i32, _p, ctypes.c_int, _p]),
     "kda_out_norm_gate_proj_workspace_size": (ctypes.c_int, [_i64, _i32, _i32, ctypes.c_int,

@@ -192,7 +192,26 @@ def _bwd(entry, q, k, v, beta, d_o, z, log_decay, g_min, initial_state, d_final_
 def dplr_recurrent_fwd(q, k, v, a, b, *, z=None, log_decay=None, g_min=-5.0, initial_state=None, out=None,
                        final_state=None):
     """General DPLR recurrence S_t = (Diag(alpha_t) - a_t b_t^T) S_{t-1} + k_t v_t^T, o_t = S_t^T q_t
-    (kda_dplr_recurrent_fwd).  q, k, a, b, z (B,S,H,D_k); v (B,S,H,D_v).  Returns (o, final_state fp32)."""
+    (kda_dplr_recurrent_fwd, token by token).  q, k, a, b, z (B,S,H,D_k); v (B,S,H,D_v).  Returns (o,
+    final_state fp32)."""
+    return _dplr(False, q, k, v, a, b, z, log_decay, g_min, initial_state, out, final_state, None)
+
+
+def dplr_chunk_fwd(q, k, v, a, b, *, z=None, log_decay=None, g_min=-5.0, initial_state=None, out=None,
+                   final_state=None, workspace=None):
+    """The same recurrence and outputs in chunk form (kda_dplr_chunk_fwd)."""
+    return _dplr(True, q, k, v, a, b, z, log_decay, g_min, initial_state, out, final_state, workspace)
+
+
+def dplr_chunk_workspace_bytes(B, S, H, Dk, Dv):
+    """Workspace bytes kda_dplr_chunk_fwd needs for these sizes."""
+    args = DplrArgs(B=B, S=S, H=H, D_k=Dk, D_v=Dv, dtype=_lib.KDA_BF16, g_min=-1.0)
+    n = ctypes.c_size_t(0)
+    check("kda_dplr_chunk_workspace_size", _lib.load().kda_dplr_chunk_workspace_size(ctypes.byref(args), ctypes.byref(n)))
+    return n.value
+
+
+def _dplr(chunked, q, k, v, a, b, z, log_decay, g_min, initial_state, out, final_state, workspace):
     _dev(q, "q")
     dt = q.dtype
     B, S, H, Dk = q.shape
@@ -213,7 +232,17 @@ def dplr_recurrent_fwd(q, k, v, a, b, *, z=None, log_decay=None, g_min=-5.0, ini
                     a=_ptr(a), b=_ptr(b), z=_ptr(z), log_decay=_ptr(log_decay), g_min=float(g_min),
                     initial_state=_ptr(initial_state), o=_ptr(out), final_state=_ptr(final_state),
                     stream=_stream(q.device))
-    check("kda_dplr_recurrent_fwd", _lib.load().kda_dplr_recurrent_fwd(ctypes.byref(args)))
+    lib = _lib.load()
+    if not chunked:
+        check("kda_dplr_recurrent_fwd", lib.kda_dplr_recurrent_fwd(ctypes.byref(args)))
+        return out, final_state
+    n = ctypes.c_size_t(0)
+    check("kda_dplr_chunk_workspace_size", lib.kda_dplr_chunk_workspace_size(ctypes.byref(args), ctypes.byref(n)))
+    ws = workspace
+    if ws is None:
+        ws = torch.empty(max(1, n.value), dtype=torch.uint8, device=q.device)
+    _dev(ws, "workspace", torch.uint8)
+    check("kda_dplr_chunk_fwd", lib.kda_dplr_chunk_fwd(ctypes.byref(args), _ptr(ws), ws.numel()))
     return out, final_state
 
 

@@ -342,8 +342,8 @@ kda_status_t kda_chunk_bwd(const kda_recurrent_bwd_args *a) {
     return launch_chunk_bwd(*a, (cudaStream_t)a->stream);
 }
 
-kda_status_t kda_dplr_recurrent_fwd(const kda_dplr_args *a) {
-    g_err[0] = 0;
+// The checks both DPLR entry points share: sizes, dtype, g_min, pointers and overlaps.
+static kda_status_t dplr_validate(const kda_dplr_args *a) {
     if (!a) return fail(KDA_ERR_INVALID_ARG, "args is NULL");
     KDA_TRY(check_dtype(a->dtype));
     KDA_TRY(check_gmin(a->g_min));
@@ -379,16 +379,58 @@ kda_status_t kda_dplr_recurrent_fwd(const kda_dplr_args *a) {
         KDA_TRY(check_no_overlap(Buf{a->final_state, ns, "final_state"}, ins, nin));
         if (a->S > 0 && overlap(a->final_state, ns, a->o, nv * es)) return fail(KDA_ERR_INVALID_ARG, "final_state overlaps o");
     }
-    if (a->S == 0) {
-        if (a->final_state) {
-            cudaError_t e = a->initial_state ? cudaMemcpyAsync(a->final_state, a->initial_state, ns,
-                                                               cudaMemcpyDeviceToDevice, (cudaStream_t)a->stream)
-                                             : cudaMemsetAsync(a->final_state, 0, ns, (cudaStream_t)a->stream);
-            if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "empty sequence: %s", cudaGetErrorString(e));
-        }
-        return KDA_OK;
+    return KDA_OK;
+}
+
+// An empty sequence: final_state = initial_state (or zero).
+static kda_status_t dplr_empty(const kda_dplr_args *a) {
+    const size_t ns = (size_t)a->B * a->H * a->D_k * a->D_v * 4;
+    if (a->final_state) {
+        cudaError_t e = a->initial_state ? cudaMemcpyAsync(a->final_state, a->initial_state, ns,
+                                                           cudaMemcpyDeviceToDevice, (cudaStream_t)a->stream)
+                                         : cudaMemsetAsync(a->final_state, 0, ns, (cudaStream_t)a->stream);
+        if (e != cudaSuccess) return fail(KDA_ERR_CUDA, "empty sequence: %s", cudaGetErrorString(e));
     }
+    return KDA_OK;
+}
+
+kda_status_t kda_dplr_recurrent_fwd(const kda_dplr_args *a) {
+    g_err[0] = 0;
+    KDA_TRY(dplr_validate(a));
+    if (a->B == 0) return KDA_OK;
+    if (a->S == 0) return dplr_empty(a);
     return launch_dplr(*a, (cudaStream_t)a->stream);
+}
+
+kda_status_t kda_dplr_chunk_workspace_size(const kda_dplr_args *a, size_t *bytes) {
+    g_err[0] = 0;
+    if (!bytes) return fail(KDA_ERR_INVALID_ARG, "bytes is NULL");
+    if (!a) return fail(KDA_ERR_INVALID_ARG, "args is NULL");
+    if (a->B < 0 || a->S < 0 || a->H < 1 || a->D_k < 1 || a->D_v < 1) return fail(KDA_ERR_INVALID_ARG, "bad sizes");
+    if (a->D_k > 128 || a->D_v > 128) return fail(KDA_ERR_UNSUPPORTED, "D_k and D_v must be <= 128");
+    *bytes = dplr_chunk_workspace(a->B, a->S, a->H, a->D_k, a->D_v);
+    return KDA_OK;
+}
+
+kda_status_t kda_dplr_chunk_fwd(const kda_dplr_args *a, void *workspace, size_t workspace_bytes) {
+    g_err[0] = 0;
+    KDA_TRY(dplr_validate(a));
+    if (a->B == 0) return KDA_OK;
+    if (a->S == 0) return dplr_empty(a);
+    KDA_OPT_PTR(workspace, "workspace", 256);
+    const size_t need = dplr_chunk_workspace(a->B, a->S, a->H, a->D_k, a->D_v);
+    if (!workspace || workspace_bytes < need)
+        return fail(KDA_ERR_WORKSPACE, "workspace needs %zu bytes (got %zu)", need, workspace ? workspace_bytes : (size_t)0);
+    const size_t es = esize(a->dtype);
+    const size_t nk = (size_t)a->B * a->S * a->H * a->D_k, nv = (size_t)a->B * a->S * a->H * a->D_v;
+    const size_t ns = (size_t)a->B * a->H * a->D_k * a->D_v * 4;
+    const Buf ins[] = {
+        {a->q, nk * es, "q"}, {a->k, nk * es, "k"}, {a->v, nv * es, "v"}, {a->a, nk * es, "a"}, {a->b, nk * es, "b"},
+        {!a->log_decay ? a->z : nullptr, nk * es, "z"}, {a->log_decay, nk * 4, "log_decay"},
+        {a->initial_state, ns, "initial_state"}, {a->o, nv * es, "o"}, {a->final_state, ns, "final_state"},
+    };
+    KDA_TRY(check_no_overlap(Buf{workspace, need, "workspace"}, ins, (int)(sizeof(ins) / sizeof(ins[0]))));
+    return launch_dplr_chunk(*a, workspace, (cudaStream_t)a->stream);
 }
 
 kda_status_t kda_decode_step(const kda_decode_args *a) {

@@ -117,8 +117,10 @@ kda_status_t launch_rec_bwd(const kda_recurrent_bwd_args &a, cudaStream_t st);
 size_t chunk_bwd_workspace(int64_t B, int64_t S, int H, int Dk, int Dv);
 kda_status_t launch_chunk_bwd(const kda_recurrent_bwd_args &a, cudaStream_t st);
 
-// General DPLR recurrence, token by token (the comparator).
+// General DPLR recurrence, token by token (the comparator), and in chunk form (per-chunk records).
 kda_status_t launch_dplr(const kda_dplr_args &a, cudaStream_t st);
+size_t dplr_chunk_workspace(int64_t B, int64_t S, int H, int Dk, int Dv);
+kda_status_t launch_dplr_chunk(const kda_dplr_args &a, void *workspace, cudaStream_t st);
 
 kda_status_t launch_norm_gate(const void *o, const void *gl, int64_t N, int H, int Dv, float eps,
                               void *x, kda_dtype_t dt, cudaStream_t st);

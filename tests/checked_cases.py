@@ -1,7 +1,7 @@
 """The calls the checked-build test runs, shared by the test and the child
 process that runs them on libkda_checked.so: the tensor-core chunk engine on
 segmented sequences (maps, combine, chains; z and log-decay inputs, gate), the
-GDN engine, the recurrent and chunkwise backward and the DPLR comparator.  As a script:
+GDN engine, the recurrent and chunkwise backward and the DPLR comparator (both forms).  As a script:
 `python tests/checked_cases.py OUT.npz` runs them on the library the binding
 loads (KDA_LIBRARY picks it) and saves the results with the device counters."""
 import ctypes
@@ -74,6 +74,9 @@ def run_cases():
     o, sf = K.dplr_recurrent_fwd(d["q"], d["k"], d["v"], d["k"], d["q"], z=d["z"], initial_state=d["S0"])
     keep("dplr_o", o)
     keep("dplr_sf", sf)
+    o, sf = K.dplr_chunk_fwd(d["q"], d["k"], d["v"], d["k"], d["q"], z=d["z"], initial_state=d["S0"])
+    keep("dplrc_o", o)
+    keep("dplrc_sf", sf)
     torch.cuda.synchronize()
     lib = K.load_library()
     n, chk = ctypes.c_uint32(0), ctypes.c_int(-1)

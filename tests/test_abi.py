@@ -219,3 +219,37 @@ def test_checked_build_reports_itself():
         assert chk.value == want
         assert st in (_lib.KDA_OK, _lib.KDA_ERR_CUDA)
         assert f(None, 0, None) == _lib.KDA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("B,S,H,Dk,Dv", [(1, 4096, 16, 128, 128), (2, 100, 3, 18, 13)])
+def test_chunk_backward_and_dplr_workspace_rules(B, S, H, Dk, Dv):
+    """The two SIMT chunk paths size their workspace as one record per (b, h, chunk): the chunkwise
+    backward's C (4 Dk + 3 Dv + 3 C) + 2 Dk Dv + ceil(Dv / 16) Dk floats, the chunked DPLR's
+    (Dk rounded to 4) + C (3 Dk + C + 2 Dv) + Dk Dv floats, each rounded up to 4 floats (C = 64)."""
+    lib = _lib.load()
+    C, nc = 64, (S + 63) // 64
+    r4 = lambda x: (x + 3) // 4 * 4
+    want_bwd = B * H * nc * r4(C * (4 * Dk + 3 * Dv + 3 * C) + 2 * Dk * Dv + (Dv + 15) // 16 * Dk) * 4
+    want_dplr = B * H * nc * r4(r4(Dk) + C * (3 * Dk + C + 2 * Dv) + Dk * Dv) * 4
+    n = ctypes.c_size_t(0)
+    rb = _lib.RecBwdArgs(B=B, S=S, H=H, D_k=Dk, D_v=Dv, dtype=_lib.KDA_BF16, g_min=-5.0)
+    assert lib.kda_chunk_bwd_workspace_size(ctypes.byref(rb), ctypes.byref(n)) == _lib.KDA_OK
+    assert n.value == want_bwd
+    da = _lib.DplrArgs(B=B, S=S, H=H, D_k=Dk, D_v=Dv, dtype=_lib.KDA_BF16, g_min=-5.0)
+    assert lib.kda_dplr_chunk_workspace_size(ctypes.byref(da), ctypes.byref(n)) == _lib.KDA_OK
+    assert n.value == want_dplr
+
+
+def test_chunked_dplr_refuses_a_short_workspace():
+    """Validated on the host before any launch (fake, aligned, non-NULL device pointers)."""
+    lib = _lib.load()
+    B, S, H, D = 1, 130, 2, 32
+    fake = [ctypes.c_void_p(0x1000000 * (i + 1)) for i in range(8)]
+    da = _lib.DplrArgs(B=B, S=S, H=H, D_k=D, D_v=D, dtype=_lib.KDA_BF16, q=fake[0], k=fake[1], v=fake[2], a=fake[3],
+                       b=fake[4], z=fake[5], g_min=-5.0, o=fake[6])
+    n = ctypes.c_size_t(0)
+    assert lib.kda_dplr_chunk_workspace_size(ctypes.byref(da), ctypes.byref(n)) == _lib.KDA_OK
+    n0 = lib.kda_launch_count()
+    assert lib.kda_dplr_chunk_fwd(ctypes.byref(da), fake[7], n.value - 16) == _lib.KDA_ERR_WORKSPACE
+    assert lib.kda_dplr_chunk_fwd(ctypes.byref(da), None, n.value) == _lib.KDA_ERR_WORKSPACE
+    assert lib.kda_launch_count() == n0
