@@ -16,6 +16,10 @@ A debugging aid beside the oracle, never used by the product path.  Two forms:
   proof of Proposition 2 fixes it as multiplying the whole bracket (reading
   recorded in the design notes), and the brute-force pin confirms it.
 
+* ``matrix_backward``: reverse-mode differentiation of the ``matrix_chunk``
+  lines, chunk by chunk (the chunkwise backward's algebra), pinned against the
+  oracle's gradient of the plain recurrence.
+
 * ``matrix_chunk``: the same chunk in matrix form, as a GPU kernel evaluates
   it: A = strictly-lower decayed beta-weighted K K^T, the unit-lower solve
   (I + A)[W | U] = [Diag(beta)(K * e^G) | Diag(beta) V], V' = U - W S_0,
@@ -124,3 +128,70 @@ def matrix_forward(q, k, v, beta, log_alpha, S0, C):
         o[s:e] = r["O"]
         S = r["S_next"]
     return o, S
+
+
+def matrix_backward(q, k, v, beta, log_alpha, S0, dO, dST, C):
+    """Gradient of one sequence through ``matrix_chunk``, chunk by chunk.  q,k,log_alpha (T,Dk), v, dO
+    (T,Dv), beta (T,), S0, dST (Dk,Dv) (dST = dL/dS_T).  Returns a dict of fp64 arrays dq, dk (T,Dk), dv
+    (T,Dv), dbeta (T,), dlog_alpha (T,Dk) and dS0 (Dk,Dv).  Per chunk, with E[r,i,c] = e^{G_rc - G_ic}:
+    the state gradient runs back through the chunks (dV' = M^T dO + Kd dS_next, dS = (Q e^G)^T dO +
+    Diag(e^{G_C}) dS_next - W^T dV'), everything else is chunk-local (through T = (I + A)^{-1}:
+    dA = -T^T dT T^T), and every decayed product contributes in its row role and its column role."""
+    f = lambda x: np.asarray(x, np.float64)
+    q, k, v, beta, log_alpha, dO = f(q), f(k), f(v), f(beta), f(log_alpha), f(dO)
+    T = q.shape[0]
+    starts = list(range(0, T, C))
+    fwd, entering = [], []
+    S = f(S0).copy()
+    for s in starts:
+        e = min(T, s + C)
+        n = e - s
+        G = np.cumsum(log_alpha[s:e], axis=0)
+        E = np.exp(G[:, None, :] - G[None, :, :])
+        low, le = np.tril(np.ones((n, n)), -1), np.tril(np.ones((n, n)))
+        P = np.einsum('rc,ic,ric->ri', k[s:e], k[s:e], E) * low
+        M = np.einsum('rc,ic,ric->ri', q[s:e], k[s:e], E) * le
+        Tm = np.linalg.inv(np.eye(n) + beta[s:e, None] * P)
+        Kg, Qg, Kd = k[s:e] * np.exp(G), q[s:e] * np.exp(G), k[s:e] * np.exp(G[-1] - G)
+        W, U = Tm @ (beta[s:e, None] * Kg), Tm @ (beta[s:e, None] * v[s:e])
+        Vp = U - W @ S
+        entering.append(S)
+        fwd.append(dict(G=G, E=E, P=P, M=M, T=Tm, Kg=Kg, Qg=Qg, Kd=Kd, W=W, Vp=Vp, low=low, le=le))
+        S = np.exp(G[-1])[:, None] * S + Kd.T @ Vp
+    out = {n: np.zeros_like(x) for n, x in (("dq", q), ("dk", k), ("dv", v), ("dbeta", beta),
+                                            ("dlog_alpha", log_alpha))}
+    dS = f(dST).copy()
+    leaving = [None] * len(starts)
+    dvp = [None] * len(starts)
+    for j in reversed(range(len(starts))):
+        s, e, c = starts[j], min(T, starts[j] + C), fwd[j]
+        leaving[j] = dS
+        dvp[j] = c["M"].T @ dO[s:e] + c["Kd"] @ dS
+        dS = c["Qg"].T @ dO[s:e] + np.exp(c["G"][-1])[:, None] * dS - c["W"].T @ dvp[j]
+    out["dS0"] = dS
+    for j, s in enumerate(starts):
+        e, c = min(T, s + C), fwd[j]
+        Sj, dSn, dVp = entering[j], leaving[j], dvp[j]
+        kk, qq, vv, bb, do = k[s:e], q[s:e], v[s:e], beta[s:e], dO[s:e]
+        dQg, dKd = do @ Sj.T, c["Vp"] @ dSn.T
+        dgam = np.sum(dSn * Sj, axis=1)
+        dM = (do @ c["Vp"].T) * c["le"]
+        dW = -dVp @ Sj.T
+        dT = dVp @ (bb[:, None] * vv).T + dW @ (bb[:, None] * c["Kg"]).T
+        dBv, dBk = c["T"].T @ dVp, c["T"].T @ dW
+        dA = -(c["T"].T @ dT @ c["T"].T) * c["low"]
+        out["dbeta"][s:e] = np.sum(dBv * vv, 1) + np.sum(dBk * c["Kg"], 1) + np.sum(dA * c["P"], 1)
+        dP, E = bb[:, None] * dA, c["E"]
+        out["dv"][s:e] = bb[:, None] * dBv
+        dKg = bb[:, None] * dBk
+        x_row = np.einsum('ri,ic,ric->rc', dP, kk, E)   # P[r,i] in its row role
+        x_col = np.einsum('ri,rc,ric->ic', dP, kk, E)   # ... and its column role
+        y_row = np.einsum('ri,ic,ric->rc', dM, kk, E)
+        y_col = np.einsum('ri,rc,ric->ic', dM, qq, E)
+        eG, eD = np.exp(c["G"]), np.exp(c["G"][-1] - c["G"])
+        out["dq"][s:e] = dQg * eG + y_row
+        out["dk"][s:e] = dKg * eG + dKd * eD + x_row + x_col + y_col
+        dG = dQg * c["Qg"] + dKg * c["Kg"] - dKd * c["Kd"] + kk * x_row - kk * x_col + qq * y_row - kk * y_col
+        dG[-1] += np.sum(dKd * c["Kd"], 0) + dgam * np.exp(c["G"][-1])
+        out["dlog_alpha"][s:e] = np.cumsum(dG[::-1], axis=0)[::-1]
+    return out
