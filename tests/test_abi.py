@@ -253,3 +253,33 @@ def test_chunked_dplr_refuses_a_short_workspace():
     assert lib.kda_dplr_chunk_fwd(ctypes.byref(da), fake[7], n.value - 16) == _lib.KDA_ERR_WORKSPACE
     assert lib.kda_dplr_chunk_fwd(ctypes.byref(da), None, n.value) == _lib.KDA_ERR_WORKSPACE
     assert lib.kda_launch_count() == n0
+
+
+def test_chunk_backward_validation():
+    """Host-side refusals of kda_chunk_bwd before any launch (fake, aligned, non-NULL device pointers)."""
+    lib = _lib.load()
+    fake = [ctypes.c_void_p(0x1000000 * (i + 1)) for i in range(13)]
+    B, S, H, D = 1, 130, 2, 32
+
+    def args(**kw):
+        base = dict(B=B, S=S, H=H, D_k=D, D_v=D, dtype=_lib.KDA_BF16, q=fake[0], k=fake[1], v=fake[2], z=fake[3],
+                    g_min=-5.0, beta=fake[4], d_o=fake[5], dq=fake[6], dk=fake[7], dv=fake[8], dbeta=fake[9],
+                    dz=fake[10])
+        base.update(kw)
+        return _lib.RecBwdArgs(**base)
+
+    n = ctypes.c_size_t(0)
+    a = args()
+    assert lib.kda_chunk_bwd_workspace_size(ctypes.byref(a), ctypes.byref(n)) == _lib.KDA_OK
+    n0 = lib.kda_launch_count()
+    a.workspace, a.workspace_bytes = fake[11], n.value - 16
+    assert lib.kda_chunk_bwd(ctypes.byref(a)) == _lib.KDA_ERR_WORKSPACE
+    big = args(D_k=129)
+    assert lib.kda_chunk_bwd_workspace_size(ctypes.byref(big), ctypes.byref(n)) == _lib.KDA_ERR_UNSUPPORTED
+    assert lib.kda_chunk_bwd(ctypes.byref(big)) == _lib.KDA_ERR_UNSUPPORTED
+    pos = args(g_min=0.5)
+    assert lib.kda_chunk_bwd(ctypes.byref(pos)) == _lib.KDA_ERR_INVALID_ARG
+    nodo = args(d_o=None)
+    nodo.workspace, nodo.workspace_bytes = fake[11], 1 << 40
+    assert lib.kda_chunk_bwd(ctypes.byref(nodo)) == _lib.KDA_ERR_INVALID_ARG
+    assert lib.kda_launch_count() == n0
