@@ -163,16 +163,16 @@ kda_status_t kda_gate(const void *z, kda_dtype_t dtype, int64_t n, float g_min, 
 
 static kda_status_t chunk_workspace_impl(const kda_chunk_args *a, size_t *bytes, bool gdn) {
     if (!bytes) return fail(KDA_ERR_INVALID_ARG, "bytes is NULL");
-    int chunk;
-    bool tc;
+    int chunk = 0;
+    bool tc = false;
     KDA_TRY(chunk_validate(a, &chunk, &tc, gdn));
     *bytes = tc ? chunk_tc_workspace(*a) : chunk_simt_workspace(*a, chunk);
     return KDA_OK;
 }
 
 static kda_status_t chunk_fwd_impl(const kda_chunk_args *a, bool gdn) {
-    int chunk;
-    bool tc;
+    int chunk = 0;
+    bool tc = false;
     KDA_TRY(chunk_validate(a, &chunk, &tc, gdn));
     if (a->B == 0) return KDA_OK;
     const size_t es = esize(a->dtype);
