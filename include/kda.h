@@ -268,7 +268,7 @@ kda_status_t kda_chunk_bwd(const kda_recurrent_bwd_args *args);
  * (KDA's).  KDA is the case a_t = beta_t k_t, b_t = k_t * alpha_t with the
  * write key beta_t k_t; without that binding the chunkwise UT/WY form of
  * kda_chunk_fwd does not apply, and this entry point evaluates the recurrence
- * token by token, exact fp32.
+ * token by token, exact fp32 (kda_dplr_chunk_fwd below is its chunk form).
  *   q, k, a, b, z (B, S, H, D_k) dtype;  log_decay (B, S, H, D_k) fp32 or NULL
  *   v (B, S, H, D_v) dtype;  initial_state (B, H, D_k, D_v) fp32 or NULL
  *   o (B, S, H, D_v) dtype out;  final_state (B, H, D_k, D_v) fp32 out or NULL

@@ -6,8 +6,9 @@
 // with free erase directions a_t, b_t, evaluated as
 //   w = b_t^T S_{t-1};  S_t = Diag(alpha_t) S_{t-1} - a_t w^T + k_t v_t^T;  o_t = S_t^T q_t.
 // It is the comparator of the KDA engines: without KDA's binding (a = beta k,
-// b = k * alpha) the chunkwise UT/WY form does not apply as is, and this is the
-// form every such transition has.  Exact fp32; a block owns one (b, h) and 16
+// b = k * alpha) the KDA engines' chunkwise UT/WY form does not apply as is;
+// this is the form every such transition has, and dplr_chunk.cu the chunk form
+// of the general case.  Exact fp32; a block owns one (b, h) and 16
 // value columns with the state slice in registers (two sums over the key rows
 // per token, one block barrier each).
 #include "rec_common.cuh"
