@@ -271,10 +271,19 @@ kda_status_t kda_recurrent_bwd_workspace_size(const kda_recurrent_bwd_args *a, s
     return KDA_OK;
 }
 
+// The SIMT chunk paths launch one CTA per (b, h, chunk): at most 2^31 - 1 of them.
+static kda_status_t check_chunk_units(int64_t B, int64_t S, int H, const char *what) {
+    const int64_t nc = (S + 63) / 64;
+    if (B > 0 && nc > 0 && B * H > 0x7fffffffLL / nc)
+        return fail(KDA_ERR_UNSUPPORTED, "%s: B*H*chunks exceeds 2^31 - 1", what);
+    return KDA_OK;
+}
+
 kda_status_t kda_chunk_bwd_workspace_size(const kda_recurrent_bwd_args *a, size_t *bytes) {
     g_err[0] = 0;
     if (!bytes) return fail(KDA_ERR_INVALID_ARG, "bytes is NULL");
     KDA_TRY(rec_bwd_validate(a));
+    KDA_TRY(check_chunk_units(a->B, a->S, a->H, "chunk backward"));
     *bytes = chunk_bwd_workspace(a->B, a->S, a->H, a->D_k, a->D_v);
     return KDA_OK;
 }
@@ -338,6 +347,7 @@ kda_status_t kda_chunk_bwd(const kda_recurrent_bwd_args *a) {
     g_err[0] = 0;
     KDA_TRY(rec_bwd_validate(a));
     if (a->B == 0) return KDA_OK;
+    KDA_TRY(check_chunk_units(a->B, a->S, a->H, "chunk backward"));
     KDA_TRY(bwd_check_buffers(a, chunk_bwd_workspace(a->B, a->S, a->H, a->D_k, a->D_v)));
     return launch_chunk_bwd(*a, (cudaStream_t)a->stream);
 }
@@ -408,6 +418,7 @@ kda_status_t kda_dplr_chunk_workspace_size(const kda_dplr_args *a, size_t *bytes
     if (!a) return fail(KDA_ERR_INVALID_ARG, "args is NULL");
     if (a->B < 0 || a->S < 0 || a->H < 1 || a->D_k < 1 || a->D_v < 1) return fail(KDA_ERR_INVALID_ARG, "bad sizes");
     if (a->D_k > 128 || a->D_v > 128) return fail(KDA_ERR_UNSUPPORTED, "D_k and D_v must be <= 128");
+    KDA_TRY(check_chunk_units(a->B, a->S, a->H, "chunked DPLR"));
     *bytes = dplr_chunk_workspace(a->B, a->S, a->H, a->D_k, a->D_v);
     return KDA_OK;
 }
@@ -416,6 +427,7 @@ kda_status_t kda_dplr_chunk_fwd(const kda_dplr_args *a, void *workspace, size_t 
     g_err[0] = 0;
     KDA_TRY(dplr_validate(a));
     if (a->B == 0) return KDA_OK;
+    KDA_TRY(check_chunk_units(a->B, a->S, a->H, "chunked DPLR"));
     if (a->S == 0) return dplr_empty(a);
     KDA_OPT_PTR(workspace, "workspace", 256);
     const size_t need = dplr_chunk_workspace(a->B, a->S, a->H, a->D_k, a->D_v);

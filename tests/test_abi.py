@@ -283,3 +283,16 @@ def test_chunk_backward_validation():
     nodo.workspace, nodo.workspace_bytes = fake[11], 1 << 40
     assert lib.kda_chunk_bwd(ctypes.byref(nodo)) == _lib.KDA_ERR_INVALID_ARG
     assert lib.kda_launch_count() == n0
+
+
+def test_simt_chunk_paths_refuse_too_many_chunks():
+    """One CTA per (b, h, chunk): a size query past 2^31 - 1 of them is refused, not wrapped."""
+    lib = _lib.load()
+    n = ctypes.c_size_t(0)
+    S = 64 * (1 << 28)                                    # 2^28 chunks per sequence, 16 heads
+    rb = _lib.RecBwdArgs(B=1, S=S, H=16, D_k=128, D_v=128, dtype=_lib.KDA_BF16, g_min=-5.0)
+    assert lib.kda_chunk_bwd_workspace_size(ctypes.byref(rb), ctypes.byref(n)) == _lib.KDA_ERR_UNSUPPORTED
+    da = _lib.DplrArgs(B=1, S=S, H=16, D_k=128, D_v=128, dtype=_lib.KDA_BF16, g_min=-5.0)
+    assert lib.kda_dplr_chunk_workspace_size(ctypes.byref(da), ctypes.byref(n)) == _lib.KDA_ERR_UNSUPPORTED
+    ok = _lib.RecBwdArgs(B=1, S=64 * (1 << 20), H=16, D_k=128, D_v=128, dtype=_lib.KDA_BF16, g_min=-5.0)
+    assert lib.kda_chunk_bwd_workspace_size(ctypes.byref(ok), ctypes.byref(n)) == _lib.KDA_OK
